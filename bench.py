@@ -1,0 +1,397 @@
+#!/usr/bin/env python3
+"""Sparse-attention decode throughput on B200: indexer + top-K + sparse MLA attention.
+
+One step = one fused ``sa_decode`` over one batch of synthetic queries (all
+three steps of the path).  Prints ONE JSON line (rank 0):
+
+  value     query-tokens/s over all ranks, device time (CUDA events), inputs
+            resident in HBM, L2 flushed (256 MiB write) before every timed step;
+  e2e       the same metric through the public API with host buffers: pinned
+            host -> device copy of the step's queries, the call, device -> host
+            copy of the outputs, all inside the timed region;
+  roofline  the dominant phase's algorithmic bytes / its event-timed duration
+            against the measured HBM copy bandwidth;
+  cpu_baseline  the fp64 oracle on a bounded sample, on this host's cores.
+
+``--impl reference`` times the fp64 oracle instead (rank 0 only).
+Multi-GPU (torchrun): every rank decodes its own batch (seeded per rank), no
+collective on the data path ("scaling": "weak").
+"""
+from __future__ import annotations
+
+import argparse
+import dataclasses
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+DEFAULT_WORKLOAD = "decode_b64_16k_32k_planted"
+METRIC = "sparse-attn decode query-tokens/s (indexer+top-K+SFA); % of HBM roofline"
+UNIT = "query-tokens/s"
+FALLBACK_HBM_GBS = 6650.0
+SPEC_HBM_GBS = 8000.0
+FLUSH_BYTES = 256 << 20
+
+
+def parse():
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="target CPU time of the oracle baseline sample")
+    return ap.parse_args()
+
+
+# --------------------------------------------------------------- helpers ---
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def algorithmic_bytes(wl, idx: np.ndarray) -> dict:
+    """Bytes the path must move per step, by phase (the metric's definition:
+    indexer keys + key scales + selected KV rows + outputs)."""
+    sp = wl.spec
+    V = wl.visible.astype(np.int64)
+    key_b = sp.d_index * (1 if sp.index_dtype == "e4m3" else 4)
+    scale_b = 4 if sp.index_dtype == "e4m3" else 0
+    indexer = int((V * (key_b + scale_b)).sum())
+    n_sel = np.minimum(V, sp.top_k)
+    if sp.kv_dtype == "e4m3":
+        row_b = sp.d_latent + 2 * sp.d_rope
+        pages = 0
+        for t in range(wl.n_q):
+            sel = idx[t][idx[t] >= 0]
+            pages += np.unique(sel // sp.page_size).size
+        rows = int((n_sel * row_b).sum()) + 4 * pages
+    else:
+        row_b = (sp.d_latent + sp.d_rope) * (2 if sp.kv_dtype == "bf16" else 4)
+        rows = int((n_sel * row_b).sum())
+    out_b = 2 if sp.kv_dtype != "f32" else 4
+    outputs = wl.n_q * sp.heads * (sp.d_latent * out_b + 4)
+    return {"indexer": indexer, "topk": 0, "attention": rows + outputs,
+            "total": indexer + rows + outputs}
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"sa_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return None
+        sm, mx, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def traffic_for(kernel: str, source_files: list[str]):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel's
+    sources are unchanged since the capture; otherwise None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        rec = json.load(open(path)).get(kernel)
+    except Exception:
+        return None
+    if not rec:
+        return None
+    h = hashlib.sha256()
+    for f in source_files:
+        h.update(open(os.path.join(ROOT, f), "rb").read())
+    if rec.get("source_sha256") != h.hexdigest():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+# -------------------------------------------------------------- oracle leg ---
+
+def time_oracle(wl, budget_s: float):
+    """Run the oracle on a growing sample of queries until ~budget_s is spent."""
+    import oracle
+    from indexed_sparse_attention_lightning_b200 import workloads as W
+    order = W.stratified_rows(wl.n_q, wl.n_q)
+    rng = np.random.default_rng(12345)
+    order = rng.permutation(order)
+    done, spent = 0, 0.0
+    while done < len(order) and spent < budget_s:
+        sub = W.subset_queries(wl, order[done:done + 1])
+        t0 = time.perf_counter()
+        oracle.run(sub)
+        spent += time.perf_counter() - t0
+        done += 1
+    return done, spent
+
+
+def run_reference(args, rank: int, world: int):
+    if rank != 0:
+        return 0
+    from indexed_sparse_attention_lightning_b200 import workloads as W
+    wl = W.make_workload(W.spec(args.workload))
+    import oracle
+    cores = oracle.threads()
+    rng = np.random.default_rng(777)
+    order = rng.permutation(wl.n_q)
+    per_step = []
+    for k in range(args.warmup + args.steps):
+        rows = order[[k % wl.n_q]]
+        sub = W.subset_queries(wl, rows)
+        t0 = time.perf_counter()
+        oracle.run(sub, nthreads=cores)
+        dt = time.perf_counter() - t0
+        if k >= args.warmup:
+            per_step.append(dt)
+    total = sum(per_step)
+    value = args.steps / total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": wl.spec.name, "sample": "1 query per step, rotating"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": "1 query of the workload per step (fp64 oracle, all steps)"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- our leg ---
+
+def run_ours(args, rank: int, world: int, dist):
+    import torch
+    from indexed_sparse_attention_lightning_b200 import _abi, api
+    from indexed_sparse_attention_lightning_b200 import workloads as W
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    sp = W.spec(args.workload)
+    if rank > 0:
+        sp = dataclasses.replace(sp, seed=sp.seed + 1000 * rank)
+    wl = W.make_workload(sp)
+    cache, queries = api.upload(wl, dev)
+    K = sp.top_k
+    odt = "f32" if sp.kv_dtype == "f32" else "bf16"
+    ws = api.workspace(api.workspace_size(cache, queries, K, _abi.SA_WS_DECODE), dev)
+    idx = torch.empty((wl.n_q, K), dtype=torch.int32, device=dev)
+    out, lse = api._outputs(queries, sp.d_latent, None, None, odt)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(events=None):
+        api.decode(cache, queries, K, out=out, lse=lse, idx=idx, out_dtype=odt, ws=ws,
+                   phase_events=events)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    st = api.device_status(ws)
+    if st[0] != _abi.SA_OK:
+        raise RuntimeError(f"device status after warm-up: {st}")
+    nbytes = algorithmic_bytes(wl, idx.cpu().numpy())
+
+    n_phase = len(_abi.DECODE_PHASES)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_phase + 1)]
+          for _ in range(args.steps)]
+    outer = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+             for _ in range(args.steps)]
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    launches0 = _abi.lib().sa_kernel_launches()
+    with ClockSampler(local) as clocks:
+        for k in range(args.steps):
+            flush.zero_()
+            outer[k][0].record(stream)
+            step(ev[k])
+            outer[k][1].record(stream)
+        torch.cuda.synchronize()
+    launches = _abi.lib().sa_kernel_launches() - launches0
+    if dist is not None:
+        dist.barrier()
+    total_ms = sum(a.elapsed_time(b) for a, b in outer)
+    phase_ms = [sum(ev[k][i].elapsed_time(ev[k][i + 1]) for k in range(args.steps)) / args.steps
+                for i in range(n_phase)]
+    st = api.device_status(ws)
+    if st[0] != _abi.SA_OK:
+        raise RuntimeError(f"device status after timing: {st}")
+
+    # end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        host_in = api.host_queries(wl, pin=True)
+        host_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        host_lse = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+        h2d = 0
+        e2e_ms = 0.0
+        for k in range(args.warmup + args.steps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            h2d = queries.copy_from(host_in, non_blocking=True)
+            step()
+            host_out.copy_(out, non_blocking=True)
+            host_lse.copy_(lse, non_blocking=True)
+            b.record(stream)
+            b.synchronize()
+            if k >= args.warmup:
+                e2e_ms += a.elapsed_time(b)
+        d2h = out.numel() * out.element_size() + lse.numel() * lse.element_size()
+        e2e = {"ms_per_step": e2e_ms / args.steps, "h2d": h2d, "d2h": d2h}
+
+    # max over ranks
+    t = torch.tensor([total_ms, e2e["ms_per_step"] if e2e else 0.0], dtype=torch.float64,
+                     device=dev)
+    q_total = torch.tensor([wl.n_q], dtype=torch.float64, device=dev)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dist.all_reduce(q_total, op=dist.ReduceOp.SUM)
+    total_ms, e2e_step_ms = float(t[0]), float(t[1])
+    n_q_all = float(q_total[0])
+    if rank != 0:
+        return 0
+
+    ms_per_step = total_ms / args.steps
+    value = n_q_all * args.steps / (total_ms / 1e3)
+    peak, peak_kind = measured_peaks()
+    dom = int(np.argmax(phase_ms))
+    dom_name = _abi.DECODE_PHASES[dom]
+    dom_bytes = nbytes[dom_name]
+    achieved = dom_bytes / (phase_ms[dom] / 1e3) / 1e9 if phase_ms[dom] > 0 else 0.0
+    step_gbs = nbytes["total"] / (ms_per_step / 1e3) / 1e9
+    kernel_src = {"indexer": ["indexed_sparse_attention_lightning_b200/csrc/indexer_simt.cu"],
+                  "topk": ["indexed_sparse_attention_lightning_b200/csrc/topk.cu"],
+                  "attention": ["indexed_sparse_attention_lightning_b200/csrc/attn_simt.cu"]}
+    traffic = traffic_for(dom_name, kernel_src[dom_name])
+
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        n, spent = time_oracle(wl, args.cpu_seconds)
+        import oracle
+        cpu = {"value": n / spent, "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
+               "sample": f"{n} of {wl.n_q} queries of the same workload (fp64 oracle: scores, "
+                         f"top-K, attention), {spent:.1f} s"}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "e4m3+bf16", "data": "synthetic",
+        "config": {
+            "workload": sp.name, "batch": int(wl.seq_len.shape[0]), "queries_per_gpu": wl.n_q,
+            "context_mean": float(wl.seq_len.mean()), "top_k": K, "heads": sp.heads,
+            "index_heads": sp.h_index, "index_dim": sp.d_index, "kv_dtype": sp.kv_dtype,
+            "page_size": sp.page_size, "l2": "flushed before every timed step (256 MiB write)",
+            "parallelism": f"replicas x{world}"},
+        "roofline": {"bound": "hbm", "kernel": dom_name, "achieved": achieved, "peak": peak,
+                     "peak_kind": peak_kind, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": traffic},
+        "path_hbm": {"bytes_per_step": nbytes["total"], "achieved_gbs": step_gbs,
+                     "frac_of_measured": step_gbs / peak, "frac_of_8tbs": step_gbs / SPEC_HBM_GBS},
+        "phases_ms": dict(zip(_abi.DECODE_PHASES, phase_ms)),
+        "gpu_launches": int(launches),
+        "clocks": clocks.summary(),
+        "cpu_baseline": cpu,
+    }
+    if e2e:
+        line["e2e"] = {"value": n_q_all / (e2e_step_ms / 1e3), "unit": UNIT,
+                       "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    dist = None
+    if args.impl == "reference":
+        return run_reference(args, rank, world)   # rank 0 only; no process group needed
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    try:
+        return run_ours(args, rank, world, dist)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,224 @@
+/*
+ * sa.h -- indexed sparse attention for NVIDIA B200 (sm_100a): C ABI.
+ *
+ * The path has three steps, which the pages present as one pipeline
+ * ("Optimizing Next-Gen LLM Inference: Sparse Attention and Mixed Parallelism
+ * in Practice", §1 and §3; "Inference Acceleration for New Large Model
+ * Architectures", §3):
+ *
+ *   1. a lightweight indexer scores every visible cached position s of a query
+ *      t and weights the per-head scores by head weights:
+ *          I[t,s] = sum_j w[t,j] * max(0, q_I[t,j,:] . k_I[s,:]);
+ *   2. a per-query top-K keeps the K best positions;
+ *   3. a sparse attention kernel reads only those rows of the MLA latent cache
+ *      (512-d latent + 64-d rope, absorbed query) and returns the 512-d output.
+ *
+ * Both caches are paged and read in place through a page table
+ * ("Optimizing Next-Gen LLM Inference" §3.1; "Inference Acceleration" §3.1).
+ * Index keys and the latent cache may be FP8 ("Optimizing Next-Gen LLM
+ * Inference" §4): index keys as e4m3 with one fp32 scale per token, the latent
+ * as e4m3 with one fp32 scale per 64-token page tile (rope stays bf16).
+ *
+ * Conventions for every entry point
+ *  - All pointers marked "device" are CUDA device pointers owned by the
+ *    caller; the library allocates no memory.  Host structs are read during
+ *    the call only.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *    default stream) and never synchronises, except sa_device_status().
+ *  - Shapes and dtypes are checked on the host before anything is launched;
+ *    a bad argument returns SA_ERR_INVALID_ARG (or SA_ERR_UNSUPPORTED for a
+ *    valid but unimplemented combination) and launches nothing.
+ *  - Data errors found on the device (a page id outside [0, num_pages), a
+ *    query position past its sequence, a selected index outside the visible
+ *    range) never fault: the offending work is skipped and a status word in
+ *    the workspace records the first error; read it with sa_device_status().
+ *  - Positions are logical (0 .. q_pos), never physical rows, so results do
+ *    not depend on where pages sit in the pools.
+ *  - Device pointers must be 16-byte aligned.
+ *  - Nothing aborts, exits or traps.
+ */
+#ifndef SA_H
+#define SA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SA_API __attribute__((visibility("default")))
+#else
+#define SA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum sa_status {
+    SA_OK = 0,
+    SA_ERR_INVALID_ARG = 1,   /* shape, dtype, pointer or size rejected on the host */
+    SA_ERR_UNSUPPORTED = 2,   /* valid combination this build does not implement */
+    SA_ERR_WORKSPACE = 3,     /* workspace missing or smaller than sa_workspace_size() */
+    SA_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed */
+    SA_ERR_DEVICE_FAULT = 5,  /* bad data detected on the device (see detail code) */
+    SA_ERR_TIMEOUT = 6        /* a bounded device-side wait gave up */
+} sa_status;
+
+typedef enum sa_dtype {
+    SA_F32 = 0,
+    SA_BF16 = 1,
+    SA_E4M3 = 2               /* OCP e4m3fn code bytes, always paired with fp32 scales */
+} sa_dtype;
+
+/* Paged caches of one attention layer.
+ *
+ * Logical position s of sequence b lives in physical row
+ *     page_table[b * max_pages + s / page_size] * page_size + s % page_size
+ * of both pools below.  page_size must be 64.
+ */
+typedef struct sa_cache {
+    const int32_t *page_table;   /* device int32 [batch, max_pages]; unused slots may hold -1 */
+    const int32_t *seq_len;      /* device int32 [batch]: tokens cached per sequence */
+    int32_t batch;
+    int32_t max_pages;
+    int32_t num_pages;           /* physical pages in each pool */
+    int32_t page_size;           /* tokens per page (64) */
+
+    /* indexer keys */
+    sa_dtype index_dtype;        /* SA_E4M3 (production) or SA_F32 */
+    const void *k_index;         /* device [num_pages, page_size, d_index] */
+    const float *k_index_scale;  /* device [num_pages, page_size] one per token (SA_E4M3 only) */
+    int32_t d_index;
+
+    /* MLA latent KV rows */
+    sa_dtype kv_dtype;           /* SA_BF16, SA_E4M3 or SA_F32 */
+    const void *kv;              /* SA_F32/SA_BF16: [num_pages, page_size, d_latent + d_rope]
+                                  * SA_E4M3: latent codes [num_pages, page_size, d_latent] */
+    const void *kv_rope;         /* SA_E4M3 only: bf16 [num_pages, page_size, d_rope] */
+    const float *kv_scale;       /* SA_E4M3 only: [num_pages], one scale per 64-token page tile */
+    int32_t d_latent;            /* 512 (production) */
+    int32_t d_rope;              /* 64 (production) */
+} sa_cache;
+
+/* A batch of query tokens.  Query t belongs to sequence q_seq[t] and sits at
+ * position q_pos[t]; it sees positions 0 .. q_pos[t] (V_t = q_pos[t] + 1,
+ * causal and inclusive).  Decode is one query per sequence at seq_len - 1;
+ * chunked prefill is many queries of one sequence. */
+typedef struct sa_query {
+    int32_t n_q;
+    const int32_t *q_seq;        /* device int32 [n_q] */
+    const int32_t *q_pos;        /* device int32 [n_q] */
+    int32_t max_visible;         /* host: an upper bound of q_pos[t] + 1 over all t */
+
+    /* indexer query, same dtype as the cache's index keys */
+    const void *q_index;         /* device [n_q, h_index, d_index] */
+    const float *q_index_scale;  /* device [n_q, h_index] one per (token, head) (SA_E4M3 only) */
+    const float *w;              /* device [n_q, h_index] head weights */
+    int32_t h_index;
+
+    /* absorbed MLA attention query */
+    sa_dtype q_dtype;            /* SA_BF16 or SA_F32 */
+    const void *q;               /* device [n_q, heads, d_latent + d_rope] */
+    int32_t heads;
+    float sm_scale;              /* softmax scale applied to q . kv */
+} sa_query;
+
+/* Which entry point a workspace is sized for. */
+enum {
+    SA_WS_INDEXER = 1,
+    SA_WS_TOPK = 2,
+    SA_WS_ATTN = 4,
+    SA_WS_DECODE = 8
+};
+
+/* Bytes of device workspace the entry points in `uses` (an OR of SA_WS_*)
+ * need for this cache/query/K.  Returns 0 if the arguments are invalid.  The
+ * workspace must be 256-byte aligned; its contents need no initialisation and
+ * are overwritten by every call.  Calls that share a workspace must be
+ * ordered (same stream, or synchronised). */
+SA_API size_t sa_workspace_size(const sa_cache *cache, const sa_query *query, int32_t top_k,
+                         int32_t uses);
+
+/* Step 1 -- indexer scores ("Optimizing Next-Gen LLM Inference" §3.1:
+ * relevance scoring and head-weight weighting; "Inference Acceleration for New
+ * Large Model Architectures" §3.1 steps 1-2).
+ * Writes scores[t * ld_scores + s] (fp32) for every s < q_pos[t] + 1; other
+ * entries are left untouched.  ld_scores >= query->max_visible. */
+SA_API sa_status sa_indexer_score(const sa_cache *cache, const sa_query *query, float *scores,
+                           int64_t ld_scores, void *workspace, size_t workspace_bytes,
+                           void *stream);
+
+/* Step 2 -- top-K ("Optimizing Next-Gen LLM Inference" §3.1 Top-K selection;
+ * "Inference Acceleration" §3.1 step 3).
+ * For each row t of scores (fp32 [n_q, ld_scores], first valid_len[t] entries
+ * valid): writes idx[t * top_k .. +top_k) = the min(top_k, valid_len[t])
+ * positions with the largest scores, ties broken towards the lower position,
+ * in ascending position order, padded with -1.  Bit-exact.
+ * valid_len: device int32 [n_q]; max_valid: host bound on valid_len. */
+SA_API sa_status sa_topk(const float *scores, int64_t ld_scores, const int32_t *valid_len,
+                  int32_t n_q, int32_t max_valid, int32_t top_k, int32_t *idx,
+                  void *workspace, size_t workspace_bytes, void *stream);
+
+/* Step 3 -- sparse MLA attention over the selected rows ("Optimizing Next-Gen
+ * LLM Inference" §3.3; "Inference Acceleration" §3.2).
+ * idx: device int32 [n_q, top_k] logical positions (ascending not required;
+ * -1 entries are skipped).  For each query t and head h:
+ *   z_s = sm_scale * q[t,h,:] . kv[s,:]   (latent + rope; an e4m3 latent is
+ *                                          scaled by its page-tile scale)
+ *   out[t,h,:] = sum_s softmax(z)_s * kv[s, 0:d_latent],  lse[t,h] = log sum_s exp(z_s)
+ * out: device [n_q, heads, d_latent] in out_dtype (SA_BF16 or SA_F32);
+ * lse: device fp32 [n_q, heads] (may be NULL).  A query with no valid index
+ * gets out = 0 and lse = -inf. */
+SA_API sa_status sa_sparse_mla_attn(const sa_cache *cache, const sa_query *query, const int32_t *idx,
+                             int32_t top_k, void *out, sa_dtype out_dtype, float *lse,
+                             void *workspace, size_t workspace_bytes, void *stream);
+
+/* Steps 1-3 fused for decode and chunked prefill ("Optimizing Next-Gen LLM
+ * Inference" §3.1: scoring, weighting and selection without writing
+ * intermediates back; "Inference Acceleration" §3.1).
+ * The only intermediate that reaches device memory is what the top-K needs.
+ * idx_out (device int32 [n_q, top_k]) may be NULL; when given it receives the
+ * selected positions exactly as sa_topk would return them. */
+SA_API sa_status sa_decode(const sa_cache *cache, const sa_query *query, int32_t top_k,
+                    int32_t *idx_out, void *out, sa_dtype out_dtype, float *lse,
+                    void *workspace, size_t workspace_bytes, void *stream);
+
+/* sa_decode with phase timing: when `phase_events` is non-NULL it points to
+ * SA_DECODE_PHASES + 1 cudaEvent_t handles (created by the caller), which are
+ * recorded on `stream` before the first phase and after each phase, so that
+ * cudaEventElapsedTime between neighbours gives each phase's device time.
+ * Phases: indexer, top-K, sparse attention. */
+#define SA_DECODE_PHASES 3
+SA_API sa_status sa_decode_traced(const sa_cache *cache, const sa_query *query, int32_t top_k,
+                                  int32_t *idx_out, void *out, sa_dtype out_dtype, float *lse,
+                                  void *workspace, size_t workspace_bytes, void *stream,
+                                  void *const *phase_events);
+
+/* Device-side status of the most recent call that used `workspace`.
+ * Synchronises `stream`.  Returns SA_OK, SA_ERR_DEVICE_FAULT or
+ * SA_ERR_TIMEOUT; *detail (may be NULL) receives an SA_DETAIL_* code. */
+enum {
+    SA_DETAIL_NONE = 0,
+    SA_DETAIL_BAD_PAGE = 1,       /* page id outside [0, num_pages) */
+    SA_DETAIL_BAD_POSITION = 2,   /* q_pos >= seq_len, or q_seq outside [0, batch) */
+    SA_DETAIL_BAD_INDEX = 3,      /* selected index outside [0, q_pos] */
+    SA_DETAIL_WAIT_TIMEOUT = 4    /* a bounded wait inside a kernel gave up */
+};
+SA_API sa_status sa_device_status(const void *workspace, size_t workspace_bytes, void *stream,
+                           int32_t *detail);
+
+/* Number of CUDA kernels this library has launched in this process so far
+ * (all devices, all threads).  For tracing: the difference across a region
+ * is the number of library kernels enqueued in it. */
+SA_API uint64_t sa_kernel_launches(void);
+
+/* Human-readable name of a status code (static storage). */
+SA_API const char *sa_status_string(sa_status status);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+SA_API int32_t sa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SA_H */

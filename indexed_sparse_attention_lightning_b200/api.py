@@ -1,0 +1,243 @@
+"""Python binding over ``libsa.so``.
+
+Argument marshalling only: torch tensors (device memory, streams) are turned
+into the C structs of ``include/sa.h`` and passed to the library, which runs
+every step of the path in its own CUDA kernels.  Nothing here computes.
+"""
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+from typing import Optional
+
+import numpy as np
+import torch
+
+from . import _abi
+from ._abi import SaCache, SaError, SaQuery, check
+
+_TORCH_RAW = {np.dtype(np.uint8): torch.uint8, np.dtype(np.uint16): torch.int16,
+              np.dtype(np.float32): torch.float32, np.dtype(np.int32): torch.int32}
+
+
+def _t(a: Optional[np.ndarray], device) -> Optional[torch.Tensor]:
+    """numpy -> torch on `device`, raw bits preserved (bf16 travels as int16)."""
+    if a is None:
+        return None
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.uint16:
+        a = a.view(np.int16)
+    return torch.from_numpy(a).to(device)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+@dataclass
+class DeviceCache:
+    """The paged index-key and latent caches of one layer, resident on the device."""
+
+    page_table: torch.Tensor
+    seq_len: torch.Tensor
+    num_pages: int
+    index_dtype: str
+    k_index: torch.Tensor
+    k_index_scale: Optional[torch.Tensor]
+    kv_dtype: str
+    kv: torch.Tensor
+    kv_rope: Optional[torch.Tensor]
+    kv_scale: Optional[torch.Tensor]
+    d_index: int
+    d_latent: int
+    d_rope: int
+    page_size: int = 64
+
+    def struct(self) -> SaCache:
+        return SaCache(
+            page_table=_ptr(self.page_table), seq_len=_ptr(self.seq_len),
+            batch=self.page_table.shape[0], max_pages=self.page_table.shape[1],
+            num_pages=self.num_pages, page_size=self.page_size,
+            index_dtype=_abi.DTYPES[self.index_dtype], k_index=_ptr(self.k_index),
+            k_index_scale=_ptr(self.k_index_scale), d_index=self.d_index,
+            kv_dtype=_abi.DTYPES[self.kv_dtype], kv=_ptr(self.kv), kv_rope=_ptr(self.kv_rope),
+            kv_scale=_ptr(self.kv_scale), d_latent=self.d_latent, d_rope=self.d_rope)
+
+
+@dataclass
+class DeviceQueries:
+    """One step's query tokens (indexer query, head weights, attention query)."""
+
+    q_seq: torch.Tensor
+    q_pos: torch.Tensor
+    max_visible: int
+    q_index: torch.Tensor
+    q_index_scale: Optional[torch.Tensor]
+    w: torch.Tensor
+    h_index: int
+    q_dtype: str
+    q: torch.Tensor
+    heads: int
+    sm_scale: float
+
+    @property
+    def n_q(self) -> int:
+        return int(self.q_seq.shape[0])
+
+    def struct(self) -> SaQuery:
+        return SaQuery(
+            n_q=self.n_q, q_seq=_ptr(self.q_seq), q_pos=_ptr(self.q_pos),
+            max_visible=self.max_visible, q_index=_ptr(self.q_index),
+            q_index_scale=_ptr(self.q_index_scale), w=_ptr(self.w), h_index=self.h_index,
+            q_dtype=_abi.DTYPES[self.q_dtype], q=_ptr(self.q), heads=self.heads,
+            sm_scale=self.sm_scale)
+
+    def tensors(self) -> dict:
+        return {"q_seq": self.q_seq, "q_pos": self.q_pos, "q_index": self.q_index,
+                "q_index_scale": self.q_index_scale, "w": self.w, "q": self.q}
+
+    def copy_from(self, host: dict, non_blocking: bool = True) -> int:
+        """Copy a step's inputs (e.g. pinned host tensors) into these buffers.
+        Returns the bytes copied."""
+        n = 0
+        for k, dst in self.tensors().items():
+            src = host.get(k)
+            if dst is None or src is None:
+                continue
+            dst.copy_(src, non_blocking=non_blocking)
+            n += src.numel() * src.element_size()
+        return n
+
+
+def upload(wl, device="cuda") -> tuple[DeviceCache, DeviceQueries]:
+    """Place a workload (numpy arrays) on the device."""
+    sp = wl.spec
+    cache = DeviceCache(
+        page_table=_t(wl.page_table, device), seq_len=_t(wl.seq_len, device),
+        num_pages=int(wl.num_pages), index_dtype=sp.index_dtype,
+        k_index=_t(wl.k_index, device), k_index_scale=_t(wl.k_index_scale, device),
+        kv_dtype=sp.kv_dtype, kv=_t(wl.kv, device), kv_rope=_t(wl.kv_rope, device),
+        kv_scale=_t(wl.kv_scale, device), d_index=sp.d_index, d_latent=sp.d_latent,
+        d_rope=sp.d_rope, page_size=sp.page_size)
+    queries = DeviceQueries(
+        q_seq=_t(wl.q_seq, device), q_pos=_t(wl.q_pos, device), max_visible=wl.max_visible,
+        q_index=_t(wl.q_index, device), q_index_scale=_t(wl.q_index_scale, device),
+        w=_t(wl.w, device), h_index=sp.h_index, q_dtype=sp.q_dtype, q=_t(wl.q, device),
+        heads=sp.heads, sm_scale=sp.softmax_scale)
+    return cache, queries
+
+
+def host_queries(wl, pin: bool = True) -> dict:
+    """A step's query inputs as (pinned) host tensors, for end-to-end timing."""
+    out = {}
+    for k in ("q_seq", "q_pos", "q_index", "q_index_scale", "w", "q"):
+        a = getattr(wl, k)
+        if a is None:
+            continue
+        t = _t(a, "cpu")
+        out[k] = t.pin_memory() if pin else t
+    return out
+
+
+# ---------------------------------------------------------------- workspace ---
+
+def workspace_size(cache: DeviceCache, queries: DeviceQueries, top_k: int, uses: int) -> int:
+    c, q = cache.struct(), queries.struct()
+    n = _abi.lib().sa_workspace_size(ctypes.byref(c), ctypes.byref(q), top_k, uses)
+    if n == 0:
+        raise SaError(_abi.SA_ERR_INVALID_ARG, "sa_workspace_size")
+    return int(n)
+
+
+def workspace(nbytes: int, device="cuda") -> torch.Tensor:
+    """Device workspace (torch allocations are at least 256-byte aligned)."""
+    return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+
+
+def device_status(ws: torch.Tensor, stream=None) -> tuple[int, int]:
+    """(status, detail) of the last call that used `ws`; synchronises the stream."""
+    detail = ctypes.c_int32(0)
+    st = _abi.lib().sa_device_status(_ptr(ws), ws.numel(), _stream(stream), ctypes.byref(detail))
+    return int(st), int(detail.value)
+
+
+# -------------------------------------------------------------- entry points ---
+
+def indexer_score(cache: DeviceCache, queries: DeviceQueries, scores=None, ws=None,
+                  stream=None) -> torch.Tensor:
+    dev = queries.q_seq.device
+    if scores is None:
+        scores = torch.full((queries.n_q, max(1, queries.max_visible)), float("nan"),
+                            dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = workspace(workspace_size(cache, queries, 1, _abi.SA_WS_INDEXER), dev)
+    c, q = cache.struct(), queries.struct()
+    check(_abi.lib().sa_indexer_score(ctypes.byref(c), ctypes.byref(q), _ptr(scores),
+                                      scores.stride(0), _ptr(ws), ws.numel(), _stream(stream)),
+          "sa_indexer_score")
+    return scores
+
+
+def topk(scores: torch.Tensor, valid_len: torch.Tensor, top_k: int, max_valid: int,
+         idx=None, ws=None, stream=None) -> torch.Tensor:
+    n_q = scores.shape[0]
+    if idx is None:
+        idx = torch.empty((n_q, top_k), dtype=torch.int32, device=scores.device)
+    if ws is None:
+        ws = workspace(256, scores.device)
+    check(_abi.lib().sa_topk(_ptr(scores), scores.stride(0), _ptr(valid_len), n_q, max_valid,
+                             top_k, _ptr(idx), _ptr(ws), ws.numel(), _stream(stream)),
+          "sa_topk")
+    return idx
+
+
+def _outputs(queries: DeviceQueries, d_latent: int, out, lse, out_dtype: str):
+    dev = queries.q_seq.device
+    if out is None:
+        dt = torch.bfloat16 if out_dtype == "bf16" else torch.float32
+        out = torch.empty((queries.n_q, queries.heads, d_latent), dtype=dt, device=dev)
+    if lse is None:
+        lse = torch.empty((queries.n_q, queries.heads), dtype=torch.float32, device=dev)
+    return out, lse
+
+
+def sparse_mla_attn(cache: DeviceCache, queries: DeviceQueries, idx: torch.Tensor, top_k: int,
+                    out=None, lse=None, out_dtype: str = "bf16", ws=None, stream=None):
+    out, lse = _outputs(queries, cache.d_latent, out, lse, out_dtype)
+    if ws is None:
+        ws = workspace(workspace_size(cache, queries, top_k, _abi.SA_WS_ATTN), idx.device)
+    c, q = cache.struct(), queries.struct()
+    check(_abi.lib().sa_sparse_mla_attn(ctypes.byref(c), ctypes.byref(q), _ptr(idx), top_k,
+                                        _ptr(out), _abi.DTYPES[out_dtype], _ptr(lse), _ptr(ws),
+                                        ws.numel(), _stream(stream)),
+          "sa_sparse_mla_attn")
+    return out, lse
+
+
+def decode(cache: DeviceCache, queries: DeviceQueries, top_k: int, out=None, lse=None,
+           idx=None, out_dtype: str = "bf16", ws=None, stream=None, phase_events=None):
+    """Fused indexer -> top-K -> sparse attention.  Returns (out, lse, idx-or-None).
+
+    ``phase_events``: optional list of len(_abi.DECODE_PHASES) + 1 torch.cuda.Event
+    objects recorded at the phase boundaries (sa_decode_traced)."""
+    out, lse = _outputs(queries, cache.d_latent, out, lse, out_dtype)
+    if ws is None:
+        ws = workspace(workspace_size(cache, queries, top_k, _abi.SA_WS_DECODE),
+                       queries.q_seq.device)
+    c, q = cache.struct(), queries.struct()
+    args = (ctypes.byref(c), ctypes.byref(q), top_k, _ptr(idx), _ptr(out),
+            _abi.DTYPES[out_dtype], _ptr(lse), _ptr(ws), ws.numel(), _stream(stream))
+    if phase_events is None:
+        check(_abi.lib().sa_decode(*args), "sa_decode")
+    else:
+        if len(phase_events) != len(_abi.DECODE_PHASES) + 1:
+            raise ValueError("need one event per phase boundary")
+        handles = (ctypes.c_void_p * len(phase_events))(*[e.cuda_event for e in phase_events])
+        check(_abi.lib().sa_decode_traced(*args, handles), "sa_decode_traced")
+    return out, lse, idx

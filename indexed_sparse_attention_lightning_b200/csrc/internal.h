@@ -1,0 +1,81 @@
+// internal.h -- parameter blocks and launchers shared between the host API
+// (sa_api.cu) and the kernel files.  Not part of the public ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "sa.h"
+
+namespace sa {
+
+// Everything a kernel needs to know about the paged caches and the queries.
+struct PathParams {
+    // paging
+    const int32_t *page_table;
+    const int32_t *seq_len;
+    int32_t batch, max_pages, num_pages;
+    // indexer keys
+    const void *k_index;
+    const float *k_index_scale;
+    int32_t d_index;
+    int32_t index_e4m3;  // 1: e4m3 codes + scales, 0: fp32
+    // latent cache
+    const void *kv;
+    const void *kv_rope;
+    const float *kv_scale;
+    int32_t d_latent, d_rope;
+    int32_t kv_dtype;  // sa_dtype
+    // queries
+    int32_t n_q;
+    const int32_t *q_seq, *q_pos;
+    int32_t max_visible;
+    const void *q_index;
+    const float *q_index_scale;
+    const float *w;
+    int32_t h_index;
+    const void *q;
+    int32_t q_dtype;  // sa_dtype
+    int32_t heads;
+    float sm_scale;
+    // status word (first 2 ints of the workspace)
+    int32_t *status;
+};
+
+// Visible length of query t after validating its sequence and position
+// against the cache; returns 0 (and reports) for an invalid query.
+__device__ __forceinline__ int32_t visible_len(const PathParams &p, int32_t t);
+
+// Count one kernel launch (see sa_kernel_launches).
+void count_launch();
+
+// ---- launchers (each returns the launch error, if any) --------------------
+cudaError_t launch_indexer_simt(const PathParams &p, float *scores, int64_t ld, cudaStream_t s);
+
+// Row-wise exact top-K.  Row t has valid_len[t] entries, or q_pos[t] + 1 when
+// valid_len is null (rows then validated as queries of `p`).
+cudaError_t launch_topk_rowwise(const float *scores, int64_t ld, const int32_t *valid_len,
+                                int32_t max_valid, const PathParams *p, int32_t n_q,
+                                int32_t top_k, int32_t *idx, int32_t *status, cudaStream_t s);
+
+cudaError_t launch_attn_simt(const PathParams &p, const int32_t *idx, int32_t top_k, void *out,
+                             int32_t out_dtype, float *lse, cudaStream_t s);
+
+}  // namespace sa
+
+// ---- inline device definitions -------------------------------------------
+#ifdef __CUDACC__
+#include "common.cuh"
+namespace sa {
+__device__ __forceinline__ int32_t visible_len(const PathParams &p, int32_t t) {
+    int32_t b = __ldg(p.q_seq + t);
+    int32_t pos = __ldg(p.q_pos + t);
+    if (b < 0 || b >= p.batch || pos < 0 || pos >= __ldg(p.seq_len + b) ||
+        pos >= p.max_visible) {
+        report(p.status, SA_ERR_DEVICE_FAULT, SA_DETAIL_BAD_POSITION);
+        return 0;
+    }
+    return pos + 1;
+}
+}  // namespace sa
+#endif

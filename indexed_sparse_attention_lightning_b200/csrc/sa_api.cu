@@ -1,0 +1,282 @@
+// sa_api.cu -- the C ABI: host-side validation, workspace layout, dispatch.
+//
+// Every entry point checks its arguments before touching the device, then
+// enqueues its kernels on the caller's stream without synchronising.
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "common.cuh"
+#include "internal.h"
+#include "sa.h"
+
+namespace sa {
+static std::atomic<uint64_t> g_launches{0};
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+}  // namespace sa
+
+namespace {
+using namespace sa;
+
+constexpr int32_t kPageSize = 64;
+constexpr int32_t kMaxQueries = 65535;
+constexpr int32_t kMaxTopK = 1 << 20;
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void *ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
+
+sa_status check_cache(const sa_cache *c) {
+    if (c == nullptr) return SA_ERR_INVALID_ARG;
+    if (c->page_size != kPageSize) return SA_ERR_UNSUPPORTED;
+    if (c->batch <= 0 || c->max_pages <= 0 || c->num_pages <= 0) return SA_ERR_INVALID_ARG;
+    if (!c->page_table || !c->seq_len || !c->k_index || !c->kv) return SA_ERR_INVALID_ARG;
+    if (!aligned16(c->k_index) || !aligned16(c->kv)) return SA_ERR_INVALID_ARG;
+    if (c->index_dtype != SA_F32 && c->index_dtype != SA_E4M3) return SA_ERR_UNSUPPORTED;
+    if (c->index_dtype == SA_E4M3 && !c->k_index_scale) return SA_ERR_INVALID_ARG;
+    if (c->d_index <= 0 || c->d_index % 16 != 0) return SA_ERR_INVALID_ARG;
+    if (c->d_index > 256) return SA_ERR_UNSUPPORTED;
+    if (c->kv_dtype != SA_F32 && c->kv_dtype != SA_BF16 && c->kv_dtype != SA_E4M3)
+        return SA_ERR_UNSUPPORTED;
+    if (c->d_latent <= 0 || c->d_rope < 0) return SA_ERR_INVALID_ARG;
+    if (c->d_latent > 512 || c->d_latent + c->d_rope > 1024) return SA_ERR_UNSUPPORTED;
+    if (c->kv_dtype == SA_E4M3) {
+        if (!c->kv_scale || (c->d_rope > 0 && !c->kv_rope)) return SA_ERR_INVALID_ARG;
+        if (c->kv_rope && !aligned16(c->kv_rope)) return SA_ERR_INVALID_ARG;
+    }
+    return SA_OK;
+}
+
+sa_status check_query(const sa_query *q, const sa_cache *c, bool need_index, bool need_attn) {
+    if (q == nullptr) return SA_ERR_INVALID_ARG;
+    if (q->n_q < 0) return SA_ERR_INVALID_ARG;
+    if (q->n_q > kMaxQueries) return SA_ERR_UNSUPPORTED;
+    if (q->n_q == 0) return SA_OK;
+    if (!q->q_seq || !q->q_pos || q->max_visible <= 0) return SA_ERR_INVALID_ARG;
+    if ((int64_t)q->max_visible > (int64_t)c->max_pages * c->page_size) return SA_ERR_INVALID_ARG;
+    if (need_index) {
+        if (!q->q_index || !q->w || q->h_index <= 0) return SA_ERR_INVALID_ARG;
+        if (q->h_index > 128) return SA_ERR_UNSUPPORTED;
+        if (c->index_dtype == SA_E4M3 && !q->q_index_scale) return SA_ERR_INVALID_ARG;
+    }
+    if (need_attn) {
+        if (!q->q || q->heads <= 0) return SA_ERR_INVALID_ARG;
+        if (q->q_dtype != SA_F32 && q->q_dtype != SA_BF16) return SA_ERR_UNSUPPORTED;
+        if (!std::isfinite(q->sm_scale)) return SA_ERR_INVALID_ARG;
+    }
+    return SA_OK;
+}
+
+PathParams make_params(const sa_cache *c, const sa_query *q, void *ws) {
+    PathParams p{};
+    p.page_table = c->page_table;
+    p.seq_len = c->seq_len;
+    p.batch = c->batch;
+    p.max_pages = c->max_pages;
+    p.num_pages = c->num_pages;
+    p.k_index = c->k_index;
+    p.k_index_scale = c->k_index_scale;
+    p.d_index = c->d_index;
+    p.index_e4m3 = c->index_dtype == SA_E4M3;
+    p.kv = c->kv;
+    p.kv_rope = c->kv_rope;
+    p.kv_scale = c->kv_scale;
+    p.d_latent = c->d_latent;
+    p.d_rope = c->d_rope;
+    p.kv_dtype = c->kv_dtype;
+    p.n_q = q->n_q;
+    p.q_seq = q->q_seq;
+    p.q_pos = q->q_pos;
+    p.max_visible = q->max_visible;
+    p.q_index = q->q_index;
+    p.q_index_scale = q->q_index_scale;
+    p.w = q->w;
+    p.h_index = q->h_index;
+    p.q = q->q;
+    p.q_dtype = q->q_dtype;
+    p.heads = q->heads;
+    p.sm_scale = q->sm_scale;
+    p.status = static_cast<int32_t *>(ws);
+    return p;
+}
+
+// Workspace of the fused path: status | scores [n_q, ld] | idx [n_q, K].
+struct DecodeLayout {
+    int64_t ld;
+    size_t scores, idx, total;
+};
+
+DecodeLayout decode_layout(const sa_query *q, int32_t top_k) {
+    DecodeLayout l{};
+    l.ld = round_up(q->max_visible > 0 ? q->max_visible : 1, 128);
+    l.scores = align_up(kStatusBytes);
+    l.idx = align_up(l.scores + sizeof(float) * (size_t)q->n_q * (size_t)l.ld);
+    l.total = align_up(l.idx + sizeof(int32_t) * (size_t)q->n_q * (size_t)top_k);
+    return l;
+}
+
+sa_status check_workspace(void *ws, size_t bytes, size_t need) {
+    if (ws == nullptr || bytes < need) return SA_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) != 0) return SA_ERR_WORKSPACE;
+    return SA_OK;
+}
+
+sa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SA_OK : SA_ERR_CUDA; }
+
+sa_status clear_status(void *ws, cudaStream_t s) {
+    return cuda_status(cudaMemsetAsync(ws, 0, kStatusBytes, s));
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t sa_workspace_size(const sa_cache *cache, const sa_query *query, int32_t top_k,
+                         int32_t uses) {
+    if (check_cache(cache) != SA_OK) return 0;
+    const bool idx = (uses & (SA_WS_INDEXER | SA_WS_DECODE)) != 0;
+    const bool att = (uses & (SA_WS_ATTN | SA_WS_DECODE)) != 0;
+    if (check_query(query, cache, idx, att) != SA_OK) return 0;
+    if ((uses & (SA_WS_TOPK | SA_WS_DECODE | SA_WS_ATTN)) && (top_k <= 0 || top_k > kMaxTopK))
+        return 0;
+    size_t need = kStatusBytes;
+    if (uses & SA_WS_DECODE) {
+        DecodeLayout l = decode_layout(query, top_k);
+        if (l.total > need) need = l.total;
+    }
+    return align_up(need);
+}
+
+sa_status sa_indexer_score(const sa_cache *cache, const sa_query *query, float *scores,
+                           int64_t ld_scores, void *workspace, size_t workspace_bytes,
+                           void *stream) {
+    sa_status st = check_cache(cache);
+    if (st != SA_OK) return st;
+    if ((st = check_query(query, cache, true, false)) != SA_OK) return st;
+    if (query->n_q > 0 && (!scores || ld_scores < query->max_visible)) return SA_ERR_INVALID_ARG;
+    if ((st = check_workspace(workspace, workspace_bytes, kStatusBytes)) != SA_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if ((st = clear_status(workspace, s)) != SA_OK) return st;
+    PathParams p = make_params(cache, query, workspace);
+    return cuda_status(launch_indexer_simt(p, scores, ld_scores, s));
+}
+
+sa_status sa_topk(const float *scores, int64_t ld_scores, const int32_t *valid_len, int32_t n_q,
+                  int32_t max_valid, int32_t top_k, int32_t *idx, void *workspace,
+                  size_t workspace_bytes, void *stream) {
+    if (n_q < 0 || top_k <= 0 || top_k > kMaxTopK) return SA_ERR_INVALID_ARG;
+    if (n_q > kMaxQueries) return SA_ERR_UNSUPPORTED;
+    if (n_q > 0 && (!scores || !valid_len || !idx || max_valid < 0 || ld_scores < max_valid))
+        return SA_ERR_INVALID_ARG;
+    sa_status st = check_workspace(workspace, workspace_bytes, kStatusBytes);
+    if (st != SA_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if ((st = clear_status(workspace, s)) != SA_OK) return st;
+    return cuda_status(launch_topk_rowwise(scores, ld_scores, valid_len, max_valid, nullptr, n_q,
+                                           top_k, idx, static_cast<int32_t *>(workspace), s));
+}
+
+sa_status sa_sparse_mla_attn(const sa_cache *cache, const sa_query *query, const int32_t *idx,
+                             int32_t top_k, void *out, sa_dtype out_dtype, float *lse,
+                             void *workspace, size_t workspace_bytes, void *stream) {
+    sa_status st = check_cache(cache);
+    if (st != SA_OK) return st;
+    if ((st = check_query(query, cache, false, true)) != SA_OK) return st;
+    if (top_k <= 0 || top_k > kMaxTopK) return SA_ERR_INVALID_ARG;
+    if (out_dtype != SA_BF16 && out_dtype != SA_F32) return SA_ERR_UNSUPPORTED;
+    if (query->n_q > 0 && (!idx || !out)) return SA_ERR_INVALID_ARG;
+    if ((st = check_workspace(workspace, workspace_bytes, kStatusBytes)) != SA_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if ((st = clear_status(workspace, s)) != SA_OK) return st;
+    PathParams p = make_params(cache, query, workspace);
+    return cuda_status(launch_attn_simt(p, idx, top_k, out, out_dtype, lse, s));
+}
+
+static sa_status decode_impl(const sa_cache *cache, const sa_query *query, int32_t top_k,
+                             int32_t *idx_out, void *out, sa_dtype out_dtype, float *lse,
+                             void *workspace, size_t workspace_bytes, void *stream,
+                             void *const *events) {
+    sa_status st = check_cache(cache);
+    if (st != SA_OK) return st;
+    if ((st = check_query(query, cache, true, true)) != SA_OK) return st;
+    if (top_k <= 0 || top_k > kMaxTopK) return SA_ERR_INVALID_ARG;
+    if (out_dtype != SA_BF16 && out_dtype != SA_F32) return SA_ERR_UNSUPPORTED;
+    if (query->n_q > 0 && !out) return SA_ERR_INVALID_ARG;
+    DecodeLayout l = decode_layout(query, top_k);
+    if ((st = check_workspace(workspace, workspace_bytes, l.total)) != SA_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    auto mark = [&](int i) -> sa_status {
+        if (events == nullptr) return SA_OK;
+        return cuda_status(cudaEventRecord(static_cast<cudaEvent_t>(events[i]), s));
+    };
+    if ((st = clear_status(workspace, s)) != SA_OK) return st;
+    if ((st = mark(0)) != SA_OK) return st;
+    if (query->n_q > 0) {
+        PathParams p = make_params(cache, query, workspace);
+        char *base = static_cast<char *>(workspace);
+        float *scores = reinterpret_cast<float *>(base + l.scores);
+        int32_t *idx = idx_out ? idx_out : reinterpret_cast<int32_t *>(base + l.idx);
+        if ((st = cuda_status(launch_indexer_simt(p, scores, l.ld, s))) != SA_OK) return st;
+        if ((st = mark(1)) != SA_OK) return st;
+        if ((st = cuda_status(launch_topk_rowwise(scores, l.ld, nullptr, query->max_visible, &p,
+                                                  query->n_q, top_k, idx, p.status, s))) != SA_OK)
+            return st;
+        if ((st = mark(2)) != SA_OK) return st;
+        if ((st = cuda_status(launch_attn_simt(p, idx, top_k, out, out_dtype, lse, s))) != SA_OK)
+            return st;
+        return mark(3);
+    }
+    for (int i = 1; i <= SA_DECODE_PHASES; ++i)
+        if ((st = mark(i)) != SA_OK) return st;
+    return SA_OK;
+}
+
+sa_status sa_decode(const sa_cache *cache, const sa_query *query, int32_t top_k,
+                    int32_t *idx_out, void *out, sa_dtype out_dtype, float *lse,
+                    void *workspace, size_t workspace_bytes, void *stream) {
+    return decode_impl(cache, query, top_k, idx_out, out, out_dtype, lse, workspace,
+                       workspace_bytes, stream, nullptr);
+}
+
+sa_status sa_decode_traced(const sa_cache *cache, const sa_query *query, int32_t top_k,
+                           int32_t *idx_out, void *out, sa_dtype out_dtype, float *lse,
+                           void *workspace, size_t workspace_bytes, void *stream,
+                           void *const *phase_events) {
+    return decode_impl(cache, query, top_k, idx_out, out, out_dtype, lse, workspace,
+                       workspace_bytes, stream, phase_events);
+}
+
+sa_status sa_device_status(const void *workspace, size_t workspace_bytes, void *stream,
+                           int32_t *detail) {
+    if (workspace == nullptr || workspace_bytes < kStatusBytes) return SA_ERR_WORKSPACE;
+    int32_t word[2] = {0, 0};
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemcpyAsync(word, workspace, sizeof word, cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return SA_ERR_CUDA;
+    if (detail) *detail = word[1];
+    if (word[0] == 0) return SA_OK;
+    if (word[0] == SA_ERR_TIMEOUT) return SA_ERR_TIMEOUT;
+    return SA_ERR_DEVICE_FAULT;
+}
+
+const char *sa_status_string(sa_status status) {
+    switch (status) {
+    case SA_OK: return "ok";
+    case SA_ERR_INVALID_ARG: return "invalid argument";
+    case SA_ERR_UNSUPPORTED: return "unsupported combination";
+    case SA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case SA_ERR_CUDA: return "CUDA error";
+    case SA_ERR_DEVICE_FAULT: return "bad data detected on the device";
+    case SA_ERR_TIMEOUT: return "bounded device wait timed out";
+    }
+    return "unknown status";
+}
+
+int32_t sa_version(void) { return 100; }
+
+uint64_t sa_kernel_launches(void) { return sa::g_launches.load(std::memory_order_relaxed); }
+
+}  // extern "C"

@@ -50,7 +50,7 @@ class WorkloadSpec:
     name: str
     seed: int
     batch: int
-    seq_len: tuple                 # ("fixed", L) or ("uniform", lo, hi) inclusive
+    seq_len: tuple                 # ("fixed", L), ("uniform", lo, hi) inclusive, ("list", (L0, L1, ...))
     queries: tuple = ("decode",)   # ("decode",) or ("prefill", first_pos, count)
     h_index: int = 64
     d_index: int = 128
@@ -199,6 +199,11 @@ def _seq_lengths(sp: WorkloadSpec, rng) -> np.ndarray:
     if kind == "uniform":
         lo, hi = int(sp.seq_len[1]), int(sp.seq_len[2])
         return rng.integers(lo, hi + 1, size=sp.batch, dtype=np.int64).astype(np.int32)
+    if kind == "list":
+        lens = np.asarray(sp.seq_len[1], dtype=np.int32)
+        if lens.shape != (sp.batch,) or lens.min() < 1:
+            raise ValueError("one positive length per sequence")
+        return lens
     raise ValueError(sp.seq_len)
 
 

@@ -1,0 +1,124 @@
+"""The C-ABI library loads, exports every declared symbol, and rejects bad
+arguments on the host before touching a device (runs without a GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from indexed_sparse_attention_lightning_b200 import _abi, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return _abi.lib()
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "sa.h")).read()
+    return sorted(set(re.findall(r"SA_API\s+[\w\s\*]*?\b(sa_\w+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = declared_symbols()
+    assert len(names) >= 8
+    assert sorted(_abi.EXPORTS) == names
+    for n in names:
+        assert hasattr(L, n), n
+    assert L.sa_version() >= 100
+
+
+def test_status_strings(L):
+    for s in range(7):
+        assert _abi.status_string(s)
+    assert _abi.status_string(99) == "unknown status"
+
+
+FAKE = 1 << 20  # a 16-byte aligned non-null stand-in; never dereferenced
+
+
+def good_cache(**kw):
+    c = _abi.SaCache(page_table=FAKE, seq_len=FAKE, batch=2, max_pages=4, num_pages=8,
+                     page_size=64, index_dtype=_abi.SA_E4M3, k_index=FAKE, k_index_scale=FAKE,
+                     d_index=128, kv_dtype=_abi.SA_BF16, kv=FAKE, kv_rope=None, kv_scale=None,
+                     d_latent=512, d_rope=64)
+    for k, v in kw.items():
+        setattr(c, k, v)
+    return c
+
+
+def good_query(**kw):
+    q = _abi.SaQuery(n_q=2, q_seq=FAKE, q_pos=FAKE, max_visible=256, q_index=FAKE,
+                     q_index_scale=FAKE, w=FAKE, h_index=64, q_dtype=_abi.SA_BF16, q=FAKE,
+                     heads=128, sm_scale=0.0416)
+    for k, v in kw.items():
+        setattr(q, k, v)
+    return q
+
+
+def ws_size(L, c, q, k=2048, uses=_abi.SA_WS_DECODE):
+    return L.sa_workspace_size(ctypes.byref(c), ctypes.byref(q), k, uses)
+
+
+def test_workspace_size_valid_and_invalid(L):
+    n = ws_size(L, good_cache(), good_query())
+    # status + scores [2, 256] + idx [2, 2048], 256-byte aligned pieces
+    assert n >= 256 + 2 * 256 * 4 + 2 * 2048 * 4 and n % 256 == 0
+    assert ws_size(L, good_cache(page_size=32), good_query()) == 0
+    assert ws_size(L, good_cache(d_index=100), good_query()) == 0
+    assert ws_size(L, good_cache(), good_query(max_visible=4 * 64 + 1)) == 0
+    assert ws_size(L, good_cache(), good_query(), k=0) == 0
+    assert ws_size(L, good_cache(kv_dtype=_abi.SA_E4M3), good_query()) == 0  # no scales
+    assert ws_size(L, good_cache(), good_query(q_index_scale=None)) == 0
+
+
+def decode_call(L, c, q, k=2048, ws=FAKE, ws_bytes=1 << 30, out=FAKE):
+    return L.sa_decode(ctypes.byref(c), ctypes.byref(q), k, None, out, _abi.SA_BF16, None, ws,
+                       ws_bytes, None)
+
+
+@pytest.mark.parametrize("mutation,expect", [
+    ({"cache": {"page_table": None}}, _abi.SA_ERR_INVALID_ARG),
+    ({"cache": {"kv": FAKE + 4}}, _abi.SA_ERR_INVALID_ARG),          # misaligned
+    ({"cache": {"page_size": 16}}, _abi.SA_ERR_UNSUPPORTED),
+    ({"cache": {"index_dtype": _abi.SA_BF16}}, _abi.SA_ERR_UNSUPPORTED),
+    ({"cache": {"kv_dtype": 7}}, _abi.SA_ERR_UNSUPPORTED),
+    ({"cache": {"num_pages": 0}}, _abi.SA_ERR_INVALID_ARG),
+    ({"query": {"n_q": -1}}, _abi.SA_ERR_INVALID_ARG),
+    ({"query": {"n_q": 70000}}, _abi.SA_ERR_UNSUPPORTED),
+    ({"query": {"w": None}}, _abi.SA_ERR_INVALID_ARG),
+    ({"query": {"q_dtype": _abi.SA_E4M3}}, _abi.SA_ERR_UNSUPPORTED),
+    ({"query": {"sm_scale": float("nan")}}, _abi.SA_ERR_INVALID_ARG),
+    ({"k": 0}, _abi.SA_ERR_INVALID_ARG),
+    ({"ws": None}, _abi.SA_ERR_WORKSPACE),
+    ({"ws_bytes": 16}, _abi.SA_ERR_WORKSPACE),
+    ({"ws": FAKE + 16}, _abi.SA_ERR_WORKSPACE),                      # not 256-aligned
+    ({"out": None}, _abi.SA_ERR_INVALID_ARG),
+])
+def test_decode_rejects_bad_arguments_before_launch(L, mutation, expect):
+    c = good_cache(**mutation.get("cache", {}))
+    q = good_query(**mutation.get("query", {}))
+    kw = {k: v for k, v in mutation.items() if k in ("k", "ws", "ws_bytes", "out")}
+    assert decode_call(L, c, q, **kw) == expect
+
+
+def test_other_entry_points_reject_bad_arguments(L):
+    c, q = good_cache(), good_query()
+    # scores leading dimension smaller than the visible range
+    assert L.sa_indexer_score(ctypes.byref(c), ctypes.byref(q), FAKE, 100, FAKE, 1 << 20,
+                              None) == _abi.SA_ERR_INVALID_ARG
+    assert L.sa_topk(FAKE, 10, FAKE, 2, 20, 4, FAKE, FAKE, 1 << 20, None) == \
+        _abi.SA_ERR_INVALID_ARG
+    assert L.sa_topk(FAKE, 10, FAKE, 2, 10, 0, FAKE, FAKE, 1 << 20, None) == \
+        _abi.SA_ERR_INVALID_ARG
+    assert L.sa_topk(FAKE, 10, FAKE, 2, 10, 4, FAKE, None, 0, None) == _abi.SA_ERR_WORKSPACE
+    assert L.sa_sparse_mla_attn(ctypes.byref(c), ctypes.byref(q), None, 2048, FAKE,
+                                _abi.SA_BF16, None, FAKE, 1 << 20, None) == \
+        _abi.SA_ERR_INVALID_ARG
+    assert L.sa_sparse_mla_attn(ctypes.byref(c), ctypes.byref(q), FAKE, 2048, FAKE,
+                                _abi.SA_E4M3, None, FAKE, 1 << 20, None) == \
+        _abi.SA_ERR_UNSUPPORTED
+    assert L.sa_device_status(None, 0, None, None) == _abi.SA_ERR_WORKSPACE

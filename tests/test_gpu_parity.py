@@ -1,0 +1,207 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+For every configuration the fused ``sa_decode`` runs on all queries -- the
+launch that ``bench.py`` times -- and the oracle checks a stratified sample of
+queries (all of them where it finishes in seconds):
+
+* top-K: bit-exact index sets, except swaps among positions whose oracle score
+  lies within ``max(1e-3 |s_K|, 1e-6 max|I|)`` of the oracle's K-th score;
+* attention, recomputed by the oracle on the GPU's own index set: max-abs
+  <= 2e-2 and mean-rel <= 5e-3 (bf16 / fp32 cache), max-abs <= 6e-2 (e4m3 latent);
+* lse within 1e-2 absolute.
+
+The unfused chain must agree with the fused path exactly, ``sa_topk`` must be
+bit-exact against the oracle's selection on the same fp32 scores, and device
+data errors must surface through the status word without a fault.
+"""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from indexed_sparse_attention_lightning_b200 import _abi, api
+from indexed_sparse_attention_lightning_b200 import workloads as W
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+
+# configuration -> number of oracle-checked queries (None = all)
+SAMPLES = {
+    "tiny_decode_b1_1k_fp32": None,
+    "decode_b8_8k": None,
+    "decode_b64_16k_32k_planted": 12,
+    "prefill_4096q_64k": 24,
+    "decode_b2_1m_fp8kv_clustered": None,
+}
+
+_WL = {}
+
+
+def workload(sp):
+    if sp.name not in _WL:
+        _WL[sp.name] = W.make_workload(sp)
+    return _WL[sp.name]
+
+
+def out_dtype(sp):
+    return "f32" if sp.kv_dtype == "f32" else "bf16"
+
+
+def run_fused(wl, dev="cuda"):
+    sp = wl.spec
+    cache, queries = api.upload(wl, dev)
+    idx = torch.full((wl.n_q, sp.top_k), -7, dtype=torch.int32, device=dev)
+    ws = api.workspace(api.workspace_size(cache, queries, sp.top_k, _abi.SA_WS_DECODE), dev)
+    out, lse, _ = api.decode(cache, queries, sp.top_k, idx=idx, out_dtype=out_dtype(sp), ws=ws)
+    st = api.device_status(ws)
+    return {"idx": idx.cpu().numpy(), "out": out.float().cpu().numpy(),
+            "lse": lse.cpu().numpy(), "status": st}
+
+
+def sample_rows(wl):
+    n = SAMPLES.get(wl.spec.name)
+    return np.arange(wl.n_q) if n is None else W.stratified_rows(wl.n_q, n)
+
+
+@pytest.mark.parametrize("sp", W.CONFIGS, ids=[s.name for s in W.CONFIGS])
+def test_decode_matches_oracle(sp):
+    wl = workload(sp)
+    res = run_fused(wl)
+    assert res["status"] == (_abi.SA_OK, 0)
+    rows = sample_rows(wl)
+    sub = W.subset_queries(wl, rows)
+    scores = oracle.index_scores(sub)
+    topk = parity.check_topk(res["idx"][rows], scores, sub.visible, sp.top_k)
+    ref_out, ref_lse = oracle.sparse_attn(sub, res["idx"][rows])
+    err = parity.check_attention(res["out"][rows], ref_out, sp.kv_dtype)
+    lse_err = parity.check_lse(res["lse"][rows], ref_lse)
+    print(f"\n{sp.name}: rows={len(rows)} swaps={topk['swaps']} "
+          f"window={topk['worst_window_fraction']:.3g} max_abs={err['max_abs']:.3g} "
+          f"mean_rel={err['mean_rel']:.3g} lse={lse_err:.3g}")
+    assert np.all(np.isfinite(res["out"])) and np.all(np.isfinite(res["lse"]))
+
+
+@pytest.mark.parametrize("sp", W.CONFIGS[:2], ids=[s.name for s in W.CONFIGS[:2]])
+def test_unfused_chain_equals_fused_and_topk_is_exact(sp):
+    wl = workload(sp)
+    fused = run_fused(wl)
+    cache, queries = api.upload(wl)
+    scores = api.indexer_score(cache, queries)
+    valid = torch.from_numpy(wl.visible).cuda()
+    idx = api.topk(scores, valid, sp.top_k, wl.max_visible)
+    out, lse = api.sparse_mla_attn(cache, queries, idx, sp.top_k, out_dtype=out_dtype(sp))
+    s = scores.cpu().numpy().astype(np.float64)
+    # scores against the oracle
+    ref = oracle.index_scores(wl)
+    for t in range(wl.n_q):
+        V = wl.visible[t]
+        rel = np.abs(s[t, :V] - ref[t, :V]).max() / np.abs(ref[t, :V]).max()
+        assert rel <= 1e-4, (t, rel)
+    # the top-K kernel is exact on its own fp32 input
+    assert np.array_equal(idx.cpu().numpy(), oracle.topk(s, wl.visible, sp.top_k))
+    # unfused chain == fused path, bit for bit
+    assert np.array_equal(idx.cpu().numpy(), fused["idx"])
+    assert np.array_equal(out.float().cpu().numpy(), fused["out"])
+    assert np.array_equal(lse.cpu().numpy(), fused["lse"])
+
+
+def test_topk_exact_on_ties_signed_zeros_and_short_rows():
+    rng = np.random.default_rng(7)
+    n_q, L, K = 9, 70000, 2048
+    s = np.round(rng.standard_normal((n_q, L)), 2).astype(np.float32)
+    s[1] = 0.0                                  # all equal: lowest positions win
+    s[2, ::2] = -0.0                            # signed zeros tie with +0
+    s[2, 1::2] = 0.0
+    s[3] = -np.abs(s[3])                        # all negative
+    s[4, :] = 1.0
+    s[4, 5000:5000 + K] = 2.0                   # a block that is exactly the top-K
+    valid = np.array([L, L, L, L, L, 1, K - 1, K, K + 1], np.int32)
+    scores = torch.from_numpy(s).cuda()
+    idx = api.topk(scores, torch.from_numpy(valid).cuda(), K, L).cpu().numpy()
+    ref = oracle.topk(s.astype(np.float64), valid, K)
+    assert np.array_equal(idx, ref)
+    assert np.array_equal(idx[1], np.arange(K))
+    assert np.array_equal(idx[4], np.arange(5000, 5000 + K))
+
+
+def test_ragged_contexts_around_k_and_page_edges():
+    sp = W.WorkloadSpec(name="ragged", seed=21, batch=8,
+                        seq_len=("list", (1, 63, 64, 65, 2047, 2048, 2049, 9000)))
+    wl = workload(sp)
+    res = run_fused(wl)
+    assert res["status"] == (_abi.SA_OK, 0)
+    scores = oracle.index_scores(wl)
+    parity.check_topk(res["idx"], scores, wl.visible, sp.top_k)
+    ref_out, ref_lse = oracle.sparse_attn(wl, res["idx"])
+    parity.check_attention(res["out"], ref_out, sp.kv_dtype)
+    parity.check_lse(res["lse"], ref_lse)
+    assert np.all(res["idx"][0, 1:] == -1) and res["idx"][0, 0] == 0
+
+
+def test_deterministic_and_independent_of_page_placement():
+    wl = workload(W.DECODE_B8_8K)
+    a = run_fused(wl)
+    b = run_fused(wl)
+    c = run_fused(W.permute_pages(wl, seed=5))
+    for k in ("idx", "out", "lse"):
+        assert np.array_equal(a[k], b[k]), k
+        assert np.array_equal(a[k], c[k]), k
+
+
+def test_fp8_latent_cache_small():
+    sp = W.WorkloadSpec(name="fp8kv_small", seed=22, batch=3, seq_len=("list", (700, 3000, 5000)),
+                        kv_dtype="e4m3", keys=("clusters", 2, 256))
+    wl = workload(sp)
+    res = run_fused(wl)
+    scores = oracle.index_scores(wl)
+    parity.check_topk(res["idx"], scores, wl.visible, sp.top_k)
+    ref_out, _ = oracle.sparse_attn(wl, res["idx"])
+    parity.check_attention(res["out"], ref_out, "e4m3")
+
+
+# ------------------------------------------------ device-side data errors ---
+
+def test_bad_page_id_is_reported_not_faulted():
+    wl = workload(W.DECODE_B8_8K)
+    cache, queries = api.upload(wl)
+    cache.page_table[3, 5] = wl.num_pages + 3
+    out, lse, _ = api.decode(cache, queries, wl.spec.top_k)
+    ws = api.workspace(api.workspace_size(cache, queries, wl.spec.top_k, _abi.SA_WS_DECODE))
+    api.decode(cache, queries, wl.spec.top_k, ws=ws)
+    assert api.device_status(ws) == (_abi.SA_ERR_DEVICE_FAULT, _abi.SA_DETAIL_BAD_PAGE)
+    # a clean call on the same workspace clears the word
+    cache.page_table[3, 5] = int(wl.page_table[3, 5])
+    api.decode(cache, queries, wl.spec.top_k, ws=ws)
+    assert api.device_status(ws) == (_abi.SA_OK, 0)
+
+
+def test_bad_query_position_is_reported():
+    wl = workload(W.DECODE_B8_8K)
+    cache, queries = api.upload(wl)
+    queries.q_pos[2] = int(wl.seq_len[2])           # one past the cached tokens
+    ws = api.workspace(api.workspace_size(cache, queries, wl.spec.top_k, _abi.SA_WS_DECODE))
+    out, lse, _ = api.decode(cache, queries, wl.spec.top_k, ws=ws)
+    assert api.device_status(ws) == (_abi.SA_ERR_DEVICE_FAULT, _abi.SA_DETAIL_BAD_POSITION)
+    assert torch.isfinite(out.float()).all()
+
+
+def test_selected_index_outside_visible_range_is_reported():
+    wl = workload(W.DECODE_B8_8K)
+    cache, queries = api.upload(wl)
+    idx = torch.zeros((wl.n_q, 16), dtype=torch.int32, device="cuda")
+    idx[1, 3] = int(wl.q_pos[1]) + 1
+    ws = api.workspace(api.workspace_size(cache, queries, 16, _abi.SA_WS_ATTN))
+    api.sparse_mla_attn(cache, queries, idx, 16, ws=ws)
+    assert api.device_status(ws) == (_abi.SA_ERR_DEVICE_FAULT, _abi.SA_DETAIL_BAD_INDEX)
+
+
+def test_empty_batch_is_a_no_op():
+    wl = workload(W.TINY)
+    cache, queries = api.upload(wl)
+    empty = dataclasses.replace(queries, q_seq=queries.q_seq[:0], q_pos=queries.q_pos[:0],
+                                q_index=queries.q_index[:0], w=queries.w[:0], q=queries.q[:0])
+    out, lse, _ = api.decode(cache, empty, wl.spec.top_k, out_dtype="f32")
+    torch.cuda.synchronize()
+    assert out.shape[0] == 0
