@@ -238,6 +238,9 @@ def decode(cache: DeviceCache, queries: DeviceQueries, top_k: int, out=None, lse
     else:
         if len(phase_events) != len(_abi.DECODE_PHASES) + 1:
             raise ValueError("need one event per phase boundary")
+        for e in phase_events:
+            if e.cuda_event == 0:       # torch creates the CUDA event on first record
+                e.record(stream if stream is not None else torch.cuda.current_stream())
         handles = (ctypes.c_void_p * len(phase_events))(*[e.cuda_event for e in phase_events])
         check(_abi.lib().sa_decode_traced(*args, handles), "sa_decode_traced")
     return out, lse, idx

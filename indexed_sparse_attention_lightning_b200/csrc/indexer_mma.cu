@@ -1,0 +1,306 @@
+// indexer_mma.cu -- FP8 lightning indexer on the 5th-generation tensor cores.
+//
+// Scores every visible cached position of every query ("Optimizing Next-Gen
+// LLM Inference" §3.1: relevance scoring, head-weight weighting; §4: index keys
+// quantised to 8-bit floats):
+//     I[t,s] = ks[s] * sum_j (w[t,j] * qs[t,j]) * max(0, q8[t,j,:] . k8[s,:])
+// which equals sum_j w * max(0, q_I . k_I) because the scales are positive.
+//
+// The contraction of 64 heads x 128 dims against every key is a dense GEMM
+// (M = 128 keys of a two-page tile, N = 64 heads, K = 128), so it runs as
+// tcgen05.mma kind::f8f6f4 (e4m3 x e4m3 -> fp32 in TMEM).  The kernel is
+// persistent: the tiles of all queries are laid end to end and every CTA takes
+// an equal contiguous share, so short and long contexts balance across SMs.
+// Roles per CTA (192 threads):
+//   warp 0     TMA producer: key pages (8 KB each, 128-byte swizzle) straight
+//              from the paged cache into a 4-stage ring, and the query's
+//              64x128 e4m3 block when the query changes;
+//   warp 1     one thread issues the MMAs and commits them to mbarriers;
+//   warps 2-5  epilogue: each thread owns one key row of the tile, reads its
+//              64 head scores from TMEM (tcgen05.ld), applies ReLU, the head
+//              weights and the key scale, and writes one fp32 score.
+// Every wait is bounded; a timeout is reported in the workspace status word.
+#include "common.cuh"
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace sa {
+namespace {
+using namespace sm100;
+
+constexpr int kKeys = 128;    // MMA M: keys per tile (two pages)
+constexpr int kHeads = 64;    // MMA N: indexer heads
+constexpr int kDim = 128;     // MMA K: index dimension (bytes of e4m3)
+constexpr int kStages = 4;
+constexpr int kAcc = 2;       // TMEM accumulators (64 columns each)
+constexpr int kThreads = 192;
+constexpr uint32_t kPageBytes = 64 * kDim;
+constexpr uint32_t kTileBytes = 2 * kPageBytes;
+constexpr uint32_t kQBytes = kHeads * kDim;
+constexpr uint32_t kTmemCols = kAcc * kHeads;
+
+struct IndexerSmem {
+    uint8_t keys[kStages][kTileBytes];  // 1024-byte aligned (128-byte swizzle atoms)
+    uint8_t q[2][kQBytes];
+    uint64_t full[kStages], empty[kStages];
+    uint64_t acc_full[kAcc], acc_empty[kAcc];
+    uint64_t q_full[2], q_empty[2];
+    uint64_t done;
+    uint32_t tmem_base;
+    int abort;
+};
+
+struct IndexerArgs {
+    PathParams p;
+    const int32_t *vis;       // [n_q] visible length (0 = invalid query)
+    const int32_t *tile_end;  // [n_q] inclusive prefix of ceil(vis / 128)
+    float *scores;
+    int64_t ld;
+};
+
+// Walks this CTA's contiguous share [k, k_end) of the global tile list.
+struct TileCursor {
+    int64_t k, k_end;
+    int32_t t, i, seg;
+
+    __device__ void init(const int32_t *tile_end, int32_t n_q, int64_t k0, int64_t k1) {
+        k = k0;
+        k_end = k1;
+        seg = 0;
+        int lo = 0, hi = n_q;  // first t with tile_end[t] > k0
+        while (lo < hi) {
+            int mid = (lo + hi) >> 1;
+            if (tile_end[mid] > k0) hi = mid;
+            else lo = mid + 1;
+        }
+        t = lo;
+        i = static_cast<int32_t>(k0 - (lo > 0 ? tile_end[lo - 1] : 0));
+    }
+    __device__ bool valid() const { return k < k_end; }
+    // Advance one tile; returns true when the next tile starts a new query.
+    __device__ bool next(const int32_t *tile_end) {
+        ++k;
+        ++i;
+        if (k >= k_end) return false;
+        bool changed = false;
+        while (k >= tile_end[t]) {
+            ++t;
+            i = 0;
+            changed = true;
+        }
+        if (changed) ++seg;
+        return changed;
+    }
+};
+
+__device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
+    return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+// One lane polls, the warp agrees on the outcome.
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                          int32_t *status) {
+    bool ok = true;
+    if (lane_id() == 0) ok = mbar_wait(bar, parity, abort_flag, status);
+    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+    __syncwarp();
+    return ok;
+}
+
+__global__ void __launch_bounds__(kThreads, 2)
+indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
+                   const __grid_constant__ CUtensorMap tm_q, const IndexerArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    IndexerSmem &sm = *reinterpret_cast<IndexerSmem *>(align1024(smem_raw));
+    const PathParams &p = a.p;
+    const int warp = warp_id(), lane = lane_id();
+    const int64_t total = p.n_q > 0 ? a.tile_end[p.n_q - 1] : 0;
+    const int64_t k0 = total * blockIdx.x / gridDim.x;
+    const int64_t k1 = total * (blockIdx.x + 1) / gridDim.x;
+    if (k0 >= k1) return;  // uniform over the CTA, before any allocation
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.empty[s], 1);
+        }
+        for (int c = 0; c < kAcc; ++c) {
+            mbar_init(&sm.acc_full[c], 1);
+            mbar_init(&sm.acc_empty[c], 4);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sm.q_full[b], 1);
+            mbar_init(&sm.q_empty[b], 1);
+        }
+        mbar_init(&sm.done, 1);
+        sm.abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0) tmem_alloc(&sm.tmem_base, kTmemCols);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    volatile int *abort_flag = &sm.abort;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer ---
+        if (lane == 0) {
+            TileCursor c;
+            c.init(a.tile_end, p.n_q, k0, k1);
+            bool seg_start = true;
+            int32_t seq = 0, V = 0;
+            for (int n = 0; c.valid(); ++n) {
+                if (seg_start) {
+                    const int b = c.seg & 1;
+                    if (!mbar_wait(&sm.q_empty[b], ((c.seg >> 1) & 1) ^ 1, abort_flag, p.status))
+                        break;
+                    mbar_arrive_expect_tx(&sm.q_full[b], kQBytes);
+                    tma_load_2d(sm.q[b], &tm_q, 0, c.t * kHeads, &sm.q_full[b]);
+                    seq = p.q_seq[c.t];
+                    V = a.vis[c.t];
+                }
+                const int stage = n % kStages;
+                if (!mbar_wait(&sm.empty[stage], ((n / kStages) & 1) ^ 1, abort_flag, p.status))
+                    break;
+                int32_t rows[2] = {-1, -1};
+                uint32_t bytes = 0;
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int64_t s = (int64_t)c.i * kKeys + 64 * h;
+                    if (s < V) {
+                        const int32_t page = p.page_table[(int64_t)seq * p.max_pages + (s >> 6)];
+                        if (page >= 0 && page < p.num_pages) {
+                            rows[h] = page * 64;
+                            bytes += kPageBytes;
+                        }
+                    }
+                }
+                mbar_arrive_expect_tx(&sm.full[stage], bytes);
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+                    if (rows[h] >= 0)
+                        tma_load_2d(sm.keys[stage] + h * kPageBytes, &tm_keys, 0, rows[h],
+                                    &sm.full[stage]);
+                seg_start = c.next(a.tile_end);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------- MMA issuer ---
+        if (lane == 0) {
+            constexpr uint32_t idesc = instr_desc(kKeys, kHeads, 0 /*e4m3*/, 0, 0);
+            TileCursor c;
+            c.init(a.tile_end, p.n_q, k0, k1);
+            bool seg_start = true;
+            for (int n = 0; c.valid(); ++n) {
+                if (seg_start) {
+                    if (c.seg > 0) mma_commit(&sm.q_empty[(c.seg - 1) & 1]);
+                    if (!mbar_wait(&sm.q_full[c.seg & 1], (c.seg >> 1) & 1, abort_flag, p.status))
+                        break;
+                }
+                const int stage = n % kStages, acc = n % kAcc;
+                if (!mbar_wait(&sm.acc_empty[acc], ((n / kAcc) & 1) ^ 1, abort_flag, p.status))
+                    break;
+                if (!mbar_wait(&sm.full[stage], (n / kStages) & 1, abort_flag, p.status)) break;
+                tc_fence_after();
+                const uint64_t adesc = desc_kmajor_sw128(smem_u32(sm.keys[stage]));
+                const uint64_t bdesc = desc_kmajor_sw128(smem_u32(sm.q[c.seg & 1]));
+                const uint32_t d = tmem + acc * kHeads;
+#pragma unroll
+                for (int kk = 0; kk < kDim / 32; ++kk)  // 32 bytes of K per instruction
+                    mma_f8(d, adesc + 2 * kk, bdesc + 2 * kk, idesc, kk > 0 ? 1u : 0u);
+                mma_commit(&sm.empty[stage]);
+                mma_commit(&sm.acc_full[acc]);
+                seg_start = c.next(a.tile_end);
+            }
+            // every issued MMA has landed before TMEM is released
+            mma_commit(&sm.done);
+            mbar_wait(&sm.done, 0, abort_flag, p.status);
+        }
+    } else {
+        // --------------------------------------------------- epilogue ---
+        const int quad = warp & 3;             // TMEM lanes this warp may read
+        const int row = quad * 32 + lane;      // key row of the tile
+        TileCursor c;
+        c.init(a.tile_end, p.n_q, k0, k1);
+        bool seg_start = true;
+        int32_t seq = 0, V = 0;
+        float wq[kHeads];
+        for (int n = 0; c.valid(); ++n) {
+            if (seg_start) {
+                seq = p.q_seq[c.t];
+                V = a.vis[c.t];
+                const float *w = p.w + (int64_t)c.t * kHeads;
+                const float *qs = p.q_index_scale + (int64_t)c.t * kHeads;
+#pragma unroll
+                for (int j = 0; j < kHeads; ++j) wq[j] = __ldg(w + j) * __ldg(qs + j);
+            }
+            const int64_t s = (int64_t)c.i * kKeys + row;
+            float kscale = 0.f;
+            bool ok = false;
+            if (s < V) {
+                const int32_t page = p.page_table[(int64_t)seq * p.max_pages + (s >> 6)];
+                if (page >= 0 && page < p.num_pages) {
+                    kscale = __ldg(p.k_index_scale + (int64_t)page * 64 + (s & 63));
+                    ok = true;
+                } else {
+                    report(p.status, SA_ERR_DEVICE_FAULT, SA_DETAIL_BAD_PAGE);
+                }
+            }
+            const int acc = n % kAcc;
+            if (!warp_wait(&sm.acc_full[acc], (n / kAcc) & 1, abort_flag, p.status)) break;
+            tc_fence_after();
+            const uint32_t taddr = tmem + (static_cast<uint32_t>(quad * 32) << 16) + acc * kHeads;
+            float v[32];
+            float sum = 0.f;
+            tmem_ld32(taddr, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) sum = fmaf(wq[j], relu_keep_nan(v[j]), sum);
+            tmem_ld32(taddr + 32, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) sum = fmaf(wq[32 + j], relu_keep_nan(v[j]), sum);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.acc_empty[acc]);
+            if (s < V) a.scores[(int64_t)c.t * a.ld + s] = ok ? sum * kscale : -INFINITY;
+            seg_start = c.next(a.tile_end);
+        }
+    }
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+}  // namespace
+
+bool indexer_mma_supported(const PathParams &p) {
+    return p.index_e4m3 && p.h_index == kHeads && p.d_index == kDim;
+}
+
+cudaError_t launch_indexer_mma(const PathParams &p, const int32_t *vis, const int32_t *tile_end,
+                               float *scores, int64_t ld, cudaStream_t s) {
+    if (p.n_q == 0) return cudaSuccess;
+    CUtensorMap tk, tq;
+    if (!encode_tmap_2d(&tk, 1, p.k_index, kDim, (uint64_t)p.num_pages * 64, kDim, kDim, 64, true) ||
+        !encode_tmap_2d(&tq, 1, p.q_index, kDim, (uint64_t)p.n_q * kHeads, kDim, kDim, kHeads,
+                        true))
+        return cudaErrorInvalidValue;
+    IndexerArgs a{p, vis, tile_end, scores, ld};
+    const int64_t max_tiles = (int64_t)p.n_q * ceil_div(p.max_visible, kKeys);
+    const int64_t grid = std::min<int64_t>(2 * num_sms(), max_tiles);
+    const size_t smem = sizeof(IndexerSmem) + 1024;
+    cudaError_t e = cudaFuncSetAttribute(indexer_mma_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    count_launch();
+    indexer_mma_kernel<<<static_cast<unsigned>(grid), kThreads, smem, s>>>(tk, tq, a);
+    return cudaGetLastError();
+}
+
+}  // namespace sa

@@ -2,8 +2,11 @@
 // (sa_api.cu) and the kernel files.  Not part of the public ABI.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+
+#include <algorithm>
 
 #include "sa.h"
 
@@ -49,8 +52,26 @@ __device__ __forceinline__ int32_t visible_len(const PathParams &p, int32_t t);
 // Count one kernel launch (see sa_kernel_launches).
 void count_launch();
 
+// SM count of the current device (cached).
+int num_sms();
+
+// 2-D TMA tensor map over a row-major [outer, inner] array (elements of
+// dtype_bytes = 1 (u8), 2 (bf16) or 4 (f32)), box [box_outer, box_inner].
+bool encode_tmap_2d(CUtensorMap *map, int dtype_bytes, const void *base, uint64_t inner,
+                    uint64_t outer, uint64_t row_stride_bytes, uint32_t box_inner,
+                    uint32_t box_outer, bool swizzle128);
+
 // ---- launchers (each returns the launch error, if any) --------------------
+// Visible length per query and the inclusive prefix of ceil(V / tile).
+cudaError_t launch_plan(const PathParams &p, int32_t *vis, int32_t *tile_end, int32_t tile,
+                        cudaStream_t s);
+
 cudaError_t launch_indexer_simt(const PathParams &p, float *scores, int64_t ld, cudaStream_t s);
+
+// Tensor-core FP8 indexer (e4m3 keys, 64 heads x 128 dims); needs the plan.
+bool indexer_mma_supported(const PathParams &p);
+cudaError_t launch_indexer_mma(const PathParams &p, const int32_t *vis, const int32_t *tile_end,
+                               float *scores, int64_t ld, cudaStream_t s);
 
 // Row-wise exact top-K.  Row t has valid_len[t] entries, or q_pos[t] + 1 when
 // valid_len is null (rows then validated as queries of `p`).

@@ -1,0 +1,76 @@
+// plan.cu -- per-call schedule: validated visible length of every query and
+// the inclusive prefix of its 128-key tile count, which the persistent
+// kernels use to split the concatenated tiles of all queries evenly.
+#include "common.cuh"
+#include "internal.h"
+
+namespace sa {
+namespace {
+
+constexpr int kThreads = 1024;
+
+__global__ void __launch_bounds__(kThreads)
+plan_kernel(const PathParams p, int32_t *vis, int32_t *tile_end, int32_t tile) {
+    __shared__ int32_t warp_sums[32];
+    __shared__ int32_t carry;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (threadIdx.x == 0) carry = 0;
+    __syncthreads();
+    for (int base = 0; base < p.n_q; base += kThreads) {
+        const int t = base + threadIdx.x;
+        const int32_t V = t < p.n_q ? visible_len(p, t) : 0;
+        const int32_t tiles = (V + tile - 1) / tile;
+        int32_t x = tiles;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            int32_t y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        if (lane == 31) warp_sums[warp] = x;
+        __syncthreads();
+        if (warp == 0) {
+            int32_t w = warp_sums[lane];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                int32_t y = __shfl_up_sync(0xffffffffu, w, o);
+                if (lane >= o) w += y;
+            }
+            warp_sums[lane] = w;  // inclusive over warps
+        }
+        __syncthreads();
+        const int32_t incl = carry + (warp > 0 ? warp_sums[warp - 1] : 0) + x;
+        if (t < p.n_q) {
+            vis[t] = V;
+            tile_end[t] = incl;
+        }
+        __syncthreads();
+        if (threadIdx.x == kThreads - 1) carry = incl;
+        __syncthreads();
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_plan(const PathParams &p, int32_t *vis, int32_t *tile_end, int32_t tile,
+                        cudaStream_t s) {
+    if (p.n_q == 0) return cudaSuccess;
+    count_launch();
+    plan_kernel<<<1, kThreads, 0, s>>>(p, vis, tile_end, tile);
+    return cudaGetLastError();
+}
+
+int num_sms() {
+    static int cached_dev = -1, cached = 0;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (dev != cached_dev) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+        cached = n;
+        cached_dev = dev;
+    }
+    return cached;
+}
+
+}  // namespace sa

@@ -28,6 +28,8 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 bool aligned16(const void *ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
 
+sa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SA_OK : SA_ERR_CUDA; }
+
 sa_status check_cache(const sa_cache *c) {
     if (c == nullptr) return SA_ERR_INVALID_ARG;
     if (c->page_size != kPageSize) return SA_ERR_UNSUPPORTED;
@@ -102,19 +104,39 @@ PathParams make_params(const sa_cache *c, const sa_query *q, void *ws) {
     return p;
 }
 
-// Workspace of the fused path: status | scores [n_q, ld] | idx [n_q, K].
-struct DecodeLayout {
+// Workspace: status | vis [n_q] | tile_end [n_q] | scores [n_q, ld] | idx [n_q, K];
+// the indexer needs the first three, the fused path all five.
+struct Layout {
     int64_t ld;
-    size_t scores, idx, total;
+    size_t vis, tile_end, scores, idx, indexer_total, decode_total;
 };
 
-DecodeLayout decode_layout(const sa_query *q, int32_t top_k) {
-    DecodeLayout l{};
+Layout make_layout(const sa_query *q, int32_t top_k) {
+    Layout l{};
+    const size_t nq = q->n_q > 0 ? (size_t)q->n_q : 0;
     l.ld = round_up(q->max_visible > 0 ? q->max_visible : 1, 128);
-    l.scores = align_up(kStatusBytes);
-    l.idx = align_up(l.scores + sizeof(float) * (size_t)q->n_q * (size_t)l.ld);
-    l.total = align_up(l.idx + sizeof(int32_t) * (size_t)q->n_q * (size_t)top_k);
+    l.vis = align_up(kStatusBytes);
+    l.tile_end = align_up(l.vis + sizeof(int32_t) * nq);
+    l.indexer_total = align_up(l.tile_end + sizeof(int32_t) * nq);
+    l.scores = l.indexer_total;
+    l.idx = align_up(l.scores + sizeof(float) * nq * (size_t)l.ld);
+    l.decode_total = align_up(l.idx + sizeof(int32_t) * nq * (size_t)(top_k > 0 ? top_k : 0));
     return l;
+}
+
+// Indexer scores into `scores` (ld): the tensor-core kernel for its shape,
+// the CUDA-core kernel otherwise.
+sa_status run_indexer(const PathParams &p, const Layout &l, void *ws, float *scores, int64_t ld,
+                      cudaStream_t s) {
+    if (indexer_mma_supported(p)) {
+        char *base = static_cast<char *>(ws);
+        int32_t *vis = reinterpret_cast<int32_t *>(base + l.vis);
+        int32_t *tile_end = reinterpret_cast<int32_t *>(base + l.tile_end);
+        sa_status st = cuda_status(launch_plan(p, vis, tile_end, 128, s));
+        if (st != SA_OK) return st;
+        return cuda_status(launch_indexer_mma(p, vis, tile_end, scores, ld, s));
+    }
+    return cuda_status(launch_indexer_simt(p, scores, ld, s));
 }
 
 sa_status check_workspace(void *ws, size_t bytes, size_t need) {
@@ -122,8 +144,6 @@ sa_status check_workspace(void *ws, size_t bytes, size_t need) {
     if ((reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) != 0) return SA_ERR_WORKSPACE;
     return SA_OK;
 }
-
-sa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SA_OK : SA_ERR_CUDA; }
 
 sa_status clear_status(void *ws, cudaStream_t s) {
     return cuda_status(cudaMemsetAsync(ws, 0, kStatusBytes, s));
@@ -141,11 +161,10 @@ size_t sa_workspace_size(const sa_cache *cache, const sa_query *query, int32_t t
     if (check_query(query, cache, idx, att) != SA_OK) return 0;
     if ((uses & (SA_WS_TOPK | SA_WS_DECODE | SA_WS_ATTN)) && (top_k <= 0 || top_k > kMaxTopK))
         return 0;
+    const Layout l = make_layout(query, top_k);
     size_t need = kStatusBytes;
-    if (uses & SA_WS_DECODE) {
-        DecodeLayout l = decode_layout(query, top_k);
-        if (l.total > need) need = l.total;
-    }
+    if (uses & SA_WS_INDEXER) need = std::max(need, l.indexer_total);
+    if (uses & SA_WS_DECODE) need = std::max(need, l.decode_total);
     return align_up(need);
 }
 
@@ -156,11 +175,13 @@ sa_status sa_indexer_score(const sa_cache *cache, const sa_query *query, float *
     if (st != SA_OK) return st;
     if ((st = check_query(query, cache, true, false)) != SA_OK) return st;
     if (query->n_q > 0 && (!scores || ld_scores < query->max_visible)) return SA_ERR_INVALID_ARG;
-    if ((st = check_workspace(workspace, workspace_bytes, kStatusBytes)) != SA_OK) return st;
+    const Layout l = make_layout(query, 1);
+    if ((st = check_workspace(workspace, workspace_bytes, l.indexer_total)) != SA_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if ((st = clear_status(workspace, s)) != SA_OK) return st;
+    if (query->n_q == 0) return SA_OK;
     PathParams p = make_params(cache, query, workspace);
-    return cuda_status(launch_indexer_simt(p, scores, ld_scores, s));
+    return run_indexer(p, l, workspace, scores, ld_scores, s);
 }
 
 sa_status sa_topk(const float *scores, int64_t ld_scores, const int32_t *valid_len, int32_t n_q,
@@ -204,8 +225,8 @@ static sa_status decode_impl(const sa_cache *cache, const sa_query *query, int32
     if (top_k <= 0 || top_k > kMaxTopK) return SA_ERR_INVALID_ARG;
     if (out_dtype != SA_BF16 && out_dtype != SA_F32) return SA_ERR_UNSUPPORTED;
     if (query->n_q > 0 && !out) return SA_ERR_INVALID_ARG;
-    DecodeLayout l = decode_layout(query, top_k);
-    if ((st = check_workspace(workspace, workspace_bytes, l.total)) != SA_OK) return st;
+    const Layout l = make_layout(query, top_k);
+    if ((st = check_workspace(workspace, workspace_bytes, l.decode_total)) != SA_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     auto mark = [&](int i) -> sa_status {
         if (events == nullptr) return SA_OK;
@@ -218,7 +239,7 @@ static sa_status decode_impl(const sa_cache *cache, const sa_query *query, int32
         char *base = static_cast<char *>(workspace);
         float *scores = reinterpret_cast<float *>(base + l.scores);
         int32_t *idx = idx_out ? idx_out : reinterpret_cast<int32_t *>(base + l.idx);
-        if ((st = cuda_status(launch_indexer_simt(p, scores, l.ld, s))) != SA_OK) return st;
+        if ((st = run_indexer(p, l, workspace, scores, l.ld, s)) != SA_OK) return st;
         if ((st = mark(1)) != SA_OK) return st;
         if ((st = cuda_status(launch_topk_rowwise(scores, l.ld, nullptr, query->max_visible, &p,
                                                   query->n_q, top_k, idx, p.status, s))) != SA_OK)
