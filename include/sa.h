@@ -193,6 +193,28 @@ SA_API sa_status sa_decode_traced(const sa_cache *cache, const sa_query *query, 
                                   void *workspace, size_t workspace_bytes, void *stream,
                                   void *const *phase_events);
 
+/* sa_decode for callers that cannot allocate device memory -- e.g. a plugin
+ * whose host application owns every device allocation, a pool with a hard cap
+ * this library may not grow, or a latency-critical loop where cudaMalloc
+ * (which can synchronise the device) is not allowed.  The paper has no
+ * counterpart; this entry point only serves such deployments.
+ * Same arguments and results as sa_decode, without a workspace: the scratch
+ * lives in a static device array of SA_NOALLOC_SCRATCH_BYTES that every
+ * device loading this library holds until the process exits.  The call
+ * allocates nothing.
+ *  - Requests needing more scratch than that (sa_workspace_size(...,
+ *    SA_WS_DECODE) > SA_NOALLOC_SCRATCH_BYTES) return SA_ERR_WORKSPACE and
+ *    launch nothing.
+ *  - The first call on a device looks the array's address up with that
+ *    device current; make it before any stream capture.
+ *  - All calls on a device share the array: calls whose GPU work overlaps
+ *    race and must not be issued.  The device status word of these calls
+ *    lives in the array and is not readable through sa_device_status(). */
+#define SA_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+SA_API sa_status sa_decode_noalloc(const sa_cache *cache, const sa_query *query, int32_t top_k,
+                                   int32_t *idx_out, void *out, sa_dtype out_dtype, float *lse,
+                                   void *stream);
+
 /* Device-side status of the most recent call that used `workspace`.
  * Synchronises `stream`.  Returns SA_OK, SA_ERR_DEVICE_FAULT or
  * SA_ERR_TIMEOUT; *detail (may be NULL) receives an SA_DETAIL_* code. */

@@ -22,8 +22,9 @@ DTYPES = {"f32": SA_F32, "bf16": SA_BF16, "e4m3": SA_E4M3}
 
 # every symbol include/sa.h declares
 EXPORTS = ("sa_workspace_size", "sa_indexer_score", "sa_topk", "sa_sparse_mla_attn",
-           "sa_decode", "sa_decode_traced", "sa_device_status", "sa_kernel_launches",
-           "sa_status_string", "sa_version")
+           "sa_decode", "sa_decode_traced", "sa_decode_noalloc", "sa_device_status",
+           "sa_kernel_launches", "sa_status_string", "sa_version")
+NOALLOC_SCRATCH_BYTES = 32 << 20
 DECODE_PHASES = ("indexer", "topk", "attention")
 
 _P, _I32, _I64, _SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
@@ -78,6 +79,8 @@ def lib():
         L.sa_decode.restype = ctypes.c_int
         L.sa_decode_traced.argtypes = [CP, QP, _I32, _P, _P, ctypes.c_int, _P, _P, _SZ, _P, _P]
         L.sa_decode_traced.restype = ctypes.c_int
+        L.sa_decode_noalloc.argtypes = [CP, QP, _I32, _P, _P, ctypes.c_int, _P, _P]
+        L.sa_decode_noalloc.restype = ctypes.c_int
         L.sa_device_status.argtypes = [_P, _SZ, _P, ctypes.POINTER(_I32)]
         L.sa_device_status.restype = ctypes.c_int
         L.sa_status_string.argtypes = [ctypes.c_int]
