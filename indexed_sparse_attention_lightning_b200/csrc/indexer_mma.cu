@@ -13,12 +13,14 @@
 // an equal contiguous share, so short and long contexts balance across SMs.
 // Roles per CTA (192 threads):
 //   warp 0     TMA producer: key pages (8 KB each, 128-byte swizzle) straight
-//              from the paged cache into a 4-stage ring, and the query's
-//              64x128 e4m3 block when the query changes;
+//              from the paged cache into a 4-stage ring together with their
+//              per-token scales (bulk copy), and the query's 64x128 e4m3 block
+//              when the query changes;
 //   warp 1     one thread issues the MMAs and commits them to mbarriers;
 //   warps 2-5  epilogue: each thread owns one key row of the tile, reads its
 //              64 head scores from TMEM (tcgen05.ld), applies ReLU, the head
-//              weights and the key scale, and writes one fp32 score.
+//              weights and the staged key scale, and writes one fp32 score;
+//              it touches only shared memory and TMEM besides that store.
 // Every wait is bounded; a timeout is reported in the workspace status word.
 #include "common.cuh"
 #include "internal.h"
@@ -42,7 +44,9 @@ constexpr uint32_t kTmemCols = kAcc * kHeads;
 struct IndexerSmem {
     uint8_t keys[kStages][kTileBytes];  // 1024-byte aligned (128-byte swizzle atoms)
     uint8_t q[2][kQBytes];
-    uint64_t full[kStages], empty[kStages];
+    float kscale[kStages][kKeys];       // per-token key scales of the staged pages
+    int32_t page_ok[kStages][2];        // 1 when the staged page id was valid
+    uint64_t full[kStages], empty[kStages], sc_empty[kStages];
     uint64_t acc_full[kAcc], acc_empty[kAcc];
     uint64_t q_full[2], q_empty[2];
     uint64_t done;
@@ -123,6 +127,7 @@ indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&sm.full[s], 1);
             mbar_init(&sm.empty[s], 1);
+            mbar_init(&sm.sc_empty[s], 4);
         }
         for (int c = 0; c < kAcc; ++c) {
             mbar_init(&sm.acc_full[c], 1);
@@ -161,7 +166,11 @@ indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
                     V = a.vis[c.t];
                 }
                 const int stage = n % kStages;
+                // the stage is free once its MMAs and its epilogue are done
                 if (!mbar_wait(&sm.empty[stage], ((n / kStages) & 1) ^ 1, abort_flag, p.status))
+                    break;
+                if (!mbar_wait(&sm.sc_empty[stage], ((n / kStages) & 1) ^ 1, abort_flag,
+                               p.status))
                     break;
                 int32_t rows[2] = {-1, -1};
                 uint32_t bytes = 0;
@@ -172,16 +181,20 @@ indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
                         const int32_t page = p.page_table[(int64_t)seq * p.max_pages + (s >> 6)];
                         if (page >= 0 && page < p.num_pages) {
                             rows[h] = page * 64;
-                            bytes += kPageBytes;
+                            bytes += kPageBytes + 64 * sizeof(float);
                         }
                     }
+                    sm.page_ok[stage][h] = rows[h] >= 0;  // published by the arrive below
                 }
                 mbar_arrive_expect_tx(&sm.full[stage], bytes);
 #pragma unroll
                 for (int h = 0; h < 2; ++h)
-                    if (rows[h] >= 0)
+                    if (rows[h] >= 0) {
                         tma_load_2d(sm.keys[stage] + h * kPageBytes, &tm_keys, 0, rows[h],
                                     &sm.full[stage]);
+                        bulk_load(&sm.kscale[stage][64 * h], p.k_index_scale + rows[h],
+                                  64 * sizeof(float), &sm.full[stage]);
+                    }
                 seg_start = c.next(a.tile_end);
             }
         }
@@ -224,11 +237,10 @@ indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
         TileCursor c;
         c.init(a.tile_end, p.n_q, k0, k1);
         bool seg_start = true;
-        int32_t seq = 0, V = 0;
+        int32_t V = 0;
         float wq[kHeads];
         for (int n = 0; c.valid(); ++n) {
             if (seg_start) {
-                seq = p.q_seq[c.t];
                 V = a.vis[c.t];
                 const float *w = p.w + (int64_t)c.t * kHeads;
                 const float *qs = p.q_index_scale + (int64_t)c.t * kHeads;
@@ -236,17 +248,14 @@ indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
                 for (int j = 0; j < kHeads; ++j) wq[j] = __ldg(w + j) * __ldg(qs + j);
             }
             const int64_t s = (int64_t)c.i * kKeys + row;
-            float kscale = 0.f;
-            bool ok = false;
-            if (s < V) {
-                const int32_t page = p.page_table[(int64_t)seq * p.max_pages + (s >> 6)];
-                if (page >= 0 && page < p.num_pages) {
-                    kscale = __ldg(p.k_index_scale + (int64_t)page * 64 + (s & 63));
-                    ok = true;
-                } else {
-                    report(p.status, SA_ERR_DEVICE_FAULT, SA_DETAIL_BAD_PAGE);
-                }
-            }
+            const int stage = n % kStages;
+            // key scales and page validity arrive with the key pages
+            if (!warp_wait(&sm.full[stage], (n / kStages) & 1, abort_flag, p.status)) break;
+            const bool ok = sm.page_ok[stage][row >> 6] != 0;
+            const float kscale = sm.kscale[stage][row];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.sc_empty[stage]);
+            if (s < V && !ok) report(p.status, SA_ERR_DEVICE_FAULT, SA_DETAIL_BAD_PAGE);
             const int acc = n % kAcc;
             if (!warp_wait(&sm.acc_full[acc], (n / kAcc) & 1, abort_flag, p.status)) break;
             tc_fence_after();

@@ -82,6 +82,16 @@ cudaError_t launch_topk_rowwise(const float *scores, int64_t ld, const int32_t *
 cudaError_t launch_attn_simt(const PathParams &p, const int32_t *idx, int32_t top_k, void *out,
                              int32_t out_dtype, float *lse, cudaStream_t s);
 
+// Tensor-core sparse attention (bf16 cache and query, 128 heads, 512 + 64
+// dims, K <= 2048) over CTA pairs; `splits` key splits per query, whose
+// partial outputs go to o_part [n_q, splits, 128, 512] / lse_part
+// [n_q, splits, 128] and are merged by a second kernel when splits > 1.
+bool sfa_mma_supported(const PathParams &p, int32_t top_k);
+int32_t sfa_splits(int32_t n_q, int32_t top_k);
+cudaError_t launch_sfa_mma(const PathParams &p, const int32_t *idx, int32_t top_k, int32_t splits,
+                           void *out, int32_t out_dtype, float *lse, float *o_part,
+                           float *lse_part, cudaStream_t s);
+
 }  // namespace sa
 
 // ---- inline device definitions -------------------------------------------

@@ -37,7 +37,8 @@ sa_status check_cache(const sa_cache *c) {
     if (!c->page_table || !c->seq_len || !c->k_index || !c->kv) return SA_ERR_INVALID_ARG;
     if (!aligned16(c->k_index) || !aligned16(c->kv)) return SA_ERR_INVALID_ARG;
     if (c->index_dtype != SA_F32 && c->index_dtype != SA_E4M3) return SA_ERR_UNSUPPORTED;
-    if (c->index_dtype == SA_E4M3 && !c->k_index_scale) return SA_ERR_INVALID_ARG;
+    if (c->index_dtype == SA_E4M3 && (!c->k_index_scale || !aligned16(c->k_index_scale)))
+        return SA_ERR_INVALID_ARG;
     if (c->d_index <= 0 || c->d_index % 16 != 0) return SA_ERR_INVALID_ARG;
     if (c->d_index > 256) return SA_ERR_UNSUPPORTED;
     if (c->kv_dtype != SA_F32 && c->kv_dtype != SA_BF16 && c->kv_dtype != SA_E4M3)
@@ -104,24 +105,53 @@ PathParams make_params(const sa_cache *c, const sa_query *q, void *ws) {
     return p;
 }
 
-// Workspace: status | vis [n_q] | tile_end [n_q] | scores [n_q, ld] | idx [n_q, K];
-// the indexer needs the first three, the fused path all five.
+// Workspace: status | vis [n_q] | tile_end [n_q] | scores [n_q, ld] | idx [n_q, K]
+// | o_part [n_q, S, 128, 512] | lse_part [n_q, S, 128]; the indexer needs the
+// first three, the fused path all of them; the attention alone needs the
+// status and the split-KV partials (placed right after the status).
 struct Layout {
     int64_t ld;
-    size_t vis, tile_end, scores, idx, indexer_total, decode_total;
+    int32_t splits;
+    size_t vis, tile_end, scores, idx, o_part, lse_part, indexer_total, decode_total;
+    size_t attn_o_part, attn_lse_part, attn_total;
 };
+
+size_t part_bytes(size_t nq, int32_t splits, size_t per) {
+    return splits > 1 ? per * nq * (size_t)splits : 0;
+}
 
 Layout make_layout(const sa_query *q, int32_t top_k) {
     Layout l{};
     const size_t nq = q->n_q > 0 ? (size_t)q->n_q : 0;
     l.ld = round_up(q->max_visible > 0 ? q->max_visible : 1, 128);
+    l.splits = sfa_splits(q->n_q, top_k > 0 ? top_k : 1);
+    const size_t o_bytes = part_bytes(nq, l.splits, sizeof(float) * 128 * 512);
+    const size_t lse_bytes = part_bytes(nq, l.splits, sizeof(float) * 128);
     l.vis = align_up(kStatusBytes);
     l.tile_end = align_up(l.vis + sizeof(int32_t) * nq);
     l.indexer_total = align_up(l.tile_end + sizeof(int32_t) * nq);
     l.scores = l.indexer_total;
     l.idx = align_up(l.scores + sizeof(float) * nq * (size_t)l.ld);
-    l.decode_total = align_up(l.idx + sizeof(int32_t) * nq * (size_t)(top_k > 0 ? top_k : 0));
+    l.o_part = align_up(l.idx + sizeof(int32_t) * nq * (size_t)(top_k > 0 ? top_k : 0));
+    l.lse_part = align_up(l.o_part + o_bytes);
+    l.decode_total = align_up(l.lse_part + lse_bytes);
+    l.attn_o_part = align_up(kStatusBytes);
+    l.attn_lse_part = align_up(l.attn_o_part + o_bytes);
+    l.attn_total = align_up(l.attn_lse_part + lse_bytes);
     return l;
+}
+
+// Sparse attention: the tensor-core kernel for its shape, CUDA cores otherwise.
+sa_status run_attention(const PathParams &p, const Layout &l, size_t o_off, size_t lse_off,
+                        void *ws, const int32_t *idx, int32_t top_k, void *out,
+                        int32_t out_dtype, float *lse, cudaStream_t s) {
+    if (sfa_mma_supported(p, top_k)) {
+        char *base = static_cast<char *>(ws);
+        return cuda_status(launch_sfa_mma(p, idx, top_k, l.splits, out, out_dtype, lse,
+                                          reinterpret_cast<float *>(base + o_off),
+                                          reinterpret_cast<float *>(base + lse_off), s));
+    }
+    return cuda_status(launch_attn_simt(p, idx, top_k, out, out_dtype, lse, s));
 }
 
 // Indexer scores into `scores` (ld): the tensor-core kernel for its shape,
@@ -164,6 +194,7 @@ size_t sa_workspace_size(const sa_cache *cache, const sa_query *query, int32_t t
     const Layout l = make_layout(query, top_k);
     size_t need = kStatusBytes;
     if (uses & SA_WS_INDEXER) need = std::max(need, l.indexer_total);
+    if (uses & SA_WS_ATTN) need = std::max(need, l.attn_total);
     if (uses & SA_WS_DECODE) need = std::max(need, l.decode_total);
     return align_up(need);
 }
@@ -208,11 +239,14 @@ sa_status sa_sparse_mla_attn(const sa_cache *cache, const sa_query *query, const
     if (top_k <= 0 || top_k > kMaxTopK) return SA_ERR_INVALID_ARG;
     if (out_dtype != SA_BF16 && out_dtype != SA_F32) return SA_ERR_UNSUPPORTED;
     if (query->n_q > 0 && (!idx || !out)) return SA_ERR_INVALID_ARG;
-    if ((st = check_workspace(workspace, workspace_bytes, kStatusBytes)) != SA_OK) return st;
+    const Layout l = make_layout(query, top_k);
+    if ((st = check_workspace(workspace, workspace_bytes, l.attn_total)) != SA_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if ((st = clear_status(workspace, s)) != SA_OK) return st;
+    if (query->n_q == 0) return SA_OK;
     PathParams p = make_params(cache, query, workspace);
-    return cuda_status(launch_attn_simt(p, idx, top_k, out, out_dtype, lse, s));
+    return run_attention(p, l, l.attn_o_part, l.attn_lse_part, workspace, idx, top_k, out,
+                         out_dtype, lse, s);
 }
 
 static sa_status decode_impl(const sa_cache *cache, const sa_query *query, int32_t top_k,
@@ -245,7 +279,8 @@ static sa_status decode_impl(const sa_cache *cache, const sa_query *query, int32
                                                   query->n_q, top_k, idx, p.status, s))) != SA_OK)
             return st;
         if ((st = mark(2)) != SA_OK) return st;
-        if ((st = cuda_status(launch_attn_simt(p, idx, top_k, out, out_dtype, lse, s))) != SA_OK)
+        if ((st = run_attention(p, l, l.o_part, l.lse_part, workspace, idx, top_k, out,
+                                out_dtype, lse, s)) != SA_OK)
             return st;
         return mark(3);
     }

@@ -1,0 +1,524 @@
+// sfa_mma.cu -- sparse MLA attention on the 5th-generation tensor cores,
+// one CTA pair (cluster of two) per (query, key split).
+//
+// For query t and its selected latent rows s ("Optimizing Next-Gen LLM
+// Inference" §3.3: attention only on the selected positions, reading the cache
+// by index; "Inference Acceleration for New Large Model Architectures" §3.2:
+// aggregated, vectorised sparse reads; "Engineering Practices for Optimizing
+// Ultra-Large Sparse Attention Model Inference" §3.1: index construction, block
+// loading with asynchronous prefetch, local attention on matrix units):
+//     z_s = sm_scale * q[t,h,:] . kv[s,:]   (576-d: 512 latent + 64 rope)
+//     out[t,h,:] = sum_s softmax(z)_s kv[s, 0:512],   lse = log sum_s exp(z_s)
+//
+// B200 mapping.  All 128 absorbed-query heads share the selected rows, so both
+// contractions are dense per key tile: S = Q K^T (M = 128 heads, N = 32 keys,
+// K = 576) and O += P V (M = 128 heads, N = 512, K = 32 keys).  O is 128 x 512
+// fp32 = all of one SM's TMEM, so the heads are split over a CTA pair with
+// tcgen05.mma.cta_group::2 (M = 128 = 64 heads per CTA, full rate): each CTA
+// keeps its 64 heads x 512 dims of O in its own TMEM (256 columns), the even
+// CTA issues every MMA for both.  The B operand of each MMA is split by
+// columns across the pair: for S each CTA holds 16 of the 32 keys (full
+// 576-d rows), for P V each CTA holds 128 of every 256 output dims of all 32
+// keys.  Rows arrive by TMA tile::gather4 straight from the paged cache
+// (128-byte swizzled boxes of 64 dims), so no dequantised or gathered copy of
+// the cache is ever written to global memory.
+//
+// Roles per CTA (192 threads):
+//   warp 0     producer: query block once, then per tile 68 gather4 loads into
+//              a 3-stage ring (lanes issue them in parallel);
+//   warp 1     even CTA: issues S and P V MMAs and commits them to both CTAs'
+//              barriers; odd CTA: relays "stage loaded" to the even CTA;
+//   warps 2-5  compact the index list into physical rows, then run the online
+//              softmax: thread L owns TMEM lane L = (head L % 64, key half /
+//              output half L / 64); the two halves of a head exchange their
+//              tile maxima through shared memory; O is rescaled in TMEM only
+//              when the running maximum grows by more than 2^8; P goes to
+//              shared memory as bf16 for the P V MMA; finally O / l is written.
+// All waits are bounded; a timeout is reported in the workspace status word.
+#include "common.cuh"
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace sa {
+namespace {
+using namespace sm100;
+
+constexpr int kHeadsCta = 64;
+constexpr int kDl = 512, kDr = 64, kD = kDl + kDr;
+constexpr int kBlocks = kD / 64;  // 64-dim (128-byte) column blocks of a row
+constexpr int kTile = 32;         // selected keys per tile
+constexpr int kHalf = kTile / 2;  // keys per CTA in the S operand
+constexpr int kStages = 3;
+constexpr int kThreads = 192;
+constexpr int kMaxK = 2048;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColO = 0;     // 256 columns: two 128-column halves of 256 output dims
+constexpr uint32_t kColS = 256;   // two S buffers of 16 columns
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kRescaleLog2 = 8.0f;
+constexpr int kGathersKs = kBlocks * (kHalf / 4);   // 36
+constexpr int kGathersPv = 4 * (kTile / 4);         // 32
+constexpr uint32_t kStageBytes = (kGathersKs + kGathersPv) * 4 * 128;
+constexpr uint32_t kQBytes = kBlocks * kHeadsCta * 128;
+
+struct SfaStage {
+    uint8_t ks[kBlocks][kHalf * 128];  // this CTA's 16 keys, full rows, K-major
+    uint8_t pv[4][kTile * 128];        // this CTA's 256 output dims of all 32 keys
+};
+
+struct SfaSmem {
+    uint8_t q[kBlocks][kHeadsCta * 128];
+    SfaStage st[kStages];
+    uint8_t p[2][kHeadsCta * 128];     // P (bf16), 32 keys used of each 128-byte row
+    int32_t rows[kMaxK];               // compacted physical rows of the selected keys
+    float xmax[2][128];
+    float lsum[128];
+    int32_t warp_cnt[4];
+    int32_t n_valid;
+    uint64_t q_full, peer_q_full, rows_ready;
+    uint64_t full[kStages], peer_full[kStages], empty[kStages];
+    uint64_t s_full[2], p_full[2], o_done[2], xch[2], lx;
+    uint32_t tmem_base;
+    int abort;
+};
+
+static_assert(sizeof(SfaSmem) + 1024 <= 232448, "shared memory budget of one CTA");
+static_assert(kStageBytes == sizeof(SfaStage), "gathers fill the stage exactly");
+
+struct SfaArgs {
+    PathParams p;
+    const int32_t *idx;  // [n_q, K]
+    int32_t K;
+    int32_t splits;
+    void *out;           // [n_q, 128, 512] (splits == 1)
+    int32_t out_dtype;
+    float *lse;          // [n_q, 128] or null (splits == 1)
+    float *o_part;       // [n_q, splits, 128, 512] (splits > 1)
+    float *lse_part;     // [n_q, splits, 128]      (splits > 1)
+};
+
+__device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
+    return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                          int32_t *status, bool cluster_scope = false) {
+    bool ok = true;
+    if (lane_id() == 0)
+        ok = cluster_scope ? mbar_wait_cluster(bar, parity, abort_flag, status)
+                           : mbar_wait(bar, parity, abort_flag, status);
+    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+    __syncwarp();
+    return ok;
+}
+
+// Tiles [j0, j1) of the compacted key list handled by this split.
+__device__ __forceinline__ void split_range(int32_t n_valid, int32_t split, int32_t splits,
+                                            int32_t &j0, int32_t &j1) {
+    const int32_t tiles = (n_valid + kTile - 1) / kTile;
+    j0 = (int32_t)((int64_t)tiles * split / splits);
+    j1 = (int32_t)((int64_t)tiles * (split + 1) / splits);
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+sfa_mma_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_constant__ CUtensorMap tm_q,
+               const SfaArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    SfaSmem &sm = *reinterpret_cast<SfaSmem *>(align1024(smem_raw));
+    const PathParams &p = a.p;
+    const uint32_t rank = cluster_ctarank();
+    const int unit = blockIdx.x >> 1;
+    const int t = unit / a.splits, split = unit % a.splits;
+    const int warp = warp_id(), lane = lane_id();
+
+    if (threadIdx.x == 0) {
+        mbar_init(&sm.q_full, 1);
+        mbar_init(&sm.peer_q_full, 1);
+        mbar_init(&sm.rows_ready, 1);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.peer_full[s], 1);
+            mbar_init(&sm.empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sm.s_full[b], 1);
+            mbar_init(&sm.p_full[b], 8);  // 4 softmax warps in each CTA of the pair
+            mbar_init(&sm.o_done[b], 1);
+            mbar_init(&sm.xch[b], 4);
+        }
+        mbar_init(&sm.lx, 4);
+        sm.abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0) tmem_alloc_pair(&sm.tmem_base, kTmemCols);
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();  // both CTAs' barriers exist before anyone arrives remotely
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    volatile int *abort_flag = &sm.abort;
+    int32_t *status = p.status;
+
+    if (warp >= 2) {
+        // --------------------------------------------- row compaction ---
+        const int et = threadIdx.x - 64, ew = et >> 5;
+        const int32_t V = visible_len(p, t);
+        const int32_t seq = p.q_seq[t];
+        const int32_t *sel = a.idx + (int64_t)t * a.K;
+        int32_t base = 0;
+        for (int k0 = 0; k0 < a.K; k0 += 128) {
+            const int k = k0 + et;
+            int32_t phys = -1;
+            if (k < a.K) {
+                const int32_t s = sel[k];
+                if (s >= V) {
+                    report(status, SA_ERR_DEVICE_FAULT, SA_DETAIL_BAD_INDEX);
+                } else if (s >= 0) {
+                    const int64_t r = phys_row(p.page_table, p.max_pages, p.num_pages, seq, s);
+                    if (r < 0) report(status, SA_ERR_DEVICE_FAULT, SA_DETAIL_BAD_PAGE);
+                    else phys = static_cast<int32_t>(r);
+                }
+            }
+            const unsigned bal = __ballot_sync(0xffffffffu, phys >= 0);
+            if (lane == 0) sm.warp_cnt[ew] = __popc(bal);
+            named_barrier(1, 128);
+            int32_t off = base, tot = 0;
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+                if (w < ew) off += sm.warp_cnt[w];
+                tot += sm.warp_cnt[w];
+            }
+            const int32_t pos = off + __popc(bal & ((1u << lane) - 1u));
+            if (phys >= 0 && pos < kMaxK) sm.rows[pos] = phys;
+            named_barrier(1, 128);
+            base += tot;
+        }
+        const int32_t n_valid = min(base, (int32_t)kMaxK);
+        const int32_t padded = ((n_valid + kTile - 1) / kTile) * kTile;
+        for (int c = n_valid + et; c < padded; c += 128) sm.rows[c] = sm.rows[0];
+        named_barrier(1, 128);
+        if (et == 0) {
+            sm.n_valid = n_valid;
+            mbar_arrive(&sm.rows_ready);  // release: rows and n_valid are visible
+        }
+
+        // ----------------------------------------------- online softmax ---
+        int32_t j0, j1;
+        split_range(n_valid, split, a.splits, j0, j1);
+        const int T = j1 - j0;
+        const int L = 32 * (warp & 3) + lane;  // TMEM lane owned by this thread
+        const int h = L & 63, hf = L >> 6;
+        const uint32_t lane_base = static_cast<uint32_t>(32 * (warp & 3)) << 16;
+        const float sl2 = p.sm_scale * kLog2e;
+        float m_run = -INFINITY, l_half = 0.f;
+        bool ok = true;
+        for (int n = 0; n < T && ok; ++n) {
+            const int sb = n & 1;
+            if (!(ok = warp_wait(&sm.s_full[sb], (n >> 1) & 1, abort_flag, status, true))) break;
+            tc_fence_after();
+            float s[16];
+            tmem_ld16(tmem + lane_base + kColS + 16 * sb, s);
+            tmem_wait_ld();
+            const int kvalid = n_valid - ((j0 + n) * kTile + kHalf * hf);
+            float tmax = -INFINITY;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                s[i] = i < kvalid ? s[i] * sl2 : -INFINITY;
+                tmax = fmaxf(tmax, s[i]);
+            }
+            sm.xmax[sb][L] = tmax;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.xch[sb]);
+            if (!(ok = warp_wait(&sm.xch[sb], (n >> 1) & 1, abort_flag, status))) break;
+            const float mt = fmaxf(tmax, sm.xmax[sb][L ^ 64]);
+            if (mt > m_run + kRescaleLog2) {
+                if (n > 0) {
+                    // O holds P V of earlier tiles: wait for the last one, then rescale
+                    if (!(ok = warp_wait(&sm.o_done[(n - 1) & 1], ((n - 1) >> 1) & 1, abort_flag,
+                                         status, true)))
+                        break;
+                    tc_fence_after();
+                    const float f = exp2f(m_run - mt);
+#pragma unroll 1
+                    for (int c = 0; c < 8; ++c) {
+                        float v[32];
+                        tmem_ld32(tmem + lane_base + kColO + 32 * c, v);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) v[i] *= f;
+                        tmem_st32(tmem + lane_base + kColO + 32 * c, v);
+                    }
+                    tmem_wait_st();
+                    l_half *= f;
+                }
+                m_run = mt;
+            }
+            uint32_t packed[8];
+#pragma unroll
+            for (int i = 0; i < 16; i += 2) {
+                const float p0 = exp2f(s[i] - m_run), p1 = exp2f(s[i + 1] - m_run);
+                l_half += p0 + p1;
+                __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
+                packed[i / 2] = *reinterpret_cast<uint32_t *>(&b2);
+            }
+            // P buffer sb was last read by the P V MMA of tile n - 2
+            if (n >= 2 && !(ok = warp_wait(&sm.o_done[sb], ((n - 2) >> 1) & 1, abort_flag, status,
+                                           true)))
+                break;
+            uint8_t *prow = sm.p[sb] + h * 128;
+            const int sw = h & 7;
+            *reinterpret_cast<uint4 *>(prow + (((2 * hf) ^ sw) << 4)) =
+                make_uint4(packed[0], packed[1], packed[2], packed[3]);
+            *reinterpret_cast<uint4 *>(prow + (((2 * hf + 1) ^ sw) << 4)) =
+                make_uint4(packed[4], packed[5], packed[6], packed[7]);
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                if (rank == 0) mbar_arrive(&sm.p_full[sb]);
+                else mbar_arrive_remote(map_to_rank(smem_u32(&sm.p_full[sb]), 0));
+            }
+        }
+        if (ok && T > 0)
+            ok = warp_wait(&sm.o_done[(T - 1) & 1], ((T - 1) >> 1) & 1, abort_flag, status, true);
+        tc_fence_after();
+        // both halves of a head hold part of its softmax denominator
+        sm.lsum[L] = l_half;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.lx);
+        if (warp_wait(&sm.lx, 0, abort_flag, status)) {
+            const float l = l_half + sm.lsum[L ^ 64];
+            const float inv = (ok && l > 0.f) ? 1.f / l : 0.f;
+            const float lse_v = (ok && l > 0.f) ? (m_run + log2f(l)) * kLn2 : -INFINITY;
+            const int head = kHeadsCta * rank + h;
+            const int64_t row = (int64_t)t * 128 + head;
+#pragma unroll 1
+            for (int c = 0; c < 8; ++c) {
+                float v[32];
+                if (ok && T > 0) {
+                    tmem_ld32(tmem + lane_base + kColO + 32 * c, v);
+                    tmem_wait_ld();
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) v[i] = 0.f;
+                }
+                const int dv = 256 * (c >> 2) + 128 * hf + 32 * (c & 3);
+                if (a.splits == 1) {
+                    if (a.out_dtype == SA_BF16) {
+                        uint32_t w[16];
+#pragma unroll
+                        for (int i = 0; i < 32; i += 2) {
+                            __nv_bfloat162 b2 = __floats2bfloat162_rn(v[i] * inv, v[i + 1] * inv);
+                            w[i / 2] = *reinterpret_cast<uint32_t *>(&b2);
+                        }
+                        uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.out) +
+                                                               row * kDl + dv);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+                    } else {
+                        float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(a.out) +
+                                                                 row * kDl + dv);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            dst[i] = make_float4(v[4 * i] * inv, v[4 * i + 1] * inv,
+                                                 v[4 * i + 2] * inv, v[4 * i + 3] * inv);
+                    }
+                } else {
+                    const int64_t prow_i = ((int64_t)t * a.splits + split) * 128 + head;
+                    float4 *dst = reinterpret_cast<float4 *>(a.o_part + prow_i * kDl + dv);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        dst[i] = make_float4(v[4 * i] * inv, v[4 * i + 1] * inv, v[4 * i + 2] * inv,
+                                             v[4 * i + 3] * inv);
+                }
+            }
+            if (hf == 0) {
+                if (a.splits == 1) {
+                    if (a.lse != nullptr) a.lse[row] = lse_v;
+                } else {
+                    a.lse_part[((int64_t)t * a.splits + split) * 128 + head] = lse_v;
+                }
+            }
+        }
+    } else {
+        // both the producer and the MMA warp need this split's tile range
+        const bool ready = warp_wait(&sm.rows_ready, 0, abort_flag, status);
+        int32_t j0 = 0, j1 = 0;
+        if (ready) split_range(sm.n_valid, split, a.splits, j0, j1);
+        const int T = j1 - j0;
+        if (warp == 0 && T > 0) {
+            // --------------------------------------------- producer ---
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&sm.q_full, kQBytes);
+                for (int b = 0; b < kBlocks; ++b)
+                    tma_load_2d(sm.q[b], &tm_q, 64 * b, t * 128 + kHeadsCta * rank, &sm.q_full);
+            }
+            for (int n = 0; n < T; ++n) {
+                const int stage = n % kStages;
+                if (!warp_wait(&sm.empty[stage], ((n / kStages) & 1) ^ 1, abort_flag, status,
+                               true))
+                    break;
+                if (lane == 0) mbar_arrive_expect_tx(&sm.full[stage], kStageBytes);
+                __syncwarp();
+                const int kb = (j0 + n) * kTile;
+                SfaStage &st = sm.st[stage];
+                for (int g = lane; g < kGathersKs + kGathersPv; g += 32) {
+                    if (g < kGathersKs) {
+                        const int b = g >> 2, grp = g & 3;
+                        const int32_t *r = &sm.rows[kb + kHalf * rank + 4 * grp];
+                        tma_gather4(st.ks[b] + grp * 512, &tm_kv, 64 * b, r[0], r[1], r[2], r[3],
+                                    &sm.full[stage]);
+                    } else {
+                        const int gp = g - kGathersKs, c = gp >> 3, grp = gp & 7;
+                        const int dvb = (c < 2 ? 0 : 4) + 2 * rank + (c & 1);
+                        const int32_t *r = &sm.rows[kb + 4 * grp];
+                        tma_gather4(st.pv[c] + grp * 512, &tm_kv, 64 * dvb, r[0], r[1], r[2], r[3],
+                                    &sm.full[stage]);
+                    }
+                }
+            }
+        } else if (warp == 1 && T > 0 && lane == 0) {
+            if (rank == 0) {
+                // ------------------------------------------ MMA issuer ---
+                constexpr uint32_t id_s = instr_desc(128, kTile, 1 /*bf16*/, 0, 0);
+                constexpr uint32_t id_pv = instr_desc(128, 256, 1 /*bf16*/, 0, 1);
+                bool ok = mbar_wait(&sm.q_full, 0, abort_flag, status) &&
+                          mbar_wait_cluster(&sm.peer_q_full, 0, abort_flag, status);
+                auto issue_s = [&](int n) -> bool {
+                    const int stage = n % kStages;
+                    const uint32_t ph = (n / kStages) & 1;
+                    if (!mbar_wait(&sm.full[stage], ph, abort_flag, status)) return false;
+                    if (!mbar_wait_cluster(&sm.peer_full[stage], ph, abort_flag, status))
+                        return false;
+                    tc_fence_after();
+                    const uint32_t d = tmem + kColS + 16 * (n & 1);
+#pragma unroll 1
+                    for (int b = 0; b < kBlocks; ++b) {
+                        const uint64_t ad = desc_kmajor_sw128(smem_u32(sm.q[b]));
+                        const uint64_t bd = desc_kmajor_sw128(smem_u32(sm.st[stage].ks[b]));
+#pragma unroll
+                        for (int k = 0; k < 4; ++k)  // 16 bf16 (32 bytes) of K per instruction
+                            mma_bf16_pair(d, ad + 2 * k, bd + 2 * k, id_s, (b | k) != 0);
+                    }
+                    mma_commit_pair_multicast(&sm.s_full[n & 1], 0x3);
+                    return true;
+                };
+                if (ok) ok = issue_s(0);
+                for (int n = 0; n < T && ok; ++n) {
+                    if (n + 1 < T && !(ok = issue_s(n + 1))) break;
+                    if (!(ok = mbar_wait_cluster(&sm.p_full[n & 1], (n >> 1) & 1, abort_flag,
+                                                 status)))
+                        break;
+                    tc_fence_after();
+                    const int stage = n % kStages;
+                    const uint64_t ad = desc_kmajor_sw128(smem_u32(sm.p[n & 1]));
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        const uint32_t va = smem_u32(sm.st[stage].pv[2 * half]);
+#pragma unroll
+                        for (int k = 0; k < 2; ++k)  // 16 keys per instruction
+                            mma_bf16_pair(tmem + kColO + 128 * half, ad + 2 * k,
+                                          desc_mnmajor_sw128(va + 2048 * k, kTile * 128, 1024),
+                                          id_pv, (n > 0 || k > 0) ? 1u : 0u);
+                    }
+                    mma_commit_pair_multicast(&sm.o_done[n & 1], 0x3);
+                    if (n + kStages < T) mma_commit_pair_multicast(&sm.empty[stage], 0x3);
+                }
+            } else {
+                // --------------------------------------------- relay ---
+                if (mbar_wait(&sm.q_full, 0, abort_flag, status))
+                    mbar_arrive_remote(map_to_rank(smem_u32(&sm.peer_q_full), 0));
+                for (int n = 0; n < T; ++n) {
+                    const int stage = n % kStages;
+                    if (!mbar_wait(&sm.full[stage], (n / kStages) & 1, abort_flag, status)) break;
+                    mbar_arrive_remote(map_to_rank(smem_u32(&sm.peer_full[stage]), 0));
+                }
+            }
+        }
+    }
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();  // the pair no longer touches each other's shared memory or TMEM
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem, kTmemCols);
+    }
+}
+
+// out = sum_s w_s o_s with w_s = exp(lse_s - lse), lse = log sum_s exp(lse_s).
+__global__ void __launch_bounds__(128)
+sfa_combine_kernel(const float *__restrict__ o_part, const float *__restrict__ lse_part,
+                   int32_t splits, void *out, int32_t out_dtype, float *lse) {
+    const int64_t row = blockIdx.x;  // t * 128 + head
+    const int64_t t = row >> 7, head = row & 127;
+    float m = -INFINITY;
+    for (int s = 0; s < splits; ++s) m = fmaxf(m, lse_part[(t * splits + s) * 128 + head]);
+    float acc[4] = {0.f, 0.f, 0.f, 0.f}, wsum = 0.f;
+    if (m != -INFINITY) {
+        for (int s = 0; s < splits; ++s) {
+            const float ls = lse_part[(t * splits + s) * 128 + head];
+            const float w = ls == -INFINITY ? 0.f : __expf(ls - m);
+            wsum += w;
+            const float4 v = reinterpret_cast<const float4 *>(
+                o_part + ((t * splits + s) * 128 + head) * kDl)[threadIdx.x];
+            acc[0] += w * v.x;
+            acc[1] += w * v.y;
+            acc[2] += w * v.z;
+            acc[3] += w * v.w;
+        }
+    }
+    const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+    if (out_dtype == SA_BF16) {
+        __nv_bfloat162 a = __floats2bfloat162_rn(acc[0] * inv, acc[1] * inv);
+        __nv_bfloat162 b = __floats2bfloat162_rn(acc[2] * inv, acc[3] * inv);
+        uint2 w = make_uint2(*reinterpret_cast<uint32_t *>(&a), *reinterpret_cast<uint32_t *>(&b));
+        reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(out) + row * kDl)[threadIdx.x] = w;
+    } else {
+        reinterpret_cast<float4 *>(static_cast<float *>(out) + row * kDl)[threadIdx.x] =
+            make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+    }
+    if (lse != nullptr && threadIdx.x == 0) lse[row] = wsum > 0.f ? m + logf(wsum) : -INFINITY;
+}
+
+}  // namespace
+
+bool sfa_mma_supported(const PathParams &p, int32_t top_k) {
+    return p.kv_dtype == SA_BF16 && p.q_dtype == SA_BF16 && p.heads == 128 &&
+           p.d_latent == kDl && p.d_rope == kDr && top_k <= kMaxK &&
+           (int64_t)p.num_pages * 64 < (int64_t(1) << 31);
+}
+
+int32_t sfa_splits(int32_t n_q, int32_t top_k) {
+    const int32_t pairs = std::max(1, num_sms() / 2);
+    const int32_t max_tiles = (top_k + kTile - 1) / kTile;
+    if (n_q <= 0) return 1;
+    return std::max(1, std::min(max_tiles, pairs / n_q));
+}
+
+cudaError_t launch_sfa_mma(const PathParams &p, const int32_t *idx, int32_t top_k, int32_t splits,
+                           void *out, int32_t out_dtype, float *lse, float *o_part,
+                           float *lse_part, cudaStream_t s) {
+    if (p.n_q == 0) return cudaSuccess;
+    CUtensorMap tkv, tq;
+    if (!encode_tmap_2d(&tkv, 2, p.kv, kD, (uint64_t)p.num_pages * 64, kD * 2, 64, 1, true) ||
+        !encode_tmap_2d(&tq, 2, p.q, kD, (uint64_t)p.n_q * 128, kD * 2, 64, kHeadsCta, true))
+        return cudaErrorInvalidValue;
+    SfaArgs a{p, idx, top_k, splits, out, out_dtype, lse, o_part, lse_part};
+    const size_t smem = sizeof(SfaSmem) + 1024;
+    cudaError_t e =
+        cudaFuncSetAttribute(sfa_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int64_t grid = 2 * (int64_t)p.n_q * splits;
+    count_launch();
+    sfa_mma_kernel<<<static_cast<unsigned>(grid), kThreads, smem, s>>>(tkv, tq, a);
+    if ((e = cudaGetLastError()) != cudaSuccess || splits == 1) return e;
+    count_launch();
+    sfa_combine_kernel<<<static_cast<unsigned>(p.n_q * 128), 128, 0, s>>>(o_part, lse_part, splits,
+                                                                         out, out_dtype, lse);
+    return cudaGetLastError();
+}
+
+}  // namespace sa

@@ -205,3 +205,21 @@ def test_empty_batch_is_a_no_op():
     out, lse, _ = api.decode(cache, empty, wl.spec.top_k, out_dtype="f32")
     torch.cuda.synchronize()
     assert out.shape[0] == 0
+
+
+def test_attention_on_unsorted_indices_with_holes():
+    """sa_sparse_mla_attn takes any index order and skips -1 entries."""
+    wl = workload(W.DECODE_B8_8K)
+    K = 700
+    rng = np.random.default_rng(31)
+    idx = np.full((wl.n_q, K), -1, np.int32)
+    for t in range(wl.n_q):
+        n = [700, 650, 33, 1, 64, 699, 320, 17][t]
+        pos = rng.choice(int(wl.visible[t]), size=n, replace=False).astype(np.int32)
+        slots = np.sort(rng.choice(K, size=n, replace=False))
+        idx[t, slots] = pos                     # unsorted positions, -1 holes anywhere
+    cache, queries = api.upload(wl)
+    out, lse = api.sparse_mla_attn(cache, queries, torch.from_numpy(idx).cuda(), K)
+    ref_out, ref_lse = oracle.sparse_attn(wl, idx)
+    parity.check_attention(out.float().cpu().numpy(), ref_out, "bf16")
+    parity.check_lse(lse.cpu().numpy(), ref_lse)
