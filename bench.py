@@ -25,7 +25,6 @@ import hashlib
 import json
 import os
 import statistics
-import subprocess
 import sys
 import time
 
@@ -101,59 +100,69 @@ def algorithmic_bytes(wl, idx: np.ndarray) -> dict:
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples during the timed region."""
+    """SM clock and clock-event (throttle) reasons sampled DURING the timed
+    region by an NVML polling thread (a sample every half millisecond or so;
+    it only reads)."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
-        self.proc = None
-        self.path = os.path.join("/tmp", f"sa_clocks_{os.getpid()}.csv")
+    def __init__(self, torch_device: int):
+        self.dev = torch_device
+        self.samples = []          # (sm_mhz, reason bitmask)
+        self.max_mhz = None
+        self.thread = None
+        self.stop = False
+
+    def _handle(self, nv):
+        import torch
+        uuid = str(torch.cuda.get_device_properties(self.dev).uuid)
+        return nv.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
 
     def __enter__(self):
+        import threading
         try:
-            self.f = open(self.path, "w")
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=self.f, stderr=subprocess.DEVNULL)
+            import pynvml as nv
+            nv.nvmlInit()
+            h = self._handle(nv)
+            self.nv, self.h = nv, h
+            self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+
+            def poll():
+                while not self.stop:
+                    try:
+                        mhz = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                        rs = int(nv.nvmlDeviceGetCurrentClocksEventReasons(h))
+                        self.samples.append((mhz, rs))
+                    except Exception:
+                        pass
+                    time.sleep(0.0005)
+
+            self.thread = threading.Thread(target=poll, daemon=True)
+            self.thread.start()
+            time.sleep(0.002)
         except Exception:
-            self.proc = None
+            self.thread = None
         return self
 
     def __exit__(self, *exc):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except Exception:
-                self.proc.kill()
-            self.f.close()
+        if self.thread is not None:
+            self.stop = True
+            self.thread.join(timeout=2)
 
     def summary(self):
-        if self.proc is None or not os.path.exists(self.path):
+        if not self.samples:
             return None
-        sm, mx, reasons = [], [], set()
-        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
-        for line in open(self.path):
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                mx.append(float(parts[2]))
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        os.unlink(self.path)
-        if not sm:
-            return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
-                "reasons": sorted(reasons), "samples": len(sm)}
+        reasons = set()
+        for _, rs in self.samples:
+            for name, attr in self.REASONS:
+                if rs & int(getattr(self.nv, attr, 0)):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(m for m, _ in self.samples),
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(reasons),
+                "samples": len(self.samples), "source": "nvml"}
 
 
 def traffic_for(kernel: str, source_files: list[str]):

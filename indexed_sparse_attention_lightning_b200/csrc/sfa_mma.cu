@@ -23,11 +23,16 @@
 // (128-byte swizzled boxes of 64 dims), so no dequantised or gathered copy of
 // the cache is ever written to global memory.
 //
-// Roles per CTA (192 threads):
-//   warp 0     producer: query block once, then per tile 68 gather4 loads into
-//              a 3-stage ring (lanes issue them in parallel);
-//   warp 1     even CTA: issues S and P V MMAs and commits them to both CTAs'
-//              barriers; odd CTA: relays "stage loaded" to the even CTA;
+// Roles per CTA (224 threads):
+//   warp 0     producer of the S operand: the query block once, then per tile
+//              36 gather4 loads (this CTA's 16 keys, all 9 column blocks) into
+//              a 4-stage ring that is freed as soon as that tile's S is done;
+//   warp 6     producer of the P V operand: per tile 32 gather4 loads (this
+//              CTA's 4 output-dim blocks of all 32 keys) into a 3-stage ring;
+//   warp 1     even CTA: issues the MMAs for both CTAs from a non-blocking
+//              loop (S of a tile as soon as its keys are in, P V as soon as P
+//              is written) and commits them to both CTAs' barriers; odd CTA:
+//              relays "stage loaded" to the even CTA;
 //   warps 2-5  compact the index list into physical rows, then run the online
 //              softmax: thread L owns TMEM lane L = (head L % 64, key half /
 //              output half L / 64); the two halves of a head exchange their
@@ -48,8 +53,9 @@ constexpr int kDl = 512, kDr = 64, kD = kDl + kDr;
 constexpr int kBlocks = kD / 64;  // 64-dim (128-byte) column blocks of a row
 constexpr int kTile = 32;         // selected keys per tile
 constexpr int kHalf = kTile / 2;  // keys per CTA in the S operand
-constexpr int kStages = 3;
-constexpr int kThreads = 192;
+constexpr int kKsStages = 4;      // S-operand ring (freed after S)
+constexpr int kPvStages = 3;      // P V-operand ring (freed after P V)
+constexpr int kThreads = 224;
 constexpr int kMaxK = 2048;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 0;     // 256 columns: two 128-column halves of 256 output dims
@@ -59,17 +65,14 @@ constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleLog2 = 8.0f;
 constexpr int kGathersKs = kBlocks * (kHalf / 4);   // 36
 constexpr int kGathersPv = 4 * (kTile / 4);         // 32
-constexpr uint32_t kStageBytes = (kGathersKs + kGathersPv) * 4 * 128;
+constexpr uint32_t kKsBytes = kGathersKs * 4 * 128;
+constexpr uint32_t kPvBytes = kGathersPv * 4 * 128;
 constexpr uint32_t kQBytes = kBlocks * kHeadsCta * 128;
-
-struct SfaStage {
-    uint8_t ks[kBlocks][kHalf * 128];  // this CTA's 16 keys, full rows, K-major
-    uint8_t pv[4][kTile * 128];        // this CTA's 256 output dims of all 32 keys
-};
 
 struct SfaSmem {
     uint8_t q[kBlocks][kHeadsCta * 128];
-    SfaStage st[kStages];
+    uint8_t ks[kKsStages][kBlocks][kHalf * 128];  // this CTA's 16 keys, full rows, K-major
+    uint8_t pv[kPvStages][4][kTile * 128];        // this CTA's 256 output dims of all 32 keys
     uint8_t p[2][kHeadsCta * 128];     // P (bf16), 32 keys used of each 128-byte row
     int32_t rows[kMaxK];               // compacted physical rows of the selected keys
     float xmax[2][128];
@@ -77,14 +80,16 @@ struct SfaSmem {
     int32_t warp_cnt[4];
     int32_t n_valid;
     uint64_t q_full, peer_q_full, rows_ready;
-    uint64_t full[kStages], peer_full[kStages], empty[kStages];
+    uint64_t ks_full[kKsStages], peer_ks_full[kKsStages], ks_empty[kKsStages];
+    uint64_t pv_full[kPvStages], peer_pv_full[kPvStages], pv_empty[kPvStages];
     uint64_t s_full[2], p_full[2], o_done[2], xch[2], lx;
     uint32_t tmem_base;
     int abort;
 };
 
 static_assert(sizeof(SfaSmem) + 1024 <= 232448, "shared memory budget of one CTA");
-static_assert(kStageBytes == sizeof(SfaStage), "gathers fill the stage exactly");
+static_assert(kKsBytes == sizeof(SfaSmem::ks[0]) && kPvBytes == sizeof(SfaSmem::pv[0]),
+              "gathers fill the stages exactly");
 
 struct SfaArgs {
     PathParams p;
@@ -136,10 +141,15 @@ sfa_mma_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_constant_
         mbar_init(&sm.q_full, 1);
         mbar_init(&sm.peer_q_full, 1);
         mbar_init(&sm.rows_ready, 1);
-        for (int s = 0; s < kStages; ++s) {
-            mbar_init(&sm.full[s], 1);
-            mbar_init(&sm.peer_full[s], 1);
-            mbar_init(&sm.empty[s], 1);
+        for (int s = 0; s < kKsStages; ++s) {
+            mbar_init(&sm.ks_full[s], 1);
+            mbar_init(&sm.peer_ks_full[s], 1);
+            mbar_init(&sm.ks_empty[s], 1);
+        }
+        for (int s = 0; s < kPvStages; ++s) {
+            mbar_init(&sm.pv_full[s], 1);
+            mbar_init(&sm.peer_pv_full[s], 1);
+            mbar_init(&sm.pv_empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sm.s_full[b], 1);
@@ -160,7 +170,7 @@ sfa_mma_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_constant_
     volatile int *abort_flag = &sm.abort;
     int32_t *status = p.status;
 
-    if (warp >= 2) {
+    if (warp >= 2 && warp <= 5) {
         // --------------------------------------------- row compaction ---
         const int et = threadIdx.x - 64, ew = et >> 5;
         const int32_t V = visible_len(p, t);
@@ -343,41 +353,48 @@ sfa_mma_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_constant_
             }
         }
     } else {
-        // both the producer and the MMA warp need this split's tile range
+        // the producers and the MMA warp need this split's tile range
         const bool ready = warp_wait(&sm.rows_ready, 0, abort_flag, status);
         int32_t j0 = 0, j1 = 0;
         if (ready) split_range(sm.n_valid, split, a.splits, j0, j1);
         const int T = j1 - j0;
         if (warp == 0 && T > 0) {
-            // --------------------------------------------- producer ---
+            // ------------------------------------ S-operand producer ---
             if (lane == 0) {
                 mbar_arrive_expect_tx(&sm.q_full, kQBytes);
                 for (int b = 0; b < kBlocks; ++b)
                     tma_load_2d(sm.q[b], &tm_q, 64 * b, t * 128 + kHeadsCta * rank, &sm.q_full);
             }
             for (int n = 0; n < T; ++n) {
-                const int stage = n % kStages;
-                if (!warp_wait(&sm.empty[stage], ((n / kStages) & 1) ^ 1, abort_flag, status,
+                const int st = n % kKsStages;
+                if (!warp_wait(&sm.ks_empty[st], ((n / kKsStages) & 1) ^ 1, abort_flag, status,
                                true))
                     break;
-                if (lane == 0) mbar_arrive_expect_tx(&sm.full[stage], kStageBytes);
+                if (lane == 0) mbar_arrive_expect_tx(&sm.ks_full[st], kKsBytes);
                 __syncwarp();
-                const int kb = (j0 + n) * kTile;
-                SfaStage &st = sm.st[stage];
-                for (int g = lane; g < kGathersKs + kGathersPv; g += 32) {
-                    if (g < kGathersKs) {
-                        const int b = g >> 2, grp = g & 3;
-                        const int32_t *r = &sm.rows[kb + kHalf * rank + 4 * grp];
-                        tma_gather4(st.ks[b] + grp * 512, &tm_kv, 64 * b, r[0], r[1], r[2], r[3],
-                                    &sm.full[stage]);
-                    } else {
-                        const int gp = g - kGathersKs, c = gp >> 3, grp = gp & 7;
-                        const int dvb = (c < 2 ? 0 : 4) + 2 * rank + (c & 1);
-                        const int32_t *r = &sm.rows[kb + 4 * grp];
-                        tma_gather4(st.pv[c] + grp * 512, &tm_kv, 64 * dvb, r[0], r[1], r[2], r[3],
-                                    &sm.full[stage]);
-                    }
+                const int32_t *r0 = &sm.rows[(j0 + n) * kTile + kHalf * rank];
+                for (int g = lane; g < kGathersKs; g += 32) {
+                    const int b = g >> 2, grp = g & 3;
+                    const int32_t *r = r0 + 4 * grp;
+                    tma_gather4(sm.ks[st][b] + grp * 512, &tm_kv, 64 * b, r[0], r[1], r[2], r[3],
+                                &sm.ks_full[st]);
                 }
+            }
+        } else if (warp == 6 && T > 0) {
+            // ---------------------------------- P V-operand producer ---
+            for (int n = 0; n < T; ++n) {
+                const int st = n % kPvStages;
+                if (!warp_wait(&sm.pv_empty[st], ((n / kPvStages) & 1) ^ 1, abort_flag, status,
+                               true))
+                    break;
+                if (lane == 0) mbar_arrive_expect_tx(&sm.pv_full[st], kPvBytes);
+                __syncwarp();
+                const int32_t *r0 = &sm.rows[(j0 + n) * kTile];
+                const int g = lane, c = g >> 3, grp = g & 7;  // 32 gathers, one per lane
+                const int dvb = (c < 2 ? 0 : 4) + 2 * rank + (c & 1);
+                const int32_t *r = r0 + 4 * grp;
+                tma_gather4(sm.pv[st][c] + grp * 512, &tm_kv, 64 * dvb, r[0], r[1], r[2], r[3],
+                            &sm.pv_full[st]);
             }
         } else if (warp == 1 && T > 0 && lane == 0) {
             if (rank == 0) {
@@ -386,54 +403,93 @@ sfa_mma_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_constant_
                 constexpr uint32_t id_pv = instr_desc(128, 256, 1 /*bf16*/, 0, 1);
                 bool ok = mbar_wait(&sm.q_full, 0, abort_flag, status) &&
                           mbar_wait_cluster(&sm.peer_q_full, 0, abort_flag, status);
-                auto issue_s = [&](int n) -> bool {
-                    const int stage = n % kStages;
-                    const uint32_t ph = (n / kStages) & 1;
-                    if (!mbar_wait(&sm.full[stage], ph, abort_flag, status)) return false;
-                    if (!mbar_wait_cluster(&sm.peer_full[stage], ph, abort_flag, status))
-                        return false;
-                    tc_fence_after();
-                    const uint32_t d = tmem + kColS + 16 * (n & 1);
+                int ns = 0, np = 0;  // next S and next P V to issue
+                long long t0 = clock64();
+                uint32_t idle = 0;
+                while (ok && np < T) {
+                    bool progressed = false;
+                    // S(ns) needs its keys in both CTAs and a free S buffer
+                    // (the softmax of tile ns - 2 is done once P V(ns - 2) was issued)
+                    if (ns < T && ns < np + 2) {
+                        const int st = ns % kKsStages;
+                        const uint32_t ph = (ns / kKsStages) & 1;
+                        if (mbar_test(&sm.ks_full[st], ph) &&
+                            mbar_test_cluster(&sm.peer_ks_full[st], ph)) {
+                            tc_fence_after();
+                            const uint32_t d = tmem + kColS + 16 * (ns & 1);
 #pragma unroll 1
-                    for (int b = 0; b < kBlocks; ++b) {
-                        const uint64_t ad = desc_kmajor_sw128(smem_u32(sm.q[b]));
-                        const uint64_t bd = desc_kmajor_sw128(smem_u32(sm.st[stage].ks[b]));
+                            for (int b = 0; b < kBlocks; ++b) {
+                                const uint64_t ad = desc_kmajor_sw128(smem_u32(sm.q[b]));
+                                const uint64_t bd = desc_kmajor_sw128(smem_u32(sm.ks[st][b]));
 #pragma unroll
-                        for (int k = 0; k < 4; ++k)  // 16 bf16 (32 bytes) of K per instruction
-                            mma_bf16_pair(d, ad + 2 * k, bd + 2 * k, id_s, (b | k) != 0);
+                                for (int k = 0; k < 4; ++k)  // 16 bf16 (32 bytes) of K each
+                                    mma_bf16_pair(d, ad + 2 * k, bd + 2 * k, id_s, (b | k) != 0);
+                            }
+                            mma_commit_pair_multicast(&sm.s_full[ns & 1], 0x3);
+                            if (ns + kKsStages < T)
+                                mma_commit_pair_multicast(&sm.ks_empty[st], 0x3);
+                            ++ns;
+                            progressed = true;
+                        }
                     }
-                    mma_commit_pair_multicast(&sm.s_full[n & 1], 0x3);
-                    return true;
-                };
-                if (ok) ok = issue_s(0);
-                for (int n = 0; n < T && ok; ++n) {
-                    if (n + 1 < T && !(ok = issue_s(n + 1))) break;
-                    if (!(ok = mbar_wait_cluster(&sm.p_full[n & 1], (n >> 1) & 1, abort_flag,
-                                                 status)))
+                    // P V(np) needs P from both CTAs and its value rows in both CTAs
+                    if (np < ns) {
+                        const int st = np % kPvStages;
+                        const uint32_t ph = (np / kPvStages) & 1;
+                        if (mbar_test_cluster(&sm.p_full[np & 1], (np >> 1) & 1) &&
+                            mbar_test(&sm.pv_full[st], ph) &&
+                            mbar_test_cluster(&sm.peer_pv_full[st], ph)) {
+                            tc_fence_after();
+                            const uint64_t ad = desc_kmajor_sw128(smem_u32(sm.p[np & 1]));
+#pragma unroll
+                            for (int half = 0; half < 2; ++half) {
+                                const uint32_t va = smem_u32(sm.pv[st][2 * half]);
+#pragma unroll
+                                for (int k = 0; k < 2; ++k)  // 16 keys per instruction
+                                    mma_bf16_pair(tmem + kColO + 128 * half, ad + 2 * k,
+                                                  desc_mnmajor_sw128(va + 2048 * k, kTile * 128,
+                                                                     1024),
+                                                  id_pv, (np > 0 || k > 0) ? 1u : 0u);
+                            }
+                            mma_commit_pair_multicast(&sm.o_done[np & 1], 0x3);
+                            if (np + kPvStages < T)
+                                mma_commit_pair_multicast(&sm.pv_empty[st], 0x3);
+                            ++np;
+                            progressed = true;
+                        }
+                    }
+                    if (progressed) {
+                        t0 = clock64();
+                    } else if ((++idle & 63) == 0 && wait_expired(t0, abort_flag, status)) {
                         break;
-                    tc_fence_after();
-                    const int stage = n % kStages;
-                    const uint64_t ad = desc_kmajor_sw128(smem_u32(sm.p[n & 1]));
-#pragma unroll
-                    for (int half = 0; half < 2; ++half) {
-                        const uint32_t va = smem_u32(sm.st[stage].pv[2 * half]);
-#pragma unroll
-                        for (int k = 0; k < 2; ++k)  // 16 keys per instruction
-                            mma_bf16_pair(tmem + kColO + 128 * half, ad + 2 * k,
-                                          desc_mnmajor_sw128(va + 2048 * k, kTile * 128, 1024),
-                                          id_pv, (n > 0 || k > 0) ? 1u : 0u);
                     }
-                    mma_commit_pair_multicast(&sm.o_done[n & 1], 0x3);
-                    if (n + kStages < T) mma_commit_pair_multicast(&sm.empty[stage], 0x3);
                 }
             } else {
                 // --------------------------------------------- relay ---
                 if (mbar_wait(&sm.q_full, 0, abort_flag, status))
                     mbar_arrive_remote(map_to_rank(smem_u32(&sm.peer_q_full), 0));
-                for (int n = 0; n < T; ++n) {
-                    const int stage = n % kStages;
-                    if (!mbar_wait(&sm.full[stage], (n / kStages) & 1, abort_flag, status)) break;
-                    mbar_arrive_remote(map_to_rank(smem_u32(&sm.peer_full[stage]), 0));
+                int nk = 0, nv = 0;
+                long long t0 = clock64();
+                uint32_t idle = 0;
+                while (nk < T || nv < T) {
+                    bool progressed = false;
+                    if (nk < T && mbar_test(&sm.ks_full[nk % kKsStages], (nk / kKsStages) & 1)) {
+                        mbar_arrive_remote(
+                            map_to_rank(smem_u32(&sm.peer_ks_full[nk % kKsStages]), 0));
+                        ++nk;
+                        progressed = true;
+                    }
+                    if (nv < T && mbar_test(&sm.pv_full[nv % kPvStages], (nv / kPvStages) & 1)) {
+                        mbar_arrive_remote(
+                            map_to_rank(smem_u32(&sm.peer_pv_full[nv % kPvStages]), 0));
+                        ++nv;
+                        progressed = true;
+                    }
+                    if (progressed) {
+                        t0 = clock64();
+                    } else if ((++idle & 63) == 0 && wait_expired(t0, abort_flag, status)) {
+                        break;
+                    }
                 }
             }
         }

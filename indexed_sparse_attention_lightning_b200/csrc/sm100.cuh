@@ -18,12 +18,6 @@ __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-__device__ __forceinline__ uint64_t global_timer_ns() {
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-
 __device__ __forceinline__ int warp_id() { return threadIdx.x >> 5; }
 __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
 
@@ -65,25 +59,47 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Longest a kernel waits on one barrier before it gives up (nanoseconds).
-constexpr uint64_t kWaitLimitNs = 2000000000ull;
+// Non-blocking probe of a phase (no suspension).
+__device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
 
-// Wait for the phase of parity `parity` to complete.  Gives up -- reporting
-// SA_ERR_TIMEOUT and raising the CTA's abort flag -- after kWaitLimitNs, or as
-// soon as another role of the CTA has raised the flag.  Returns false when it
-// gave up.
+// Longest a kernel waits on one barrier before it gives up, in SM clock
+// cycles (about two seconds at the B200's clocks).  The bound is checked
+// every 64 polls with the cheap per-SM cycle counter.
+constexpr long long kWaitLimitCycles = 4000000000ll;
+
+// Gives up -- reporting SA_ERR_TIMEOUT and raising the CTA's abort flag -- when
+// the wait that started at `t0` has lasted too long.  Returns true to stop.
+__device__ __forceinline__ bool wait_expired(long long t0, volatile int *abort_flag,
+                                             int32_t *status) {
+    if (*abort_flag) return true;
+    if (clock64() - t0 > kWaitLimitCycles) {
+        report(status, SA_ERR_TIMEOUT, SA_DETAIL_WAIT_TIMEOUT);
+        *abort_flag = 1;
+        return true;
+    }
+    return false;
+}
+
+// Wait for the phase of parity `parity` to complete.  Gives up after
+// kWaitLimitCycles, or as soon as another role of the CTA has raised the
+// abort flag; returns false when it gave up.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
                                           int32_t *status) {
     if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = global_timer_ns();
-    while (true) {
+    const long long t0 = clock64();
+    for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
-        if (*abort_flag) return false;
-        if (global_timer_ns() - t0 > kWaitLimitNs) {
-            report(status, SA_ERR_TIMEOUT, SA_DETAIL_WAIT_TIMEOUT);
-            *abort_flag = 1;
-            return false;
-        }
+        if ((it & 63) == 0 && wait_expired(t0, abort_flag, status)) return false;
     }
 }
 
@@ -297,16 +313,24 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t pa
 __device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity,
                                                   volatile int *abort_flag, int32_t *status) {
     if (mbar_try_wait_cluster(bar, parity)) return true;
-    const uint64_t t0 = global_timer_ns();
-    while (true) {
+    const long long t0 = clock64();
+    for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait_cluster(bar, parity)) return true;
-        if (*abort_flag) return false;
-        if (global_timer_ns() - t0 > kWaitLimitNs) {
-            report(status, SA_ERR_TIMEOUT, SA_DETAIL_WAIT_TIMEOUT);
-            *abort_flag = 1;
-            return false;
-        }
+        if ((it & 63) == 0 && wait_expired(t0, abort_flag, status)) return false;
     }
+}
+
+// Non-blocking probe with acquire at cluster scope.
+__device__ __forceinline__ bool mbar_test_cluster(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
 }
 
 // Generic-proxy writes to shared memory become visible to the async proxy
