@@ -49,6 +49,11 @@ __device__ __forceinline__ uint32_t order_key(float f) {
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// Radix buckets of the score histogram built by the indexer for top-K: the
+// top kHistBits bits of order_key().
+constexpr int kHistBits = 12;
+constexpr int kHistBins = 1 << kHistBits;
+
 // ReLU that lets a NaN through, so a poisoned slot stays visible.
 __device__ __forceinline__ float relu_keep_nan(float x) { return x < 0.f ? 0.f : x; }
 

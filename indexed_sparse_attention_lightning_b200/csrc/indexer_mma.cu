@@ -20,7 +20,9 @@
 //   warps 2-5  epilogue: each thread owns one key row of the tile, reads its
 //              64 head scores from TMEM (tcgen05.ld), applies ReLU, the head
 //              weights and the staged key scale, and writes one fp32 score;
-//              it touches only shared memory and TMEM besides that store.
+//              for the fused top-K it also counts the score's 12-bit radix
+//              bucket in a shared-memory histogram per query, which is added
+//              to the query's global histogram when the CTA leaves the query.
 // Every wait is bounded; a timeout is reported in the workspace status word.
 #include "common.cuh"
 #include "internal.h"
@@ -43,6 +45,7 @@ constexpr uint32_t kTmemCols = kAcc * kHeads;
 
 struct IndexerSmem {
     uint8_t keys[kStages][kTileBytes];  // 1024-byte aligned (128-byte swizzle atoms)
+    uint32_t hist[kHistBins];           // score-key histogram of the current query
     uint8_t q[2][kQBytes];
     float kscale[kStages][kKeys];       // per-token key scales of the staged pages
     int32_t page_ok[kStages][2];        // 1 when the staged page id was valid
@@ -60,6 +63,7 @@ struct IndexerArgs {
     const int32_t *tile_end;  // [n_q] inclusive prefix of ceil(vis / 128)
     float *scores;
     int64_t ld;
+    uint32_t *hist;           // [n_q, kHistBins] (zeroed by the caller) or null
 };
 
 // Walks this CTA's contiguous share [k, k_end) of the global tile list.
@@ -232,15 +236,39 @@ indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
         }
     } else {
         // --------------------------------------------------- epilogue ---
+        // The loop never leaves early: after a failed (timed-out) wait it
+        // carries on without waiting, so the four warps meet at the same
+        // named barriers when they flush the histogram.
         const int quad = warp & 3;             // TMEM lanes this warp may read
         const int row = quad * 32 + lane;      // key row of the tile
+        const int et = threadIdx.x - 64;       // 0..127 over the epilogue warps
+        const bool histo = a.hist != nullptr;
+        if (histo) {
+            for (int b = et; b < kHistBins; b += 128) sm.hist[b] = 0;
+            named_barrier(1, 128);
+        }
+        // add this CTA's counts of query t to the global histogram, then clear
+        auto flush = [&](int32_t t) {
+            named_barrier(1, 128);
+            uint32_t *g = a.hist + (int64_t)t * kHistBins;
+            for (int b = et; b < kHistBins; b += 128) {
+                const uint32_t v = sm.hist[b];
+                if (v != 0) {
+                    atomicAdd(g + b, v);
+                    sm.hist[b] = 0;
+                }
+            }
+            named_barrier(1, 128);
+        };
         TileCursor c;
         c.init(a.tile_end, p.n_q, k0, k1);
-        bool seg_start = true;
-        int32_t V = 0;
+        bool seg_start = true, ok = true;
+        int32_t V = 0, t_cur = -1;
         float wq[kHeads];
         for (int n = 0; c.valid(); ++n) {
             if (seg_start) {
+                if (histo && t_cur >= 0) flush(t_cur);
+                t_cur = c.t;
                 V = a.vis[c.t];
                 const float *w = p.w + (int64_t)c.t * kHeads;
                 const float *qs = p.q_index_scale + (int64_t)c.t * kHeads;
@@ -250,32 +278,40 @@ indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
             const int64_t s = (int64_t)c.i * kKeys + row;
             const int stage = n % kStages;
             // key scales and page validity arrive with the key pages
-            if (!warp_wait(&sm.full[stage], (n / kStages) & 1, abort_flag, p.status)) break;
-            const bool ok = sm.page_ok[stage][row >> 6] != 0;
-            const float kscale = sm.kscale[stage][row];
+            if (ok) ok = warp_wait(&sm.full[stage], (n / kStages) & 1, abort_flag, p.status);
+            const bool page_ok = ok && sm.page_ok[stage][row >> 6] != 0;
+            const float kscale = ok ? sm.kscale[stage][row] : 0.f;
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.sc_empty[stage]);
-            if (s < V && !ok) report(p.status, SA_ERR_DEVICE_FAULT, SA_DETAIL_BAD_PAGE);
+            if (ok && s < V && !page_ok) report(p.status, SA_ERR_DEVICE_FAULT, SA_DETAIL_BAD_PAGE);
             const int acc = n % kAcc;
-            if (!warp_wait(&sm.acc_full[acc], (n / kAcc) & 1, abort_flag, p.status)) break;
-            tc_fence_after();
-            const uint32_t taddr = tmem + (static_cast<uint32_t>(quad * 32) << 16) + acc * kHeads;
-            float v[32];
+            if (ok) ok = warp_wait(&sm.acc_full[acc], (n / kAcc) & 1, abort_flag, p.status);
             float sum = 0.f;
-            tmem_ld32(taddr, v);
-            tmem_wait_ld();
+            if (ok) {
+                tc_fence_after();
+                const uint32_t taddr =
+                    tmem + (static_cast<uint32_t>(quad * 32) << 16) + acc * kHeads;
+                float v[32];
+                tmem_ld32(taddr, v);
+                tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 32; ++j) sum = fmaf(wq[j], relu_keep_nan(v[j]), sum);
-            tmem_ld32(taddr + 32, v);
-            tmem_wait_ld();
+                for (int j = 0; j < 32; ++j) sum = fmaf(wq[j], relu_keep_nan(v[j]), sum);
+                tmem_ld32(taddr + 32, v);
+                tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 32; ++j) sum = fmaf(wq[32 + j], relu_keep_nan(v[j]), sum);
+                for (int j = 0; j < 32; ++j) sum = fmaf(wq[32 + j], relu_keep_nan(v[j]), sum);
+            }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.acc_empty[acc]);
-            if (s < V) a.scores[(int64_t)c.t * a.ld + s] = ok ? sum * kscale : -INFINITY;
+            if (s < V) {
+                const float score = page_ok ? sum * kscale : -INFINITY;
+                a.scores[(int64_t)c.t * a.ld + s] = score;
+                if (histo) atomicAdd(&sm.hist[order_key(score) >> (32 - kHistBits)], 1u);
+            }
             seg_start = c.next(a.tile_end);
         }
+        if (histo && t_cur >= 0) flush(t_cur);
     }
     __syncwarp();
     tc_fence_before();
@@ -293,14 +329,14 @@ bool indexer_mma_supported(const PathParams &p) {
 }
 
 cudaError_t launch_indexer_mma(const PathParams &p, const int32_t *vis, const int32_t *tile_end,
-                               float *scores, int64_t ld, cudaStream_t s) {
+                               float *scores, int64_t ld, uint32_t *hist, cudaStream_t s) {
     if (p.n_q == 0) return cudaSuccess;
     CUtensorMap tk, tq;
     if (!encode_tmap_2d(&tk, 1, p.k_index, kDim, (uint64_t)p.num_pages * 64, kDim, kDim, 64, true) ||
         !encode_tmap_2d(&tq, 1, p.q_index, kDim, (uint64_t)p.n_q * kHeads, kDim, kDim, kHeads,
                         true))
         return cudaErrorInvalidValue;
-    IndexerArgs a{p, vis, tile_end, scores, ld};
+    IndexerArgs a{p, vis, tile_end, scores, ld, hist};
     const int64_t max_tiles = (int64_t)p.n_q * ceil_div(p.max_visible, kKeys);
     const int64_t grid = std::min<int64_t>(2 * num_sms(), max_tiles);
     const size_t smem = sizeof(IndexerSmem) + 1024;

@@ -62,22 +62,32 @@ bool encode_tmap_2d(CUtensorMap *map, int dtype_bytes, const void *base, uint64_
                     uint32_t box_outer, bool swizzle128);
 
 // ---- launchers (each returns the launch error, if any) --------------------
-// Visible length per query and the inclusive prefix of ceil(V / tile).
+// Visible length per query and the inclusive prefix of ceil(V / tile); also
+// zeroes `zero_words` 32-bit words at `zero` (histograms and counters).
 cudaError_t launch_plan(const PathParams &p, int32_t *vis, int32_t *tile_end, int32_t tile,
-                        cudaStream_t s);
+                        uint32_t *zero, size_t zero_words, cudaStream_t s);
 
 cudaError_t launch_indexer_simt(const PathParams &p, float *scores, int64_t ld, cudaStream_t s);
 
 // Tensor-core FP8 indexer (e4m3 keys, 64 heads x 128 dims); needs the plan.
 bool indexer_mma_supported(const PathParams &p);
 cudaError_t launch_indexer_mma(const PathParams &p, const int32_t *vis, const int32_t *tile_end,
-                               float *scores, int64_t ld, cudaStream_t s);
+                               float *scores, int64_t ld, uint32_t *hist, cudaStream_t s);
 
 // Row-wise exact top-K.  Row t has valid_len[t] entries, or q_pos[t] + 1 when
 // valid_len is null (rows then validated as queries of `p`).
 cudaError_t launch_topk_rowwise(const float *scores, int64_t ld, const int32_t *valid_len,
                                 int32_t max_valid, const PathParams *p, int32_t n_q,
                                 int32_t top_k, int32_t *idx, int32_t *status, cudaStream_t s);
+
+// Histogram-guided exact top-K for rows scored by the tensor-core indexer
+// (which filled `hist`, [n_q, kHistBins]).  Scratch: sel [n_q, top_k],
+// counts [n_q, 2] (zeroed), cand [n_q, cap].
+constexpr int32_t kTopkCandCap = 8192;
+cudaError_t launch_topk_hist(const float *scores, int64_t ld, const int32_t *vis,
+                             const uint32_t *hist, int32_t n_q, int32_t max_valid, int32_t top_k,
+                             int32_t *sel, int32_t *counts, uint64_t *cand, int32_t cap,
+                             int32_t *idx, cudaStream_t s);
 
 cudaError_t launch_attn_simt(const PathParams &p, const int32_t *idx, int32_t top_k, void *out,
                              int32_t out_dtype, float *lse, cudaStream_t s);

@@ -1,6 +1,7 @@
 // plan.cu -- per-call schedule: validated visible length of every query and
 // the inclusive prefix of its 128-key tile count, which the persistent
-// kernels use to split the concatenated tiles of all queries evenly.
+// kernels use to split the concatenated tiles of all queries evenly.  The
+// same launch clears the per-call histograms and counters.
 #include "common.cuh"
 #include "internal.h"
 
@@ -10,7 +11,12 @@ namespace {
 constexpr int kThreads = 1024;
 
 __global__ void __launch_bounds__(kThreads)
-plan_kernel(const PathParams p, int32_t *vis, int32_t *tile_end, int32_t tile) {
+plan_kernel(const PathParams p, int32_t *vis, int32_t *tile_end, int32_t tile, uint32_t *zero,
+            size_t zero_words) {
+    for (size_t i = (size_t)blockIdx.x * kThreads + threadIdx.x; i < zero_words;
+         i += (size_t)gridDim.x * kThreads)
+        zero[i] = 0u;
+    if (blockIdx.x != 0) return;
     __shared__ int32_t warp_sums[32];
     __shared__ int32_t carry;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -52,10 +58,13 @@ plan_kernel(const PathParams p, int32_t *vis, int32_t *tile_end, int32_t tile) {
 }  // namespace
 
 cudaError_t launch_plan(const PathParams &p, int32_t *vis, int32_t *tile_end, int32_t tile,
-                        cudaStream_t s) {
+                        uint32_t *zero, size_t zero_words, cudaStream_t s) {
     if (p.n_q == 0) return cudaSuccess;
+    const int64_t blocks =
+        std::max<int64_t>(1, std::min<int64_t>(num_sms(), ceil_div(zero_words, 4 * kThreads)));
     count_launch();
-    plan_kernel<<<1, kThreads, 0, s>>>(p, vis, tile_end, tile);
+    plan_kernel<<<static_cast<unsigned>(blocks), kThreads, 0, s>>>(p, vis, tile_end, tile, zero,
+                                                                  zero_words);
     return cudaGetLastError();
 }
 

@@ -106,13 +106,15 @@ PathParams make_params(const sa_cache *c, const sa_query *q, void *ws) {
 }
 
 // Workspace: status | vis [n_q] | tile_end [n_q] | scores [n_q, ld] | idx [n_q, K]
+// | hist [n_q, 4096] | counts [n_q, 2] | sel [n_q, K] | cand [n_q, cap]
 // | o_part [n_q, S, 128, 512] | lse_part [n_q, S, 128]; the indexer needs the
 // first three, the fused path all of them; the attention alone needs the
 // status and the split-KV partials (placed right after the status).
 struct Layout {
     int64_t ld;
     int32_t splits;
-    size_t vis, tile_end, scores, idx, o_part, lse_part, indexer_total, decode_total;
+    size_t vis, tile_end, scores, idx, hist, counts, sel, cand, o_part, lse_part;
+    size_t indexer_total, decode_total;
     size_t attn_o_part, attn_lse_part, attn_total;
 };
 
@@ -131,8 +133,13 @@ Layout make_layout(const sa_query *q, int32_t top_k) {
     l.tile_end = align_up(l.vis + sizeof(int32_t) * nq);
     l.indexer_total = align_up(l.tile_end + sizeof(int32_t) * nq);
     l.scores = l.indexer_total;
+    const size_t kk = top_k > 0 ? (size_t)top_k : 0;
     l.idx = align_up(l.scores + sizeof(float) * nq * (size_t)l.ld);
-    l.o_part = align_up(l.idx + sizeof(int32_t) * nq * (size_t)(top_k > 0 ? top_k : 0));
+    l.hist = align_up(l.idx + sizeof(int32_t) * nq * kk);
+    l.counts = align_up(l.hist + sizeof(uint32_t) * nq * kHistBins);  // follows hist: one clear
+    l.sel = align_up(l.counts + sizeof(int32_t) * 2 * nq);
+    l.cand = align_up(l.sel + sizeof(int32_t) * nq * kk);
+    l.o_part = align_up(l.cand + sizeof(uint64_t) * nq * kTopkCandCap);
     l.lse_part = align_up(l.o_part + o_bytes);
     l.decode_total = align_up(l.lse_part + lse_bytes);
     l.attn_o_part = align_up(kStatusBytes);
@@ -155,16 +162,24 @@ sa_status run_attention(const PathParams &p, const Layout &l, size_t o_off, size
 }
 
 // Indexer scores into `scores` (ld): the tensor-core kernel for its shape,
-// the CUDA-core kernel otherwise.
+// the CUDA-core kernel otherwise.  With `want_hist` (fused path) the
+// tensor-core kernel also fills the per-query score histograms, which the
+// plan kernel clears first together with the counters behind them;
+// *have_hist reports whether they were built.
 sa_status run_indexer(const PathParams &p, const Layout &l, void *ws, float *scores, int64_t ld,
-                      cudaStream_t s) {
+                      bool want_hist, bool *have_hist, cudaStream_t s) {
+    *have_hist = false;
     if (indexer_mma_supported(p)) {
         char *base = static_cast<char *>(ws);
         int32_t *vis = reinterpret_cast<int32_t *>(base + l.vis);
         int32_t *tile_end = reinterpret_cast<int32_t *>(base + l.tile_end);
-        sa_status st = cuda_status(launch_plan(p, vis, tile_end, 128, s));
+        uint32_t *hist = want_hist ? reinterpret_cast<uint32_t *>(base + l.hist) : nullptr;
+        const size_t zero_words = want_hist ? (l.sel - l.hist) / 4 : 0;
+        sa_status st = cuda_status(launch_plan(p, vis, tile_end, 128, hist, zero_words, s));
         if (st != SA_OK) return st;
-        return cuda_status(launch_indexer_mma(p, vis, tile_end, scores, ld, s));
+        st = cuda_status(launch_indexer_mma(p, vis, tile_end, scores, ld, hist, s));
+        *have_hist = want_hist && st == SA_OK;
+        return st;
     }
     return cuda_status(launch_indexer_simt(p, scores, ld, s));
 }
@@ -212,7 +227,8 @@ sa_status sa_indexer_score(const sa_cache *cache, const sa_query *query, float *
     if ((st = clear_status(workspace, s)) != SA_OK) return st;
     if (query->n_q == 0) return SA_OK;
     PathParams p = make_params(cache, query, workspace);
-    return run_indexer(p, l, workspace, scores, ld_scores, s);
+    bool have_hist;
+    return run_indexer(p, l, workspace, scores, ld_scores, false, &have_hist, s);
 }
 
 sa_status sa_topk(const float *scores, int64_t ld_scores, const int32_t *valid_len, int32_t n_q,
@@ -273,11 +289,22 @@ static sa_status decode_impl(const sa_cache *cache, const sa_query *query, int32
         char *base = static_cast<char *>(workspace);
         float *scores = reinterpret_cast<float *>(base + l.scores);
         int32_t *idx = idx_out ? idx_out : reinterpret_cast<int32_t *>(base + l.idx);
-        if ((st = run_indexer(p, l, workspace, scores, l.ld, s)) != SA_OK) return st;
-        if ((st = mark(1)) != SA_OK) return st;
-        if ((st = cuda_status(launch_topk_rowwise(scores, l.ld, nullptr, query->max_visible, &p,
-                                                  query->n_q, top_k, idx, p.status, s))) != SA_OK)
+        bool have_hist = false;
+        if ((st = run_indexer(p, l, workspace, scores, l.ld, true, &have_hist, s)) != SA_OK)
             return st;
+        if ((st = mark(1)) != SA_OK) return st;
+        if (have_hist) {
+            st = cuda_status(launch_topk_hist(
+                scores, l.ld, reinterpret_cast<const int32_t *>(base + l.vis),
+                reinterpret_cast<const uint32_t *>(base + l.hist), query->n_q, query->max_visible,
+                top_k, reinterpret_cast<int32_t *>(base + l.sel),
+                reinterpret_cast<int32_t *>(base + l.counts),
+                reinterpret_cast<uint64_t *>(base + l.cand), kTopkCandCap, idx, s));
+        } else {
+            st = cuda_status(launch_topk_rowwise(scores, l.ld, nullptr, query->max_visible, &p,
+                                                 query->n_q, top_k, idx, p.status, s));
+        }
+        if (st != SA_OK) return st;
         if ((st = mark(2)) != SA_OK) return st;
         if ((st = run_attention(p, l, l.o_part, l.lse_part, workspace, idx, top_k, out,
                                 out_dtype, lse, s)) != SA_OK)

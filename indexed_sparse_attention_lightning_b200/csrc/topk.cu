@@ -17,6 +17,7 @@ namespace sa {
 namespace {
 
 constexpr int kThreads = 1024;
+constexpr size_t kTopkSmemLimit = 200 * 1024;  // dynamic shared memory of the finalize CTA
 
 // Exclusive prefix of `flag` over the block in thread order; returns the
 // block total through *total.  Uses warp ballots plus one scan of the warp
@@ -45,33 +46,49 @@ __device__ __forceinline__ int block_exclusive_count(bool flag, int *warp_sums, 
     return r;
 }
 
-__global__ void __launch_bounds__(kThreads)
-topk_rowwise_kernel(const float *__restrict__ scores, int64_t ld,
-                    const int32_t *__restrict__ valid_len, int32_t max_valid, const PathParams p,
-                    int32_t top_k, int32_t *__restrict__ idx, int32_t *status) {
+// Exclusive prefix sum of `v` over the block in thread order (total through
+// *total).  All threads must call it.
+__device__ __forceinline__ int block_exclusive_prefix(int v, int *warp_sums, int *total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        int n = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += n;
+    }
+    if (lane == 31) warp_sums[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        const int nw = blockDim.x >> 5;
+        int w = lane < nw ? warp_sums[lane] : 0;
+        int wi = w;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            int n = __shfl_up_sync(0xffffffffu, wi, o);
+            if (lane >= o) wi += n;
+        }
+        warp_sums[lane] = wi - w;
+        if (lane == 31) warp_sums[32] = wi;
+    }
+    __syncthreads();
+    const int r = warp_sums[warp] + incl - v;
+    *total = warp_sums[32];
+    __syncthreads();
+    return r;
+}
+
+// Exact top-K of one row by four 8-bit radix passes, written in ascending
+// position order.  All kThreads threads of the block call it.
+__device__ void select_row(const float *__restrict__ row, int32_t V, int32_t top_k,
+                           int32_t *__restrict__ out) {
     __shared__ unsigned hist[256];
     __shared__ int warp_sums[33];
     __shared__ unsigned sel_digit, sel_above;
-
-    const int t = blockIdx.x;
-    int32_t V;
-    if (valid_len != nullptr) {
-        V = valid_len[t];
-        if (V < 0 || V > max_valid) {
-            if (threadIdx.x == 0) report(status, SA_ERR_DEVICE_FAULT, SA_DETAIL_BAD_POSITION);
-            V = 0;
-        }
-    } else {
-        V = visible_len(p, t);
-    }
-    const float *row = scores + (int64_t)t * ld;
-    int32_t *out = idx + (int64_t)t * top_k;
 
     if (V <= top_k) {
         for (int i = threadIdx.x; i < top_k; i += kThreads) out[i] = i < V ? i : -1;
         return;
     }
-
     uint32_t prefix = 0, mask = 0;
     unsigned remaining = top_k;  // how many still to take at or below the prefix
     const int lane = threadIdx.x & 31;
@@ -83,7 +100,7 @@ topk_rowwise_kernel(const float *__restrict__ scores, int64_t ld,
             const int64_t i = base + threadIdx.x;
             uint32_t key = i < V ? order_key(row[i]) : 0u;
             bool match = i < V && (key & mask) == prefix;
-            unsigned digit = match ? (key >> shift) & 255u : 256u + 0u;
+            unsigned digit = match ? (key >> shift) & 255u : 256u;
             unsigned same = __match_any_sync(0xffffffffu, digit);
             if (match && lane == __ffs(same) - 1) atomicAdd(&hist[digit], __popc(same));
         }
@@ -140,7 +157,293 @@ topk_rowwise_kernel(const float *__restrict__ scores, int64_t ld,
     }
 }
 
+__global__ void __launch_bounds__(kThreads)
+topk_rowwise_kernel(const float *__restrict__ scores, int64_t ld,
+                    const int32_t *__restrict__ valid_len, int32_t max_valid, const PathParams p,
+                    int32_t top_k, int32_t *__restrict__ idx, int32_t *status) {
+    const int t = blockIdx.x;
+    int32_t V;
+    if (valid_len != nullptr) {
+        V = valid_len[t];
+        if (V < 0 || V > max_valid) {
+            if (threadIdx.x == 0) report(status, SA_ERR_DEVICE_FAULT, SA_DETAIL_BAD_POSITION);
+            V = 0;
+        }
+    } else {
+        V = visible_len(p, t);
+    }
+    select_row(scores + (int64_t)t * ld, V, top_k, idx + (int64_t)t * top_k);
+}
+
+// ---------------------------------------------------------------------------
+// Histogram-guided top-K for the fused path.  The indexer has counted every
+// query's score keys in kHistBins radix buckets (the top kHistBits bits of
+// the order-preserving key).  The bucket b* where the count from the top
+// reaches K splits the row: keys above it are selected outright, keys inside
+// it are candidates whose exact order is settled later, keys below are out.
+// ---------------------------------------------------------------------------
+constexpr int kCollectThreads = 256;
+
+// Bucket b* and the number of keys in buckets above it, for a histogram of
+// kHistBins bins with at least K keys.  All threads of the block call it.
+__device__ void threshold_bucket(const uint32_t *__restrict__ h, int32_t K, int *b_out,
+                                 uint32_t *above_out) {
+    constexpr int kPer = kHistBins / kCollectThreads;  // 16 bins per thread
+    __shared__ uint32_t part[kCollectThreads];
+    __shared__ int sb;
+    __shared__ uint32_t sa;
+    const int tid = threadIdx.x;
+    uint32_t c[kPer], mine = 0;
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+        c[j] = h[tid * kPer + j];
+        mine += c[j];
+    }
+    part[tid] = mine;
+    if (tid == 0) {
+        sb = 0;   // only used when the histogram holds fewer than K keys; the
+        sa = 0;   // finalize step then falls back to the row-wise select
+    }
+    __syncthreads();
+    if (tid < 32) {
+        // suffix sums over the 256 thread partials, 8 per lane
+        uint32_t v[8], s8 = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            v[j] = part[tid * 8 + j];
+            s8 += v[j];
+        }
+        uint32_t suffix = s8;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            uint32_t n = __shfl_down_sync(0xffffffffu, suffix, o);
+            if (tid + o < 32) suffix += n;
+        }
+        uint32_t acc = suffix - s8;  // partials of threads > 8 * tid + 7
+#pragma unroll
+        for (int j = 7; j >= 0; --j) {
+            const uint32_t hi = acc;  // partials strictly above thread 8*tid+j
+            acc += v[j];
+            part[tid * 8 + j] = hi;   // counts in buckets above this thread's range
+        }
+    }
+    __syncthreads();
+    uint32_t acc = part[tid];
+    if (acc < (uint32_t)K && acc + mine >= (uint32_t)K) {
+#pragma unroll
+        for (int j = kPer - 1; j >= 0; --j) {
+            if (acc + c[j] >= (uint32_t)K) {
+                sb = tid * kPer + j;
+                sa = acc;
+                break;
+            }
+            acc += c[j];
+        }
+    }
+    __syncthreads();
+    *b_out = sb;
+    *above_out = sa;
+}
+
+__global__ void __launch_bounds__(kCollectThreads)
+topk_collect_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *__restrict__ vis,
+                    const uint32_t *__restrict__ hist, int32_t top_k, int32_t chunk,
+                    int32_t *__restrict__ sel, int32_t *__restrict__ counts,
+                    uint64_t *__restrict__ cand, int32_t cap) {
+    __shared__ int32_t cnt_s[2], base_s[2];
+    const int t = blockIdx.y;
+    const int32_t V = vis[t];
+    const int64_t c0 = (int64_t)blockIdx.x * chunk;
+    if (V <= top_k || c0 >= V) return;
+    const int64_t c1 = min((int64_t)V, c0 + chunk);
+    int bstar;
+    uint32_t above;
+    threshold_bucket(hist + (int64_t)t * kHistBins, top_k, &bstar, &above);
+    const float *row = scores + (int64_t)t * ld;
+    const int lane = threadIdx.x & 31;
+    const unsigned lt = (1u << lane) - 1u;
+    // pass 1: this chunk's counts, then one global reservation per list
+    if (threadIdx.x < 2) cnt_s[threadIdx.x] = 0;
+    __syncthreads();
+    int32_t nh = 0, ne = 0;
+    for (int64_t i = c0 + threadIdx.x; i < c1; i += kCollectThreads) {
+        const int b = static_cast<int>(order_key(row[i]) >> (32 - kHistBits));
+        nh += b > bstar;
+        ne += b == bstar;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        nh += __shfl_xor_sync(0xffffffffu, nh, o);
+        ne += __shfl_xor_sync(0xffffffffu, ne, o);
+    }
+    if (lane == 0) {
+        atomicAdd(&cnt_s[0], nh);
+        atomicAdd(&cnt_s[1], ne);
+    }
+    __syncthreads();
+    if (threadIdx.x < 2) {
+        base_s[threadIdx.x] = cnt_s[threadIdx.x] > 0
+                                  ? atomicAdd(&counts[2 * t + threadIdx.x], cnt_s[threadIdx.x])
+                                  : 0;
+        cnt_s[threadIdx.x] = 0;
+    }
+    __syncthreads();
+    // pass 2: write into the reserved ranges (slots from shared-memory counters)
+    int32_t *sel_t = sel + (int64_t)t * top_k;
+    uint64_t *cand_t = cand + (int64_t)t * cap;
+    for (int64_t base = c0; base < c1; base += kCollectThreads) {
+        const int64_t i = base + threadIdx.x;
+        const uint32_t key = i < c1 ? order_key(row[i]) : 0u;
+        const int b = static_cast<int>(key >> (32 - kHistBits));
+        const bool hi = i < c1 && b > bstar, eq = i < c1 && b == bstar;
+        const unsigned bh = __ballot_sync(0xffffffffu, hi), be = __ballot_sync(0xffffffffu, eq);
+        int32_t oh = 0, oe = 0;
+        if (lane == 0) {
+            if (bh) oh = atomicAdd(&cnt_s[0], __popc(bh));
+            if (be) oe = atomicAdd(&cnt_s[1], __popc(be));
+        }
+        oh = base_s[0] + __shfl_sync(0xffffffffu, oh, 0) + __popc(bh & lt);
+        oe = base_s[1] + __shfl_sync(0xffffffffu, oe, 0) + __popc(be & lt);
+        if (hi && oh < top_k) sel_t[oh] = static_cast<int32_t>(i);
+        if (eq && oe < cap)
+            cand_t[oe] = (static_cast<uint64_t>(key) << 32) | (0xFFFFFFFFu - static_cast<uint32_t>(i));
+    }
+}
+
+// One CTA per query: exact order inside the threshold bucket, then every
+// selected position set in a bitmap and read back in ascending order.  Rows
+// the candidate buffer or the bitmap cannot hold (massive exact ties, very
+// long rows) take the row-wise radix select instead.
+__global__ void __launch_bounds__(kThreads)
+topk_finalize_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *__restrict__ vis,
+                     int32_t top_k, const int32_t *__restrict__ sel,
+                     const int32_t *__restrict__ counts, const uint64_t *__restrict__ cand,
+                     int32_t cap, int32_t bitmap_words, int32_t *__restrict__ idx) {
+    extern __shared__ uint64_t fin_smem[];
+    __shared__ unsigned hist[256];
+    __shared__ int warp_sums[33];
+    __shared__ unsigned sel_digit, sel_above;
+    const int t = blockIdx.x;
+    const int32_t V = vis[t];
+    int32_t *out = idx + (int64_t)t * top_k;
+    const int32_t n_sel = counts[2 * t], n_cand = counts[2 * t + 1];
+    const int32_t need = top_k - n_sel;
+    const bool fits = V > top_k && n_cand <= cap && V <= bitmap_words * 32 && need > 0 &&
+                      need <= n_cand;
+    if (!fits) {
+        select_row(scores + (int64_t)t * ld, V, top_k, out);
+        return;
+    }
+    uint64_t *cs = fin_smem;                                       // [cap]
+    uint32_t *bits = reinterpret_cast<uint32_t *>(fin_smem + cap);  // [bitmap_words]
+    const uint64_t *cg = cand + (int64_t)t * cap;
+    for (int i = threadIdx.x; i < n_cand; i += kThreads) cs[i] = cg[i];
+    const int words = (V + 31) / 32;
+    for (int w = threadIdx.x; w < words; w += kThreads) bits[w] = 0;
+    __syncthreads();
+    // the need-th largest 64-bit candidate key (all distinct: the low word
+    // holds the inverted position), by 8-bit radix passes from the top
+    uint64_t prefix = 0, mask = 0;
+    unsigned remaining = need;
+    const int lane = threadIdx.x & 31;
+    for (int pass = 0; pass < 8; ++pass) {
+        const int shift = 56 - 8 * pass;
+        for (int i = threadIdx.x; i < 256; i += kThreads) hist[i] = 0;
+        __syncthreads();
+        for (int i = threadIdx.x; i < n_cand; i += kThreads) {
+            const uint64_t k = cs[i];
+            if ((k & mask) == prefix) atomicAdd(&hist[(k >> shift) & 255u], 1u);
+        }
+        __syncthreads();
+        if (threadIdx.x < 32) {
+            unsigned c[8], lane_sum = 0;
+#pragma unroll
+            for (int b = 0; b < 8; ++b) {
+                c[b] = hist[8 * lane + b];
+                lane_sum += c[b];
+            }
+            unsigned suffix = lane_sum;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                unsigned n = __shfl_down_sync(0xffffffffu, suffix, o);
+                if (lane + o < 32) suffix += n;
+            }
+            const unsigned above_lane = suffix - lane_sum;
+            if (above_lane < remaining && remaining <= suffix) {
+                unsigned acc = above_lane;
+                for (int b = 7; b >= 0; --b) {
+                    if (acc + c[b] >= remaining) {
+                        sel_digit = 8 * lane + b;
+                        sel_above = acc;
+                        break;
+                    }
+                    acc += c[b];
+                }
+            }
+        }
+        __syncthreads();
+        prefix |= static_cast<uint64_t>(sel_digit) << shift;
+        mask |= static_cast<uint64_t>(255u) << shift;
+        remaining -= sel_above;
+        __syncthreads();
+    }
+    // keys are distinct, so exactly `need` candidates are >= prefix
+    for (int i = threadIdx.x; i < n_cand; i += kThreads)
+        if (cs[i] >= prefix) {
+            const uint32_t pos = 0xFFFFFFFFu - static_cast<uint32_t>(cs[i]);
+            atomicOr(&bits[pos >> 5], 1u << (pos & 31));
+        }
+    const int32_t *st = sel + (int64_t)t * top_k;
+    for (int i = threadIdx.x; i < n_sel; i += kThreads) {
+        const uint32_t pos = static_cast<uint32_t>(st[i]);
+        atomicOr(&bits[pos >> 5], 1u << (pos & 31));
+    }
+    __syncthreads();
+    // ascending order: each thread owns a contiguous run of words
+    const int per = (words + kThreads - 1) / kThreads;
+    const int w0 = min(words, threadIdx.x * per), w1 = min(words, w0 + per);
+    int cnt = 0;
+    for (int w = w0; w < w1; ++w) cnt += __popc(bits[w]);
+    int total;
+    int pos = block_exclusive_prefix(cnt, warp_sums, &total);
+    for (int w = w0; w < w1; ++w) {
+        uint32_t b = bits[w];
+        while (b) {
+            const int j = __ffs(b) - 1;
+            b &= b - 1;
+            if (pos < top_k) out[pos] = w * 32 + j;
+            ++pos;
+        }
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_topk_hist(const float *scores, int64_t ld, const int32_t *vis,
+                             const uint32_t *hist, int32_t n_q, int32_t max_valid, int32_t top_k,
+                             int32_t *sel, int32_t *counts, uint64_t *cand, int32_t cap,
+                             int32_t *idx, cudaStream_t s) {
+    if (n_q == 0) return cudaSuccess;
+    constexpr int32_t kChunk = 8192;
+    const dim3 grid_c(static_cast<unsigned>(ceil_div(std::max(max_valid, 1), kChunk)), n_q);
+    count_launch();
+    topk_collect_kernel<<<grid_c, kCollectThreads, 0, s>>>(scores, ld, vis, hist, top_k, kChunk,
+                                                           sel, counts, cand, cap);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    // candidates plus a bitmap of the longest row, within one CTA's shared memory
+    const int32_t words = static_cast<int32_t>(ceil_div(std::max(max_valid, 1), 32));
+    const int32_t max_words = static_cast<int32_t>((kTopkSmemLimit - (size_t)cap * 8) / 4);
+    const int32_t bw = std::min(words, max_words);
+    const size_t smem = (size_t)cap * 8 + (size_t)bw * 4;
+    e = cudaFuncSetAttribute(topk_finalize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+    if (e != cudaSuccess) return e;
+    count_launch();
+    topk_finalize_kernel<<<n_q, kThreads, smem, s>>>(scores, ld, vis, top_k, sel, counts, cand,
+                                                      cap, bw, idx);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_topk_rowwise(const float *scores, int64_t ld, const int32_t *valid_len,
                                 int32_t max_valid, const PathParams *p, int32_t n_q,

@@ -223,3 +223,30 @@ def test_attention_on_unsorted_indices_with_holes():
     ref_out, ref_lse = oracle.sparse_attn(wl, idx)
     parity.check_attention(out.float().cpu().numpy(), ref_out, "bf16")
     parity.check_lse(lse.cpu().numpy(), ref_lse)
+
+
+@pytest.mark.parametrize("pattern", ["all_zero", "three_values"])
+def test_fused_topk_on_massive_ties(pattern):
+    """All-equal or few-valued scores: the fused top-K must still pick the
+    lowest positions among ties (exercising its exact tie-bucket select and
+    its fall-back to the row-wise select when the tie bucket overflows)."""
+    sp = W.WorkloadSpec(name=f"ties_{pattern}", seed=23, batch=4,
+                        seq_len=("list", (3000, 7000, 9000, 30000)))
+    wl = W.make_workload(sp)
+    k = wl.k_index.copy()
+    valid = np.isfinite(wl.k_index_scale)                  # written (non-poisoned) slots
+    if pattern == "all_zero":
+        k[valid] = 0                                       # e4m3 code 0: every score is 0
+    else:
+        rng = np.random.default_rng(5)
+        protos = rng.integers(0, 0x7E, size=(3, sp.d_index), dtype=np.uint8)
+        pick = rng.integers(0, 3, size=valid.sum())
+        k[valid] = protos[pick]
+    scale = np.where(valid, np.float32(0.01), wl.k_index_scale).astype(np.float32)
+    wl = dataclasses.replace(wl, k_index=k, k_index_scale=scale)
+    res = run_fused(wl)
+    assert res["status"] == (_abi.SA_OK, 0)
+    scores = oracle.index_scores(wl)
+    ref = oracle.topk(scores, wl.visible, sp.top_k)
+    # with exact ties the only correct answer is the oracle's (lower positions win)
+    assert np.array_equal(res["idx"], ref)
