@@ -93,14 +93,17 @@ cudaError_t launch_attn_simt(const PathParams &p, const int32_t *idx, int32_t to
                              int32_t out_dtype, float *lse, cudaStream_t s);
 
 // Tensor-core sparse attention (bf16 cache and query, 128 heads, 512 + 64
-// dims, K <= 2048) over CTA pairs; `splits` key splits per query, whose
-// partial outputs go to o_part [n_q, splits, 128, 512] / lse_part
-// [n_q, splits, 128] and are merged by a second kernel when splits > 1.
+// dims, K <= 2048): a compaction kernel turns the selected positions into
+// physical rows (rows [n_q, sfa_rows_ld(K)], n_valid [n_q]), then one CTA per
+// 64 heads of a query and key split; with `splits` > 1 the partial outputs go
+// to o_part [n_q, splits, 128, 512] / lse_part [n_q, splits, 128] and a third
+// kernel merges them.
 bool sfa_mma_supported(const PathParams &p, int32_t top_k);
 int32_t sfa_splits(int32_t n_q, int32_t top_k);
+int32_t sfa_rows_ld(int32_t top_k);
 cudaError_t launch_sfa_mma(const PathParams &p, const int32_t *idx, int32_t top_k, int32_t splits,
-                           void *out, int32_t out_dtype, float *lse, float *o_part,
-                           float *lse_part, cudaStream_t s);
+                           int32_t *rows, int32_t *n_valid, void *out, int32_t out_dtype,
+                           float *lse, float *o_part, float *lse_part, cudaStream_t s);
 
 }  // namespace sa
 

@@ -107,15 +107,16 @@ PathParams make_params(const sa_cache *c, const sa_query *q, void *ws) {
 
 // Workspace: status | vis [n_q] | tile_end [n_q] | scores [n_q, ld] | idx [n_q, K]
 // | hist [n_q, 4096] | counts [n_q, 2] | sel [n_q, K] | cand [n_q, cap]
-// | o_part [n_q, S, 128, 512] | lse_part [n_q, S, 128]; the indexer needs the
-// first three, the fused path all of them; the attention alone needs the
-// status and the split-KV partials (placed right after the status).
+// | rows [n_q, R] | n_valid [n_q] | o_part [n_q, S, 128, 512]
+// | lse_part [n_q, S, 128]; the indexer needs the first three, the fused path
+// all of them; the attention alone needs the status, the compacted rows and
+// the split-KV partials (placed right after the status).
 struct Layout {
     int64_t ld;
     int32_t splits;
-    size_t vis, tile_end, scores, idx, hist, counts, sel, cand, o_part, lse_part;
+    size_t vis, tile_end, scores, idx, hist, counts, sel, cand, rows, n_valid, o_part, lse_part;
     size_t indexer_total, decode_total;
-    size_t attn_o_part, attn_lse_part, attn_total;
+    size_t attn_rows, attn_n_valid, attn_o_part, attn_lse_part, attn_total;
 };
 
 size_t part_bytes(size_t nq, int32_t splits, size_t per) {
@@ -139,24 +140,32 @@ Layout make_layout(const sa_query *q, int32_t top_k) {
     l.counts = align_up(l.hist + sizeof(uint32_t) * nq * kHistBins);  // follows hist: one clear
     l.sel = align_up(l.counts + sizeof(int32_t) * 2 * nq);
     l.cand = align_up(l.sel + sizeof(int32_t) * nq * kk);
-    l.o_part = align_up(l.cand + sizeof(uint64_t) * nq * kTopkCandCap);
+    const size_t rows_bytes = sizeof(int32_t) * nq * (size_t)sfa_rows_ld(top_k);
+    l.rows = align_up(l.cand + sizeof(uint64_t) * nq * kTopkCandCap);
+    l.n_valid = align_up(l.rows + rows_bytes);
+    l.o_part = align_up(l.n_valid + sizeof(int32_t) * nq);
     l.lse_part = align_up(l.o_part + o_bytes);
     l.decode_total = align_up(l.lse_part + lse_bytes);
-    l.attn_o_part = align_up(kStatusBytes);
+    l.attn_rows = align_up(kStatusBytes);
+    l.attn_n_valid = align_up(l.attn_rows + rows_bytes);
+    l.attn_o_part = align_up(l.attn_n_valid + sizeof(int32_t) * nq);
     l.attn_lse_part = align_up(l.attn_o_part + o_bytes);
     l.attn_total = align_up(l.attn_lse_part + lse_bytes);
     return l;
 }
 
 // Sparse attention: the tensor-core kernel for its shape, CUDA cores otherwise.
-sa_status run_attention(const PathParams &p, const Layout &l, size_t o_off, size_t lse_off,
-                        void *ws, const int32_t *idx, int32_t top_k, void *out,
-                        int32_t out_dtype, float *lse, cudaStream_t s) {
+sa_status run_attention(const PathParams &p, const Layout &l, bool fused, void *ws,
+                        const int32_t *idx, int32_t top_k, void *out, int32_t out_dtype,
+                        float *lse, cudaStream_t s) {
     if (sfa_mma_supported(p, top_k)) {
         char *base = static_cast<char *>(ws);
-        return cuda_status(launch_sfa_mma(p, idx, top_k, l.splits, out, out_dtype, lse,
-                                          reinterpret_cast<float *>(base + o_off),
-                                          reinterpret_cast<float *>(base + lse_off), s));
+        return cuda_status(launch_sfa_mma(
+            p, idx, top_k, l.splits,
+            reinterpret_cast<int32_t *>(base + (fused ? l.rows : l.attn_rows)),
+            reinterpret_cast<int32_t *>(base + (fused ? l.n_valid : l.attn_n_valid)), out,
+            out_dtype, lse, reinterpret_cast<float *>(base + (fused ? l.o_part : l.attn_o_part)),
+            reinterpret_cast<float *>(base + (fused ? l.lse_part : l.attn_lse_part)), s));
     }
     return cuda_status(launch_attn_simt(p, idx, top_k, out, out_dtype, lse, s));
 }
@@ -261,8 +270,7 @@ sa_status sa_sparse_mla_attn(const sa_cache *cache, const sa_query *query, const
     if ((st = clear_status(workspace, s)) != SA_OK) return st;
     if (query->n_q == 0) return SA_OK;
     PathParams p = make_params(cache, query, workspace);
-    return run_attention(p, l, l.attn_o_part, l.attn_lse_part, workspace, idx, top_k, out,
-                         out_dtype, lse, s);
+    return run_attention(p, l, false, workspace, idx, top_k, out, out_dtype, lse, s);
 }
 
 static sa_status decode_impl(const sa_cache *cache, const sa_query *query, int32_t top_k,
@@ -306,8 +314,8 @@ static sa_status decode_impl(const sa_cache *cache, const sa_query *query, int32
         }
         if (st != SA_OK) return st;
         if ((st = mark(2)) != SA_OK) return st;
-        if ((st = run_attention(p, l, l.o_part, l.lse_part, workspace, idx, top_k, out,
-                                out_dtype, lse, s)) != SA_OK)
+        if ((st = run_attention(p, l, true, workspace, idx, top_k, out, out_dtype, lse, s)) !=
+            SA_OK)
             return st;
         return mark(3);
     }

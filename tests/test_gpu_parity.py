@@ -225,6 +225,20 @@ def test_attention_on_unsorted_indices_with_holes():
     parity.check_lse(lse.cpu().numpy(), ref_lse)
 
 
+def test_attention_with_large_logits_rescales_output():
+    """Queries scaled by 16 (exact in bf16): each head's running maximum jumps
+    by far more than 2^8 between key tiles, so the kernel must rescale the
+    partial output it keeps on the tensor cores' accumulator."""
+    wl = workload(W.DECODE_B8_8K)
+    qf = (wl.q.astype(np.uint32) << 16).view(np.float32) * np.float32(16.0)
+    wl = dataclasses.replace(wl, q=W.to_bf16_bits(qf))
+    res = run_fused(wl)
+    assert res["status"] == (_abi.SA_OK, 0)
+    ref_out, ref_lse = oracle.sparse_attn(wl, res["idx"])
+    parity.check_attention(res["out"], ref_out, "bf16")
+    parity.check_lse(res["lse"], ref_lse)
+
+
 @pytest.mark.parametrize("pattern", ["all_zero", "three_values"])
 def test_fused_topk_on_massive_ties(pattern):
     """All-equal or few-valued scores: the fused top-K must still pick the
