@@ -22,18 +22,23 @@
 // rows are copied once into a 128-byte-swizzled stage that is the K-major B
 // operand of S and, read MN-major, the B operand of P V.
 //
-// Roles (256 threads, one CTA per SM):
-//   warp 0     lane 0 issues the MMAs from a non-blocking loop -- S of a tile
-//              as soon as its rows are in and an S buffer is free, P V as soon
-//              as P is written -- and commits them to mbarriers;
-//   warps 1-3  copy the selected rows (16-byte cp.async, the swizzle applied
+// Roles (384 threads, one CTA per SM):
+//   warp 0     lane 0 loads Q by TMA (into the third ring stage), then issues
+//              the MMAs from a non-blocking loop -- S of a tile as soon as its
+//              rows are in and an S buffer is free, P V as soon as P is
+//              written -- and commits them to mbarriers;
+//   warps 1-7  copy the selected rows (16-byte cp.async, the swizzle applied
 //              in the addresses) into a 3-stage ring freed by each tile's P V;
-//   warps 4-7  put Q into TMEM, then run the online softmax: lane l < 16 of
-//              warp 4 + j owns head 16j + l (a whole 64-key S row, no
-//              exchange); P goes to shared memory as bf16; O is rescaled in
-//              TMEM (16-lane accesses that leave Q and S alone) only when a
+//              random 1152-byte rows reach shared memory fastest this way;
+//   warps 8-11 move Q into TMEM, then run the online softmax.  Warp 8 + j
+//              owns heads 16j .. 16j + 15 and reads their S rows with 16-lane
+//              loads: thread i holds heads 16j + i/4 and 16j + i/4 + 8, keys
+//              8r + 2(i%4) and 8r + 2(i%4) + 1 of each 8-key group r, so a row
+//              maximum takes two shuffles and P goes to shared memory in
+//              bf16 pairs.  O is rescaled in TMEM (16-lane accesses with the
+//              same thread-to-head mapping, leaving Q and S alone) only when a
 //              head's running maximum grows by more than 2^8; finally lanes
-//              16-31 write O / l.
+//              16-31 read O with 32-lane loads and write O / l.
 // Selected positions are turned into physical cache rows by a small kernel
 // first (sfa_rows_kernel).  All waits are bounded; a timeout is reported in
 // the workspace status word.
@@ -50,8 +55,10 @@ constexpr int kDl = 512, kDr = 64, kD = kDl + kDr;
 constexpr int kBlocks = kD / 64;  // 64-dim (128-byte) column blocks of a row
 constexpr int kTile = 64;         // selected keys per tile
 constexpr int kStages = 3;
-constexpr int kProducerWarps = 3;
-constexpr int kThreads = 256;
+constexpr int kPrefetch = 4;      // tiles of rows prefetched into L2 ahead of the copies
+constexpr int kProducerWarps = 7;
+constexpr int kSoftmaxWarp0 = 8;  // warps 8-11, one per TMEM subpartition
+constexpr int kThreads = 384;
 constexpr int kMaxK = 2048;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColQ = 0;    // lower half-lanes: Q, 288 columns
@@ -61,12 +68,20 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleLog2 = 8.0f;
 constexpr int kChunksPerRow = kD * 2 / 16;  // 72 sixteen-byte pieces of a row
+// Stage layout: key k of a tile, 64-dim block b -> byte (k/8)*kGroupBytes +
+// b*1024 + (k%8)*128 (+ the 16-byte swizzle): the S view (K-major, 8-key
+// groups kGroupBytes apart) and the P V view (MN-major, 64-dim atoms 1024
+// bytes apart, 8-key groups kGroupBytes apart) read the same bytes.
+constexpr uint32_t kGroupBytes = kBlocks * 1024;             // 9216
+constexpr uint32_t kStageBytes = (kTile / 8) * kGroupBytes;  // 73728
 
 struct SfaSmem {
-    uint8_t kv[kStages][kBlocks][kTile * 128];  // 64 full rows, 128-byte swizzle per block
+    // ring stage: 8 groups of 8 rows; a group holds the 9 column blocks of its
+    // rows, each 8 x 128 bytes with the 128-byte swizzle (see kGroupBytes)
+    uint8_t kv[kStages][kStageBytes];
     uint8_t p[kHeadsCta * 128];                 // P (bf16), K-major, 128-byte swizzle
     uint64_t kv_full[kStages], kv_empty[kStages];
-    uint64_t s_full[2], p_full, o_done, q_ready;
+    uint64_t s_full[2], p_full, o_done, q_full, q_ready;
     uint32_t tmem_base;
     int abort;
 };
@@ -98,6 +113,13 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volati
     ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
     __syncwarp();
     return ok;
+}
+
+// 2^x on the special-function unit (ex2.approx: relative error ~2^-22, -inf -> 0).
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
 
 // Tiles [j0, j1) of the compacted key list handled by this split.
@@ -173,7 +195,8 @@ sfa_rows_kernel(const PathParams p, const int32_t *__restrict__ idx, int32_t K, 
     if (et == 0) n_valid_out[t] = n_valid;
 }
 
-__global__ void __launch_bounds__(kThreads, 1) sfa_mma_kernel(const SfaArgs a) {
+__global__ void __launch_bounds__(kThreads, 1)
+sfa_mma_kernel(const __grid_constant__ CUtensorMap tm_q, const SfaArgs a) {
     extern __shared__ uint8_t smem_raw[];
     SfaSmem &sm = *reinterpret_cast<SfaSmem *>(align1024(smem_raw));
     const PathParams &p = a.p;
@@ -190,6 +213,7 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_mma_kernel(const SfaArgs a) {
         for (int b = 0; b < 2; ++b) mbar_init(&sm.s_full[b], 1);
         mbar_init(&sm.p_full, 4);  // the four softmax warps
         mbar_init(&sm.o_done, 1);
+        mbar_init(&sm.q_full, 1);
         mbar_init(&sm.q_ready, 4);
         sm.abort = 0;
         fence_barrier_init();
@@ -206,112 +230,136 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_mma_kernel(const SfaArgs a) {
     split_range(n_valid, split, a.splits, j0, j1);
     const int T = j1 - j0;
 
-    if (warp >= 4) {
+    if (warp >= kSoftmaxWarp0) {
         const int j = warp & 3;  // TMEM subpartition of this warp
-        const bool owner = lane < 16;
-        const int h = 16 * j + (lane & 15);  // head within this CTA (owner: S row, else O row)
+        const int q4 = lane & 3;
+        const int ha = 16 * j + (lane >> 2), hb = ha + 8;  // the two heads of this thread
         const uint32_t lane_lo = static_cast<uint32_t>(32 * j) << 16;
         const uint32_t lane_hi = static_cast<uint32_t>(32 * j + kLaneO) << 16;
+        bool ok = true;
         // ----------------------------------------------- Q into TMEM ---
-        // 32-lane stores: lanes 16-31 receive a copy on O's columns, which
-        // the first P V overwrites.
+        // Q (128-byte-swizzled, in ring stage 2) -> lanes 32j .. 32j + 15;
+        // the 32-lane stores also put a copy on O's columns of lanes 16-31,
+        // which the first P V overwrites.
         if (T > 0) {
-            const uint4 *qrow = reinterpret_cast<const uint4 *>(
-                static_cast<const __nv_bfloat16 *>(p.q) +
-                ((int64_t)t * 128 + kHeadsCta * hh + h) * kD);
+            ok = warp_wait(&sm.q_full, 0, abort_flag, status);
+            if (ok) {
+                const int h = 16 * j + (lane & 15);
 #pragma unroll 1
-            for (int c = 0; c < kBlocks; ++c) {
-                uint32_t v[32];
+                for (int b = 0; b < kBlocks; ++b) {
+                    const uint8_t *qr = sm.kv[2] + b * (kHeadsCta * 128) + h * 128;
+                    uint32_t v[32];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const uint4 x = __ldg(qrow + 8 * c + i);
-                    v[4 * i] = x.x;
-                    v[4 * i + 1] = x.y;
-                    v[4 * i + 2] = x.z;
-                    v[4 * i + 3] = x.w;
+                    for (int c = 0; c < 8; ++c) {
+                        const uint4 x = *reinterpret_cast<const uint4 *>(qr + ((c ^ (h & 7)) << 4));
+                        v[4 * c] = x.x;
+                        v[4 * c + 1] = x.y;
+                        v[4 * c + 2] = x.z;
+                        v[4 * c + 3] = x.w;
+                    }
+                    tmem_st32_u(tmem + lane_lo + kColQ + 32 * b, v);
                 }
-                tmem_st32_u(tmem + lane_lo + kColQ + 32 * c, v);
+                tmem_wait_st();
             }
-            tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.q_ready);
+            if (lane == 0) mbar_arrive(&sm.q_ready);  // also frees ring stage 2
         }
 
         // ----------------------------------------------- online softmax ---
         // The loop never leaves early: after a failed wait (a timeout raised
         // the abort flag) it keeps going without waiting or touching TMEM.
         const float sl2 = p.sm_scale * kLog2e;
-        float m_run = -INFINITY, l_sum = 0.f;
-        bool ok = true;
+        float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
         for (int n = 0; n < T; ++n) {
             const int sb = n & 1;
             if (ok) ok = warp_wait(&sm.s_full[sb], (n >> 1) & 1, abort_flag, status);
-            float s0[32], s1[32];
+            uint32_t v[32];
             if (ok) {
                 tc_fence_after();
-                tmem_ld32(tmem + lane_lo + kColS + kTile * sb, s0);
-                tmem_ld32(tmem + lane_lo + kColS + kTile * sb + 32, s1);
+                tmem_ld_16x256b_x8(tmem + lane_lo + kColS + kTile * sb, v);
                 tmem_wait_ld();
             }
-            const int kvalid = owner ? n_valid - (j0 + n) * kTile : 0;
-            float tmax = -INFINITY;
+            const int kvalid = ok ? n_valid - (j0 + n) * kTile : 0;
+            float xa[16], xb[16];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                s0[i] = (ok && i < kvalid) ? s0[i] * sl2 : -INFINITY;
-                s1[i] = (ok && i + 32 < kvalid) ? s1[i] * sl2 : -INFINITY;
-                tmax = fmaxf(tmax, fmaxf(s0[i], s1[i]));
+            for (int r = 0; r < 8; ++r) {
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    xa[2 * r + e] = __uint_as_float(v[4 * r + e]) * sl2;
+                    xb[2 * r + e] = __uint_as_float(v[4 * r + 2 + e]) * sl2;
+                }
             }
-            // lazy rescaling: the running maximum moves only on a large jump
-            const bool grow = tmax > m_run + kRescaleLog2;
-            const float m_new = grow ? tmax : m_run;
-            const float f = (grow && n > 0) ? exp2f(m_run - m_new) : 1.f;
-            uint32_t packed[32];
-            float l_tile = 0.f;
+            if (kvalid < kTile) {  // the last tile: mask the padding
 #pragma unroll
-            for (int i = 0; i < 32; i += 2) {
-                const float a0 = exp2f(s0[i] - m_new), a1 = exp2f(s0[i + 1] - m_new);
-                const float b0 = exp2f(s1[i] - m_new), b1 = exp2f(s1[i + 1] - m_new);
-                l_tile += (a0 + a1) + (b0 + b1);
+                for (int r = 0; r < 8; ++r) {
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const bool valid = 8 * r + 2 * q4 + e < kvalid;
+                        xa[2 * r + e] = valid ? xa[2 * r + e] : -INFINITY;
+                        xb[2 * r + e] = valid ? xb[2 * r + e] : -INFINITY;
+                    }
+                }
+            }
+            float ta = xa[0], tb = xb[0];
+#pragma unroll
+            for (int i = 1; i < 16; ++i) {
+                ta = fmaxf(ta, xa[i]);
+                tb = fmaxf(tb, xb[i]);
+            }
+            ta = fmaxf(ta, __shfl_xor_sync(0xffffffffu, ta, 1));
+            ta = fmaxf(ta, __shfl_xor_sync(0xffffffffu, ta, 2));
+            tb = fmaxf(tb, __shfl_xor_sync(0xffffffffu, tb, 1));
+            tb = fmaxf(tb, __shfl_xor_sync(0xffffffffu, tb, 2));
+            // lazy rescaling: a running maximum moves only on a large jump
+            const bool grow_a = ta > m_a + kRescaleLog2, grow_b = tb > m_b + kRescaleLog2;
+            const float mn_a = grow_a ? ta : m_a, mn_b = grow_b ? tb : m_b;
+            const float f_a = (grow_a && n > 0) ? exp2f(m_a - mn_a) : 1.f;
+            const float f_b = (grow_b && n > 0) ? exp2f(m_b - mn_b) : 1.f;
+            uint32_t pa[8], pb[8];
+            float la = 0.f, lb = 0.f;
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {
+                const float a0 = ex2(xa[2 * r] - mn_a), a1 = ex2(xa[2 * r + 1] - mn_a);
+                const float b0 = ex2(xb[2 * r] - mn_b), b1 = ex2(xb[2 * r + 1] - mn_b);
+                la += a0 + a1;
+                lb += b0 + b1;
                 __nv_bfloat162 x = __floats2bfloat162_rn(a0, a1);
                 __nv_bfloat162 y = __floats2bfloat162_rn(b0, b1);
-                packed[i / 2] = *reinterpret_cast<uint32_t *>(&x);
-                packed[16 + i / 2] = *reinterpret_cast<uint32_t *>(&y);
+                pa[r] = *reinterpret_cast<uint32_t *>(&x);
+                pb[r] = *reinterpret_cast<uint32_t *>(&y);
             }
             // O and the P buffer belong to P V of the previous tile until it is done
             if (n > 0 && ok) ok = warp_wait(&sm.o_done, (n - 1) & 1, abort_flag, status);
-            if (ok && __any_sync(0xffffffffu, grow && n > 0)) {
+            if (ok && __any_sync(0xffffffffu, (grow_a || grow_b) && n > 0)) {
                 tc_fence_after();
-                // 16-lane accesses to lanes 16-31: thread i holds rows i/4
-                // and i/4 + 8 of them (registers 4r, 4r+1 and 4r+2, 4r+3)
-                const float fa = __shfl_sync(0xffffffffu, f, lane >> 2);
-                const float fb = __shfl_sync(0xffffffffu, f, (lane >> 2) + 8);
 #pragma unroll 1
                 for (int c = 0; c < 4; ++c) {
-                    uint32_t v[64];
-                    tmem_ld_16x256b_x16(tmem + lane_hi + 128 * c, v);
+                    uint32_t w[64];
+                    tmem_ld_16x256b_x16(tmem + lane_hi + 128 * c, w);
                     tmem_wait_ld();
 #pragma unroll
                     for (int r = 0; r < 16; ++r) {
-                        v[4 * r] = __float_as_uint(__uint_as_float(v[4 * r]) * fa);
-                        v[4 * r + 1] = __float_as_uint(__uint_as_float(v[4 * r + 1]) * fa);
-                        v[4 * r + 2] = __float_as_uint(__uint_as_float(v[4 * r + 2]) * fb);
-                        v[4 * r + 3] = __float_as_uint(__uint_as_float(v[4 * r + 3]) * fb);
+                        w[4 * r] = __float_as_uint(__uint_as_float(w[4 * r]) * f_a);
+                        w[4 * r + 1] = __float_as_uint(__uint_as_float(w[4 * r + 1]) * f_a);
+                        w[4 * r + 2] = __float_as_uint(__uint_as_float(w[4 * r + 2]) * f_b);
+                        w[4 * r + 3] = __float_as_uint(__uint_as_float(w[4 * r + 3]) * f_b);
                     }
-                    tmem_st_16x256b_x16(tmem + lane_hi + 128 * c, v);
+                    tmem_st_16x256b_x16(tmem + lane_hi + 128 * c, w);
                 }
                 tmem_wait_st();
             }
-            l_sum = l_sum * f + l_tile;
-            m_run = m_new;
-            if (owner) {
-                uint8_t *prow = sm.p + h * 128;
-                const int sw = h & 7;
+            l_a = l_a * f_a + la;
+            l_b = l_b * f_b + lb;
+            m_a = mn_a;
+            m_b = mn_b;
+            // P rows ha, hb: keys 8r + 2 q4 (+1) -> bytes 16r + 4 q4 of the row
+            uint8_t *row_a = sm.p + ha * 128 + 4 * q4;
+            uint8_t *row_b = sm.p + hb * 128 + 4 * q4;
 #pragma unroll
-                for (int c = 0; c < 8; ++c)
-                    *reinterpret_cast<uint4 *>(prow + ((c ^ sw) << 4)) =
-                        make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2],
-                                   packed[4 * c + 3]);
+            for (int r = 0; r < 8; ++r) {
+                *reinterpret_cast<uint32_t *>(row_a + ((r ^ (ha & 7)) << 4)) = pa[r];
+                *reinterpret_cast<uint32_t *>(row_b + ((r ^ (hb & 7)) << 4)) = pb[r];
             }
             fence_proxy_async_smem();
             tc_fence_before();
@@ -320,12 +368,22 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_mma_kernel(const SfaArgs a) {
         }
         if (ok && T > 0) ok = warp_wait(&sm.o_done, (T - 1) & 1, abort_flag, status);
         tc_fence_after();
-        const float inv = (ok && l_sum > 0.f) ? 1.f / l_sum : 0.f;
-        const float lse_v = (ok && l_sum > 0.f) ? (m_run + log2f(l_sum)) * kLn2 : -INFINITY;
-        const float inv_o = __shfl_sync(0xffffffffu, inv, lane & 15);
-        const int head = kHeadsCta * hh + h;
+        // full row sums: the four threads of a head each hold a quarter
+        l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
+        l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
+        l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
+        l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
+        const float inv_a = (ok && l_a > 0.f) ? 1.f / l_a : 0.f;
+        const float inv_b = (ok && l_b > 0.f) ? 1.f / l_b : 0.f;
+        // 32-lane loads: lane 16 + r receives the O row of head 16j + r, whose
+        // sums sit in thread 4(r % 8) (as its first head for r < 8)
+        const int r_o = lane & 15;
+        const float inv_ra = __shfl_sync(0xffffffffu, inv_a, 4 * (r_o & 7));
+        const float inv_rb = __shfl_sync(0xffffffffu, inv_b, 4 * (r_o & 7));
+        const float inv_o = r_o < 8 ? inv_ra : inv_rb;
+        const bool o_lane = lane >= 16;
+        const int head = kHeadsCta * hh + 16 * j + r_o;
         const int64_t row = (int64_t)t * 128 + head;
-        // 32-lane loads: lanes 16-31 receive the O rows
 #pragma unroll 1
         for (int c = 0; c < kDl / 32; ++c) {
             float v[32];
@@ -336,7 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_mma_kernel(const SfaArgs a) {
 #pragma unroll
                 for (int i = 0; i < 32; ++i) v[i] = 0.f;
             }
-            if (owner) continue;
+            if (!o_lane) continue;
             const int dv = 32 * c;
             if (a.splits == 1) {
                 if (a.out_dtype == SA_BF16) {
@@ -369,49 +427,113 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_mma_kernel(const SfaArgs a) {
                                          v[4 * i + 2] * inv_o, v[4 * i + 3] * inv_o);
             }
         }
-        if (owner) {
+        if (q4 == 0) {
+            const float lse_a = (ok && l_a > 0.f) ? (m_a + log2f(l_a)) * kLn2 : -INFINITY;
+            const float lse_b = (ok && l_b > 0.f) ? (m_b + log2f(l_b)) * kLn2 : -INFINITY;
+            const int64_t row_a = (int64_t)t * 128 + kHeadsCta * hh + ha;
+            const int64_t row_b = row_a + 8;
             if (a.splits == 1) {
-                if (a.lse != nullptr) a.lse[row] = lse_v;
+                if (a.lse != nullptr) {
+                    a.lse[row_a] = lse_a;
+                    a.lse[row_b] = lse_b;
+                }
             } else {
-                a.lse_part[((int64_t)t * a.splits + split) * 128 + head] = lse_v;
+                const int64_t base = ((int64_t)t * a.splits + split) * 128 + kHeadsCta * hh;
+                a.lse_part[base + ha] = lse_a;
+                a.lse_part[base + hb] = lse_b;
             }
         }
     } else if (warp >= 1) {
         // ---------------------------------------------- row producers ---
-        // warp 1 + w copies keys w, w + 3, ... of each tile; a key's 72
-        // sixteen-byte pieces go to lanes (piece % 32) in three steps.
+        // warp 1 + w copies keys w, w + 7, ... of each tile; a key's 72
+        // sixteen-byte pieces go to lanes (piece % 32) in three steps.  Ring
+        // stage 2 holds Q until the softmax warps have moved it to TMEM.
         const int pw = warp - 1;
         const uint8_t *kv = static_cast<const uint8_t *>(p.kv);
         const int32_t *rows = a.rows + (int64_t)t * a.ld_rows;
+        // The ring holds about one tile in flight per SM, too little to cover
+        // the latency of random row reads from HBM; so the rows of tile
+        // n + kPrefetch are pulled into L2 (one bulk prefetch per row, by
+        // warps 1-2) while tile n is copied, and the copies mostly hit L2.
+        // Row indices are loaded one iteration before they are used, so no
+        // global load latency sits between a freed stage and its copies.
+        const int pk = pw * 32 + lane;  // key prefetched by this thread
+        const bool prefetcher = pk < kTile;
+        const int32_t *tile_rows = rows + (int64_t)j0 * kTile;
+        if (prefetcher) {
+            int32_t r0[kPrefetch];
+#pragma unroll
+            for (int n = 0; n < kPrefetch; ++n) r0[n] = n < T ? __ldg(tile_rows + n * kTile + pk) : 0;
+#pragma unroll
+            for (int n = 0; n < kPrefetch; ++n)
+                if (n < T) prefetch_l2(kv + (int64_t)r0[n] * (kD * 2), kD * 2);
+        }
+        int32_t pf_row =
+            (prefetcher && kPrefetch < T) ? __ldg(tile_rows + kPrefetch * kTile + pk) : 0;
+        int32_t r_lo = T > 0 ? __ldg(tile_rows + lane) : 0;
+        int32_t r_hi = T > 0 ? __ldg(tile_rows + 32 + lane) : 0;
         for (int n = 0; n < T; ++n) {
             const int st = n % kStages;
+            if (prefetcher && n + kPrefetch < T) prefetch_l2(kv + (int64_t)pf_row * (kD * 2), kD * 2);
+            const bool more = n + 1 < T;
+            const int32_t pf_next = (prefetcher && n + 1 + kPrefetch < T)
+                                        ? __ldg(tile_rows + (n + 1 + kPrefetch) * kTile + pk)
+                                        : 0;
+            const int32_t lo_next = more ? __ldg(tile_rows + (n + 1) * kTile + lane) : 0;
+            const int32_t hi_next = more ? __ldg(tile_rows + (n + 1) * kTile + 32 + lane) : 0;
             if (!warp_wait(&sm.kv_empty[st], ((n / kStages) & 1) ^ 1, abort_flag, status)) break;
-            const int32_t *rr = rows + (j0 + n) * kTile;
-            const int32_t r_lo = __ldg(rr + lane), r_hi = __ldg(rr + 32 + lane);
-            const uint32_t dst0 = smem_u32(sm.kv[st][0]);
+            if (n == 2 && !warp_wait(&sm.q_ready, 0, abort_flag, status)) break;
+            const uint32_t dst0 = smem_u32(sm.kv[st]);
 #pragma unroll 2
             for (int k = pw; k < kTile; k += kProducerWarps) {
                 const int32_t r = __shfl_sync(0xffffffffu, k < 32 ? r_lo : r_hi, k & 31);
                 const uint8_t *src = kv + (int64_t)r * (kD * 2);
-                const uint32_t dk = dst0 + k * 128;
+                const uint32_t dk = dst0 + (k >> 3) * kGroupBytes + (k & 7) * 128;
                 const int sw = k & 7;
 #pragma unroll
                 for (int i = 0; i < 3; ++i) {
                     const int c = lane + 32 * i;
                     if (c < kChunksPerRow)
-                        cp_async16(dk + (c >> 3) * (kTile * 128) + (((c & 7) ^ sw) << 4),
-                                   src + c * 16);
+                        cp_async16(dk + (c >> 3) * 1024 + (((c & 7) ^ sw) << 4), src + c * 16);
                 }
             }
             cp_async_arrive(&sm.kv_full[st]);
+            pf_row = pf_next;
+            r_lo = lo_next;
+            r_hi = hi_next;
         }
         cp_async_wait_all();
     } else if (lane == 0 && T > 0) {
-        // ---------------------------------------------------- MMA issuer ---
+        // ------------------------------------------ Q load, MMA issuer ---
+        mbar_arrive_expect_tx(&sm.q_full, kBlocks * kHeadsCta * 128);
+        for (int b = 0; b < kBlocks; ++b)
+            tma_load_2d(sm.kv[2] + b * (kHeadsCta * 128), &tm_q, 64 * b, t * 128 + kHeadsCta * hh,
+                        &sm.q_full);
         constexpr uint32_t id_s = instr_desc(64, kTile, 1 /*bf16*/, 0, 0);
         constexpr uint32_t id_pv = instr_desc(64, 256, 1 /*bf16*/, 0, 1);
         bool ok = mbar_wait(&sm.q_ready, 0, abort_flag, status);
         int ns = 0, np = 0;  // next S and next P V to issue
+        // P V(np) needs P of tile np
+        auto try_pv = [&]() -> bool {
+            if (!(np < ns && mbar_test(&sm.p_full, np & 1))) return false;
+            fence_proxy_async_smem();
+            tc_fence_after();
+            const int st = np % kStages;
+            const uint64_t ad = desc_kmajor_sw128(smem_u32(sm.p));
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                const uint32_t vb = smem_u32(sm.kv[st]) + 4 * half * 1024;
+#pragma unroll
+                for (int k = 0; k < 4; ++k)  // 16 keys (two groups) per instruction
+                    mma_bf16(tmem + (kLaneO << 16) + 256 * half, ad + 2 * k,
+                             desc_mnmajor_sw128(vb + 2 * k * kGroupBytes, 1024, kGroupBytes),
+                             id_pv, (np > 0 || k > 0) ? 1u : 0u);
+            }
+            mma_commit(&sm.o_done);
+            if (np + kStages < T) mma_commit(&sm.kv_empty[st]);
+            ++np;
+            return true;
+        };
         long long t0 = clock64();
         uint32_t idle = 0;
         while (ok && np < T) {
@@ -424,9 +546,10 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_mma_kernel(const SfaArgs a) {
                     fence_proxy_async_smem();
                     tc_fence_after();
                     const uint32_t d = tmem + kColS + kTile * (ns & 1);
+                    const uint32_t stage = smem_u32(sm.kv[st]);
 #pragma unroll 1
                     for (int b = 0; b < kBlocks; ++b) {
-                        const uint64_t bd = desc_kmajor_sw128(smem_u32(sm.kv[st][b]));
+                        const uint64_t bd = desc_kmajor_sw128_sbo(stage + b * 1024, kGroupBytes);
 #pragma unroll
                         for (int k = 0; k < 4; ++k)  // 16 dims (32 bytes) per instruction
                             mma_bf16_ts(d, tmem + kColQ + 32 * b + 8 * k, bd + 2 * k, id_s,
@@ -437,26 +560,7 @@ __global__ void __launch_bounds__(kThreads, 1) sfa_mma_kernel(const SfaArgs a) {
                     progressed = true;
                 }
             }
-            // P V(np) needs P of tile np
-            if (np < ns && mbar_test(&sm.p_full, np & 1)) {
-                fence_proxy_async_smem();
-                tc_fence_after();
-                const int st = np % kStages;
-                const uint64_t ad = desc_kmajor_sw128(smem_u32(sm.p));
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    const uint32_t vb = smem_u32(sm.kv[st][4 * half]);
-#pragma unroll
-                    for (int k = 0; k < 4; ++k)  // 16 keys per instruction
-                        mma_bf16(tmem + (kLaneO << 16) + 256 * half, ad + 2 * k,
-                                 desc_mnmajor_sw128(vb + 2048 * k, kTile * 128, 1024), id_pv,
-                                 (np > 0 || k > 0) ? 1u : 0u);
-                }
-                mma_commit(&sm.o_done);
-                if (np + kStages < T) mma_commit(&sm.kv_empty[st]);
-                ++np;
-                progressed = true;
-            }
+            if (try_pv()) progressed = true;
             if (progressed) {
                 t0 = clock64();
                 idle = 0;
@@ -536,6 +640,9 @@ cudaError_t launch_sfa_mma(const PathParams &p, const int32_t *idx, int32_t top_
                                                                  n_valid);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
+    CUtensorMap tq;
+    if (!encode_tmap_2d(&tq, 2, p.q, kD, (uint64_t)p.n_q * 128, kD * 2, 64, kHeadsCta, true))
+        return cudaErrorInvalidValue;
     SfaArgs a{p, rows, n_valid, ld_rows, splits, out, out_dtype, lse, o_part, lse_part};
     const size_t smem = sizeof(SfaSmem) + 1024;
     e = cudaFuncSetAttribute(sfa_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -543,7 +650,7 @@ cudaError_t launch_sfa_mma(const PathParams &p, const int32_t *idx, int32_t top_
     if (e != cudaSuccess) return e;
     const int64_t grid = 2 * (int64_t)p.n_q * splits;
     count_launch();
-    sfa_mma_kernel<<<static_cast<unsigned>(grid), kThreads, smem, s>>>(a);
+    sfa_mma_kernel<<<static_cast<unsigned>(grid), kThreads, smem, s>>>(tq, a);
     if ((e = cudaGetLastError()) != cudaSuccess || splits == 1) return e;
     count_launch();
     sfa_combine_kernel<<<static_cast<unsigned>(p.n_q * 128), 128, 0, s>>>(o_part, lse_part, splits,
