@@ -285,10 +285,17 @@ def run_ours(args, rank: int, world: int, dist):
         for k in range(args.steps):
             flush.zero_()
             outer[k][0].record(stream)
-            step(ev[k])
+            step()
             outer[k][1].record(stream)
         torch.cuda.synchronize()
     launches = _abi.lib().sa_kernel_launches() - launches0
+    # Phase attribution: the same steps again with events between the phases
+    # (an event between two kernels stops the next one from launching early,
+    # so these steps run a little slower than the timed ones above).
+    for k in range(args.steps):
+        flush.zero_()
+        step(ev[k])
+    torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
     total_ms = sum(a.elapsed_time(b) for a, b in outer)

@@ -44,6 +44,8 @@ template <int HG>
 __global__ void __launch_bounds__(kThreads)
 attn_simt_kernel(const PathParams p, const int32_t *__restrict__ idx, int32_t K, void *out,
                  int32_t out_dtype, float *__restrict__ lse) {
+    pdl_wait();
+    pdl_trigger();
     extern __shared__ float smem[];
     const int D = p.d_latent + p.d_rope, dl = p.d_latent, ldr = D + 1;
     float *q_s = smem;                      // [HG][D]
@@ -172,8 +174,8 @@ cudaError_t launch_hg(const PathParams &p, const int32_t *idx, int32_t K, void *
                          (int)smem);
     dim3 grid(p.heads / HG, p.n_q);
     count_launch();
-    attn_simt_kernel<HG><<<grid, kThreads, smem, s>>>(p, idx, K, out, out_dtype, lse);
-    return cudaGetLastError();
+    return launch_pdl(attn_simt_kernel<HG>, grid, dim3(kThreads), smem, s, p, idx, K, out,
+                      out_dtype, lse);
 }
 
 }  // namespace

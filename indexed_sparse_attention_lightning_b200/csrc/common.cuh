@@ -70,6 +70,15 @@ __device__ __forceinline__ int64_t phys_row(const int32_t *page_table, int32_t m
     return (int64_t)page * 64 + (s & 63);
 }
 
+// Programmatic dependent launch.  pdl_wait: block until the kernel before
+// this one in the stream has completed and its writes are visible (a no-op
+// when launched without the attribute).  pdl_trigger: let the next kernel in
+// the stream start launching; its blocks still stop in their pdl_wait.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __host__ __device__ constexpr int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 __host__ __device__ constexpr int64_t round_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }
 

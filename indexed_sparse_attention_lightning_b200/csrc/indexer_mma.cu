@@ -118,6 +118,7 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volati
 __global__ void __launch_bounds__(kThreads, 2)
 indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
                    const __grid_constant__ CUtensorMap tm_q, const IndexerArgs a) {
+    pdl_wait();
     extern __shared__ uint8_t smem_raw[];
     IndexerSmem &sm = *reinterpret_cast<IndexerSmem *>(align1024(smem_raw));
     const PathParams &p = a.p;
@@ -149,25 +150,48 @@ indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    pdl_trigger();  // after the TMEM allocation: a waiting successor holds none
     const uint32_t tmem = sm.tmem_base;
     volatile int *abort_flag = &sm.abort;
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer ---
         if (lane == 0) {
+            // Page-table entries are looked up one tile ahead, so their load
+            // latency overlaps the wait for a free stage instead of sitting
+            // between that wait and the TMA copies.
             TileCursor c;
             c.init(a.tile_end, p.n_q, k0, k1);
             bool seg_start = true;
-            int32_t seq = 0, V = 0;
+            int32_t seq = p.q_seq[c.t], V = a.vis[c.t];
+            int32_t pg[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int64_t s = (int64_t)c.i * kKeys + 64 * h;
+                pg[h] = s < V ? p.page_table[(int64_t)seq * p.max_pages + (s >> 6)] : -1;
+            }
             for (int n = 0; c.valid(); ++n) {
+                // look-ahead: the next tile of this CTA
+                TileCursor nx = c;
+                const bool nx_seg = nx.next(a.tile_end);
+                int32_t nseq = seq, nV = V, npg[2] = {-1, -1};
+                if (nx.valid()) {
+                    if (nx_seg) {
+                        nseq = p.q_seq[nx.t];
+                        nV = a.vis[nx.t];
+                    }
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int64_t s = (int64_t)nx.i * kKeys + 64 * h;
+                        if (s < nV) npg[h] = p.page_table[(int64_t)nseq * p.max_pages + (s >> 6)];
+                    }
+                }
                 if (seg_start) {
                     const int b = c.seg & 1;
                     if (!mbar_wait(&sm.q_empty[b], ((c.seg >> 1) & 1) ^ 1, abort_flag, p.status))
                         break;
                     mbar_arrive_expect_tx(&sm.q_full[b], kQBytes);
                     tma_load_2d(sm.q[b], &tm_q, 0, c.t * kHeads, &sm.q_full[b]);
-                    seq = p.q_seq[c.t];
-                    V = a.vis[c.t];
                 }
                 const int stage = n % kStages;
                 // the stage is free once its MMAs and its epilogue are done
@@ -181,12 +205,9 @@ indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     const int64_t s = (int64_t)c.i * kKeys + 64 * h;
-                    if (s < V) {
-                        const int32_t page = p.page_table[(int64_t)seq * p.max_pages + (s >> 6)];
-                        if (page >= 0 && page < p.num_pages) {
-                            rows[h] = page * 64;
-                            bytes += kPageBytes + 64 * sizeof(float);
-                        }
+                    if (s < V && pg[h] >= 0 && pg[h] < p.num_pages) {
+                        rows[h] = pg[h] * 64;
+                        bytes += kPageBytes + 64 * sizeof(float);
                     }
                     sm.page_ok[stage][h] = rows[h] >= 0;  // published by the arrive below
                 }
@@ -199,7 +220,12 @@ indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
                         bulk_load(&sm.kscale[stage][64 * h], p.k_index_scale + rows[h],
                                   64 * sizeof(float), &sm.full[stage]);
                     }
-                seg_start = c.next(a.tile_end);
+                c = nx;
+                seg_start = nx_seg;
+                seq = nseq;
+                V = nV;
+                pg[0] = npg[0];
+                pg[1] = npg[1];
             }
         }
     } else if (warp == 1) {
@@ -344,8 +370,8 @@ cudaError_t launch_indexer_mma(const PathParams &p, const int32_t *vis, const in
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     count_launch();
-    indexer_mma_kernel<<<static_cast<unsigned>(grid), kThreads, smem, s>>>(tk, tq, a);
-    return cudaGetLastError();
+    return launch_pdl(indexer_mma_kernel, dim3(static_cast<unsigned>(grid)), dim3(kThreads), smem,
+                      s, tk, tq, a);
 }
 
 }  // namespace sa

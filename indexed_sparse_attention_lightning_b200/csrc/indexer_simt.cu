@@ -19,6 +19,8 @@ constexpr int kHeadBlock = 16;  // head dot products kept in registers at once
 template <bool kE4M3>
 __global__ void __launch_bounds__(kThreads)
 indexer_simt_kernel(const PathParams p, float *__restrict__ scores, int64_t ld) {
+    pdl_wait();
+    pdl_trigger();
     extern __shared__ float smem[];
     const int32_t H = p.h_index, d = p.d_index;
     float *q_s = smem;          // [H][d] query codes as floats (scale folded into w)
@@ -108,14 +110,14 @@ cudaError_t launch_indexer_simt(const PathParams &p, float *scores, int64_t ld, 
         cudaFuncSetAttribute(indexer_simt_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem);
         count_launch();
-        indexer_simt_kernel<true><<<grid, kThreads, smem, s>>>(p, scores, ld);
+        return launch_pdl(indexer_simt_kernel<true>, grid, dim3(kThreads), smem, s, p, scores, ld);
     } else {
         cudaFuncSetAttribute(indexer_simt_kernel<false>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         count_launch();
-        indexer_simt_kernel<false><<<grid, kThreads, smem, s>>>(p, scores, ld);
+        return launch_pdl(indexer_simt_kernel<false>, grid, dim3(kThreads), smem, s, p, scores,
+                          ld);
     }
-    return cudaGetLastError();
 }
 
 }  // namespace sa

@@ -7,10 +7,31 @@
 #include <stdint.h>
 
 #include <algorithm>
+#include <utility>
 
 #include "sa.h"
 
 namespace sa {
+
+// Launches `kernel` with programmatic stream serialization, so that its
+// launch overlaps the tail of the previous kernel in the stream (the kernel
+// itself calls pdl_wait before touching anything that kernel wrote).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t s, Args &&...args) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 
 // Everything a kernel needs to know about the paged caches and the queries.
 struct PathParams {
@@ -84,17 +105,22 @@ cudaError_t launch_topk_rowwise(const float *scores, int64_t ld, const int32_t *
 // (which filled `hist`, [n_q, kHistBins]).  Scratch: sel [n_q, top_k],
 // counts [n_q, 2] (zeroed), cand [n_q, cap].
 constexpr int32_t kTopkCandCap = 8192;
+// With `rows` non-null it also writes the physical cache rows of the
+// selection for the tensor-core attention (compact_rows layout, tile 64,
+// leading dimension ld_rows) and their count n_valid [n_q].
 cudaError_t launch_topk_hist(const float *scores, int64_t ld, const int32_t *vis,
                              const uint32_t *hist, int32_t n_q, int32_t max_valid, int32_t top_k,
                              int32_t *sel, int32_t *counts, uint64_t *cand, int32_t cap,
-                             int32_t *idx, cudaStream_t s);
+                             int32_t *idx, const PathParams &p, int32_t *rows, int32_t ld_rows,
+                             int32_t *n_valid, cudaStream_t s);
 
 cudaError_t launch_attn_simt(const PathParams &p, const int32_t *idx, int32_t top_k, void *out,
                              int32_t out_dtype, float *lse, cudaStream_t s);
 
 // Tensor-core sparse attention (bf16 cache and query, 128 heads, 512 + 64
 // dims, K <= 2048): a compaction kernel turns the selected positions into
-// physical rows (rows [n_q, sfa_rows_ld(K)], n_valid [n_q]), then one CTA per
+// physical rows (rows [n_q, sfa_rows_ld(K)], n_valid [n_q]; skipped when
+// `rows_ready`, i.e. the top-K kernel already wrote them), then one CTA per
 // 64 heads of a query and key split; with `splits` > 1 the partial outputs go
 // to o_part [n_q, splits, 128, 512] / lse_part [n_q, splits, 128] and a third
 // kernel merges them.
@@ -102,8 +128,9 @@ bool sfa_mma_supported(const PathParams &p, int32_t top_k);
 int32_t sfa_splits(int32_t n_q, int32_t top_k);
 int32_t sfa_rows_ld(int32_t top_k);
 cudaError_t launch_sfa_mma(const PathParams &p, const int32_t *idx, int32_t top_k, int32_t splits,
-                           int32_t *rows, int32_t *n_valid, void *out, int32_t out_dtype,
-                           float *lse, float *o_part, float *lse_part, cudaStream_t s);
+                           int32_t *rows, int32_t *n_valid, bool rows_ready, void *out,
+                           int32_t out_dtype, float *lse, float *o_part, float *lse_part,
+                           cudaStream_t s);
 
 }  // namespace sa
 
@@ -120,6 +147,51 @@ __device__ __forceinline__ int32_t visible_len(const PathParams &p, int32_t t) {
         return 0;
     }
     return pos + 1;
+}
+
+// Physical cache rows of query t's selected positions sel[0, K): list order,
+// -1 entries dropped, out-of-range positions and bad page ids skipped and
+// reported; then padded with the first row up to a multiple of `tile`.
+// Writes rows[0, padded) and *n_valid.  Called by every thread of a CTA
+// (blockDim.x a multiple of 32); `scratch` is shared memory of 33 ints.
+__device__ __forceinline__ void compact_rows(const PathParams &p, int32_t t, const int32_t *sel,
+                                             int32_t K, int32_t tile, int32_t *rows,
+                                             int32_t *n_valid, int32_t *scratch) {
+    const int nwarps = blockDim.x >> 5, w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int32_t V = visible_len(p, t);
+    const int32_t seq = __ldg(p.q_seq + t);
+    int32_t base = 0;
+    for (int32_t r0 = 0; r0 < K; r0 += blockDim.x) {
+        const int32_t k = r0 + threadIdx.x;
+        const int32_t s = k < K ? sel[k] : -1;
+        int32_t v = -1;
+        if (s >= V) {
+            report(p.status, SA_ERR_DEVICE_FAULT, SA_DETAIL_BAD_INDEX);
+        } else if (s >= 0) {
+            const int64_t row = phys_row(p.page_table, p.max_pages, p.num_pages, seq, s);
+            if (row < 0) report(p.status, SA_ERR_DEVICE_FAULT, SA_DETAIL_BAD_PAGE);
+            else v = static_cast<int32_t>(row);
+        }
+        const unsigned bal = __ballot_sync(0xffffffffu, v >= 0);
+        if (lane == 0) scratch[w] = __popc(bal);
+        __syncthreads();
+        int32_t off = base, tot = 0;
+        for (int i = 0; i < nwarps; ++i) {
+            if (i < w) off += scratch[i];
+            tot += scratch[i];
+        }
+        const int32_t pos = off + __popc(bal & ((1u << lane) - 1u));
+        if (v >= 0) {
+            rows[pos] = v;
+            if (pos == 0) scratch[32] = v;
+        }
+        __syncthreads();
+        base += tot;
+    }
+    const int32_t padded = (base + tile - 1) / tile * tile;
+    if (base > 0)
+        for (int32_t c = base + threadIdx.x; c < padded; c += blockDim.x) rows[c] = scratch[32];
+    if (threadIdx.x == 0) *n_valid = base;
 }
 }  // namespace sa
 #endif

@@ -13,6 +13,8 @@ constexpr int kThreads = 1024;
 __global__ void __launch_bounds__(kThreads)
 plan_kernel(const PathParams p, int32_t *vis, int32_t *tile_end, int32_t tile, uint32_t *zero,
             size_t zero_words) {
+    pdl_wait();
+    pdl_trigger();
     for (size_t i = (size_t)blockIdx.x * kThreads + threadIdx.x; i < zero_words;
          i += (size_t)gridDim.x * kThreads)
         zero[i] = 0u;
@@ -63,9 +65,8 @@ cudaError_t launch_plan(const PathParams &p, int32_t *vis, int32_t *tile_end, in
     const int64_t blocks =
         std::max<int64_t>(1, std::min<int64_t>(num_sms(), ceil_div(zero_words, 4 * kThreads)));
     count_launch();
-    plan_kernel<<<static_cast<unsigned>(blocks), kThreads, 0, s>>>(p, vis, tile_end, tile, zero,
-                                                                  zero_words);
-    return cudaGetLastError();
+    return launch_pdl(plan_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kThreads), 0, s, p,
+                      vis, tile_end, tile, zero, zero_words);
 }
 
 int num_sms() {

@@ -155,16 +155,16 @@ Layout make_layout(const sa_query *q, int32_t top_k) {
 }
 
 // Sparse attention: the tensor-core kernel for its shape, CUDA cores otherwise.
-sa_status run_attention(const PathParams &p, const Layout &l, bool fused, void *ws,
-                        const int32_t *idx, int32_t top_k, void *out, int32_t out_dtype,
-                        float *lse, cudaStream_t s) {
+sa_status run_attention(const PathParams &p, const Layout &l, bool fused, bool rows_ready,
+                        void *ws, const int32_t *idx, int32_t top_k, void *out,
+                        int32_t out_dtype, float *lse, cudaStream_t s) {
     if (sfa_mma_supported(p, top_k)) {
         char *base = static_cast<char *>(ws);
         return cuda_status(launch_sfa_mma(
             p, idx, top_k, l.splits,
             reinterpret_cast<int32_t *>(base + (fused ? l.rows : l.attn_rows)),
-            reinterpret_cast<int32_t *>(base + (fused ? l.n_valid : l.attn_n_valid)), out,
-            out_dtype, lse, reinterpret_cast<float *>(base + (fused ? l.o_part : l.attn_o_part)),
+            reinterpret_cast<int32_t *>(base + (fused ? l.n_valid : l.attn_n_valid)), rows_ready,
+            out, out_dtype, lse, reinterpret_cast<float *>(base + (fused ? l.o_part : l.attn_o_part)),
             reinterpret_cast<float *>(base + (fused ? l.lse_part : l.attn_lse_part)), s));
     }
     return cuda_status(launch_attn_simt(p, idx, top_k, out, out_dtype, lse, s));
@@ -270,7 +270,7 @@ sa_status sa_sparse_mla_attn(const sa_cache *cache, const sa_query *query, const
     if ((st = clear_status(workspace, s)) != SA_OK) return st;
     if (query->n_q == 0) return SA_OK;
     PathParams p = make_params(cache, query, workspace);
-    return run_attention(p, l, false, workspace, idx, top_k, out, out_dtype, lse, s);
+    return run_attention(p, l, false, false, workspace, idx, top_k, out, out_dtype, lse, s);
 }
 
 static sa_status decode_impl(const sa_cache *cache, const sa_query *query, int32_t top_k,
@@ -301,21 +301,26 @@ static sa_status decode_impl(const sa_cache *cache, const sa_query *query, int32
         if ((st = run_indexer(p, l, workspace, scores, l.ld, true, &have_hist, s)) != SA_OK)
             return st;
         if ((st = mark(1)) != SA_OK) return st;
+        // the top-K kernel also emits the physical rows for the tensor-core attention
+        const bool rows_ready = have_hist && sfa_mma_supported(p, top_k);
         if (have_hist) {
             st = cuda_status(launch_topk_hist(
                 scores, l.ld, reinterpret_cast<const int32_t *>(base + l.vis),
                 reinterpret_cast<const uint32_t *>(base + l.hist), query->n_q, query->max_visible,
                 top_k, reinterpret_cast<int32_t *>(base + l.sel),
                 reinterpret_cast<int32_t *>(base + l.counts),
-                reinterpret_cast<uint64_t *>(base + l.cand), kTopkCandCap, idx, s));
+                reinterpret_cast<uint64_t *>(base + l.cand), kTopkCandCap, idx, p,
+                rows_ready ? reinterpret_cast<int32_t *>(base + l.rows) : nullptr,
+                sfa_rows_ld(top_k),
+                rows_ready ? reinterpret_cast<int32_t *>(base + l.n_valid) : nullptr, s));
         } else {
             st = cuda_status(launch_topk_rowwise(scores, l.ld, nullptr, query->max_visible, &p,
                                                  query->n_q, top_k, idx, p.status, s));
         }
         if (st != SA_OK) return st;
         if ((st = mark(2)) != SA_OK) return st;
-        if ((st = run_attention(p, l, true, workspace, idx, top_k, out, out_dtype, lse, s)) !=
-            SA_OK)
+        if ((st = run_attention(p, l, true, rows_ready, workspace, idx, top_k, out, out_dtype,
+                                lse, s)) != SA_OK)
             return st;
         return mark(3);
     }

@@ -130,73 +130,23 @@ __device__ __forceinline__ void split_range(int32_t n_valid, int32_t split, int3
     j1 = (int32_t)((int64_t)tiles * (split + 1) / splits);
 }
 
-// Query t's selected positions -> physical cache rows, in list order with the
-// -1 padding dropped, then padded with the first row to whole tiles (the
-// softmax masks the padding).  Out-of-range positions and bad page ids are
-// skipped and reported.  One CTA of 128 threads per query.
-__global__ void __launch_bounds__(128)
+// Query t's selected positions -> physical cache rows (compact_rows): one
+// CTA per query.  The fused decode path gets the rows from the top-K kernel.
+constexpr int kRowsThreads = 512;
+__global__ void __launch_bounds__(kRowsThreads)
 sfa_rows_kernel(const PathParams p, const int32_t *__restrict__ idx, int32_t K, int32_t ld_rows,
                 int32_t *__restrict__ rows, int32_t *__restrict__ n_valid_out) {
-    __shared__ int32_t warp_cnt[4];
-    __shared__ int32_t first_row;
-    const int t = blockIdx.x, et = threadIdx.x, ew = et >> 5, lane = et & 31;
-    const int32_t V = visible_len(p, t);
-    const int32_t seq = p.q_seq[t];
-    const int32_t *sel = idx + (int64_t)t * K;
-    int32_t *out = rows + (int64_t)t * ld_rows;
-    // all index and page-table loads in flight at once (16 per thread), then
-    // an ordered compaction over the 16 rounds of 128 entries
-    constexpr int kRounds = kMaxK / 128;
-    int32_t phys[kRounds];
-#pragma unroll
-    for (int r = 0; r < kRounds; ++r) {
-        const int k = r * 128 + et;
-        phys[r] = k < K ? __ldg(sel + k) : -1;
-    }
-#pragma unroll
-    for (int r = 0; r < kRounds; ++r) {
-        const int32_t s = phys[r];
-        int32_t v = -1;
-        if (s >= V) {
-            report(p.status, SA_ERR_DEVICE_FAULT, SA_DETAIL_BAD_INDEX);
-        } else if (s >= 0) {
-            const int64_t row = phys_row(p.page_table, p.max_pages, p.num_pages, seq, s);
-            if (row < 0) report(p.status, SA_ERR_DEVICE_FAULT, SA_DETAIL_BAD_PAGE);
-            else v = static_cast<int32_t>(row);
-        }
-        phys[r] = v;
-    }
-    int32_t base = 0;
-#pragma unroll
-    for (int r = 0; r < kRounds; ++r) {
-        const unsigned bal = __ballot_sync(0xffffffffu, phys[r] >= 0);
-        if (lane == 0) warp_cnt[ew] = __popc(bal);
-        __syncthreads();
-        int32_t off = base, tot = 0;
-#pragma unroll
-        for (int w = 0; w < 4; ++w) {
-            if (w < ew) off += warp_cnt[w];
-            tot += warp_cnt[w];
-        }
-        const int32_t pos = off + __popc(bal & ((1u << lane) - 1u));
-        if (phys[r] >= 0) {
-            out[pos] = phys[r];
-            if (pos == 0) first_row = phys[r];
-        }
-        __syncthreads();
-        base += tot;
-    }
-    const int32_t n_valid = base;
-    const int32_t padded = ((n_valid + kTile - 1) / kTile) * kTile;
-    if (n_valid > 0) {
-        const int32_t r0 = first_row;  // written before the last barrier above
-        for (int c = n_valid + et; c < padded; c += 128) out[c] = r0;
-    }
-    if (et == 0) n_valid_out[t] = n_valid;
+    pdl_wait();
+    pdl_trigger();
+    __shared__ int32_t scratch[33];
+    const int t = blockIdx.x;
+    compact_rows(p, t, idx + (int64_t)t * K, K, kTile, rows + (int64_t)t * ld_rows,
+                 n_valid_out + t, scratch);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
 sfa_mma_kernel(const __grid_constant__ CUtensorMap tm_q, const SfaArgs a) {
+    pdl_wait();
     extern __shared__ uint8_t smem_raw[];
     SfaSmem &sm = *reinterpret_cast<SfaSmem *>(align1024(smem_raw));
     const PathParams &p = a.p;
@@ -222,6 +172,7 @@ sfa_mma_kernel(const __grid_constant__ CUtensorMap tm_q, const SfaArgs a) {
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    pdl_trigger();  // after the TMEM allocation: a waiting successor holds none
     const uint32_t tmem = sm.tmem_base;
     volatile int *abort_flag = &sm.abort;
     int32_t *status = p.status;
@@ -582,6 +533,8 @@ sfa_mma_kernel(const __grid_constant__ CUtensorMap tm_q, const SfaArgs a) {
 __global__ void __launch_bounds__(128)
 sfa_combine_kernel(const float *__restrict__ o_part, const float *__restrict__ lse_part,
                    int32_t splits, void *out, int32_t out_dtype, float *lse) {
+    pdl_wait();
+    pdl_trigger();
     const int64_t row = blockIdx.x;  // t * 128 + head
     const int64_t t = row >> 7, head = row & 127;
     float m = -INFINITY;
@@ -631,15 +584,18 @@ int32_t sfa_splits(int32_t n_q, int32_t top_k) {
 int32_t sfa_rows_ld(int32_t top_k) { return (int32_t)round_up(top_k > 0 ? top_k : 1, kTile); }
 
 cudaError_t launch_sfa_mma(const PathParams &p, const int32_t *idx, int32_t top_k, int32_t splits,
-                           int32_t *rows, int32_t *n_valid, void *out, int32_t out_dtype,
-                           float *lse, float *o_part, float *lse_part, cudaStream_t s) {
+                           int32_t *rows, int32_t *n_valid, bool rows_ready, void *out,
+                           int32_t out_dtype, float *lse, float *o_part, float *lse_part,
+                           cudaStream_t s) {
     if (p.n_q == 0) return cudaSuccess;
     const int32_t ld_rows = sfa_rows_ld(top_k);
-    count_launch();
-    sfa_rows_kernel<<<static_cast<unsigned>(p.n_q), 128, 0, s>>>(p, idx, top_k, ld_rows, rows,
-                                                                 n_valid);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
+    cudaError_t e;
+    if (!rows_ready) {
+        count_launch();
+        e = launch_pdl(sfa_rows_kernel, dim3(static_cast<unsigned>(p.n_q)), dim3(kRowsThreads), 0,
+                       s, p, idx, top_k, ld_rows, rows, n_valid);
+        if (e != cudaSuccess) return e;
+    }
     CUtensorMap tq;
     if (!encode_tmap_2d(&tq, 2, p.q, kD, (uint64_t)p.n_q * 128, kD * 2, 64, kHeadsCta, true))
         return cudaErrorInvalidValue;
@@ -650,12 +606,13 @@ cudaError_t launch_sfa_mma(const PathParams &p, const int32_t *idx, int32_t top_
     if (e != cudaSuccess) return e;
     const int64_t grid = 2 * (int64_t)p.n_q * splits;
     count_launch();
-    sfa_mma_kernel<<<static_cast<unsigned>(grid), kThreads, smem, s>>>(tq, a);
-    if ((e = cudaGetLastError()) != cudaSuccess || splits == 1) return e;
+    e = launch_pdl(sfa_mma_kernel, dim3(static_cast<unsigned>(grid)), dim3(kThreads), smem, s, tq,
+                   a);
+    if (e != cudaSuccess || splits == 1) return e;
     count_launch();
-    sfa_combine_kernel<<<static_cast<unsigned>(p.n_q * 128), 128, 0, s>>>(o_part, lse_part, splits,
-                                                                         out, out_dtype, lse);
-    return cudaGetLastError();
+    return launch_pdl(sfa_combine_kernel, dim3(static_cast<unsigned>(p.n_q * 128)), dim3(128), 0,
+                      s, (const float *)o_part, (const float *)lse_part, splits, out, out_dtype,
+                      lse);
 }
 
 }  // namespace sa

@@ -161,6 +161,8 @@ __global__ void __launch_bounds__(kThreads)
 topk_rowwise_kernel(const float *__restrict__ scores, int64_t ld,
                     const int32_t *__restrict__ valid_len, int32_t max_valid, const PathParams p,
                     int32_t top_k, int32_t *__restrict__ idx, int32_t *status) {
+    pdl_wait();
+    pdl_trigger();
     const int t = blockIdx.x;
     int32_t V;
     if (valid_len != nullptr) {
@@ -250,6 +252,8 @@ topk_collect_kernel(const float *__restrict__ scores, int64_t ld, const int32_t 
                     const uint32_t *__restrict__ hist, int32_t top_k, int32_t chunk,
                     int32_t *__restrict__ sel, int32_t *__restrict__ counts,
                     uint64_t *__restrict__ cand, int32_t cap) {
+    pdl_wait();
+    pdl_trigger();
     __shared__ int32_t cnt_s[2], base_s[2];
     const int t = blockIdx.y;
     const int32_t V = vis[t];
@@ -318,7 +322,11 @@ __global__ void __launch_bounds__(kThreads)
 topk_finalize_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *__restrict__ vis,
                      int32_t top_k, const int32_t *__restrict__ sel,
                      const int32_t *__restrict__ counts, const uint64_t *__restrict__ cand,
-                     int32_t cap, int32_t bitmap_words, int32_t *__restrict__ idx) {
+                     int32_t cap, int32_t bitmap_words, int32_t *__restrict__ idx,
+                     const PathParams p, int32_t *__restrict__ rows_all, int32_t ld_rows,
+                     int32_t *__restrict__ n_valid_all) {
+    pdl_wait();
+    pdl_trigger();
     extern __shared__ uint64_t fin_smem[];
     __shared__ unsigned hist[256];
     __shared__ int warp_sums[33];
@@ -332,8 +340,16 @@ topk_finalize_kernel(const float *__restrict__ scores, int64_t ld, const int32_t
                       need <= n_cand;
     if (!fits) {
         select_row(scores + (int64_t)t * ld, V, top_k, out);
+        if (rows_all != nullptr) {
+            __syncthreads();
+            compact_rows(p, t, out, top_k, 64, rows_all + (int64_t)t * ld_rows, n_valid_all + t,
+                         warp_sums);
+        }
         return;
     }
+    // physical cache rows for the attention, written beside the positions
+    int32_t *rows = rows_all != nullptr ? rows_all + (int64_t)t * ld_rows : nullptr;
+    const int32_t seq = rows != nullptr ? __ldg(p.q_seq + t) : 0;
     uint64_t *cs = fin_smem;                                       // [cap]
     uint32_t *bits = reinterpret_cast<uint32_t *>(fin_smem + cap);  // [bitmap_words]
     const uint64_t *cg = cand + (int64_t)t * cap;
@@ -406,15 +422,34 @@ topk_finalize_kernel(const float *__restrict__ scores, int64_t ld, const int32_t
     for (int w = w0; w < w1; ++w) cnt += __popc(bits[w]);
     int total;
     int pos = block_exclusive_prefix(cnt, warp_sums, &total);
+    int bad_page = 0;
     for (int w = w0; w < w1; ++w) {
         uint32_t b = bits[w];
         while (b) {
             const int j = __ffs(b) - 1;
             b &= b - 1;
-            if (pos < top_k) out[pos] = w * 32 + j;
+            if (pos < top_k) {
+                const int32_t s = w * 32 + j;
+                out[pos] = s;
+                if (rows != nullptr) {
+                    const int64_t row = phys_row(p.page_table, p.max_pages, p.num_pages, seq, s);
+                    if (row < 0) bad_page = 1;
+                    else rows[pos] = static_cast<int32_t>(row);
+                }
+            }
             ++pos;
         }
     }
+    if (rows == nullptr) return;
+    if (__syncthreads_or(bad_page)) {  // rare: drop (and report) the unmapped rows
+        compact_rows(p, t, out, top_k, 64, rows, n_valid_all + t, warp_sums);
+        return;
+    }
+    const int32_t nv = min(total, top_k);
+    const int32_t padded = (nv + 63) / 64 * 64;
+    if (nv > 0)
+        for (int c = nv + threadIdx.x; c < padded; c += kThreads) rows[c] = rows[0];
+    if (threadIdx.x == 0) n_valid_all[t] = nv;
 }
 
 }  // namespace
@@ -422,14 +457,14 @@ topk_finalize_kernel(const float *__restrict__ scores, int64_t ld, const int32_t
 cudaError_t launch_topk_hist(const float *scores, int64_t ld, const int32_t *vis,
                              const uint32_t *hist, int32_t n_q, int32_t max_valid, int32_t top_k,
                              int32_t *sel, int32_t *counts, uint64_t *cand, int32_t cap,
-                             int32_t *idx, cudaStream_t s) {
+                             int32_t *idx, const PathParams &p, int32_t *rows, int32_t ld_rows,
+                             int32_t *n_valid, cudaStream_t s) {
     if (n_q == 0) return cudaSuccess;
     constexpr int32_t kChunk = 8192;
     const dim3 grid_c(static_cast<unsigned>(ceil_div(std::max(max_valid, 1), kChunk)), n_q);
     count_launch();
-    topk_collect_kernel<<<grid_c, kCollectThreads, 0, s>>>(scores, ld, vis, hist, top_k, kChunk,
-                                                           sel, counts, cand, cap);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(topk_collect_kernel, grid_c, dim3(kCollectThreads), 0, s, scores, ld,
+                               vis, hist, top_k, kChunk, sel, counts, cand, cap);
     if (e != cudaSuccess) return e;
     // candidates plus a bitmap of the longest row, within one CTA's shared memory
     const int32_t words = static_cast<int32_t>(ceil_div(std::max(max_valid, 1), 32));
@@ -440,9 +475,8 @@ cudaError_t launch_topk_hist(const float *scores, int64_t ld, const int32_t *vis
                              (int)smem);
     if (e != cudaSuccess) return e;
     count_launch();
-    topk_finalize_kernel<<<n_q, kThreads, smem, s>>>(scores, ld, vis, top_k, sel, counts, cand,
-                                                      cap, bw, idx);
-    return cudaGetLastError();
+    return launch_pdl(topk_finalize_kernel, dim3(n_q), dim3(kThreads), smem, s, scores, ld, vis,
+                      top_k, sel, counts, cand, cap, bw, idx, p, rows, ld_rows, n_valid);
 }
 
 cudaError_t launch_topk_rowwise(const float *scores, int64_t ld, const int32_t *valid_len,
@@ -452,9 +486,8 @@ cudaError_t launch_topk_rowwise(const float *scores, int64_t ld, const int32_t *
     PathParams pp{};
     if (p != nullptr) pp = *p;
     count_launch();
-    topk_rowwise_kernel<<<n_q, kThreads, 0, s>>>(scores, ld, valid_len, max_valid, pp, top_k,
-                                                 idx, status);
-    return cudaGetLastError();
+    return launch_pdl(topk_rowwise_kernel, dim3(n_q), dim3(kThreads), 0, s, scores, ld, valid_len,
+                      max_valid, pp, top_k, idx, status);
 }
 
 }  // namespace sa
