@@ -452,6 +452,231 @@ topk_finalize_kernel(const float *__restrict__ scores, int64_t ld, const int32_t
     if (threadIdx.x == 0) n_valid_all[t] = nv;
 }
 
+// ---------------------------------------------------------------------------
+// Rows of at most kSingleMaxV positions (decode at up to 64K context): the
+// whole selection in one CTA per query.  One pass over the row (from L2: the
+// indexer has just written it) marks the keys above the threshold bucket in
+// a shared-memory bitmap and collects the bucket's keys; the need-th largest
+// candidate follows from 10-bit radix passes over composite keys (score key,
+// inverted position: distinct, ties to the lower position), normally two;
+// the bitmap is then read back in ascending order.
+// ---------------------------------------------------------------------------
+constexpr int32_t kSingleMaxV = 65536;
+constexpr int32_t kSingleCap = 8192;  // candidates held in shared memory
+constexpr size_t kSingleSmem = (size_t)kSingleCap * 8 + (size_t)kSingleMaxV / 8;
+
+// Writes the selected positions (bits set in `bits`, `words` words) to out in
+// ascending order, -1 after them, and -- when rows != null -- their physical
+// cache rows (compact_rows layout, tile 64) and count.  All threads call it.
+__device__ void emit_selection(const uint32_t *bits, int words, int32_t top_k, int32_t *out,
+                               const PathParams &p, int32_t t, int32_t *rows, int32_t *n_valid,
+                               int *warp_sums) {
+    const int32_t seq = rows != nullptr ? __ldg(p.q_seq + t) : 0;
+    const int per = (words + kThreads - 1) / kThreads;
+    const int w0 = min(words, (int)threadIdx.x * per), w1 = min(words, w0 + per);
+    int cnt = 0;
+    for (int w = w0; w < w1; ++w) cnt += __popc(bits[w]);
+    int total;
+    int pos = block_exclusive_prefix(cnt, warp_sums, &total);
+    int bad_page = 0;
+    for (int w = w0; w < w1; ++w) {
+        uint32_t b = bits[w];
+        while (b) {
+            const int j = __ffs(b) - 1;
+            b &= b - 1;
+            if (pos < top_k) {
+                const int32_t s = w * 32 + j;
+                out[pos] = s;
+                if (rows != nullptr) {
+                    const int64_t row = phys_row(p.page_table, p.max_pages, p.num_pages, seq, s);
+                    if (row < 0) bad_page = 1;
+                    else rows[pos] = static_cast<int32_t>(row);
+                }
+            }
+            ++pos;
+        }
+    }
+    const int32_t nv = min(total, top_k);
+    for (int i = nv + threadIdx.x; i < top_k; i += kThreads) out[i] = -1;
+    if (rows == nullptr) return;
+    if (__syncthreads_or(bad_page)) {  // rare: drop (and report) the unmapped rows
+        compact_rows(p, t, out, top_k, 64, rows, n_valid, warp_sums);
+        return;
+    }
+    const int32_t padded = (nv + 63) / 64 * 64;
+    if (nv > 0)
+        for (int c = nv + threadIdx.x; c < padded; c += kThreads) rows[c] = rows[0];
+    if (threadIdx.x == 0) *n_valid = nv;
+}
+
+__global__ void __launch_bounds__(kThreads)
+topk_single_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *__restrict__ vis,
+                   const uint32_t *__restrict__ hist, int32_t top_k, int32_t *__restrict__ idx,
+                   const PathParams p, int32_t *__restrict__ rows_all, int32_t ld_rows,
+                   int32_t *__restrict__ n_valid_all) {
+    pdl_wait();
+    pdl_trigger();
+    extern __shared__ uint64_t single_smem[];
+    uint64_t *cs = single_smem;                                           // [kSingleCap]
+    uint32_t *bits = reinterpret_cast<uint32_t *>(single_smem + kSingleCap);  // [V / 32]
+    __shared__ unsigned dh[1024];
+    __shared__ int warp_sums[33];
+    __shared__ int n_cand_s, bstar_s, above_s, sel_digit_s, sel_above_s, sel_count_s;
+    const int t = blockIdx.x, tid = threadIdx.x, lane = tid & 31;
+    const int32_t V = vis[t];
+    int32_t *out = idx + (int64_t)t * top_k;
+    int32_t *rows = rows_all != nullptr ? rows_all + (int64_t)t * ld_rows : nullptr;
+    int32_t *nv_out = n_valid_all != nullptr ? n_valid_all + t : nullptr;
+    const int words = (V + 31) / 32;
+    if (V <= top_k) {  // everything visible is selected
+        for (int w = tid; w < words; w += kThreads)
+            bits[w] = (32 * w + 32 <= V) ? 0xFFFFFFFFu : ((1u << (V & 31)) - 1u);
+        __syncthreads();
+        emit_selection(bits, words, top_k, out, p, t, rows, nv_out, warp_sums);
+        return;
+    }
+    // threshold bucket b*: thread i holds the buckets of rank 4i .. 4i+3 from the top
+    const uint32_t *h = hist + (int64_t)t * kHistBins;
+    uint32_t c[4], mine = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        c[j] = h[kHistBins - 1 - 4 * tid - j];
+        mine += c[j];
+    }
+    if (tid == 0) {
+        bstar_s = -1;
+        above_s = 0;
+        n_cand_s = 0;
+    }
+    int tot;
+    int excl = block_exclusive_prefix((int)mine, warp_sums, &tot);
+    if (excl < top_k && excl + (int)mine >= top_k) {
+        int acc = excl;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            if (acc + (int)c[j] >= top_k) {
+                bstar_s = kHistBins - 1 - 4 * tid - j;
+                above_s = acc;
+                break;
+            }
+            acc += c[j];
+        }
+    }
+    for (int w = tid; w < words; w += kThreads) bits[w] = 0;
+    __syncthreads();
+    const int bstar = bstar_s;
+    const int32_t need = top_k - above_s;
+    bool fallback = bstar < 0;
+    if (!fallback) {
+        // one pass over the row: keys above b* into the bitmap, b*'s keys collected
+        const float *row = scores + (int64_t)t * ld;
+        for (int32_t b0 = 0; b0 < V; b0 += 4 * kThreads) {  // same trip count in every lane
+            const int32_t i0 = b0 + 4 * tid;
+            float x[4];
+            if (i0 + 4 <= V) {
+                const float4 v4 = *reinterpret_cast<const float4 *>(row + i0);
+                x[0] = v4.x;
+                x[1] = v4.y;
+                x[2] = v4.z;
+                x[3] = v4.w;
+            } else {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) x[e] = i0 + e < V ? row[i0 + e] : 0.f;
+            }
+            uint32_t above_mask = 0;
+            int n_eq = 0;
+            uint32_t keys[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                keys[e] = order_key(x[e]);
+                const int b = static_cast<int>(keys[e] >> (32 - kHistBits));
+                const bool valid = i0 + e < V;
+                if (valid && b > bstar) above_mask |= 1u << e;
+                if (valid && b == bstar) ++n_eq;
+            }
+            if (above_mask) atomicOr(&bits[i0 >> 5], above_mask << (i0 & 31));
+            // warp-aggregated slots for the bucket's keys
+            int incl = n_eq;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int n = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += n;
+            }
+            int base = 0;
+            if (lane == 31 && incl > 0) base = atomicAdd(&n_cand_s, incl);
+            base = __shfl_sync(0xffffffffu, base, 31) + incl - n_eq;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int b = static_cast<int>(keys[e] >> (32 - kHistBits));
+                if (i0 + e < V && b == bstar) {
+                    if (base < kSingleCap)
+                        cs[base] = (static_cast<uint64_t>(keys[e]) << 32) |
+                                   (0xFFFFFFFFu - static_cast<uint32_t>(i0 + e));
+                    ++base;
+                }
+            }
+        }
+        __syncthreads();
+        fallback = n_cand_s > kSingleCap || need < 1 || need > n_cand_s;
+    }
+    if (fallback) {  // histogram and scores disagree, or too many candidates
+        select_row(scores + (int64_t)t * ld, V, top_k, out);
+        if (rows != nullptr) {
+            __syncthreads();
+            compact_rows(p, t, out, top_k, 64, rows, nv_out, warp_sums);
+        }
+        return;
+    }
+    // the need-th largest composite key among the candidates: digits of 10
+    // bits below the fixed bucket bits, stopping once a whole digit bin is taken
+    const int n_cand = n_cand_s;
+    uint64_t prefix = static_cast<uint64_t>(bstar) << (64 - kHistBits);
+    uint64_t mask = ~0ull << (64 - kHistBits);
+    int remaining = need;
+    int shift = 64 - kHistBits - 10, width = 10;
+    for (;;) {
+        const uint64_t dmask = (1ull << width) - 1;
+        dh[tid] = 0;
+        __syncthreads();
+        for (int i = tid; i < n_cand; i += kThreads) {
+            const uint64_t k = cs[i];
+            if ((k & mask) == prefix) atomicAdd(&dh[(k >> shift) & dmask], 1u);
+        }
+        __syncthreads();
+        const int d = 1023 - tid;  // digits in descending order
+        const int cd = static_cast<int>(dh[d]);
+        const int ex = block_exclusive_prefix(cd, warp_sums, &tot);
+        if (ex < remaining && ex + cd >= remaining) {
+            sel_digit_s = d;
+            sel_above_s = ex;
+            sel_count_s = cd;
+        }
+        __syncthreads();
+        prefix |= static_cast<uint64_t>(sel_digit_s) << shift;
+        mask |= dmask << shift;
+        remaining -= sel_above_s;
+        const bool whole = remaining == sel_count_s;
+        __syncthreads();
+        if (whole || shift == 0) break;
+        if (shift >= 10) {
+            shift -= 10;
+        } else {
+            width = shift;
+            shift = 0;
+        }
+    }
+    // exactly `need` candidates satisfy (k & mask) >= prefix
+    for (int i = tid; i < n_cand; i += kThreads) {
+        const uint64_t k = cs[i];
+        if ((k & mask) >= prefix) {
+            const uint32_t pos = 0xFFFFFFFFu - static_cast<uint32_t>(k);
+            atomicOr(&bits[pos >> 5], 1u << (pos & 31));
+        }
+    }
+    __syncthreads();
+    emit_selection(bits, words, top_k, out, p, t, rows, nv_out, warp_sums);
+}
+
 }  // namespace
 
 cudaError_t launch_topk_hist(const float *scores, int64_t ld, const int32_t *vis,
@@ -460,6 +685,14 @@ cudaError_t launch_topk_hist(const float *scores, int64_t ld, const int32_t *vis
                              int32_t *idx, const PathParams &p, int32_t *rows, int32_t ld_rows,
                              int32_t *n_valid, cudaStream_t s) {
     if (n_q == 0) return cudaSuccess;
+    if (max_valid <= kSingleMaxV) {
+        cudaError_t e = cudaFuncSetAttribute(
+            topk_single_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSingleSmem);
+        if (e != cudaSuccess) return e;
+        count_launch();
+        return launch_pdl(topk_single_kernel, dim3(n_q), dim3(kThreads), kSingleSmem, s, scores,
+                          ld, vis, hist, top_k, idx, p, rows, ld_rows, n_valid);
+    }
     constexpr int32_t kChunk = 8192;
     const dim3 grid_c(static_cast<unsigned>(ceil_div(std::max(max_valid, 1), kChunk)), n_q);
     count_launch();
