@@ -129,6 +129,9 @@ class ClockSampler:
             h = self._handle(nv)
             self.nv, self.h = nv, h
             self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+            # pay the first-query cost of each call before the timed region
+            nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+            nv.nvmlDeviceGetCurrentClocksEventReasons(h)
 
             def poll():
                 while not self.stop:

@@ -55,7 +55,13 @@ constexpr int kHistBits = 12;
 constexpr int kHistBins = 1 << kHistBits;
 
 // ReLU that lets a NaN through, so a poisoned slot stays visible.
-__device__ __forceinline__ float relu_keep_nan(float x) { return x < 0.f ? 0.f : x; }
+// max(x, 0) that keeps NaN (a poisoned key must not turn into a finite
+// score): one max.NaN instruction instead of a compare and a select.
+__device__ __forceinline__ float relu_keep_nan(float x) {
+    float y;
+    asm("max.NaN.f32 %0, %1, 0f00000000;" : "=f"(y) : "f"(x));
+    return y;
+}
 
 // ---------------------------------------------------------------------------
 // Paged addressing: physical row of logical position s of sequence seq, or -1

@@ -24,6 +24,8 @@
 //              bucket in a shared-memory histogram per query, which is added
 //              to the query's global histogram when the CTA leaves the query.
 // Every wait is bounded; a timeout is reported in the workspace status word.
+#include <cstddef>
+
 #include "common.cuh"
 #include "internal.h"
 #include "sm100.cuh"
@@ -35,9 +37,11 @@ using namespace sm100;
 constexpr int kKeys = 128;    // MMA M: keys per tile (two pages)
 constexpr int kHeads = 64;    // MMA N: indexer heads
 constexpr int kDim = 128;     // MMA K: index dimension (bytes of e4m3)
-constexpr int kStages = 4;
-constexpr int kAcc = 2;       // TMEM accumulators (64 columns each)
-constexpr int kThreads = 192;
+constexpr int kStages = 3;
+constexpr int kAcc = 4;       // TMEM accumulators (64 columns each)
+constexpr int kScaleSlots = 8;  // key-scale ring: the epilogue frees these, not the key stages
+constexpr int kEpiGroups = 2;  // epilogue warp groups, alternating tiles
+constexpr int kThreads = 64 + kEpiGroups * 128;
 constexpr uint32_t kPageBytes = 64 * kDim;
 constexpr uint32_t kTileBytes = 2 * kPageBytes;
 constexpr uint32_t kQBytes = kHeads * kDim;
@@ -45,17 +49,24 @@ constexpr uint32_t kTmemCols = kAcc * kHeads;
 
 struct IndexerSmem {
     uint8_t keys[kStages][kTileBytes];  // 1024-byte aligned (128-byte swizzle atoms)
-    uint32_t hist[kHistBins];           // score-key histogram of the current query
-    uint8_t q[2][kQBytes];
-    float kscale[kStages][kKeys];       // per-token key scales of the staged pages
-    int32_t page_ok[kStages][2];        // 1 when the staged page id was valid
-    uint64_t full[kStages], empty[kStages], sc_empty[kStages];
+    uint32_t hist[kEpiGroups][kHistBins];  // score-key histogram of each group's current query
+    uint8_t q[2][kQBytes];                 // 1024-byte aligned like the key stages
+    float wq[kEpiGroups][kHeads];          // head weights x query scales of that query
+    float kscale[kScaleSlots][kKeys];   // per-token key scales of the staged pages
+    int32_t page_ok[kScaleSlots][2];    // 1 when the staged page id was valid
+    uint64_t full[kStages], empty[kStages];
+    uint64_t sc_full[kScaleSlots], sc_empty[kScaleSlots];
     uint64_t acc_full[kAcc], acc_empty[kAcc];
     uint64_t q_full[2], q_empty[2];
     uint64_t done;
     uint32_t tmem_base;
+    int32_t start_t, start_i;           // this CTA's first tile (query, tile in query)
     int abort;
 };
+
+static_assert(offsetof(IndexerSmem, q) % 1024 == 0, "128-byte-swizzled Q tiles need 1024-byte alignment");
+static_assert(offsetof(IndexerSmem, wq) % 16 == 0, "head weights are read as float4");
+static_assert(2 * (sizeof(IndexerSmem) + 2048) <= 233472, "two CTAs per SM");
 
 struct IndexerArgs {
     PathParams p;
@@ -70,19 +81,16 @@ struct IndexerArgs {
 struct TileCursor {
     int64_t k, k_end;
     int32_t t, i, seg;
+    int32_t t_end;  // tile_end[t], loaded once per query
 
-    __device__ void init(const int32_t *tile_end, int32_t n_q, int64_t k0, int64_t k1) {
+    __device__ void init_at(const int32_t *tile_end, int32_t t0, int32_t i0, int64_t k0,
+                            int64_t k1) {
         k = k0;
         k_end = k1;
         seg = 0;
-        int lo = 0, hi = n_q;  // first t with tile_end[t] > k0
-        while (lo < hi) {
-            int mid = (lo + hi) >> 1;
-            if (tile_end[mid] > k0) hi = mid;
-            else lo = mid + 1;
-        }
-        t = lo;
-        i = static_cast<int32_t>(k0 - (lo > 0 ? tile_end[lo - 1] : 0));
+        t = t0;
+        i = i0;
+        t_end = tile_end[t0];
     }
     __device__ bool valid() const { return k < k_end; }
     // Advance one tile; returns true when the next tile starts a new query.
@@ -90,14 +98,14 @@ struct TileCursor {
         ++k;
         ++i;
         if (k >= k_end) return false;
-        bool changed = false;
-        while (k >= tile_end[t]) {
+        if (k < t_end) return false;
+        do {  // skip queries without tiles
             ++t;
-            i = 0;
-            changed = true;
-        }
-        if (changed) ++seg;
-        return changed;
+            t_end = tile_end[t];
+        } while (k >= t_end);
+        i = 0;
+        ++seg;
+        return true;
     }
 };
 
@@ -132,6 +140,9 @@ indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&sm.full[s], 1);
             mbar_init(&sm.empty[s], 1);
+        }
+        for (int s = 0; s < kScaleSlots; ++s) {
+            mbar_init(&sm.sc_full[s], 1);
             mbar_init(&sm.sc_empty[s], 4);
         }
         for (int c = 0; c < kAcc; ++c) {
@@ -146,7 +157,25 @@ indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
         sm.abort = 0;
         fence_barrier_init();
     }
-    if (warp == 0) tmem_alloc(&sm.tmem_base, kTmemCols);
+    if (warp == 0) {
+        // this CTA's first tile: the first query t with tile_end[t] > k0, by a
+        // 32-way search (a few dependent loads instead of a binary search's
+        // dozen), shared with the other roles through shared memory
+        int lo = 0, hi = p.n_q - 1;
+        while (lo < hi) {
+            const int step = (hi - lo + 32) / 32;
+            const int q = min(hi, lo + (lane + 1) * step - 1);
+            const unsigned bal = __ballot_sync(0xffffffffu, a.tile_end[q] > k0);
+            const int j = __ffs(bal) - 1;  // lane 31 probes hi, which qualifies
+            hi = min(hi, lo + (j + 1) * step - 1);
+            lo += j * step;
+        }
+        if (lane == 0) {
+            sm.start_t = lo;
+            sm.start_i = static_cast<int32_t>(k0 - (lo > 0 ? a.tile_end[lo - 1] : 0));
+        }
+        tmem_alloc(&sm.tmem_base, kTmemCols);
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -161,7 +190,7 @@ indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
             // latency overlaps the wait for a free stage instead of sitting
             // between that wait and the TMA copies.
             TileCursor c;
-            c.init(a.tile_end, p.n_q, k0, k1);
+            c.init_at(a.tile_end, sm.start_t, sm.start_i, k0, k1);
             bool seg_start = true;
             int32_t seq = p.q_seq[c.t], V = a.vis[c.t];
             int32_t pg[2];
@@ -197,7 +226,8 @@ indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
                 // the stage is free once its MMAs and its epilogue are done
                 if (!mbar_wait(&sm.empty[stage], ((n / kStages) & 1) ^ 1, abort_flag, p.status))
                     break;
-                if (!mbar_wait(&sm.sc_empty[stage], ((n / kStages) & 1) ^ 1, abort_flag,
+                const int slot = n % kScaleSlots;
+                if (!mbar_wait(&sm.sc_empty[slot], ((n / kScaleSlots) & 1) ^ 1, abort_flag,
                                p.status))
                     break;
                 int32_t rows[2] = {-1, -1};
@@ -207,18 +237,19 @@ indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
                     const int64_t s = (int64_t)c.i * kKeys + 64 * h;
                     if (s < V && pg[h] >= 0 && pg[h] < p.num_pages) {
                         rows[h] = pg[h] * 64;
-                        bytes += kPageBytes + 64 * sizeof(float);
+                        bytes += kPageBytes;
                     }
-                    sm.page_ok[stage][h] = rows[h] >= 0;  // published by the arrive below
+                    sm.page_ok[slot][h] = rows[h] >= 0;  // published by the arrive below
                 }
+                mbar_arrive_expect_tx(&sm.sc_full[slot], (bytes / kPageBytes) * 64 * sizeof(float));
                 mbar_arrive_expect_tx(&sm.full[stage], bytes);
 #pragma unroll
                 for (int h = 0; h < 2; ++h)
                     if (rows[h] >= 0) {
                         tma_load_2d(sm.keys[stage] + h * kPageBytes, &tm_keys, 0, rows[h],
                                     &sm.full[stage]);
-                        bulk_load(&sm.kscale[stage][64 * h], p.k_index_scale + rows[h],
-                                  64 * sizeof(float), &sm.full[stage]);
+                        bulk_load(&sm.kscale[slot][64 * h], p.k_index_scale + rows[h],
+                                  64 * sizeof(float), &sm.sc_full[slot]);
                     }
                 c = nx;
                 seg_start = nx_seg;
@@ -233,7 +264,7 @@ indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
         if (lane == 0) {
             constexpr uint32_t idesc = instr_desc(kKeys, kHeads, 0 /*e4m3*/, 0, 0);
             TileCursor c;
-            c.init(a.tile_end, p.n_q, k0, k1);
+            c.init_at(a.tile_end, sm.start_t, sm.start_i, k0, k1);
             bool seg_start = true;
             for (int n = 0; c.valid(); ++n) {
                 if (seg_start) {
@@ -262,53 +293,62 @@ indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
         }
     } else {
         // --------------------------------------------------- epilogue ---
-        // The loop never leaves early: after a failed (timed-out) wait it
-        // carries on without waiting, so the four warps meet at the same
-        // named barriers when they flush the histogram.
-        const int quad = warp & 3;             // TMEM lanes this warp may read
-        const int row = quad * 32 + lane;      // key row of the tile
-        const int et = threadIdx.x - 64;       // 0..127 over the epilogue warps
+        // Two groups of four warps take alternate tiles, so two tiles' chains
+        // (scale wait, accumulator wait, TMEM loads, weighted ReLU sum, score
+        // store, histogram) run side by side.  Within a group, warp w reads
+        // TMEM lanes 32 (w % 4) .. +31: one key row per thread.  The loop
+        // never leaves early: after a failed (timed-out) wait it carries on
+        // without waiting, so a group's warps meet at the same named barriers.
+        const int g = (warp - 2) >> 2;          // epilogue group
+        const int quad = warp & 3;              // TMEM lanes this warp may read
+        const int row = quad * 32 + lane;       // key row of the tile
+        const int et = threadIdx.x - 64 - 128 * g;  // 0..127 within the group
+        const int bar = 1 + g;                  // the group's named barrier
         const bool histo = a.hist != nullptr;
+        uint32_t *hist = sm.hist[g];
+        float *wq = sm.wq[g];
         if (histo) {
-            for (int b = et; b < kHistBins; b += 128) sm.hist[b] = 0;
-            named_barrier(1, 128);
+            for (int b = et; b < kHistBins; b += 128) hist[b] = 0;
+            named_barrier(bar, 128);
         }
-        // add this CTA's counts of query t to the global histogram, then clear
+        // add this group's counts of query t to the global histogram, then clear
         auto flush = [&](int32_t t) {
-            named_barrier(1, 128);
-            uint32_t *g = a.hist + (int64_t)t * kHistBins;
+            named_barrier(bar, 128);
+            uint32_t *gh = a.hist + (int64_t)t * kHistBins;
             for (int b = et; b < kHistBins; b += 128) {
-                const uint32_t v = sm.hist[b];
+                const uint32_t v = hist[b];
                 if (v != 0) {
-                    atomicAdd(g + b, v);
-                    sm.hist[b] = 0;
+                    atomicAdd(gh + b, v);
+                    hist[b] = 0;
                 }
             }
-            named_barrier(1, 128);
+            named_barrier(bar, 128);
         };
         TileCursor c;
-        c.init(a.tile_end, p.n_q, k0, k1);
-        bool seg_start = true, ok = true;
+        c.init_at(a.tile_end, sm.start_t, sm.start_i, k0, k1);
+        bool ok = true;
         int32_t V = 0, t_cur = -1;
-        float wq[kHeads];
-        for (int n = 0; c.valid(); ++n) {
-            if (seg_start) {
+        for (int n = 0; c.valid(); ++n, c.next(a.tile_end)) {
+            if ((n & 1) != g) continue;
+            if (c.t != t_cur) {  // this group's first tile of a query
                 if (histo && t_cur >= 0) flush(t_cur);
+                named_barrier(bar, 128);  // the old weights are no longer read
                 t_cur = c.t;
                 V = a.vis[c.t];
-                const float *w = p.w + (int64_t)c.t * kHeads;
-                const float *qs = p.q_index_scale + (int64_t)c.t * kHeads;
-#pragma unroll
-                for (int j = 0; j < kHeads; ++j) wq[j] = __ldg(w + j) * __ldg(qs + j);
+                if (et < kHeads)
+                    wq[et] = __ldg(p.w + (int64_t)c.t * kHeads + et) *
+                             __ldg(p.q_index_scale + (int64_t)c.t * kHeads + et);
+                named_barrier(bar, 128);
             }
             const int64_t s = (int64_t)c.i * kKeys + row;
-            const int stage = n % kStages;
-            // key scales and page validity arrive with the key pages
-            if (ok) ok = warp_wait(&sm.full[stage], (n / kStages) & 1, abort_flag, p.status);
-            const bool page_ok = ok && sm.page_ok[stage][row >> 6] != 0;
-            const float kscale = ok ? sm.kscale[stage][row] : 0.f;
+            // key scales and page validity have a ring of their own
+            const int slot = n % kScaleSlots;
+            if (ok)
+                ok = warp_wait(&sm.sc_full[slot], (n / kScaleSlots) & 1, abort_flag, p.status);
+            const bool page_ok = ok && sm.page_ok[slot][row >> 6] != 0;
+            const float kscale = ok ? sm.kscale[slot][row] : 0.f;
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.sc_empty[stage]);
+            if (lane == 0) mbar_arrive(&sm.sc_empty[slot]);
             if (ok && s < V && !page_ok) report(p.status, SA_ERR_DEVICE_FAULT, SA_DETAIL_BAD_PAGE);
             const int acc = n % kAcc;
             if (ok) ok = warp_wait(&sm.acc_full[acc], (n / kAcc) & 1, abort_flag, p.status);
@@ -317,15 +357,25 @@ indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
                 tc_fence_after();
                 const uint32_t taddr =
                     tmem + (static_cast<uint32_t>(quad * 32) << 16) + acc * kHeads;
-                float v[32];
+                float v[32], u[32];
                 tmem_ld32(taddr, v);
+                tmem_ld32(taddr + 32, u);
                 tmem_wait_ld();
+                const float4 *w4 = reinterpret_cast<const float4 *>(wq);
+                float part[4] = {0.f, 0.f, 0.f, 0.f};  // four independent chains
 #pragma unroll
-                for (int j = 0; j < 32; ++j) sum = fmaf(wq[j], relu_keep_nan(v[j]), sum);
-                tmem_ld32(taddr + 32, v);
-                tmem_wait_ld();
-#pragma unroll
-                for (int j = 0; j < 32; ++j) sum = fmaf(wq[32 + j], relu_keep_nan(v[j]), sum);
+                for (int j4 = 0; j4 < 8; ++j4) {
+                    const float4 wa = w4[j4], wb = w4[8 + j4];
+                    part[0] = fmaf(wa.x, relu_keep_nan(v[4 * j4]), part[0]);
+                    part[1] = fmaf(wa.y, relu_keep_nan(v[4 * j4 + 1]), part[1]);
+                    part[2] = fmaf(wa.z, relu_keep_nan(v[4 * j4 + 2]), part[2]);
+                    part[3] = fmaf(wa.w, relu_keep_nan(v[4 * j4 + 3]), part[3]);
+                    part[0] = fmaf(wb.x, relu_keep_nan(u[4 * j4]), part[0]);
+                    part[1] = fmaf(wb.y, relu_keep_nan(u[4 * j4 + 1]), part[1]);
+                    part[2] = fmaf(wb.z, relu_keep_nan(u[4 * j4 + 2]), part[2]);
+                    part[3] = fmaf(wb.w, relu_keep_nan(u[4 * j4 + 3]), part[3]);
+                }
+                sum = (part[0] + part[1]) + (part[2] + part[3]);
             }
             tc_fence_before();
             __syncwarp();
@@ -333,9 +383,8 @@ indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
             if (s < V) {
                 const float score = page_ok ? sum * kscale : -INFINITY;
                 a.scores[(int64_t)c.t * a.ld + s] = score;
-                if (histo) atomicAdd(&sm.hist[order_key(score) >> (32 - kHistBits)], 1u);
+                if (histo) atomicAdd(&hist[order_key(score) >> (32 - kHistBits)], 1u);
             }
-            seg_start = c.next(a.tile_end);
         }
         if (histo && t_cur >= 0) flush(t_cur);
     }
