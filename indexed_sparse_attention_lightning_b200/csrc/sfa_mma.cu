@@ -95,6 +95,7 @@ struct SfaArgs {
     const int32_t *n_valid;  // [n_q]
     int32_t ld_rows;
     int32_t splits;
+    int32_t fp8;             // e4m3 latent + fp32 page scale + bf16 rope (else bf16 rows)
     void *out;               // [n_q, 128, 512] (splits == 1)
     int32_t out_dtype;
     float *lse;              // [n_q, 128] or null (splits == 1)
@@ -411,13 +412,22 @@ sfa_mma_kernel(const __grid_constant__ CUtensorMap tm_q, const SfaArgs a) {
         const int pk = pw * 32 + lane;  // key prefetched by this thread
         const bool prefetcher = pk < kTile;
         const int32_t *tile_rows = rows + (int64_t)j0 * kTile;
+        const uint8_t *rope = static_cast<const uint8_t *>(p.kv_rope);
+        auto prefetch_row = [&](int32_t r) {
+            if (a.fp8) {
+                prefetch_l2(kv + (int64_t)r * kDl, kDl);
+                prefetch_l2(rope + (int64_t)r * (kDr * 2), kDr * 2);
+            } else {
+                prefetch_l2(kv + (int64_t)r * (kD * 2), kD * 2);
+            }
+        };
         if (prefetcher) {
             int32_t r0[kPrefetch];
 #pragma unroll
             for (int n = 0; n < kPrefetch; ++n) r0[n] = n < T ? __ldg(tile_rows + n * kTile + pk) : 0;
 #pragma unroll
             for (int n = 0; n < kPrefetch; ++n)
-                if (n < T) prefetch_l2(kv + (int64_t)r0[n] * (kD * 2), kD * 2);
+                if (n < T) prefetch_row(r0[n]);
         }
         int32_t pf_row =
             (prefetcher && kPrefetch < T) ? __ldg(tile_rows + kPrefetch * kTile + pk) : 0;
@@ -425,7 +435,7 @@ sfa_mma_kernel(const __grid_constant__ CUtensorMap tm_q, const SfaArgs a) {
         int32_t r_hi = T > 0 ? __ldg(tile_rows + 32 + lane) : 0;
         for (int n = 0; n < T; ++n) {
             const int st = n % kStages;
-            if (prefetcher && n + kPrefetch < T) prefetch_l2(kv + (int64_t)pf_row * (kD * 2), kD * 2);
+            if (prefetcher && n + kPrefetch < T) prefetch_row(pf_row);
             const bool more = n + 1 < T;
             const int32_t pf_next = (prefetcher && n + 1 + kPrefetch < T)
                                         ? __ldg(tile_rows + (n + 1 + kPrefetch) * kTile + pk)
@@ -434,21 +444,57 @@ sfa_mma_kernel(const __grid_constant__ CUtensorMap tm_q, const SfaArgs a) {
             const int32_t hi_next = more ? __ldg(tile_rows + (n + 1) * kTile + 32 + lane) : 0;
             if (!warp_wait(&sm.kv_empty[st], ((n / kStages) & 1) ^ 1, abort_flag, status)) break;
             if (n == 2 && !warp_wait(&sm.q_ready, 0, abort_flag, status)) break;
-            const uint32_t dst0 = smem_u32(sm.kv[st]);
+            if (!a.fp8) {
+                const uint32_t dst0 = smem_u32(sm.kv[st]);
 #pragma unroll 2
-            for (int k = pw; k < kTile; k += kProducerWarps) {
-                const int32_t r = __shfl_sync(0xffffffffu, k < 32 ? r_lo : r_hi, k & 31);
-                const uint8_t *src = kv + (int64_t)r * (kD * 2);
-                const uint32_t dk = dst0 + (k >> 3) * kGroupBytes + (k & 7) * 128;
-                const int sw = k & 7;
+                for (int k = pw; k < kTile; k += kProducerWarps) {
+                    const int32_t r = __shfl_sync(0xffffffffu, k < 32 ? r_lo : r_hi, k & 31);
+                    const uint8_t *src = kv + (int64_t)r * (kD * 2);
+                    const uint32_t dk = dst0 + (k >> 3) * kGroupBytes + (k & 7) * 128;
+                    const int sw = k & 7;
 #pragma unroll
-                for (int i = 0; i < 3; ++i) {
-                    const int c = lane + 32 * i;
-                    if (c < kChunksPerRow)
-                        cp_async16(dk + (c >> 3) * 1024 + (((c & 7) ^ sw) << 4), src + c * 16);
+                    for (int i = 0; i < 3; ++i) {
+                        const int c = lane + 32 * i;
+                        if (c < kChunksPerRow)
+                            cp_async16(dk + (c >> 3) * 1024 + (((c & 7) ^ sw) << 4), src + c * 16);
+                    }
                 }
+                cp_async_arrive(&sm.kv_full[st]);
+            } else {
+                // e4m3 latent: lane c dequantises dims 16c .. 16c + 15 of a row
+                // (x its page's scale, rounded to bf16) into the same swizzled
+                // layout; lanes 0-7 copy the bf16 rope.  Plain stores, so a
+                // proxy fence and an ordinary arrive publish them.
+                uint8_t *stage = sm.kv[st];
+#pragma unroll 2
+                for (int k = pw; k < kTile; k += kProducerWarps) {
+                    const int32_t r = __shfl_sync(0xffffffffu, k < 32 ? r_lo : r_hi, k & 31);
+                    const float sc = __ldg(p.kv_scale + (r >> 6));
+                    const uint4 x = __ldg(reinterpret_cast<const uint4 *>(kv + (int64_t)r * kDl) + lane);
+                    uint4 rp = make_uint4(0, 0, 0, 0);
+                    if (lane < 8)
+                        rp = __ldg(reinterpret_cast<const uint4 *>(rope + (int64_t)r * (kDr * 2)) + lane);
+                    const uint32_t xw[4] = {x.x, x.y, x.z, x.w};
+                    uint32_t o[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const uint16_t two = static_cast<uint16_t>(xw[i >> 1] >> (16 * (i & 1)));
+                        const float2 f = e4m3x2_to_float2(two);
+                        __nv_bfloat162 b2 = __floats2bfloat162_rn(f.x * sc, f.y * sc);
+                        o[i] = *reinterpret_cast<uint32_t *>(&b2);
+                    }
+                    uint8_t *dk = stage + (k >> 3) * kGroupBytes + (k & 7) * 128;
+                    const int sw = k & 7, b = lane >> 2, c0 = 2 * (lane & 3);
+                    *reinterpret_cast<uint4 *>(dk + b * 1024 + ((c0 ^ sw) << 4)) =
+                        make_uint4(o[0], o[1], o[2], o[3]);
+                    *reinterpret_cast<uint4 *>(dk + b * 1024 + (((c0 + 1) ^ sw) << 4)) =
+                        make_uint4(o[4], o[5], o[6], o[7]);
+                    if (lane < 8)
+                        *reinterpret_cast<uint4 *>(dk + 8 * 1024 + ((lane ^ sw) << 4)) = rp;
+                }
+                fence_proxy_async_smem();
+                mbar_arrive(&sm.kv_full[st]);
             }
-            cp_async_arrive(&sm.kv_full[st]);
             pf_row = pf_next;
             r_lo = lo_next;
             r_hi = hi_next;
@@ -569,7 +615,9 @@ sfa_combine_kernel(const float *__restrict__ o_part, const float *__restrict__ l
 }  // namespace
 
 bool sfa_mma_supported(const PathParams &p, int32_t top_k) {
-    return p.kv_dtype == SA_BF16 && p.q_dtype == SA_BF16 && p.heads == 128 &&
+    const bool kv_ok = p.kv_dtype == SA_BF16 ||
+                       (p.kv_dtype == SA_E4M3 && p.kv_rope != nullptr && p.kv_scale != nullptr);
+    return kv_ok && p.q_dtype == SA_BF16 && p.heads == 128 &&
            p.d_latent == kDl && p.d_rope == kDr && top_k <= kMaxK &&
            (int64_t)p.num_pages * 64 < (int64_t(1) << 31);
 }
@@ -599,7 +647,8 @@ cudaError_t launch_sfa_mma(const PathParams &p, const int32_t *idx, int32_t top_
     CUtensorMap tq;
     if (!encode_tmap_2d(&tq, 2, p.q, kD, (uint64_t)p.n_q * 128, kD * 2, 64, kHeadsCta, true))
         return cudaErrorInvalidValue;
-    SfaArgs a{p, rows, n_valid, ld_rows, splits, out, out_dtype, lse, o_part, lse_part};
+    SfaArgs a{p,         rows,   n_valid,  ld_rows,  splits, p.kv_dtype == SA_E4M3,
+              out,       out_dtype, lse,    o_part,   lse_part};
     const size_t smem = sizeof(SfaSmem) + 1024;
     e = cudaFuncSetAttribute(sfa_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem);
