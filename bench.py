@@ -351,9 +351,11 @@ def run_ours(args, rank: int, world: int, dist):
     dom_bytes = nbytes[dom_name]
     achieved = dom_bytes / (phase_ms[dom] / 1e3) / 1e9 if phase_ms[dom] > 0 else 0.0
     step_gbs = nbytes["total"] / (ms_per_step / 1e3) / 1e9
-    kernel_src = {"indexer": ["indexed_sparse_attention_lightning_b200/csrc/indexer_simt.cu"],
-                  "topk": ["indexed_sparse_attention_lightning_b200/csrc/topk.cu"],
-                  "attention": ["indexed_sparse_attention_lightning_b200/csrc/attn_simt.cu"]}
+    csrc = "indexed_sparse_attention_lightning_b200/csrc/"
+    shared = [csrc + f for f in ("common.cuh", "sm100.cuh", "internal.h")]
+    kernel_src = {"indexer": [csrc + "indexer_mma.cu", csrc + "plan.cu"] + shared,
+                  "topk": [csrc + "topk.cu"] + shared,
+                  "attention": [csrc + "sfa_mma.cu"] + shared}
     traffic = traffic_for(dom_name, kernel_src[dom_name])
 
     cpu = None

@@ -84,9 +84,10 @@ bool encode_tmap_2d(CUtensorMap *map, int dtype_bytes, const void *base, uint64_
 
 // ---- launchers (each returns the launch error, if any) --------------------
 // Visible length per query and the inclusive prefix of ceil(V / tile); also
-// zeroes `zero_words` 32-bit words at `zero` (histograms and counters).
+// zeroes `zero_words` 32-bit words at `zero` (histograms and counters) and,
+// with `clear_status`, the status word before anything can report into it.
 cudaError_t launch_plan(const PathParams &p, int32_t *vis, int32_t *tile_end, int32_t tile,
-                        uint32_t *zero, size_t zero_words, cudaStream_t s);
+                        uint32_t *zero, size_t zero_words, bool clear_status, cudaStream_t s);
 
 cudaError_t launch_indexer_simt(const PathParams &p, float *scores, int64_t ld, cudaStream_t s);
 

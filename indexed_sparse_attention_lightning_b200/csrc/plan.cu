@@ -12,13 +12,16 @@ constexpr int kThreads = 1024;
 
 __global__ void __launch_bounds__(kThreads)
 plan_kernel(const PathParams p, int32_t *vis, int32_t *tile_end, int32_t tile, uint32_t *zero,
-            size_t zero_words) {
+            size_t zero_words, int32_t clear_status) {
     pdl_wait();
     pdl_trigger();
+    // CTA 0 is the only one that reports, so it clears the status word first
+    if (clear_status && blockIdx.x == 0 && threadIdx.x < kStatusBytes / 4) p.status[threadIdx.x] = 0;
     for (size_t i = (size_t)blockIdx.x * kThreads + threadIdx.x; i < zero_words;
          i += (size_t)gridDim.x * kThreads)
         zero[i] = 0u;
     if (blockIdx.x != 0) return;
+    __syncthreads();
     __shared__ int32_t warp_sums[32];
     __shared__ int32_t carry;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -60,13 +63,13 @@ plan_kernel(const PathParams p, int32_t *vis, int32_t *tile_end, int32_t tile, u
 }  // namespace
 
 cudaError_t launch_plan(const PathParams &p, int32_t *vis, int32_t *tile_end, int32_t tile,
-                        uint32_t *zero, size_t zero_words, cudaStream_t s) {
+                        uint32_t *zero, size_t zero_words, bool clear_status, cudaStream_t s) {
     if (p.n_q == 0) return cudaSuccess;
     const int64_t blocks =
         std::max<int64_t>(1, std::min<int64_t>(num_sms(), ceil_div(zero_words, 4 * kThreads)));
     count_launch();
     return launch_pdl(plan_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kThreads), 0, s, p,
-                      vis, tile_end, tile, zero, zero_words);
+                      vis, tile_end, tile, zero, zero_words, clear_status ? 1 : 0);
 }
 
 int num_sms() {

@@ -175,8 +175,12 @@ sa_status run_attention(const PathParams &p, const Layout &l, bool fused, bool r
 // tensor-core kernel also fills the per-query score histograms, which the
 // plan kernel clears first together with the counters behind them;
 // *have_hist reports whether they were built.
+sa_status clear_status(void *ws, cudaStream_t s);
+
+// With `clear`, the status word is cleared first: by the plan kernel when
+// there is one (saving a separate memset in front of it), else by a memset.
 sa_status run_indexer(const PathParams &p, const Layout &l, void *ws, float *scores, int64_t ld,
-                      bool want_hist, bool *have_hist, cudaStream_t s) {
+                      bool want_hist, bool clear, bool *have_hist, cudaStream_t s) {
     *have_hist = false;
     if (indexer_mma_supported(p)) {
         char *base = static_cast<char *>(ws);
@@ -184,11 +188,16 @@ sa_status run_indexer(const PathParams &p, const Layout &l, void *ws, float *sco
         int32_t *tile_end = reinterpret_cast<int32_t *>(base + l.tile_end);
         uint32_t *hist = want_hist ? reinterpret_cast<uint32_t *>(base + l.hist) : nullptr;
         const size_t zero_words = want_hist ? (l.sel - l.hist) / 4 : 0;
-        sa_status st = cuda_status(launch_plan(p, vis, tile_end, 128, hist, zero_words, s));
+        sa_status st =
+            cuda_status(launch_plan(p, vis, tile_end, 128, hist, zero_words, clear, s));
         if (st != SA_OK) return st;
         st = cuda_status(launch_indexer_mma(p, vis, tile_end, scores, ld, hist, s));
         *have_hist = want_hist && st == SA_OK;
         return st;
+    }
+    if (clear) {
+        const sa_status st = clear_status(ws, s);
+        if (st != SA_OK) return st;
     }
     return cuda_status(launch_indexer_simt(p, scores, ld, s));
 }
@@ -237,7 +246,7 @@ sa_status sa_indexer_score(const sa_cache *cache, const sa_query *query, float *
     if (query->n_q == 0) return SA_OK;
     PathParams p = make_params(cache, query, workspace);
     bool have_hist;
-    return run_indexer(p, l, workspace, scores, ld_scores, false, &have_hist, s);
+    return run_indexer(p, l, workspace, scores, ld_scores, false, false, &have_hist, s);
 }
 
 sa_status sa_topk(const float *scores, int64_t ld_scores, const int32_t *valid_len, int32_t n_q,
@@ -290,7 +299,7 @@ static sa_status decode_impl(const sa_cache *cache, const sa_query *query, int32
         if (events == nullptr) return SA_OK;
         return cuda_status(cudaEventRecord(static_cast<cudaEvent_t>(events[i]), s));
     };
-    if ((st = clear_status(workspace, s)) != SA_OK) return st;
+    if (query->n_q == 0 && (st = clear_status(workspace, s)) != SA_OK) return st;
     if ((st = mark(0)) != SA_OK) return st;
     if (query->n_q > 0) {
         PathParams p = make_params(cache, query, workspace);
@@ -298,7 +307,7 @@ static sa_status decode_impl(const sa_cache *cache, const sa_query *query, int32
         float *scores = reinterpret_cast<float *>(base + l.scores);
         int32_t *idx = idx_out ? idx_out : reinterpret_cast<int32_t *>(base + l.idx);
         bool have_hist = false;
-        if ((st = run_indexer(p, l, workspace, scores, l.ld, true, &have_hist, s)) != SA_OK)
+        if ((st = run_indexer(p, l, workspace, scores, l.ld, true, true, &have_hist, s)) != SA_OK)
             return st;
         if ((st = mark(1)) != SA_OK) return st;
         // the top-K kernel also emits the physical rows for the tensor-core attention

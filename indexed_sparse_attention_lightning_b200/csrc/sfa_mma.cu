@@ -23,7 +23,8 @@
 // operand of S and, read MN-major, the B operand of P V.
 //
 // Roles (384 threads, one CTA per SM):
-//   warp 0     lane 0 loads Q by TMA (into the third ring stage), then issues
+//   warp 0     lane 0 loads Q by TMA (into the third ring stage; this copy
+//              starts before the wait on the top-K kernel), then issues
 //              the MMAs from a non-blocking loop -- S of a tile as soon as its
 //              rows are in and an S buffer is free, P V as soon as P is
 //              written -- and commits them to mbarriers;
@@ -147,7 +148,6 @@ sfa_rows_kernel(const PathParams p, const int32_t *__restrict__ idx, int32_t K, 
 
 __global__ void __launch_bounds__(kThreads, 1)
 sfa_mma_kernel(const __grid_constant__ CUtensorMap tm_q, const SfaArgs a) {
-    pdl_wait();
     extern __shared__ uint8_t smem_raw[];
     SfaSmem &sm = *reinterpret_cast<SfaSmem *>(align1024(smem_raw));
     const PathParams &p = a.p;
@@ -174,6 +174,15 @@ sfa_mma_kernel(const __grid_constant__ CUtensorMap tm_q, const SfaArgs a) {
     __syncthreads();
     tc_fence_after();
     pdl_trigger();  // after the TMEM allocation: a waiting successor holds none
+    // Q is an input, not the previous kernel's output: its copy (into ring
+    // stage 2) starts before the wait on that kernel
+    if (warp == 0 && lane == 0) {
+        mbar_arrive_expect_tx(&sm.q_full, kBlocks * kHeadsCta * 128);
+        for (int b = 0; b < kBlocks; ++b)
+            tma_load_2d(sm.kv[2] + b * (kHeadsCta * 128), &tm_q, 64 * b, t * 128 + kHeadsCta * hh,
+                        &sm.q_full);
+    }
+    pdl_wait();  // the selected rows come from the top-K kernel
     const uint32_t tmem = sm.tmem_base;
     volatile int *abort_flag = &sm.abort;
     int32_t *status = p.status;
@@ -501,11 +510,7 @@ sfa_mma_kernel(const __grid_constant__ CUtensorMap tm_q, const SfaArgs a) {
         }
         cp_async_wait_all();
     } else if (lane == 0 && T > 0) {
-        // ------------------------------------------ Q load, MMA issuer ---
-        mbar_arrive_expect_tx(&sm.q_full, kBlocks * kHeadsCta * 128);
-        for (int b = 0; b < kBlocks; ++b)
-            tma_load_2d(sm.kv[2] + b * (kHeadsCta * 128), &tm_q, 64 * b, t * 128 + kHeadsCta * hh,
-                        &sm.q_full);
+        // ------------------------------------------------- MMA issuer ---
         constexpr uint32_t id_s = instr_desc(64, kTile, 1 /*bf16*/, 0, 0);
         constexpr uint32_t id_pv = instr_desc(64, 256, 1 /*bf16*/, 0, 1);
         bool ok = mbar_wait(&sm.q_ready, 0, abort_flag, status);
@@ -566,6 +571,8 @@ sfa_mma_kernel(const __grid_constant__ CUtensorMap tm_q, const SfaArgs a) {
             }
         }
     }
+    // with no tiles nobody waited for Q: its copy must land before the CTA ends
+    if (warp == 0 && lane == 0 && T == 0) mbar_wait(&sm.q_full, 0, abort_flag, status);
     __syncwarp();
     tc_fence_before();
     __syncthreads();

@@ -102,12 +102,20 @@ DECODE_B2_1M_FP8KV = WorkloadSpec(
 CONFIGS = (TINY, DECODE_B8_8K, DECODE_B64_16K_32K, PREFILL_4096Q_64K,
            DECODE_B2_1M_FP8KV)
 
+# A smaller decode case for full profiler captures: the same kernels and
+# per-query work as the 64-sequence decode, at a fixed 16K context (138 MB of
+# index keys, more than L2; about 1.7 GB on the device).
+PROFILE_B64_16K = WorkloadSpec(
+    name="profile_decode_b64_16k", seed=3, batch=64, seq_len=("fixed", 16384))
+
+EXTRA = (PROFILE_B64_16K,)
+
 
 def spec(which) -> WorkloadSpec:
     """Look a spec up by index (0..4) or by name."""
     if isinstance(which, int):
         return CONFIGS[which]
-    for s in CONFIGS:
+    for s in CONFIGS + EXTRA:
         if s.name == which:
             return s
     raise KeyError(which)
