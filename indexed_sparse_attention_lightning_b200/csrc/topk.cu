@@ -314,6 +314,68 @@ topk_collect_kernel(const float *__restrict__ scores, int64_t ld, const int32_t 
     }
 }
 
+// Writes the selected positions (bits set in `bits`, `words` words) to out in
+// ascending order, -1 after them, and -- when rows != null -- their physical
+// cache rows (compact_rows layout, tile 64) and count.  Positions first (each
+// thread owns a run of words; selected keys may crowd into a few runs), then
+// the rows in a second pass spread evenly over the threads, so no thread
+// serialises many page-table loads.  All threads call it.
+__device__ void emit_selection(const uint32_t *bits, int words, int32_t top_k, int32_t *out,
+                               const PathParams &p, int32_t t, int32_t *rows, int32_t *n_valid,
+                               int *warp_sums) {
+    // each warp owns a run of words and walks it 32 words at a time, one
+    // word per lane, so a run dense with selected keys is shared by 32 lanes
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    constexpr int kWarps = kThreads / 32;
+    const int per = (words + kWarps - 1) / kWarps;
+    const int w0 = min(words, warp * per), w1 = min(words, w0 + per);
+    int cnt = 0;
+    for (int w = w0 + lane; w < w1; w += 32) cnt += __popc(bits[w]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+    int total;
+    int pos = block_exclusive_prefix(lane == 0 ? cnt : 0, warp_sums, &total);
+    pos = __shfl_sync(0xffffffffu, pos, 0);  // the warp's first slot
+    for (int c0 = w0; c0 < w1; c0 += 32) {
+        const int w = c0 + lane;
+        uint32_t b = w < w1 ? bits[w] : 0u;
+        const int c = __popc(b);
+        int incl = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        int q = pos + incl - c;
+        while (b) {
+            const int j = __ffs(b) - 1;
+            b &= b - 1;
+            if (q < top_k) out[q] = w * 32 + j;
+            ++q;
+        }
+        pos += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    const int32_t nv = min(total, top_k);
+    for (int i = nv + threadIdx.x; i < top_k; i += kThreads) out[i] = -1;
+    if (rows == nullptr) return;
+    __syncthreads();  // the positions are visible to the whole block
+    const int32_t seq = __ldg(p.q_seq + t);
+    int bad_page = 0;
+    for (int i = threadIdx.x; i < nv; i += kThreads) {
+        const int64_t row = phys_row(p.page_table, p.max_pages, p.num_pages, seq, out[i]);
+        if (row < 0) bad_page = 1;
+        else rows[i] = static_cast<int32_t>(row);
+    }
+    if (__syncthreads_or(bad_page)) {  // rare: drop (and report) the unmapped rows
+        compact_rows(p, t, out, top_k, 64, rows, n_valid, warp_sums);
+        return;
+    }
+    const int32_t padded = (nv + 63) / 64 * 64;
+    if (nv > 0)
+        for (int c = nv + threadIdx.x; c < padded; c += kThreads) rows[c] = rows[0];
+    if (threadIdx.x == 0) *n_valid = nv;
+}
+
 // One CTA per query: exact order inside the threshold bucket, then every
 // selected position set in a bitmap and read back in ascending order.  Rows
 // the candidate buffer or the bitmap cannot hold (massive exact ties, very
@@ -347,9 +409,7 @@ topk_finalize_kernel(const float *__restrict__ scores, int64_t ld, const int32_t
         }
         return;
     }
-    // physical cache rows for the attention, written beside the positions
     int32_t *rows = rows_all != nullptr ? rows_all + (int64_t)t * ld_rows : nullptr;
-    const int32_t seq = rows != nullptr ? __ldg(p.q_seq + t) : 0;
     uint64_t *cs = fin_smem;                                       // [cap]
     uint32_t *bits = reinterpret_cast<uint32_t *>(fin_smem + cap);  // [bitmap_words]
     const uint64_t *cg = cand + (int64_t)t * cap;
@@ -415,41 +475,8 @@ topk_finalize_kernel(const float *__restrict__ scores, int64_t ld, const int32_t
         atomicOr(&bits[pos >> 5], 1u << (pos & 31));
     }
     __syncthreads();
-    // ascending order: each thread owns a contiguous run of words
-    const int per = (words + kThreads - 1) / kThreads;
-    const int w0 = min(words, threadIdx.x * per), w1 = min(words, w0 + per);
-    int cnt = 0;
-    for (int w = w0; w < w1; ++w) cnt += __popc(bits[w]);
-    int total;
-    int pos = block_exclusive_prefix(cnt, warp_sums, &total);
-    int bad_page = 0;
-    for (int w = w0; w < w1; ++w) {
-        uint32_t b = bits[w];
-        while (b) {
-            const int j = __ffs(b) - 1;
-            b &= b - 1;
-            if (pos < top_k) {
-                const int32_t s = w * 32 + j;
-                out[pos] = s;
-                if (rows != nullptr) {
-                    const int64_t row = phys_row(p.page_table, p.max_pages, p.num_pages, seq, s);
-                    if (row < 0) bad_page = 1;
-                    else rows[pos] = static_cast<int32_t>(row);
-                }
-            }
-            ++pos;
-        }
-    }
-    if (rows == nullptr) return;
-    if (__syncthreads_or(bad_page)) {  // rare: drop (and report) the unmapped rows
-        compact_rows(p, t, out, top_k, 64, rows, n_valid_all + t, warp_sums);
-        return;
-    }
-    const int32_t nv = min(total, top_k);
-    const int32_t padded = (nv + 63) / 64 * 64;
-    if (nv > 0)
-        for (int c = nv + threadIdx.x; c < padded; c += kThreads) rows[c] = rows[0];
-    if (threadIdx.x == 0) n_valid_all[t] = nv;
+    emit_selection(bits, words, top_k, out, p, t, rows,
+                   n_valid_all != nullptr ? n_valid_all + t : nullptr, warp_sums);
 }
 
 // ---------------------------------------------------------------------------
@@ -464,50 +491,6 @@ topk_finalize_kernel(const float *__restrict__ scores, int64_t ld, const int32_t
 constexpr int32_t kSingleMaxV = 65536;
 constexpr int32_t kSingleCap = 8192;  // candidates held in shared memory
 constexpr size_t kSingleSmem = (size_t)kSingleCap * 8 + (size_t)kSingleMaxV / 8;
-
-// Writes the selected positions (bits set in `bits`, `words` words) to out in
-// ascending order, -1 after them, and -- when rows != null -- their physical
-// cache rows (compact_rows layout, tile 64) and count.  All threads call it.
-__device__ void emit_selection(const uint32_t *bits, int words, int32_t top_k, int32_t *out,
-                               const PathParams &p, int32_t t, int32_t *rows, int32_t *n_valid,
-                               int *warp_sums) {
-    const int32_t seq = rows != nullptr ? __ldg(p.q_seq + t) : 0;
-    const int per = (words + kThreads - 1) / kThreads;
-    const int w0 = min(words, (int)threadIdx.x * per), w1 = min(words, w0 + per);
-    int cnt = 0;
-    for (int w = w0; w < w1; ++w) cnt += __popc(bits[w]);
-    int total;
-    int pos = block_exclusive_prefix(cnt, warp_sums, &total);
-    int bad_page = 0;
-    for (int w = w0; w < w1; ++w) {
-        uint32_t b = bits[w];
-        while (b) {
-            const int j = __ffs(b) - 1;
-            b &= b - 1;
-            if (pos < top_k) {
-                const int32_t s = w * 32 + j;
-                out[pos] = s;
-                if (rows != nullptr) {
-                    const int64_t row = phys_row(p.page_table, p.max_pages, p.num_pages, seq, s);
-                    if (row < 0) bad_page = 1;
-                    else rows[pos] = static_cast<int32_t>(row);
-                }
-            }
-            ++pos;
-        }
-    }
-    const int32_t nv = min(total, top_k);
-    for (int i = nv + threadIdx.x; i < top_k; i += kThreads) out[i] = -1;
-    if (rows == nullptr) return;
-    if (__syncthreads_or(bad_page)) {  // rare: drop (and report) the unmapped rows
-        compact_rows(p, t, out, top_k, 64, rows, n_valid, warp_sums);
-        return;
-    }
-    const int32_t padded = (nv + 63) / 64 * 64;
-    if (nv > 0)
-        for (int c = nv + threadIdx.x; c < padded; c += kThreads) rows[c] = rows[0];
-    if (threadIdx.x == 0) *n_valid = nv;
-}
 
 __global__ void __launch_bounds__(kThreads)
 topk_single_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *__restrict__ vis,
