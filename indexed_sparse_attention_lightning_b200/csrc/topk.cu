@@ -553,49 +553,58 @@ topk_single_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *
     if (!fallback) {
         // one pass over the row: keys above b* into the bitmap, b*'s keys collected
         const float *row = scores + (int64_t)t * ld;
-        for (int32_t b0 = 0; b0 < V; b0 += 4 * kThreads) {  // same trip count in every lane
-            const int32_t i0 = b0 + 4 * tid;
-            float x[4];
-            if (i0 + 4 <= V) {
-                const float4 v4 = *reinterpret_cast<const float4 *>(row + i0);
-                x[0] = v4.x;
-                x[1] = v4.y;
-                x[2] = v4.z;
-                x[3] = v4.w;
-            } else {
+        // all loads of a batch in flight before any is used (a row of up to
+        // 32K positions is one batch); the trip count is the same in every lane
+        constexpr int kBatch = 8;
+        for (int32_t b0 = 0; b0 < V; b0 += 4 * kThreads * kBatch) {
+            float4 xs[kBatch];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) x[e] = i0 + e < V ? row[i0 + e] : 0.f;
+            for (int u = 0; u < kBatch; ++u) {
+                const int32_t i0 = b0 + 4 * (tid + u * kThreads);
+                if (i0 + 4 <= V) {
+                    xs[u] = *reinterpret_cast<const float4 *>(row + i0);
+                } else {
+                    xs[u].x = i0 < V ? row[i0] : 0.f;
+                    xs[u].y = i0 + 1 < V ? row[i0 + 1] : 0.f;
+                    xs[u].z = i0 + 2 < V ? row[i0 + 2] : 0.f;
+                    xs[u].w = i0 + 3 < V ? row[i0 + 3] : 0.f;
+                }
             }
-            uint32_t above_mask = 0;
-            int n_eq = 0;
-            uint32_t keys[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                keys[e] = order_key(x[e]);
-                const int b = static_cast<int>(keys[e] >> (32 - kHistBits));
-                const bool valid = i0 + e < V;
-                if (valid && b > bstar) above_mask |= 1u << e;
-                if (valid && b == bstar) ++n_eq;
-            }
-            if (above_mask) atomicOr(&bits[i0 >> 5], above_mask << (i0 & 31));
-            // warp-aggregated slots for the bucket's keys
-            int incl = n_eq;
+            for (int u = 0; u < kBatch; ++u) {
+                const int32_t i0 = b0 + 4 * (tid + u * kThreads);
+                const float x[4] = {xs[u].x, xs[u].y, xs[u].z, xs[u].w};
+                uint32_t above_mask = 0;
+                int n_eq = 0;
+                uint32_t keys[4];
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int n = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += n;
-            }
-            int base = 0;
-            if (lane == 31 && incl > 0) base = atomicAdd(&n_cand_s, incl);
-            base = __shfl_sync(0xffffffffu, base, 31) + incl - n_eq;
+                for (int e = 0; e < 4; ++e) {
+                    keys[e] = order_key(x[e]);
+                    const int b = static_cast<int>(keys[e] >> (32 - kHistBits));
+                    const bool valid = i0 + e < V;
+                    if (valid && b > bstar) above_mask |= 1u << e;
+                    if (valid && b == bstar) ++n_eq;
+                }
+                if (above_mask) atomicOr(&bits[i0 >> 5], above_mask << (i0 & 31));
+                // warp-aggregated slots for the bucket's keys
+                int incl = n_eq;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int b = static_cast<int>(keys[e] >> (32 - kHistBits));
-                if (i0 + e < V && b == bstar) {
-                    if (base < kSingleCap)
-                        cs[base] = (static_cast<uint64_t>(keys[e]) << 32) |
-                                   (0xFFFFFFFFu - static_cast<uint32_t>(i0 + e));
-                    ++base;
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int n = __shfl_up_sync(0xffffffffu, incl, o);
+                    if (lane >= o) incl += n;
+                }
+                int base = 0;
+                if (lane == 31 && incl > 0) base = atomicAdd(&n_cand_s, incl);
+                base = __shfl_sync(0xffffffffu, base, 31) + incl - n_eq;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int b = static_cast<int>(keys[e] >> (32 - kHistBits));
+                    if (i0 + e < V && b == bstar) {
+                        if (base < kSingleCap)
+                            cs[base] = (static_cast<uint64_t>(keys[e]) << 32) |
+                                       (0xFFFFFFFFu - static_cast<uint32_t>(i0 + e));
+                        ++base;
+                    }
                 }
             }
         }
