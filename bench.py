@@ -308,28 +308,62 @@ def run_ours(args, rank: int, world: int, dist):
     if st[0] != _abi.SA_OK:
         raise RuntimeError(f"device status after timing: {st}")
 
-    # end to end through the public API with host buffers
+    # end to end through the public API with host buffers: every step copies
+    # its inputs from pinned host memory and reads its output back.  Steps are
+    # pipelined the way a serving loop runs them -- the copies of one step
+    # overlap the compute of its neighbours (copy-in stream, compute stream,
+    # copy-out stream; inputs and outputs double-buffered) -- and the time
+    # runs from the first copy-in to the last copy-out.
     e2e = None
     if not args.no_e2e:
+        import dataclasses as _dc
         host_in = api.host_queries(wl, pin=True)
-        host_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
-        host_lse = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
-        h2d = 0
-        e2e_ms = 0.0
-        for k in range(args.warmup + args.steps):
-            flush.zero_()
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            h2d = queries.copy_from(host_in, non_blocking=True)
-            step()
-            host_out.copy_(out, non_blocking=True)
-            host_lse.copy_(lse, non_blocking=True)
-            b.record(stream)
-            b.synchronize()
-            if k >= args.warmup:
-                e2e_ms += a.elapsed_time(b)
+        comp = stream
+        s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+        qbuf = [queries, _dc.replace(queries, **{k: torch.empty_like(v)
+                                                 for k, v in queries.tensors().items()
+                                                 if v is not None})]
+        obuf = [(out, lse), (torch.empty_like(out), torch.empty_like(lse))]
+        hout = [(torch.empty(out.shape, dtype=out.dtype, pin_memory=True),
+                 torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)) for _ in range(2)]
+
+        def pipelined(n):
+            if n <= 0:
+                return 0.0, 0
+            in_done = [torch.cuda.Event() for _ in range(n)]
+            comp_done = [torch.cuda.Event() for _ in range(n)]
+            out_done = [torch.cuda.Event() for _ in range(n)]
+            t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            h2d = 0
+            t0.record(s_in)
+            for k in range(n):
+                b = k % 2
+                with torch.cuda.stream(s_in):
+                    if k >= 2:
+                        s_in.wait_event(comp_done[k - 2])  # buffer b no longer read
+                    h2d = qbuf[b].copy_from(host_in, non_blocking=True)
+                    in_done[k].record(s_in)
+                comp.wait_event(in_done[k])
+                if k >= 2:
+                    comp.wait_event(out_done[k - 2])  # output b has been read back
+                flush.zero_()
+                api.decode(cache, qbuf[b], K, out=obuf[b][0], lse=obuf[b][1], idx=idx,
+                           out_dtype=odt, ws=ws)
+                comp_done[k].record(comp)
+                with torch.cuda.stream(s_out):
+                    s_out.wait_event(comp_done[k])
+                    hout[b][0].copy_(obuf[b][0], non_blocking=True)
+                    hout[b][1].copy_(obuf[b][1], non_blocking=True)
+                    out_done[k].record(s_out)
+            s_out.wait_event(out_done[n - 1])
+            t1.record(s_out)
+            torch.cuda.synchronize()
+            return t0.elapsed_time(t1), h2d
+
+        pipelined(args.warmup)
+        e2e_total, h2d = pipelined(args.steps)
         d2h = out.numel() * out.element_size() + lse.numel() * lse.element_size()
-        e2e = {"ms_per_step": e2e_ms / args.steps, "h2d": h2d, "d2h": d2h}
+        e2e = {"ms_per_step": e2e_total / args.steps, "h2d": h2d, "d2h": d2h}
 
     # max over ranks
     t = torch.tensor([total_ms, e2e["ms_per_step"] if e2e else 0.0], dtype=torch.float64,
