@@ -37,7 +37,7 @@ using namespace sm100;
 constexpr int kKeys = 128;    // MMA M: keys per tile (two pages)
 constexpr int kHeads = 64;    // MMA N: indexer heads
 constexpr int kDim = 128;     // MMA K: index dimension (bytes of e4m3)
-constexpr int kStages = 3;
+constexpr int kStages = 4;
 constexpr int kAcc = 4;       // TMEM accumulators (64 columns each)
 constexpr int kScaleSlots = 8;  // key-scale ring: the epilogue frees these, not the key stages
 constexpr int kEpiGroups = 2;  // epilogue warp groups, alternating tiles
@@ -49,7 +49,7 @@ constexpr uint32_t kTmemCols = kAcc * kHeads;
 
 struct IndexerSmem {
     uint8_t keys[kStages][kTileBytes];  // 1024-byte aligned (128-byte swizzle atoms)
-    uint32_t hist[kEpiGroups][kHistBins];  // score-key histogram of each group's current query
+    uint32_t hist[kHistBins];              // score-key histogram of the current query
     uint8_t q[2][kQBytes];                 // 1024-byte aligned like the key stages
     float wq[kEpiGroups][kHeads];          // head weights x query scales of that query
     float kscale[kScaleSlots][kKeys];   // per-token key scales of the staged pages
@@ -302,35 +302,35 @@ indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
         const int g = (warp - 2) >> 2;          // epilogue group
         const int quad = warp & 3;              // TMEM lanes this warp may read
         const int row = quad * 32 + lane;       // key row of the tile
-        const int et = threadIdx.x - 64 - 128 * g;  // 0..127 within the group
-        const int bar = 1 + g;                  // the group's named barrier
+        const int ea = threadIdx.x - 64;        // 0..255 over both groups
+        const int et = ea - 128 * g;            // 0..127 within the group
+        const int bar = 2 + g;                  // the group's named barrier (1: both groups)
         const bool histo = a.hist != nullptr;
-        uint32_t *hist = sm.hist[g];
         float *wq = sm.wq[g];
         if (histo) {
-            for (int b = et; b < kHistBins; b += 128) hist[b] = 0;
-            named_barrier(bar, 128);
+            for (int b = ea; b < kHistBins; b += 256) sm.hist[b] = 0;
+            named_barrier(1, 256);
         }
-        // add this group's counts of query t to the global histogram, then clear
+        // add the CTA's counts of query t to the global histogram, then clear;
+        // both groups walk every tile, so they get here at the same query change
         auto flush = [&](int32_t t) {
-            named_barrier(bar, 128);
+            named_barrier(1, 256);
             uint32_t *gh = a.hist + (int64_t)t * kHistBins;
-            for (int b = et; b < kHistBins; b += 128) {
-                const uint32_t v = hist[b];
+            for (int b = ea; b < kHistBins; b += 256) {
+                const uint32_t v = sm.hist[b];
                 if (v != 0) {
                     atomicAdd(gh + b, v);
-                    hist[b] = 0;
+                    sm.hist[b] = 0;
                 }
             }
-            named_barrier(bar, 128);
+            named_barrier(1, 256);
         };
         TileCursor c;
         c.init_at(a.tile_end, sm.start_t, sm.start_i, k0, k1);
         bool ok = true;
         int32_t V = 0, t_cur = -1;
         for (int n = 0; c.valid(); ++n, c.next(a.tile_end)) {
-            if ((n & 1) != g) continue;
-            if (c.t != t_cur) {  // this group's first tile of a query
+            if (c.t != t_cur) {  // a new query: both groups see it at the same tile
                 if (histo && t_cur >= 0) flush(t_cur);
                 named_barrier(bar, 128);  // the old weights are no longer read
                 t_cur = c.t;
@@ -340,6 +340,7 @@ indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
                              __ldg(p.q_index_scale + (int64_t)c.t * kHeads + et);
                 named_barrier(bar, 128);
             }
+            if ((n & 1) != g) continue;  // the other group's tile
             const int64_t s = (int64_t)c.i * kKeys + row;
             // key scales and page validity have a ring of their own
             const int slot = n % kScaleSlots;
@@ -383,7 +384,7 @@ indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
             if (s < V) {
                 const float score = page_ok ? sum * kscale : -INFINITY;
                 a.scores[(int64_t)c.t * a.ld + s] = score;
-                if (histo) atomicAdd(&hist[order_key(score) >> (32 - kHistBits)], 1u);
+                if (histo) atomicAdd(&sm.hist[order_key(score) >> (32 - kHistBits)], 1u);
             }
         }
         if (histo && t_cur >= 0) flush(t_cur);
