@@ -583,40 +583,61 @@ sfa_mma_kernel(const __grid_constant__ CUtensorMap tm_q, const SfaArgs a) {
 }
 
 // out = sum_s w_s o_s with w_s = exp(lse_s - lse), lse = log sum_s exp(lse_s).
+// One CTA per (query, head): the split weights are computed once in shared
+// memory, then each thread merges four output dims over all splits with the
+// partial loads unrolled.
+constexpr int kMaxSplits = 128;
 __global__ void __launch_bounds__(128)
 sfa_combine_kernel(const float *__restrict__ o_part, const float *__restrict__ lse_part,
                    int32_t splits, void *out, int32_t out_dtype, float *lse) {
     pdl_wait();
     pdl_trigger();
+    __shared__ float w_s[kMaxSplits];
     const int64_t row = blockIdx.x;  // t * 128 + head
     const int64_t t = row >> 7, head = row & 127;
-    float m = -INFINITY;
-    for (int s = 0; s < splits; ++s) m = fmaxf(m, lse_part[(t * splits + s) * 128 + head]);
-    float acc[4] = {0.f, 0.f, 0.f, 0.f}, wsum = 0.f;
-    if (m != -INFINITY) {
-        for (int s = 0; s < splits; ++s) {
-            const float ls = lse_part[(t * splits + s) * 128 + head];
-            const float w = ls == -INFINITY ? 0.f : __expf(ls - m);
-            wsum += w;
-            const float4 v = reinterpret_cast<const float4 *>(
-                o_part + ((t * splits + s) * 128 + head) * kDl)[threadIdx.x];
-            acc[0] += w * v.x;
-            acc[1] += w * v.y;
-            acc[2] += w * v.z;
-            acc[3] += w * v.w;
+    if (threadIdx.x < splits) w_s[threadIdx.x] = lse_part[(t * splits + threadIdx.x) * 128 + head];
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        float m = -INFINITY;
+        for (int s = threadIdx.x; s < splits; s += 32) m = fmaxf(m, w_s[s]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        float sum = 0.f;
+        for (int s = threadIdx.x; s < splits; s += 32) {
+            const float ls = w_s[s];
+            const float w = (m == -INFINITY || ls == -INFINITY) ? 0.f : __expf(ls - m);
+            w_s[s] = w;
+            sum += w;
         }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        const float inv = sum > 0.f ? 1.f / sum : 0.f;
+        for (int s = threadIdx.x; s < splits; s += 32) w_s[s] *= inv;
+        if (lse != nullptr && threadIdx.x == 0) lse[row] = sum > 0.f ? m + logf(sum) : -INFINITY;
     }
-    const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+    __syncthreads();
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    const float4 *src = reinterpret_cast<const float4 *>(o_part + (t * splits * 128 + head) * kDl) +
+                        threadIdx.x;
+    const int64_t stride = 128 * kDl / 4;  // one split, in float4
+#pragma unroll 8
+    for (int s = 0; s < splits; ++s) {
+        const float w = w_s[s];
+        const float4 v = src[s * stride];
+        acc[0] += w * v.x;
+        acc[1] += w * v.y;
+        acc[2] += w * v.z;
+        acc[3] += w * v.w;
+    }
     if (out_dtype == SA_BF16) {
-        __nv_bfloat162 a = __floats2bfloat162_rn(acc[0] * inv, acc[1] * inv);
-        __nv_bfloat162 b = __floats2bfloat162_rn(acc[2] * inv, acc[3] * inv);
+        __nv_bfloat162 a = __floats2bfloat162_rn(acc[0], acc[1]);
+        __nv_bfloat162 b = __floats2bfloat162_rn(acc[2], acc[3]);
         uint2 w = make_uint2(*reinterpret_cast<uint32_t *>(&a), *reinterpret_cast<uint32_t *>(&b));
         reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(out) + row * kDl)[threadIdx.x] = w;
     } else {
         reinterpret_cast<float4 *>(static_cast<float *>(out) + row * kDl)[threadIdx.x] =
-            make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+            make_float4(acc[0], acc[1], acc[2], acc[3]);
     }
-    if (lse != nullptr && threadIdx.x == 0) lse[row] = wsum > 0.f ? m + logf(wsum) : -INFINITY;
 }
 
 }  // namespace
@@ -633,7 +654,7 @@ int32_t sfa_splits(int32_t n_q, int32_t top_k) {
     const int32_t ctas = std::max(1, num_sms());
     const int32_t max_tiles = (top_k + kTile - 1) / kTile;
     if (n_q <= 0) return 1;
-    return std::max(1, std::min(max_tiles, ctas / (2 * n_q)));
+    return std::max(1, std::min({max_tiles, ctas / (2 * n_q), kMaxSplits}));
 }
 
 int32_t sfa_rows_ld(int32_t top_k) { return (int32_t)round_up(top_k > 0 ? top_k : 1, kTile); }
