@@ -94,9 +94,20 @@ typedef struct sa_cache {
     const void *kv;              /* SA_F32/SA_BF16: [num_pages, page_size, d_latent + d_rope]
                                   * SA_E4M3: latent codes [num_pages, page_size, d_latent] */
     const void *kv_rope;         /* SA_E4M3 only: bf16 [num_pages, page_size, d_rope] */
-    const float *kv_scale;       /* SA_E4M3 only: [num_pages], one scale per 64-token page tile */
+    const float *kv_scale;       /* SA_E4M3 only: fp32 [num_pages, page_size / kv_scale_tokens,
+                                  * d_latent / kv_scale_dims], one scale per tile */
     int32_t d_latent;            /* 512 (production) */
     int32_t d_rope;              /* 64 (production) */
+    /* SA_E4M3 scale tile: one fp32 scale per kv_scale_tokens tokens of a page
+     * x kv_scale_dims latent dims.  The pages quantise the main cache per token
+     * and per 128 elements ("Optimizing Next-Gen LLM Inference" §4, table;
+     * "Inference Acceleration for New Large Model Architectures" §4.2;
+     * "Long-Context LLM Inference Optimization", Layered Quantization): that is
+     * (1, 128).  kv_scale_tokens divides page_size; kv_scale_dims divides
+     * d_latent and is a multiple of 16.  0 and 0 mean one scale per page
+     * (page_size x d_latent). */
+    int32_t kv_scale_tokens;
+    int32_t kv_scale_dims;
 } sa_cache;
 
 /* A batch of query tokens.  Query t belongs to sequence q_seq[t] and sits at

@@ -36,7 +36,8 @@ class SaCache(ctypes.Structure):
                 ("index_dtype", ctypes.c_int), ("k_index", _P), ("k_index_scale", _P),
                 ("d_index", _I32),
                 ("kv_dtype", ctypes.c_int), ("kv", _P), ("kv_rope", _P), ("kv_scale", _P),
-                ("d_latent", _I32), ("d_rope", _I32)]
+                ("d_latent", _I32), ("d_rope", _I32),
+                ("kv_scale_tokens", _I32), ("kv_scale_dims", _I32)]
 
 
 class SaQuery(ctypes.Structure):

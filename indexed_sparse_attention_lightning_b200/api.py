@@ -58,6 +58,7 @@ class DeviceCache:
     d_latent: int
     d_rope: int
     page_size: int = 64
+    kv_scale_tile: tuple = (0, 0)   # (tokens, dims) per e4m3 scale; (0, 0): one per page
 
     def struct(self) -> SaCache:
         return SaCache(
@@ -67,7 +68,8 @@ class DeviceCache:
             index_dtype=_abi.DTYPES[self.index_dtype], k_index=_ptr(self.k_index),
             k_index_scale=_ptr(self.k_index_scale), d_index=self.d_index,
             kv_dtype=_abi.DTYPES[self.kv_dtype], kv=_ptr(self.kv), kv_rope=_ptr(self.kv_rope),
-            kv_scale=_ptr(self.kv_scale), d_latent=self.d_latent, d_rope=self.d_rope)
+            kv_scale=_ptr(self.kv_scale), d_latent=self.d_latent, d_rope=self.d_rope,
+            kv_scale_tokens=int(self.kv_scale_tile[0]), kv_scale_dims=int(self.kv_scale_tile[1]))
 
 
 @dataclass
@@ -124,7 +126,7 @@ def upload(wl, device="cuda") -> tuple[DeviceCache, DeviceQueries]:
         k_index=_t(wl.k_index, device), k_index_scale=_t(wl.k_index_scale, device),
         kv_dtype=sp.kv_dtype, kv=_t(wl.kv, device), kv_rope=_t(wl.kv_rope, device),
         kv_scale=_t(wl.kv_scale, device), d_index=sp.d_index, d_latent=sp.d_latent,
-        d_rope=sp.d_rope, page_size=sp.page_size)
+        d_rope=sp.d_rope, page_size=sp.page_size, kv_scale_tile=tuple(sp.kv_scale_tile))
     queries = DeviceQueries(
         q_seq=_t(wl.q_seq, device), q_pos=_t(wl.q_pos, device), max_visible=wl.max_visible,
         q_index=_t(wl.q_index, device), q_index_scale=_t(wl.q_index_scale, device),

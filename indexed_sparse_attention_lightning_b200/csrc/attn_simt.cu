@@ -33,7 +33,7 @@ __device__ __forceinline__ float load_kv(const PathParams &p, int64_t row, int d
     default:
         if (dd < p.d_latent) {
             uint8_t c = static_cast<const uint8_t *>(p.kv)[row * p.d_latent + dd];
-            return e4m3x2_to_float2(c).x * p.kv_scale[row >> 6];
+            return e4m3x2_to_float2(c).x * kv_scale_at(p, row, dd);
         }
         return bf16_bits_to_float(
             static_cast<const uint16_t *>(p.kv_rope)[row * p.d_rope + (dd - p.d_latent)]);

@@ -50,6 +50,7 @@ struct PathParams {
     const float *kv_scale;
     int32_t d_latent, d_rope;
     int32_t kv_dtype;  // sa_dtype
+    int32_t kv_scale_tokens, kv_scale_dims;  // e4m3 scale tile (resolved, > 0)
     // queries
     int32_t n_q;
     const int32_t *q_seq, *q_pos;
@@ -148,6 +149,17 @@ __device__ __forceinline__ int32_t visible_len(const PathParams &p, int32_t t) {
         return 0;
     }
     return pos + 1;
+}
+
+// Scale of latent dim d of physical row `row` of the e4m3 cache: one fp32 per
+// tile of kv_scale_tokens tokens x kv_scale_dims dims of a 64-token page,
+// laid out [num_pages, 64 / kv_scale_tokens, d_latent / kv_scale_dims].
+__device__ __forceinline__ float kv_scale_at(const PathParams &p, int64_t row, int32_t d) {
+    const int64_t page = row >> 6;
+    const int32_t tok = static_cast<int32_t>(row & 63);
+    const int32_t tiles_t = 64 / p.kv_scale_tokens, tiles_d = p.d_latent / p.kv_scale_dims;
+    return __ldg(p.kv_scale + (page * tiles_t + tok / p.kv_scale_tokens) * tiles_d +
+                 d / p.kv_scale_dims);
 }
 
 // Physical cache rows of query t's selected positions sel[0, K): list order,

@@ -48,6 +48,13 @@ sa_status check_cache(const sa_cache *c) {
     if (c->kv_dtype == SA_E4M3) {
         if (!c->kv_scale || (c->d_rope > 0 && !c->kv_rope)) return SA_ERR_INVALID_ARG;
         if (c->kv_rope && !aligned16(c->kv_rope)) return SA_ERR_INVALID_ARG;
+        const bool page_tile = c->kv_scale_tokens == 0 && c->kv_scale_dims == 0;
+        if (!page_tile) {
+            if (c->kv_scale_tokens <= 0 || c->kv_scale_dims <= 0) return SA_ERR_INVALID_ARG;
+            if (c->page_size % c->kv_scale_tokens != 0 || c->d_latent % c->kv_scale_dims != 0 ||
+                c->kv_scale_dims % 16 != 0)
+                return SA_ERR_UNSUPPORTED;
+        }
     }
     return SA_OK;
 }
@@ -89,6 +96,9 @@ PathParams make_params(const sa_cache *c, const sa_query *q, void *ws) {
     p.d_latent = c->d_latent;
     p.d_rope = c->d_rope;
     p.kv_dtype = c->kv_dtype;
+    const bool page_tile = c->kv_scale_tokens == 0 && c->kv_scale_dims == 0;
+    p.kv_scale_tokens = page_tile ? c->page_size : c->kv_scale_tokens;
+    p.kv_scale_dims = page_tile ? c->d_latent : c->kv_scale_dims;
     p.n_q = q->n_q;
     p.q_seq = q->q_seq;
     p.q_pos = q->q_pos;

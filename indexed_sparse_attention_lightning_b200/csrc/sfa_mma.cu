@@ -478,7 +478,7 @@ sfa_mma_kernel(const __grid_constant__ CUtensorMap tm_q, const SfaArgs a) {
 #pragma unroll 2
                 for (int k = pw; k < kTile; k += kProducerWarps) {
                     const int32_t r = __shfl_sync(0xffffffffu, k < 32 ? r_lo : r_hi, k & 31);
-                    const float sc = __ldg(p.kv_scale + (r >> 6));
+                    const float sc = kv_scale_at(p, r, 16 * lane);  // this lane's 16 dims
                     const uint4 x = __ldg(reinterpret_cast<const uint4 *>(kv + (int64_t)r * kDl) + lane);
                     uint4 rp = make_uint4(0, 0, 0, 0);
                     if (lane < 8)

@@ -15,8 +15,9 @@ indexer and the sparse attention kernel -- "Optimizing Next-Gen LLM Inference"
 * index keys ``k_index[P, 64, d_index]`` (fp32, or e4m3 codes with one fp32
   scale per token in ``k_index_scale[P, 64]``);
 * MLA latent rows ``kv[P, 64, d_latent + d_rope]`` (fp32 or bf16), or for the
-  FP8 cache ``kv[P, 64, d_latent]`` e4m3 codes, ``kv_scale[P]`` (one fp32 scale
-  per 64-token page tile) and ``kv_rope[P, 64, d_rope]`` bf16.
+  FP8 cache ``kv[P, 64, d_latent]`` e4m3 codes, ``kv_scale[P, 64 / ts, d_latent / td]``
+  (one fp32 scale per tile of ts tokens x td latent dims of a page; the default
+  (64, d_latent) is one per page) and ``kv_rope[P, 64, d_rope]`` bf16.
 
 Slots past a sequence's end and pages no sequence owns are filled with NaN, so
 that any read outside the visible range shows up as NaN in a result.
@@ -64,12 +65,21 @@ class WorkloadSpec:
     page_size: int = 64
     paging: str = "permuted"       # "identity" or "permuted"
     keys: tuple = ("iid",)         # ("iid",), ("planted", frac, sigma), ("clusters", n, span)
-    sm_scale: Optional[float] = None  # default 1/sqrt(d_latent + d_rope)
+    sm_scale: Optional[float] = None
+    # e4m3 latent cache: one fp32 scale per tile of (tokens of a page, latent
+    # dims); (0, 0) is one scale per page
+    kv_scale_tile: tuple = (0, 0)  # default 1/sqrt(d_latent + d_rope)
     poison_pages: int = 2
 
     @property
     def d_qk(self) -> int:
         return self.d_latent + self.d_rope
+
+    @property
+    def kv_tile(self) -> tuple:
+        """(tokens, latent dims) covered by one e4m3 scale."""
+        st, sd = self.kv_scale_tile
+        return (st or self.page_size, sd or self.d_latent)
 
     @property
     def softmax_scale(self) -> float:
@@ -141,7 +151,7 @@ class Workload:
     w: np.ndarray                # f32 [n_q, h_index]
     kv: np.ndarray               # f32/uint16(bf16) [P, ps, d_qk] or uint8 [P, ps, d_latent]
     kv_rope: Optional[np.ndarray]  # uint16 (bf16) [P, ps, d_rope] for the e4m3 cache
-    kv_scale: Optional[np.ndarray]  # f32 [P] for the e4m3 cache
+    kv_scale: Optional[np.ndarray]  # f32 [P, 64 / tile tokens, d_latent / tile dims] (e4m3)
     q: np.ndarray                # f32 or uint16 (bf16) [n_q, heads, d_qk]
     planted: dict = field(default_factory=dict)  # seq -> sorted planted positions
     clusters: dict = field(default_factory=dict)  # seq -> list of (start, len)
@@ -358,7 +368,10 @@ def make_workload(sp: WorkloadSpec) -> Workload:
             raise ValueError("the e4m3 cache keeps one scale per 64-token page")
         kv = np.full((rows, dl), E4M3_NAN, dtype=np.uint8)
         kv_rope = np.full((rows, dr), BF16_NAN, dtype=np.uint16)
-        kv_scale = np.full((num_pages,), np.nan, dtype=np.float32)
+        st, sd = sp.kv_tile
+        if ps % st or dl % sd:
+            raise ValueError("scale tiles must divide the page and the latent dims")
+        kv_scale = np.full((num_pages, ps // st, dl // sd), np.nan, dtype=np.float32)
     else:
         raise ValueError(sp.kv_dtype)
     for b in range(sp.batch):
@@ -373,16 +386,18 @@ def make_workload(sp: WorkloadSpec) -> Workload:
             elif sp.kv_dtype == "bf16":
                 kv[dst] = to_bf16_bits(x)
             else:
-                # one scale per page tile of the latent part; the chunk is a
-                # multiple of the page size, so pages never straddle chunks
+                # one scale per (st tokens x sd dims) tile of each page's
+                # latent part; the chunk is a multiple of the page size, so
+                # pages never straddle chunks
                 lat = x[:, :dl]
                 n = c1 - c0
                 npg = (n + ps - 1) // ps
                 pad = npg * ps - n
                 lat_p = np.concatenate([lat, np.zeros((pad, dl), np.float32)]) if pad else lat
-                amax = np.abs(lat_p.reshape(npg, ps * dl)).max(axis=1)
-                sc = amax_scale(amax)
-                codes = to_e4m3_codes(lat / np.repeat(sc, ps)[:n, None])
+                tiles = np.abs(lat_p).reshape(npg, ps // st, st, dl // sd, sd)
+                sc = amax_scale(tiles.max(axis=(2, 4)))            # [npg, ps/st, dl/sd]
+                full = np.repeat(np.repeat(sc, st, axis=1), sd, axis=2).reshape(npg * ps, dl)
+                codes = to_e4m3_codes(lat / full[:n])
                 kv[dst] = codes
                 kv_rope[dst] = to_bf16_bits(x[:, dl:])
                 kv_scale[pt[c0 // ps: c0 // ps + npg]] = sc

@@ -57,7 +57,8 @@ def _load():
         lib.oracle_topk.argtypes = [I32, P, I64, P, I32, P]
         lib.oracle_topk.restype = ctypes.c_int
         lib.oracle_sparse_attn.argtypes = [I32, P, P, I32, I32, I32, I32, P, D, I32, P, P, P,
-                                           P, I32, I32, I32, P, I32, P, P, ctypes.c_int]
+                                           I32, I32, P, I32, I32, I32, P, I32, P, P,
+                                           ctypes.c_int]
         lib.oracle_sparse_attn.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -142,7 +143,8 @@ def sparse_attn(wl, idx: np.ndarray, nthreads: int | None = None):
     rc = _load().oracle_sparse_attn(
         n_q, _ptr(q_seq), _ptr(q_pos), sp.heads, sp.d_latent, sp.d_rope,
         _DT[sp.q_dtype], _ptr(q), sp.softmax_scale, _DT[sp.kv_dtype], _ptr(kv), _ptr(rope),
-        _ptr(ksc), _ptr(pt), pt.shape[1], sp.page_size, wl.num_pages, _ptr(idx), K,
+        _ptr(ksc), sp.kv_tile[0], sp.kv_tile[1],
+        _ptr(pt), pt.shape[1], sp.page_size, wl.num_pages, _ptr(idx), K,
         _ptr(out), _ptr(lse), nthreads or threads())
     _check(rc, "sparse_attn")
     return out, lse

@@ -337,7 +337,10 @@ typedef struct {
     int32_t kv_dtype;          /* OR_F32, OR_BF16 or OR_E4M3 */
     const void *kv;            /* f32/bf16: [rows, d_latent + d_rope]; e4m3: [rows, d_latent] */
     const void *kv_rope;       /* e4m3 cache: bf16 [rows, d_rope] */
-    const float *kv_scale;     /* e4m3 cache: [num_pages], one per page tile */
+    const float *kv_scale;     /* e4m3 cache: [num_pages, page_size / scale_tokens,
+                                *   d_latent / scale_dims], one per tile */
+    int32_t scale_tokens;      /* tokens of a page per scale tile */
+    int32_t scale_dims;        /* latent dims per scale tile */
     pages_t pg;
     const int32_t *idx;
     int32_t K;
@@ -387,9 +390,15 @@ static int attn_item(pool_t *p, int64_t t)
         }
         double *dst = rows + (int64_t)r * D;
         if (c->kv_dtype == OR_E4M3) {
-            double sc = (double)c->kv_scale[row / c->pg.page_size];
+            /* the scale of (token, dim) is that of its tile within its page */
+            const int64_t page = row / c->pg.page_size;
+            const int32_t tok = (int32_t)(row % c->pg.page_size);
+            const int32_t tiles_t = c->pg.page_size / c->scale_tokens;
+            const int32_t tiles_d = dl / c->scale_dims;
+            const float *ps = c->kv_scale + (page * tiles_t + tok / c->scale_tokens) * tiles_d;
             for (int32_t i = 0; i < dl; i++)
-                dst[i] = e4m3_value(((const uint8_t *)c->kv)[row * dl + i]) * sc;
+                dst[i] = e4m3_value(((const uint8_t *)c->kv)[row * dl + i]) *
+                         (double)ps[i / c->scale_dims];
             for (int32_t i = 0; i < dr; i++)
                 dst[dl + i] = bf16_value(((const uint16_t *)c->kv_rope)[row * dr + i]);
         } else {
@@ -438,7 +447,7 @@ int oracle_sparse_attn(int32_t n_q, const int32_t *q_seq, const int32_t *q_pos,
                        int32_t heads, int32_t d_latent, int32_t d_rope,
                        int32_t q_dtype, const void *q, double sm_scale,
                        int32_t kv_dtype, const void *kv, const void *kv_rope,
-                       const float *kv_scale,
+                       const float *kv_scale, int32_t scale_tokens, int32_t scale_dims,
                        const int32_t *page_table, int32_t max_pages, int32_t page_size,
                        int32_t num_pages, const int32_t *idx, int32_t K,
                        double *out, double *lse, int nthreads)
@@ -449,8 +458,12 @@ int oracle_sparse_attn(int32_t n_q, const int32_t *q_seq, const int32_t *q_pos,
         return OR_BAD_ARG;
     if (kv_dtype == OR_E4M3 && (!kv_rope || !kv_scale))
         return OR_BAD_ARG;
+    if (kv_dtype == OR_E4M3 &&
+        (scale_tokens <= 0 || page_size % scale_tokens != 0 || scale_dims <= 0 ||
+         d_latent % scale_dims != 0))
+        return OR_BAD_ARG;
     attn_ctx c = { n_q, q_seq, q_pos, heads, d_latent, d_rope, q_dtype, q, sm_scale,
-                   kv_dtype, kv, kv_rope, kv_scale,
+                   kv_dtype, kv, kv_rope, kv_scale, scale_tokens, scale_dims,
                    { page_table, max_pages, page_size, num_pages }, idx, K, out, lse };
     return pool_run(attn_item, &c, n_q, nthreads);
 }

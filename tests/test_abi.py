@@ -75,6 +75,23 @@ def test_workspace_size_valid_and_invalid(L):
     assert ws_size(L, good_cache(), good_query(q_index_scale=None)) == 0
 
 
+FP8_KV = {"kv_dtype": _abi.SA_E4M3, "kv_rope": FAKE, "kv_scale": FAKE}
+
+
+@pytest.mark.parametrize("tile,ok", [
+    ((0, 0), True),       # one scale per page
+    ((1, 128), True),     # per token and 128 latent dims
+    ((64, 512), True), ((4, 16), True),
+    ((3, 128), False),    # does not divide the page
+    ((1, 100), False),    # does not divide the latent dims
+    ((1, 8), False),      # not a multiple of 16 dims
+    ((-1, 128), False), ((1, 0), False),
+])
+def test_fp8_scale_tile_validation(L, tile, ok):
+    c = good_cache(**FP8_KV, kv_scale_tokens=tile[0], kv_scale_dims=tile[1])
+    assert (ws_size(L, c, good_query()) > 0) == ok
+
+
 def decode_call(L, c, q, k=2048, ws=FAKE, ws_bytes=1 << 30, out=FAKE):
     return L.sa_decode(ctypes.byref(c), ctypes.byref(q), k, None, out, _abi.SA_BF16, None, ws,
                        ws_bytes, None)

@@ -150,9 +150,15 @@ def test_deterministic_and_independent_of_page_placement():
         assert np.array_equal(a[k], c[k]), k
 
 
-def test_fp8_latent_cache_small():
-    sp = W.WorkloadSpec(name="fp8kv_small", seed=22, batch=3, seq_len=("list", (700, 3000, 5000)),
-                        kv_dtype="e4m3", keys=("clusters", 2, 256))
+@pytest.mark.parametrize("tile,heads", [((0, 0), 128), ((1, 128), 128), ((1, 128), 64),
+                                        ((16, 256), 128)])
+def test_fp8_latent_cache_small(tile, heads):
+    """e4m3 latent with one scale per page or per finer tile (the pages'
+    per-token, per-128-element blocks are (1, 128)); 128 heads take the
+    tensor-core attention, 64 the CUDA-core one."""
+    sp = W.WorkloadSpec(name=f"fp8kv_small_{tile[0]}_{tile[1]}_{heads}", seed=22, batch=3,
+                        seq_len=("list", (700, 3000, 5000)), kv_dtype="e4m3",
+                        keys=("clusters", 2, 256), kv_scale_tile=tile, heads=heads)
     wl = workload(sp)
     res = run_fused(wl)
     scores = oracle.index_scores(wl)

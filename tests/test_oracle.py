@@ -68,7 +68,11 @@ def np_latent_rows(wl, b, positions):
     rows = np_rows(wl, b, positions)
     if sp.kv_dtype == "e4m3":
         lat = np_values("e4m3", wl.kv.reshape(-1, sp.d_latent)[rows])
-        lat = lat * wl.kv_scale[rows // sp.page_size][:, None].astype(np.float64)
+        # scale tile of (token, dim): (page, token // tile tokens, dim // tile dims)
+        st, sd = sp.kv_tile
+        sc = wl.kv_scale.reshape(wl.num_pages, sp.page_size // st, sp.d_latent // sd)
+        per_row = sc[rows // sp.page_size, (rows % sp.page_size) // st]   # [n, d_latent / sd]
+        lat = lat * np.repeat(per_row, sd, axis=1).astype(np.float64)
         rope = np_values("bf16", wl.kv_rope.reshape(-1, sp.d_rope)[rows])
         return np.concatenate([lat, rope], axis=1)
     return np_values(sp.kv_dtype, wl.kv.reshape(-1, sp.d_qk)[rows])
@@ -214,9 +218,12 @@ def test_attention_equals_dense_when_k_covers_context(kv_dtype, q_dtype):
     np.testing.assert_allclose(lse, ref_lse, rtol=1e-12, atol=1e-12)
 
 
-def test_attention_fp8_latent_equals_dense():
+@pytest.mark.parametrize("tile", [(64, 32), (1, 16), (8, 8), (16, 32)])
+def test_attention_fp8_latent_equals_dense(tile):
+    """Every scale tile shape: the oracle's dequantisation (C, its own tile
+    lookup) against numpy's restatement of the tile layout."""
     sp = small_spec(kv_dtype="e4m3", page_size=64, seq_len=("uniform", 130, 260), top_k=300,
-                    d_latent=32, d_rope=8)
+                    d_latent=32, d_rope=8, kv_scale_tile=tile)
     wl = W.make_workload(sp)
     idx = oracle.topk(oracle.index_scores(wl), wl.visible, sp.top_k)
     out, lse = oracle.sparse_attn(wl, idx)
