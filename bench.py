@@ -241,6 +241,23 @@ def run_reference(args, rank: int, world: int):
 
 # ---------------------------------------------------------------- our leg ---
 
+def rank_spec(sp, rank: int):
+    """Replicas: every rank decodes its own batch, drawn with its own seed."""
+    return sp if rank == 0 else dataclasses.replace(sp, seed=sp.seed + 1000 * rank)
+
+
+def reduce_over_ranks(dist, device, step_ms: float, e2e_ms: float, n_q: int):
+    """(max step time, max end-to-end step time, total queries) over all ranks:
+    the job is as slow as its slowest rank and serves every rank's queries."""
+    import torch
+    t = torch.tensor([step_ms, e2e_ms], dtype=torch.float64, device=device)
+    q = torch.tensor([float(n_q)], dtype=torch.float64, device=device)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dist.all_reduce(q, op=dist.ReduceOp.SUM)
+    return float(t[0]), float(t[1]), float(q[0])
+
+
 def run_ours(args, rank: int, world: int, dist):
     import torch
     from indexed_sparse_attention_lightning_b200 import _abi, api
@@ -249,9 +266,7 @@ def run_ours(args, rank: int, world: int, dist):
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    sp = W.spec(args.workload)
-    if rank > 0:
-        sp = dataclasses.replace(sp, seed=sp.seed + 1000 * rank)
+    sp = rank_spec(W.spec(args.workload), rank)
     wl = W.make_workload(sp)
     cache, queries = api.upload(wl, dev)
     K = sp.top_k
@@ -365,15 +380,8 @@ def run_ours(args, rank: int, world: int, dist):
         d2h = out.numel() * out.element_size() + lse.numel() * lse.element_size()
         e2e = {"ms_per_step": e2e_total / args.steps, "h2d": h2d, "d2h": d2h}
 
-    # max over ranks
-    t = torch.tensor([total_ms, e2e["ms_per_step"] if e2e else 0.0], dtype=torch.float64,
-                     device=dev)
-    q_total = torch.tensor([wl.n_q], dtype=torch.float64, device=dev)
-    if dist is not None:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        dist.all_reduce(q_total, op=dist.ReduceOp.SUM)
-    total_ms, e2e_step_ms = float(t[0]), float(t[1])
-    n_q_all = float(q_total[0])
+    total_ms, e2e_step_ms, n_q_all = reduce_over_ranks(
+        dist, dev, total_ms, e2e["ms_per_step"] if e2e else 0.0, wl.n_q)
     if rank != 0:
         return 0
 
