@@ -37,6 +37,7 @@ DEFAULT_WORKLOAD = "decode_b64_16k_32k_planted"
 METRIC = "sparse-attn decode query-tokens/s (indexer+top-K+SFA); % of HBM roofline"
 UNIT = "query-tokens/s"
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 SPEC_HBM_GBS = 8000.0
 FLUSH_BYTES = 256 << 20
 
@@ -65,13 +66,46 @@ def host_cores() -> int:
 
 
 def measured_peaks():
+    """(HBM GB/s, dense bf16 TFLOP/s for a kernel timed alone, "measured" or "fallback")."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
         with open(path) as f:
             d = json.load(f)
-        return float(d["hbm_gbs"]), "measured"
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
     except Exception:
-        return FALLBACK_HBM_GBS, "fallback"
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def algorithmic_flops(wl, idx: np.ndarray) -> dict:
+    """Tensor-core work per step, by phase: the indexer does 2 * h_index * d_index
+    flops per visible (query, position); the attention 2 * heads * (d_latent + d_rope
+    + d_latent) per selected row (Q K^T over 576 dims, P V over 512)."""
+    sp = wl.spec
+    V = wl.visible.astype(np.int64)
+    n_sel = int((idx >= 0).sum())
+    return {"indexer": int(V.sum()) * 2 * sp.h_index * sp.d_index,
+            "attention": n_sel * 2 * sp.heads * (2 * sp.d_latent + sp.d_rope)}
+
+
+def roofline(wl, name: str, ms: float, nbytes: dict, flops: dict) -> dict:
+    """Roofline of one phase.  Decode (one query per sequence) streams every key
+    and selected row once: HBM-bound, algorithmic bytes over the measured copy
+    bandwidth.  Chunked prefill (many queries of one sequence) reuses keys and rows
+    from L2, so the tensor pipe bounds it: algorithmic flops over the dtype's
+    peak (e4m3 = 2 x the measured bf16 GEMM, the nominal fp8:bf16 ratio)."""
+    hbm, bf16, kind = measured_peaks()
+    sp = wl.spec
+    shared = wl.n_q > wl.seq_len.shape[0]
+    secs = ms / 1e3
+    if shared and name in flops and sp.index_dtype == "e4m3":
+        peak = bf16 * (2.0 if name == "indexer" else 1.0)
+        achieved = flops[name] / secs / 1e12 if secs > 0 else 0.0
+        return {"bound": "tensor", "kernel": name, "achieved": achieved, "peak": peak,
+                "peak_kind": kind + (" (fp8 = 2 x bf16)" if name == "indexer" else " (bf16)"),
+                "unit": "TFLOP/s", "frac": achieved / peak}
+    achieved = nbytes[name] / secs / 1e9 if secs > 0 else 0.0
+    return {"bound": "hbm", "kernel": name, "achieved": achieved, "peak": hbm,
+            "peak_kind": kind, "unit": "GB/s", "frac": achieved / hbm}
 
 
 def algorithmic_bytes(wl, idx: np.ndarray) -> dict:
@@ -84,12 +118,14 @@ def algorithmic_bytes(wl, idx: np.ndarray) -> dict:
     indexer = int((V * (key_b + scale_b)).sum())
     n_sel = np.minimum(V, sp.top_k)
     if sp.kv_dtype == "e4m3":
+        # codes + bf16 rope per row, and 4 B per scale tile the selection touches
         row_b = sp.d_latent + 2 * sp.d_rope
-        pages = 0
+        tile_t, tile_d = sp.kv_tile
+        tiles = 0
         for t in range(wl.n_q):
             sel = idx[t][idx[t] >= 0]
-            pages += np.unique(sel // sp.page_size).size
-        rows = int((n_sel * row_b).sum()) + 4 * pages
+            tiles += np.unique(sel // tile_t).size * (sp.d_latent // tile_d)
+        rows = int((n_sel * row_b).sum()) + 4 * tiles
     else:
         row_b = (sp.d_latent + sp.d_rope) * (2 if sp.kv_dtype == "bf16" else 4)
         rows = int((n_sel * row_b).sum())
@@ -168,15 +204,15 @@ class ClockSampler:
                 "samples": len(self.samples), "source": "nvml"}
 
 
-def traffic_for(kernel: str, source_files: list[str]):
-    """DRAM bytes per launch from the committed ncu summary, if the kernel's
-    sources are unchanged since the capture; otherwise None."""
+def traffic_for(kernel: str, source_files: list[str], workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    this workload and the kernel's sources are unchanged since; otherwise None."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         rec = json.load(open(path)).get(kernel)
     except Exception:
         return None
-    if not rec:
+    if not rec or rec.get("workload") != workload:
         return None
     h = hashlib.sha256()
     for f in source_files:
@@ -288,7 +324,8 @@ def run_ours(args, rank: int, world: int, dist):
     st = api.device_status(ws)
     if st[0] != _abi.SA_OK:
         raise RuntimeError(f"device status after warm-up: {st}")
-    nbytes = algorithmic_bytes(wl, idx.cpu().numpy())
+    idx_host = idx.cpu().numpy()
+    nbytes = algorithmic_bytes(wl, idx_host)
 
     n_phase = len(_abi.DECODE_PHASES)
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_phase + 1)]
@@ -387,18 +424,17 @@ def run_ours(args, rank: int, world: int, dist):
 
     ms_per_step = total_ms / args.steps
     value = n_q_all * args.steps / (total_ms / 1e3)
-    peak, peak_kind = measured_peaks()
+    peak, _, peak_kind = measured_peaks()
     dom = int(np.argmax(phase_ms))
     dom_name = _abi.DECODE_PHASES[dom]
-    dom_bytes = nbytes[dom_name]
-    achieved = dom_bytes / (phase_ms[dom] / 1e3) / 1e9 if phase_ms[dom] > 0 else 0.0
+    roof = roofline(wl, dom_name, phase_ms[dom], nbytes, algorithmic_flops(wl, idx_host))
     step_gbs = nbytes["total"] / (ms_per_step / 1e3) / 1e9
     csrc = "indexed_sparse_attention_lightning_b200/csrc/"
     shared = [csrc + f for f in ("common.cuh", "sm100.cuh", "internal.h")]
     kernel_src = {"indexer": [csrc + "indexer_mma.cu", csrc + "plan.cu"] + shared,
                   "topk": [csrc + "topk.cu"] + shared,
                   "attention": [csrc + "sfa_mma.cu"] + shared}
-    traffic = traffic_for(dom_name, kernel_src[dom_name])
+    traffic = traffic_for(dom_name, kernel_src[dom_name], sp.name)
 
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
@@ -418,9 +454,7 @@ def run_ours(args, rank: int, world: int, dist):
             "index_heads": sp.h_index, "index_dim": sp.d_index, "kv_dtype": sp.kv_dtype,
             "page_size": sp.page_size, "l2": "flushed before every timed step (256 MiB write)",
             "parallelism": f"replicas x{world}"},
-        "roofline": {"bound": "hbm", "kernel": dom_name, "achieved": achieved, "peak": peak,
-                     "peak_kind": peak_kind, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": traffic},
+        "roofline": dict(roof, traffic=traffic if roof["bound"] == "hbm" else None),
         "path_hbm": {"bytes_per_step": nbytes["total"], "achieved_gbs": step_gbs,
                      "frac_of_measured": step_gbs / peak, "frac_of_8tbs": step_gbs / SPEC_HBM_GBS},
         "phases_ms": dict(zip(_abi.DECODE_PHASES, phase_ms)),
