@@ -65,10 +65,10 @@ class WorkloadSpec:
     page_size: int = 64
     paging: str = "permuted"       # "identity" or "permuted"
     keys: tuple = ("iid",)         # ("iid",), ("planted", frac, sigma), ("clusters", n, span)
-    sm_scale: Optional[float] = None
+    sm_scale: Optional[float] = None  # default 1/sqrt(d_latent + d_rope)
     # e4m3 latent cache: one fp32 scale per tile of (tokens of a page, latent
     # dims); (0, 0) is one scale per page
-    kv_scale_tile: tuple = (0, 0)  # default 1/sqrt(d_latent + d_rope)
+    kv_scale_tile: tuple = (0, 0)
     poison_pages: int = 2
 
     @property

@@ -1,0 +1,64 @@
+"""Host-side accounting of bench.py: algorithmic bytes and flops per phase and
+the choice of roofline (decode against HBM, chunked prefill against the
+tensor pipe).  No GPU: the selections are made up on the host."""
+import numpy as np
+
+import bench
+from indexed_sparse_attention_lightning_b200 import workloads as W
+
+
+def _first_k(wl, K):
+    """Positions 0 .. min(K, V_t) - 1 of every query, -1 padded."""
+    idx = np.full((wl.n_q, K), -1, dtype=np.int32)
+    for t, v in enumerate(wl.visible):
+        n = min(K, int(v))
+        idx[t, :n] = np.arange(n)
+    return idx
+
+
+def test_decode_bytes_and_hbm_roofline():
+    wl = W.make_workload(W.spec("tiny_decode_b1_1k_fp32"))
+    sp = wl.spec
+    idx = _first_k(wl, sp.top_k)
+    nb = bench.algorithmic_bytes(wl, idx)
+    V = int(wl.visible.sum())
+    assert nb["indexer"] == V * sp.d_index * 4                     # fp32 keys, no scales
+    rows = int(np.minimum(wl.visible, sp.top_k).sum()) * (sp.d_latent + sp.d_rope) * 4
+    outs = wl.n_q * sp.heads * (sp.d_latent * 4 + 4)
+    assert nb["attention"] == rows + outs
+    assert nb["total"] == nb["indexer"] + nb["attention"]
+    r = bench.roofline(wl, "attention", 1.0, nb, bench.algorithmic_flops(wl, idx))
+    hbm, _, _ = bench.measured_peaks()
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s"
+    assert np.isclose(r["achieved"], nb["attention"] / 1e-3 / 1e9)
+    assert np.isclose(r["frac"], r["achieved"] / hbm)
+
+
+def test_fp8_cache_counts_each_scale_tile_once():
+    import dataclasses
+    sp = dataclasses.replace(W.spec("decode_b8_8k"), batch=1, seq_len=("fixed", 256),
+                             kv_dtype="e4m3", kv_scale_tile=(1, 128), top_k=64)
+    wl = W.make_workload(sp)
+    idx = _first_k(wl, sp.top_k)
+    nb = bench.algorithmic_bytes(wl, idx)
+    per_row = sp.d_latent + 2 * sp.d_rope + 4 * (sp.d_latent // 128)
+    assert nb["attention"] == 64 * per_row + sp.heads * (sp.d_latent * 2 + 4)
+
+
+def test_prefill_is_reported_against_the_tensor_pipe():
+    import dataclasses
+    sp = dataclasses.replace(W.spec("prefill_4096q_64k"), seq_len=("fixed", 4096),
+                             queries=("prefill", 4032, 64))
+    wl = W.make_workload(sp)
+    assert wl.n_q > wl.seq_len.shape[0]
+    idx = _first_k(wl, sp.top_k)
+    fl = bench.algorithmic_flops(wl, idx)
+    assert fl["indexer"] == int(wl.visible.sum()) * 2 * sp.h_index * sp.d_index
+    assert fl["attention"] == int((idx >= 0).sum()) * 2 * sp.heads * (2 * sp.d_latent + sp.d_rope)
+    _, bf16, _ = bench.measured_peaks()
+    r = bench.roofline(wl, "indexer", 2.0, bench.algorithmic_bytes(wl, idx), fl)
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
+    assert np.isclose(r["peak"], 2 * bf16)                          # e4m3 indexer
+    assert np.isclose(r["achieved"], fl["indexer"] / 2e-3 / 1e12)
+    r = bench.roofline(wl, "attention", 2.0, bench.algorithmic_bytes(wl, idx), fl)
+    assert np.isclose(r["peak"], bf16)
