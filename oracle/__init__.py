@@ -60,6 +60,12 @@ def _load():
                                            I32, I32, P, I32, I32, I32, P, I32, P, P,
                                            ctypes.c_int]
         lib.oracle_sparse_attn.restype = ctypes.c_int
+        lib.oracle_quantize_e4m3.argtypes = [I64, I32, P, P, P]
+        lib.oracle_quantize_e4m3.restype = ctypes.c_int
+        lib.oracle_e4m3_encode.argtypes = [I64, P, P]
+        lib.oracle_e4m3_encode.restype = ctypes.c_int
+        lib.oracle_to_bf16.argtypes = [I64, P, P]
+        lib.oracle_to_bf16.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -148,6 +154,103 @@ def sparse_attn(wl, idx: np.ndarray, nthreads: int | None = None):
         _ptr(out), _ptr(lse), nthreads or threads())
     _check(rc, "sparse_attn")
     return out, lse
+
+
+# ---------------------------------------------------------------------------
+# Input preparation ("Optimizing Next-Gen LLM Inference", §3.2 and the §4
+# table; "Inference Acceleration for New Large Model Architectures", §3.3 and
+# §4.1-4.2).  The arithmetic (scale, quotient, rounding) is in sa_oracle.c;
+# this part only reshapes and scatters.
+# ---------------------------------------------------------------------------
+
+def widen(dtype: str, a: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns (uint16) or fp32 values -> fp32 values, exactly."""
+    if dtype == "bf16":
+        return (np.ascontiguousarray(a, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
+    return np.ascontiguousarray(a, dtype=np.float32)
+
+
+def quantize_e4m3(x: np.ndarray, group: int):
+    """Dynamic FP8 quantisation of the last axis in groups of ``group`` values:
+    (codes uint8, same shape; scales f32 [..., last / group])."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    if x.shape[-1] % group:
+        raise ValueError("the last axis must be a multiple of the group")
+    codes = np.empty(x.shape, dtype=np.uint8)
+    scales = np.empty(x.shape[:-1] + (x.shape[-1] // group,), dtype=np.float32)
+    rc = _load().oracle_quantize_e4m3(x.size // group, group, _ptr(x), _ptr(codes), _ptr(scales))
+    _check(rc, "quantize_e4m3")
+    return codes, scales
+
+
+def e4m3_encode(x: np.ndarray) -> np.ndarray:
+    """fp32 values -> e4m3 codes (round to nearest even, saturating), no scale."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    codes = np.empty(x.shape, dtype=np.uint8)
+    _check(_load().oracle_e4m3_encode(x.size, _ptr(x), _ptr(codes)), "e4m3_encode")
+    return codes
+
+
+def to_bf16(x: np.ndarray) -> np.ndarray:
+    """fp32 values -> bf16 bit patterns (uint16), round to nearest even."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    bits = np.empty(x.shape, dtype=np.uint16)
+    _check(_load().oracle_to_bf16(x.size, _ptr(x), _ptr(bits)), "to_bf16")
+    return bits
+
+
+def quantize_index_query(q: np.ndarray):
+    """Indexer query [n_q, h, d] (fp32 values) -> e4m3 codes + one scale per
+    (token, head): the form the FP8 indexer consumes."""
+    codes, scales = quantize_e4m3(q, q.shape[-1])
+    return codes, scales[..., 0]
+
+
+def append_tokens(pools: dict, layout: dict, seq, pos, k_new=None, kv_new=None):
+    """Write new tokens into copies of the paged pools.
+
+    pools: ``k_index``, ``k_index_scale``, ``kv``, ``kv_rope``, ``kv_scale`` (numpy
+    arrays shaped as the cache stores them; absent entries are None).
+    layout: ``page_table`` [batch, max_pages], ``page_size``, ``num_pages``,
+    ``index_dtype`` ("e4m3"/"f32"), ``kv_dtype`` ("e4m3"/"bf16"/"f32"), ``d_latent``,
+    ``kv_scale_dims`` (latent dims per scale; one token per scale).
+    k_new [n, d_index], kv_new [n, d_latent + d_rope]: fp32 values.
+    Token i goes to physical row page_table[seq, pos // page_size] * page_size +
+    pos % page_size; a token whose sequence, position or page id is out of range
+    is skipped.  Returns (new pools, list of (token, "position" | "page") skips)."""
+    out = {k: (None if v is None else v.copy()) for k, v in pools.items()}
+    pt = layout["page_table"]
+    ps, n_pages = layout["page_size"], layout["num_pages"]
+    dl = layout["d_latent"]
+    skipped = []
+    for i, (b, p) in enumerate(zip(np.asarray(seq).tolist(), np.asarray(pos).tolist())):
+        if not (0 <= b < pt.shape[0]) or p < 0 or p // ps >= pt.shape[1]:
+            skipped.append((i, "position"))
+            continue
+        page = int(pt[b, p // ps])
+        if not (0 <= page < n_pages):
+            skipped.append((i, "page"))
+            continue
+        slot = p % ps
+        if k_new is not None:
+            if layout["index_dtype"] == "e4m3":
+                codes, sc = quantize_e4m3(k_new[i], k_new.shape[-1])
+                out["k_index"][page, slot] = codes
+                out["k_index_scale"][page, slot] = sc[0]
+            else:
+                out["k_index"][page, slot] = k_new[i]
+        if kv_new is not None:
+            row = np.asarray(kv_new[i], dtype=np.float32)
+            if layout["kv_dtype"] == "e4m3":
+                codes, sc = quantize_e4m3(row[:dl], layout["kv_scale_dims"])
+                out["kv"][page, slot] = codes
+                out["kv_scale"][page, slot] = sc
+                out["kv_rope"][page, slot] = to_bf16(row[dl:])
+            elif layout["kv_dtype"] == "bf16":
+                out["kv"][page, slot] = to_bf16(row)
+            else:
+                out["kv"][page, slot] = row
+    return out, skipped
 
 
 def run(wl, nthreads: int | None = None) -> dict:

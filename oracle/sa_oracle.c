@@ -467,3 +467,125 @@ int oracle_sparse_attn(int32_t n_q, const int32_t *q_seq, const int32_t *q_pos,
                    { page_table, max_pages, page_size, num_pages }, idx, K, out, lse };
     return pool_run(attn_item, &c, n_q, nthreads);
 }
+
+/* ---------------------------------------------------------------------------
+ * Input preparation ("Optimizing Next-Gen LLM Inference", §3.2 and the §4
+ * table; "Inference Acceleration for New Large Model Architectures", §3.3 and
+ * §4.1-4.2): dynamic FP8 quantisation of the indexer query and of new index
+ * keys, and block-quantised rows appended to the latent cache.
+ *
+ * The pages fix the format (8-bit float, one scale per group) but not the
+ * arithmetic.  The reading used here: per group of values, in fp32,
+ *     amax  = max |x|,   scale = amax / 448   (1 when amax is 0),
+ *     code  = e4m3(x / scale), rounded to nearest, ties to even, saturated
+ *             to +-448,
+ * so that the largest magnitude lands on e4m3's largest finite value.  The
+ * scale and the quotient are fp32 operations (what the kernel does), because
+ * they decide an integer code; the rounding to e4m3 is then taken exactly,
+ * in double, from that fp32 value.
+ * ------------------------------------------------------------------------- */
+
+/* Exact fp32 value -> OCP e4m3fn code.  e4m3 values are integers times
+ * 2^(e-3) for the binade [2^e, 2^(e+1)), e >= -6; below 2^-6 the spacing
+ * stays 2^-9 (subnormals).  The value must not be NaN. */
+static uint8_t e4m3_code(float xf)
+{
+    double x = (double)xf;
+    uint8_t sign = signbit(x) ? 0x80 : 0x00;
+    double a = fabs(x);
+    if (a >= 448.0)
+        return sign | 0x7E;                  /* saturate: S.1111.110 = 448 */
+    if (a == 0.0)
+        return sign;
+    int e2;
+    frexp(a, &e2);                           /* a = f * 2^e2, f in [0.5, 1) */
+    int e = e2 - 1;                          /* a in [2^e, 2^(e+1)) */
+    if (e < -6)
+        e = -6;
+    double step = ldexp(1.0, e - 3);
+    double q = nearbyint(a / step) * step;   /* a / step is exact; ties to even */
+    if (q < ldexp(1.0, -6))                  /* subnormal: m * 2^-9, m in 0..7 */
+        return sign | (uint8_t)(q / ldexp(1.0, -9));
+    frexp(q, &e2);
+    e = e2 - 1;                              /* rounding may have moved q up a binade */
+    int m = (int)((q / ldexp(1.0, e) - 1.0) * 8.0);
+    return sign | (uint8_t)((e + 7) << 3) | (uint8_t)m;
+}
+
+/* Exact fp32 value -> bf16 bits, round to nearest, ties to even (finite
+ * values; bf16 keeps fp32's exponent and the top 7 fraction bits). */
+static uint16_t bf16_code(float xf)
+{
+    double x = (double)xf;
+    double a = fabs(x);
+    uint16_t sign = signbit(x) ? 0x8000 : 0x0000;
+    if (a == 0.0)
+        return sign;
+    int e2;
+    frexp(a, &e2);
+    int e = e2 - 1;
+    if (e < -126)
+        e = -126;                            /* bf16 subnormals share fp32's range */
+    double step = ldexp(1.0, e - 7);
+    double q = nearbyint(a / step) * step;
+    if (q >= ldexp(1.0, 128))
+        return sign | 0x7F80;                /* overflow rounds to infinity */
+    if (q < ldexp(1.0, -126))
+        return sign | (uint16_t)(q / ldexp(1.0, -133));
+    frexp(q, &e2);
+    e = e2 - 1;
+    int m = (int)((q / ldexp(1.0, e) - 1.0) * 128.0);
+    return sign | (uint16_t)((e + 127) << 7) | (uint16_t)m;
+}
+
+/* n_groups groups of `group` consecutive fp32 values -> e4m3 codes and one
+ * fp32 scale per group (rule above). */
+int oracle_quantize_e4m3(int64_t n_groups, int32_t group, const float *x, uint8_t *codes,
+                         float *scales)
+{
+    if (n_groups < 0 || group <= 0 || (n_groups > 0 && (!x || !codes || !scales)))
+        return OR_BAD_ARG;
+    for (int64_t g = 0; g < n_groups; g++) {
+        const float *v = x + g * group;
+        float amax = 0.0f;
+        for (int32_t i = 0; i < group; i++) {
+            if (isnan(v[i]))
+                return OR_NAN;
+            if (fabsf(v[i]) > amax)
+                amax = fabsf(v[i]);
+        }
+        float scale = amax > 0.0f ? amax / 448.0f : 1.0f;
+        scales[g] = scale;
+        for (int32_t i = 0; i < group; i++) {
+            float r = v[i] / scale;
+            codes[g * group + i] = e4m3_code(r);
+        }
+    }
+    return OR_OK;
+}
+
+/* n fp32 values -> bf16 bits. */
+int oracle_to_bf16(int64_t n, const float *x, uint16_t *bits)
+{
+    if (n < 0 || (n > 0 && (!x || !bits)))
+        return OR_BAD_ARG;
+    for (int64_t i = 0; i < n; i++) {
+        if (isnan(x[i]))
+            return OR_NAN;
+        bits[i] = bf16_code(x[i]);
+    }
+    return OR_OK;
+}
+
+/* n fp32 values -> e4m3 codes directly (no scale), for pinning the encoder. */
+int oracle_e4m3_encode(int64_t n, const float *x, uint8_t *codes)
+{
+    if (n < 0 || (n > 0 && (!x || !codes)))
+        return OR_BAD_ARG;
+    for (int64_t i = 0; i < n; i++) {
+        if (isnan(x[i]))
+            return OR_NAN;
+        codes[i] = e4m3_code(x[i]);
+    }
+    return OR_OK;
+}

@@ -378,3 +378,165 @@ def test_parity_checker_accepts_tie_swaps_and_rejects_real_errors():
     scores2 = np.array([[5.0, 1.0, 3.0, 3.0000001, 0.5, 3.0000002]])
     r = check_topk(np.array([[0, 2, 5]]), scores2, valid, 3)
     assert r["swaps"] == 1
+
+
+# ------------------------------------------------------- input preparation ---
+# Pins for the FP8 / bf16 encoders and the append scatter of the oracle.
+
+def torch_e4m3(x):
+    """torch's own fp32 -> e4m3fn conversion (round to nearest even)."""
+    return torch.from_numpy(np.asarray(x, dtype=np.float32)).to(torch.float8_e4m3fn) \
+        .view(torch.uint8).numpy()
+
+
+def e4m3_table():
+    """All finite e4m3 codes and their values, from torch."""
+    codes = np.array([c for c in range(256) if c & 0x7F != 0x7F], dtype=np.uint8)
+    vals = torch.from_numpy(codes).view(torch.float8_e4m3fn).float().numpy()
+    return codes, vals
+
+
+def test_e4m3_encoder_round_trips_every_finite_code():
+    codes, vals = e4m3_table()
+    got = oracle.e4m3_encode(vals)
+    # -0 and +0 both encode by sign; every other value has exactly one code
+    assert np.array_equal(got, codes)
+
+
+def test_e4m3_encoder_matches_torch_including_ties():
+    rng = np.random.default_rng(11)
+    mags = np.exp2(rng.uniform(-12, np.log2(448.0), 20000)).astype(np.float32)
+    x = mags * rng.choice([-1.0, 1.0], mags.size).astype(np.float32)
+    _, vals = e4m3_table()
+    v = np.unique(vals[vals > 0])
+    mids = ((v[:-1].astype(np.float64) + v[1:]) / 2).astype(np.float32)  # exact in fp32
+    x = np.concatenate([x, mids, -mids, np.float32(2.0 ** -10) * np.arange(1, 9,
+                                                                            dtype=np.float32)])
+    assert np.array_equal(oracle.e4m3_encode(x), torch_e4m3(x))
+
+
+def test_e4m3_encoder_closed_forms():
+    x = np.array([449, 464, 1e30, -1e30, 2 ** -10, 3 * 2 ** -10, 2 ** -9, 1.0625, 1.1875, 0.0,
+                  -0.0, 240, 248, 256], dtype=np.float32)
+    # 464 is the midpoint of 448 and (non-finite) 480: saturation keeps 448;
+    # 2^-10 ties to 0 (even), 3*2^-10 to 2*2^-9, 1.0625 to 1.0, 1.1875 to 1.25;
+    # 248 is the midpoint of 240 (mantissa 7, odd) and 256 (mantissa 0, even)
+    want = [0x7E, 0x7E, 0x7E, 0xFE, 0x00, 0x02, 0x01, 0x38, 0x3A, 0x00, 0x80, 0x77, 0x78,
+            0x78]
+    assert oracle.e4m3_encode(x).tolist() == want
+
+
+def test_bf16_encoder_matches_torch():
+    rng = np.random.default_rng(12)
+    bits = rng.integers(0, 2 ** 32, 50000, dtype=np.uint64).astype(np.uint32)
+    bits = bits[(bits & 0x7F800000) != 0x7F800000]          # finite only
+    ties = (rng.integers(0, 2 ** 16, 2000).astype(np.uint32) << 16) | 0x8000
+    ties = ties[(ties & 0x7F800000) != 0x7F800000]
+    x = np.concatenate([bits, ties]).view(np.float32)
+    want = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(oracle.to_bf16(x), want)
+
+
+def test_group_quantisation_rule():
+    rng = np.random.default_rng(13)
+    x = (rng.standard_normal((300, 128)) * np.exp2(rng.uniform(-8, 8, (300, 1)))) \
+        .astype(np.float32)
+    x[7] = 0.0                                               # an all-zero group
+    codes, scales = oracle.quantize_e4m3(x, 32)
+    assert codes.shape == x.shape and scales.shape == (300, 4)
+    g = x.reshape(300, 4, 32)
+    amax = np.abs(g).max(axis=-1)
+    want_scale = np.where(amax > 0, amax / np.float32(448.0), np.float32(1.0)).astype(np.float32)
+    assert np.array_equal(scales, want_scale)                # fp32 division, as numpy does it
+    assert np.all(codes[7] == 0) and np.all(scales[7] == 1.0)
+    # each code is torch's rounding of the fp32 quotient, so the largest
+    # magnitude of every group lands on +-448
+    q = (g / want_scale[..., None]).astype(np.float32)
+    assert np.array_equal(codes.reshape(300, 4, 32), torch_e4m3(q))
+    c = codes.reshape(300, 4, 32)
+    top = np.take_along_axis(c, np.abs(g).argmax(axis=-1)[..., None], axis=-1)[..., 0]
+    live = amax > 0
+    assert np.all((top[live] & 0x7F) == 0x7E)
+    # dequantised error within half an e4m3 step of the quotient
+    _, vals = e4m3_table()
+    deq = torch.from_numpy(c.copy()).view(torch.float8_e4m3fn).float().numpy()
+    step = np.exp2(np.maximum(np.floor(np.log2(np.maximum(np.abs(q), 2.0 ** -9))), -6) - 3)
+    assert np.all(np.abs(deq - q) <= step / 2 + 1e-12)
+
+
+def test_query_quantisation_agrees_with_the_input_generator():
+    rng = np.random.default_rng(14)
+    q = rng.standard_normal((9, 64, 128)).astype(np.float32)
+    codes, scales = oracle.quantize_index_query(q)
+    gen_codes, gen_scales = W.quantize_rows_e4m3(q)
+    assert np.array_equal(codes, gen_codes) and np.array_equal(scales, gen_scales)
+
+
+def _pools(rng, kv_dtype, P=6, ps=64, d_index=32, d_latent=64, d_rope=16, dims=16):
+    pools = {"k_index": rng.integers(0, 255, (P, ps, d_index), dtype=np.uint8),
+             "k_index_scale": rng.random((P, ps), dtype=np.float32),
+             "kv_rope": None, "kv_scale": None}
+    if kv_dtype == "e4m3":
+        pools["kv"] = rng.integers(0, 255, (P, ps, d_latent), dtype=np.uint8)
+        pools["kv_rope"] = rng.integers(0, 2 ** 15, (P, ps, d_rope), dtype=np.uint16)
+        pools["kv_scale"] = rng.random((P, ps, d_latent // dims), dtype=np.float32)
+    elif kv_dtype == "bf16":
+        pools["kv"] = rng.integers(0, 2 ** 15, (P, ps, d_latent + d_rope), dtype=np.uint16)
+    else:
+        pools["kv"] = rng.random((P, ps, d_latent + d_rope), dtype=np.float32)
+    return pools
+
+
+@pytest.mark.parametrize("kv_dtype", ["e4m3", "bf16", "f32"])
+def test_append_scatters_through_the_page_table(kv_dtype):
+    rng = np.random.default_rng(15)
+    P, ps, d_index, d_latent, d_rope, dims = 6, 64, 32, 64, 16, 16
+    pools = _pools(rng, kv_dtype)
+    table_a = np.array([[4, 1, -1], [0, 5, 9]], dtype=np.int32)   # 9: bad page id
+    layout = {"page_table": table_a, "page_size": ps, "num_pages": P, "index_dtype": "e4m3",
+              "kv_dtype": kv_dtype, "d_latent": d_latent, "kv_scale_dims": dims}
+    seq = np.array([0, 0, 1, 1, 2, 0, -1, 1, 0])
+    pos = np.array([3, 127, 64, 130, 0, 128, 0, 200, -5])
+    k_new = rng.standard_normal((9, d_index)).astype(np.float32)
+    kv_new = rng.standard_normal((9, d_latent + d_rope)).astype(np.float32)
+    out, skipped = oracle.append_tokens(pools, layout, seq, pos, k_new, kv_new)
+    # seq 0 pos 128 hits a -1 slot; seq 1 pos 130 hits page 9; pos 200 is past max_pages
+    assert sorted(skipped) == [(3, "page"), (4, "position"), (5, "page"), (6, "position"),
+                               (7, "position"), (8, "position")]
+    written = {(4, 3): 0, (1, 63): 1, (5, 0): 2}                # (page, slot) -> token
+    for name, a in pools.items():
+        if a is None:
+            continue
+        changed = {(p, s) for p, s in zip(*np.nonzero(
+            (out[name] != a).reshape(P, ps, -1).any(axis=-1)))}
+        assert changed <= set(written), name
+    for (page, slot), i in written.items():
+        assert np.array_equal(out["k_index"][page, slot], torch_e4m3(
+            k_new[i] / out["k_index_scale"][page, slot]))
+        assert out["k_index_scale"][page, slot] == np.abs(k_new[i]).max() / np.float32(448)
+        if kv_dtype == "e4m3":
+            sc = out["kv_scale"][page, slot]
+            lat = kv_new[i, :d_latent].reshape(-1, dims)
+            assert np.array_equal(sc, np.abs(lat).max(axis=-1) / np.float32(448))
+            assert np.array_equal(out["kv"][page, slot].reshape(-1, dims),
+                                  torch_e4m3(lat / sc[:, None]))
+            want_rope = torch.from_numpy(kv_new[i, d_latent:]).to(torch.bfloat16) \
+                .view(torch.int16).numpy().view(np.uint16)
+            assert np.array_equal(out["kv_rope"][page, slot], want_rope)
+        elif kv_dtype == "bf16":
+            want = torch.from_numpy(kv_new[i]).to(torch.bfloat16).view(torch.int16).numpy() \
+                .view(np.uint16)
+            assert np.array_equal(out["kv"][page, slot], want)
+        else:
+            assert np.array_equal(out["kv"][page, slot], kv_new[i])
+    # the same tokens through a permuted table land at the same logical rows
+    perm = np.array([2, 3, 0, 5, 1, 4])
+    layout_b = dict(layout, page_table=np.where(table_a >= 0, perm[np.clip(table_a, 0, 5)],
+                                                table_a).astype(np.int32))
+    layout_b["page_table"][1, 2] = 9
+    pools_b = {k: None if v is None else v[np.argsort(perm)] for k, v in pools.items()}
+    out_b, skipped_b = oracle.append_tokens(pools_b, layout_b, seq, pos, k_new, kv_new)
+    assert skipped_b == skipped
+    for name in pools:
+        if pools[name] is not None:
+            assert np.array_equal(out_b[name][perm], out[name])
