@@ -38,7 +38,7 @@ def _rank_main(rank: int, world: int, port: int, results):
 
 def test_two_gloo_ranks_take_max_time_and_total_queries():
     world = 2
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:
         results = m.dict()
         mp.start_processes(_rank_main, args=(world, _free_port(), results), nprocs=world,
                            join=True, start_method="spawn")
