@@ -294,6 +294,78 @@ def reduce_over_ranks(dist, device, step_ms: float, e2e_ms: float, n_q: int):
     return float(t[0]), float(t[1]), float(q[0])
 
 
+def input_prep_bytes(wl, with_kv: bool) -> int:
+    """Algorithmic bytes of one step's input preparation: the bf16 indexer query
+    read, its e4m3 codes and scales written; per new token the bf16 key read and
+    its code row and scale written, and (with_kv) the bf16 latent row read and
+    its stored form written."""
+    sp = wl.spec
+    n, h, d = wl.n_q, sp.h_index, sp.d_index
+    b = n * h * d * 2 + n * h * d + n * h * 4
+    b += n * (d * 2 + d + 4)
+    if with_kv:
+        D = sp.d_latent + sp.d_rope
+        if sp.kv_dtype == "e4m3":
+            stored = sp.d_latent + 2 * sp.d_rope + 4 * (sp.d_latent // sp.kv_tile[1])
+        else:
+            stored = D * (2 if sp.kv_dtype == "bf16" else 4)
+        b += n * (D * 2 + stored)
+    return b
+
+
+def time_input_prep(args, wl, cache, dev, flush):
+    """One step's input preparation, timed on its own after the decode timing:
+    the indexer query quantised from bf16, and one new token per query (decode's
+    newest token, a prefill chunk's tokens) appended at the query's position to
+    both caches.  A latent cache with one scale per page cannot take single
+    tokens; there only the keys are appended."""
+    import torch
+    from indexed_sparse_attention_lightning_b200 import api
+    sp = wl.spec
+    if sp.index_dtype != "e4m3":
+        return None
+    with_kv = not (sp.kv_dtype == "e4m3" and sp.kv_tile[0] != 1)
+    g = torch.Generator(device=dev)
+    g.manual_seed(sp.seed + 77)
+    qi = torch.randn((wl.n_q, sp.h_index, sp.d_index), generator=g, device=dev).bfloat16()
+    k_new = torch.randn((wl.n_q, sp.d_index), generator=g, device=dev).bfloat16()
+    kv_new = (torch.randn((wl.n_q, sp.d_latent + sp.d_rope), generator=g, device=dev)
+              .bfloat16() if with_kv else None)
+    seq = torch.from_numpy(wl.q_seq).to(dev)
+    pos = torch.from_numpy(wl.q_pos).to(dev)
+    q_out = torch.empty((wl.n_q, sp.h_index, sp.d_index), dtype=torch.uint8, device=dev)
+    q_scale = torch.empty((wl.n_q, sp.h_index), dtype=torch.float32, device=dev)
+    ws = api.workspace(256, dev)
+
+    def step():
+        api.quantize_index_query(qi, out=q_out, scale=q_scale)
+        api.append_tokens(cache, seq, pos, k_index=k_new, kv=kv_new, ws=ws)
+
+    stream = torch.cuda.current_stream()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    for k in range(args.steps):
+        flush.zero_()
+        ev[k][0].record(stream)
+        step()
+        ev[k][1].record(stream)
+    torch.cuda.synchronize()
+    st = api.device_status(ws)
+    if st[0] != 0:
+        raise RuntimeError(f"device status after input preparation: {st}")
+    ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
+    nb = input_prep_bytes(wl, with_kv)
+    hbm, _, kind = measured_peaks()
+    gbs = nb / (ms / 1e3) / 1e9
+    return {"ms": ms, "bytes": nb, "achieved_gbs": gbs, "frac": gbs / hbm, "peak_kind": kind,
+            "launches": 2, "appends_latent": with_kv,
+            "what": "bf16 indexer query -> e4m3 + scales; one bf16 key (and latent row) "
+                    "per query appended at its position"}
+
+
 def run_ours(args, rank: int, world: int, dist):
     import torch
     from indexed_sparse_attention_lightning_b200 import _abi, api
@@ -417,6 +489,8 @@ def run_ours(args, rank: int, world: int, dist):
         d2h = out.numel() * out.element_size() + lse.numel() * lse.element_size()
         e2e = {"ms_per_step": e2e_total / args.steps, "h2d": h2d, "d2h": d2h}
 
+    prep = time_input_prep(args, wl, cache, dev, flush)
+
     total_ms, e2e_step_ms, n_q_all = reduce_over_ranks(
         dist, dev, total_ms, e2e["ms_per_step"] if e2e else 0.0, wl.n_q)
     if rank != 0:
@@ -461,6 +535,7 @@ def run_ours(args, rank: int, world: int, dist):
         "gpu_launches": int(launches),
         "clocks": clocks.summary(),
         "cpu_baseline": cpu,
+        "input_prep": prep,
     }
     if e2e:
         line["e2e"] = {"value": n_q_all / (e2e_step_ms / 1e3), "unit": UNIT,

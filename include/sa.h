@@ -17,7 +17,9 @@
  * ("Optimizing Next-Gen LLM Inference" §3.1; "Inference Acceleration" §3.1).
  * Index keys and the latent cache may be FP8 ("Optimizing Next-Gen LLM
  * Inference" §4): index keys as e4m3 with one fp32 scale per token, the latent
- * as e4m3 with one fp32 scale per 64-token page tile (rope stays bf16).
+ * as e4m3 with one fp32 scale per tile of tokens x latent dims (a whole page
+ * by default; rope stays bf16).  Input preparation quantises the query and
+ * appends new tokens in these formats.
  *
  * Conventions for every entry point
  *  - All pointers marked "device" are CUDA device pointers owned by the
@@ -138,7 +140,8 @@ enum {
     SA_WS_INDEXER = 1,
     SA_WS_TOPK = 2,
     SA_WS_ATTN = 4,
-    SA_WS_DECODE = 8
+    SA_WS_DECODE = 8,
+    SA_WS_APPEND = 16             /* sa_append_tokens alone: `query` may be NULL */
 };
 
 /* Bytes of device workspace the entry points in `uses` (an OR of SA_WS_*)
@@ -225,6 +228,62 @@ SA_API sa_status sa_decode_traced(const sa_cache *cache, const sa_query *query, 
 SA_API sa_status sa_decode_noalloc(const sa_cache *cache, const sa_query *query, int32_t top_k,
                                    int32_t *idx_out, void *out, sa_dtype out_dtype, float *lse,
                                    void *stream);
+
+/* ---- Input preparation -------------------------------------------------
+ * Before the indexer runs, the query is quantised and the step's new tokens
+ * are written into the paged caches ("Optimizing Next-Gen LLM Inference"
+ * §3.2 input preparation and the §4 table; "Inference Acceleration for New
+ * Large Model Architectures" §3.3 and §4.1-4.2).  Projections and key
+ * normalisation stay with the caller (they need the model's weights); these
+ * calls take their bf16 or fp32 outputs.
+ *
+ * FP8 rule, per group of values, in fp32: amax = max |x|, scale = amax / 448
+ * (1 for an all-zero group), code = e4m3(x / scale) with an IEEE
+ * round-to-nearest division, rounded to nearest even and saturated to +-448.
+ * Inputs must be finite: a NaN or infinity gives unspecified codes. */
+
+/* Indexer query -> e4m3 codes + one fp32 scale per (token, head): the form
+ * sa_query.q_index / q_index_scale take for an SA_E4M3 index cache.
+ *   q_in:    device [n_q, h_index, d_index] in in_dtype (SA_BF16 or SA_F32)
+ *   q_out:   device uint8 [n_q, h_index, d_index]
+ *   q_scale: device fp32 [n_q, h_index]
+ * Needs no workspace and cannot fail on the device. */
+SA_API sa_status sa_quantize_index_query(const void *q_in, sa_dtype in_dtype, int32_t n_q,
+                                         int32_t h_index, int32_t d_index, void *q_out,
+                                         float *q_scale, void *stream);
+
+/* New tokens of one step: token i belongs to sequence seq[i] at logical
+ * position pos[i]. */
+typedef struct sa_new_tokens {
+    int32_t n_new;
+    const int32_t *seq;          /* device int32 [n_new] */
+    const int32_t *pos;          /* device int32 [n_new] */
+    sa_dtype in_dtype;           /* SA_BF16 or SA_F32, for both inputs below */
+    const void *k_index;         /* device [n_new, d_index] index keys, or NULL (not written) */
+    const void *kv;              /* device [n_new, d_latent + d_rope] latent + rope rows,
+                                  * or NULL (not written) */
+} sa_new_tokens;
+
+/* Writes each new token into the pools of `cache` at its physical row
+ * (page_table[seq * max_pages + pos / page_size] * page_size + pos % page_size):
+ *  - index key: SA_E4M3 pool -> codes + the token's scale (one group of
+ *    d_index values); SA_F32 pool -> the values;
+ *  - latent row: SA_BF16 / SA_F32 pool -> the row (fp32 inputs rounded to
+ *    nearest even for bf16); SA_E4M3 pool -> the latent quantised in groups of
+ *    kv_scale_dims values with its scales, the rope as bf16.  An SA_E4M3 pool
+ *    needs kv_scale_tokens == 1: a scale shared by several tokens would force
+ *    the others to be requantised, so other tiles return SA_ERR_UNSUPPORTED.
+ * The pools named by `cache` (k_index, k_index_scale, kv, kv_rope, kv_scale)
+ * are written in place and must be writable device memory; seq_len is neither
+ * read nor changed (the caller advances it).  Tokens must not share a row.
+ * A token whose sequence is outside [0, batch), whose position is negative or
+ * at or past max_pages * page_size, or whose page-table entry is outside
+ * [0, num_pages) is skipped and recorded in the workspace status word
+ * (SA_DETAIL_BAD_POSITION / SA_DETAIL_BAD_PAGE; read it with
+ * sa_device_status).  workspace: at least
+ * sa_workspace_size(cache, NULL, 0, SA_WS_APPEND) bytes, 256-byte aligned. */
+SA_API sa_status sa_append_tokens(const sa_cache *cache, const sa_new_tokens *tokens,
+                                  void *workspace, size_t workspace_bytes, void *stream);
 
 /* Device-side status of the most recent call that used `workspace`.
  * Synchronises `stream`.  Returns SA_OK, SA_ERR_DEVICE_FAULT or

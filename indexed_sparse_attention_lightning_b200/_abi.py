@@ -14,7 +14,7 @@ LIB_PATH = os.path.join(_HERE, "libsa.so")
 SA_OK, SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED, SA_ERR_WORKSPACE, SA_ERR_CUDA, \
     SA_ERR_DEVICE_FAULT, SA_ERR_TIMEOUT = range(7)
 SA_F32, SA_BF16, SA_E4M3 = 0, 1, 2
-SA_WS_INDEXER, SA_WS_TOPK, SA_WS_ATTN, SA_WS_DECODE = 1, 2, 4, 8
+SA_WS_INDEXER, SA_WS_TOPK, SA_WS_ATTN, SA_WS_DECODE, SA_WS_APPEND = 1, 2, 4, 8, 16
 SA_DETAIL_NONE, SA_DETAIL_BAD_PAGE, SA_DETAIL_BAD_POSITION, SA_DETAIL_BAD_INDEX, \
     SA_DETAIL_WAIT_TIMEOUT = range(5)
 
@@ -22,7 +22,8 @@ DTYPES = {"f32": SA_F32, "bf16": SA_BF16, "e4m3": SA_E4M3}
 
 # every symbol include/sa.h declares
 EXPORTS = ("sa_workspace_size", "sa_indexer_score", "sa_topk", "sa_sparse_mla_attn",
-           "sa_decode", "sa_decode_traced", "sa_decode_noalloc", "sa_device_status",
+           "sa_decode", "sa_decode_traced", "sa_decode_noalloc", "sa_quantize_index_query",
+           "sa_append_tokens", "sa_device_status",
            "sa_kernel_launches", "sa_status_string", "sa_version")
 NOALLOC_SCRATCH_BYTES = 32 << 20
 DECODE_PHASES = ("indexer", "topk", "attention")
@@ -45,6 +46,11 @@ class SaQuery(ctypes.Structure):
                 ("q_index", _P), ("q_index_scale", _P), ("w", _P), ("h_index", _I32),
                 ("q_dtype", ctypes.c_int), ("q", _P), ("heads", _I32),
                 ("sm_scale", ctypes.c_float)]
+
+
+class SaNewTokens(ctypes.Structure):
+    _fields_ = [("n_new", _I32), ("seq", _P), ("pos", _P), ("in_dtype", ctypes.c_int),
+                ("k_index", _P), ("kv", _P)]
 
 
 class SaError(RuntimeError):
@@ -82,6 +88,10 @@ def lib():
         L.sa_decode_traced.restype = ctypes.c_int
         L.sa_decode_noalloc.argtypes = [CP, QP, _I32, _P, _P, ctypes.c_int, _P, _P]
         L.sa_decode_noalloc.restype = ctypes.c_int
+        L.sa_quantize_index_query.argtypes = [_P, ctypes.c_int, _I32, _I32, _I32, _P, _P, _P]
+        L.sa_quantize_index_query.restype = ctypes.c_int
+        L.sa_append_tokens.argtypes = [CP, ctypes.POINTER(SaNewTokens), _P, _SZ, _P]
+        L.sa_append_tokens.restype = ctypes.c_int
         L.sa_device_status.argtypes = [_P, _SZ, _P, ctypes.POINTER(_I32)]
         L.sa_device_status.restype = ctypes.c_int
         L.sa_status_string.argtypes = [ctypes.c_int]

@@ -14,7 +14,7 @@ import numpy as np
 import torch
 
 from . import _abi
-from ._abi import SaCache, SaError, SaQuery, check
+from ._abi import SaCache, SaError, SaNewTokens, SaQuery, check
 
 _TORCH_RAW = {np.dtype(np.uint8): torch.uint8, np.dtype(np.uint16): torch.int16,
               np.dtype(np.float32): torch.float32, np.dtype(np.int32): torch.int32}
@@ -246,3 +246,56 @@ def decode(cache: DeviceCache, queries: DeviceQueries, top_k: int, out=None, lse
         handles = (ctypes.c_void_p * len(phase_events))(*[e.cuda_event for e in phase_events])
         check(_abi.lib().sa_decode_traced(*args, handles), "sa_decode_traced")
     return out, lse, idx
+
+
+# ------------------------------------------------------- input preparation ---
+
+_IN_DTYPES = {torch.bfloat16: "bf16", torch.float32: "f32"}
+
+
+def _in_dtype(t: torch.Tensor) -> int:
+    if t.dtype not in _IN_DTYPES:
+        raise SaError(_abi.SA_ERR_UNSUPPORTED, "input dtype (bfloat16 or float32)")
+    return _abi.DTYPES[_IN_DTYPES[t.dtype]]
+
+
+def quantize_index_query(q: torch.Tensor, out=None, scale=None, stream=None):
+    """Indexer query [n_q, h_index, d_index] (bfloat16 or float32) -> (e4m3 codes
+    uint8 [n_q, h_index, d_index], fp32 scales [n_q, h_index])."""
+    q = q.contiguous()
+    n_q, h, d = q.shape
+    if out is None:
+        out = torch.empty((n_q, h, d), dtype=torch.uint8, device=q.device)
+    if scale is None:
+        scale = torch.empty((n_q, h), dtype=torch.float32, device=q.device)
+    check(_abi.lib().sa_quantize_index_query(_ptr(q), _in_dtype(q), n_q, h, d, _ptr(out),
+                                             _ptr(scale), _stream(stream)),
+          "sa_quantize_index_query")
+    return out, scale
+
+
+def append_tokens(cache: DeviceCache, seq: torch.Tensor, pos: torch.Tensor,
+                  k_index: Optional[torch.Tensor] = None, kv: Optional[torch.Tensor] = None,
+                  ws=None, stream=None) -> torch.Tensor:
+    """Write new tokens (sequence, position) into the cache's pools in place:
+    index keys [n_new, d_index] and latent + rope rows [n_new, d_latent + d_rope],
+    both bfloat16 or both float32 (either may be None).  Returns the workspace,
+    whose status word records skipped tokens (see device_status)."""
+    ins = [t for t in (k_index, kv) if t is not None]
+    if len({t.dtype for t in ins}) > 1:
+        raise SaError(_abi.SA_ERR_INVALID_ARG, "append_tokens: k_index and kv dtypes differ")
+    k_index = None if k_index is None else k_index.contiguous()
+    kv = None if kv is None else kv.contiguous()
+    dt = _in_dtype(ins[0]) if ins else _abi.SA_BF16
+    c = cache.struct()
+    if ws is None:
+        n = _abi.lib().sa_workspace_size(ctypes.byref(c), None, 0, _abi.SA_WS_APPEND)
+        if n == 0:
+            raise SaError(_abi.SA_ERR_INVALID_ARG, "sa_workspace_size")
+        ws = workspace(n, seq.device)
+    t = SaNewTokens(n_new=int(seq.numel()), seq=_ptr(seq), pos=_ptr(pos), in_dtype=dt,
+                    k_index=_ptr(k_index), kv=_ptr(kv))
+    check(_abi.lib().sa_append_tokens(ctypes.byref(c), ctypes.byref(t), _ptr(ws), ws.numel(),
+                                      _stream(stream)),
+          "sa_append_tokens")
+    return ws

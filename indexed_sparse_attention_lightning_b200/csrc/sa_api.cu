@@ -9,6 +9,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "prep.h"
 #include "sa.h"
 
 namespace sa {
@@ -229,6 +230,7 @@ extern "C" {
 size_t sa_workspace_size(const sa_cache *cache, const sa_query *query, int32_t top_k,
                          int32_t uses) {
     if (check_cache(cache) != SA_OK) return 0;
+    if (uses == SA_WS_APPEND) return align_up(kStatusBytes);
     const bool idx = (uses & (SA_WS_INDEXER | SA_WS_DECODE)) != 0;
     const bool att = (uses & (SA_WS_ATTN | SA_WS_DECODE)) != 0;
     if (check_query(query, cache, idx, att) != SA_OK) return 0;
@@ -361,6 +363,66 @@ sa_status sa_decode_traced(const sa_cache *cache, const sa_query *query, int32_t
                            void *const *phase_events) {
     return decode_impl(cache, query, top_k, idx_out, out, out_dtype, lse, workspace,
                        workspace_bytes, stream, phase_events);
+}
+
+sa_status sa_quantize_index_query(const void *q_in, sa_dtype in_dtype, int32_t n_q,
+                                  int32_t h_index, int32_t d_index, void *q_out, float *q_scale,
+                                  void *stream) {
+    if (n_q < 0 || h_index <= 0 || d_index <= 0) return SA_ERR_INVALID_ARG;
+    if (in_dtype != SA_BF16 && in_dtype != SA_F32) return SA_ERR_UNSUPPORTED;
+    if (n_q == 0) return SA_OK;
+    if (!q_in || !q_out || !q_scale) return SA_ERR_INVALID_ARG;
+    if (!aligned16(q_in) || !aligned16(q_out) || !aligned16(q_scale)) return SA_ERR_INVALID_ARG;
+    return cuda_status(launch_quantize_rows(q_in, in_dtype, (int64_t)n_q * h_index, d_index,
+                                            static_cast<uint8_t *>(q_out), q_scale,
+                                            static_cast<cudaStream_t>(stream)));
+}
+
+sa_status sa_append_tokens(const sa_cache *cache, const sa_new_tokens *tokens, void *workspace,
+                           size_t workspace_bytes, void *stream) {
+    sa_status st = check_cache(cache);
+    if (st != SA_OK) return st;
+    if (tokens == nullptr || tokens->n_new < 0) return SA_ERR_INVALID_ARG;
+    if (tokens->in_dtype != SA_BF16 && tokens->in_dtype != SA_F32) return SA_ERR_UNSUPPORTED;
+    const bool page_tile = cache->kv_scale_tokens == 0 && cache->kv_scale_dims == 0;
+    if (tokens->kv && cache->kv_dtype == SA_E4M3 && (page_tile || cache->kv_scale_tokens != 1))
+        return SA_ERR_UNSUPPORTED;  // a scale shared by several tokens cannot take one more
+    if (tokens->n_new > 0) {
+        if (!tokens->seq || !tokens->pos) return SA_ERR_INVALID_ARG;
+        if ((tokens->k_index && !aligned16(tokens->k_index)) ||
+            (tokens->kv && !aligned16(tokens->kv)))
+            return SA_ERR_INVALID_ARG;
+    }
+    if ((st = check_workspace(workspace, workspace_bytes, kStatusBytes)) != SA_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if ((st = clear_status(workspace, s)) != SA_OK) return st;
+    if (tokens->n_new == 0 || (!tokens->k_index && !tokens->kv)) return SA_OK;
+    AppendParams p{};
+    p.page_table = cache->page_table;
+    p.batch = cache->batch;
+    p.max_pages = cache->max_pages;
+    p.num_pages = cache->num_pages;
+    p.n_new = tokens->n_new;
+    p.seq = tokens->seq;
+    p.pos = tokens->pos;
+    p.in_bf16 = tokens->in_dtype == SA_BF16;
+    p.k_new = tokens->k_index;
+    p.kv_new = tokens->kv;
+    // The pools are caller-owned writable device memory; sa_cache holds them
+    // as const because the decode path only reads them.
+    p.k_index = const_cast<void *>(cache->k_index);
+    p.k_index_scale = const_cast<float *>(cache->k_index_scale);
+    p.d_index = cache->d_index;
+    p.index_e4m3 = cache->index_dtype == SA_E4M3;
+    p.kv = const_cast<void *>(cache->kv);
+    p.kv_rope = const_cast<void *>(cache->kv_rope);
+    p.kv_scale = const_cast<float *>(cache->kv_scale);
+    p.d_latent = cache->d_latent;
+    p.d_rope = cache->d_rope;
+    p.kv_dtype = cache->kv_dtype;
+    p.kv_scale_dims = page_tile ? cache->d_latent : cache->kv_scale_dims;
+    p.status = static_cast<int32_t *>(workspace);
+    return cuda_status(launch_append(p, s));
 }
 
 sa_status sa_device_status(const void *workspace, size_t workspace_bytes, void *stream,

@@ -139,3 +139,49 @@ def test_other_entry_points_reject_bad_arguments(L):
                                 _abi.SA_E4M3, None, FAKE, 1 << 20, None) == \
         _abi.SA_ERR_UNSUPPORTED
     assert L.sa_device_status(None, 0, None, None) == _abi.SA_ERR_WORKSPACE
+
+
+def test_quantize_index_query_checks_arguments_before_launch(L):
+    q = L.sa_quantize_index_query
+    assert q(FAKE, _abi.SA_BF16, -1, 64, 128, FAKE, FAKE, None) == _abi.SA_ERR_INVALID_ARG
+    assert q(FAKE, _abi.SA_BF16, 4, 0, 128, FAKE, FAKE, None) == _abi.SA_ERR_INVALID_ARG
+    assert q(FAKE, _abi.SA_E4M3, 4, 64, 128, FAKE, FAKE, None) == _abi.SA_ERR_UNSUPPORTED
+    assert q(None, _abi.SA_BF16, 4, 64, 128, FAKE, FAKE, None) == _abi.SA_ERR_INVALID_ARG
+    assert q(FAKE + 8, _abi.SA_F32, 4, 64, 128, FAKE, FAKE, None) == _abi.SA_ERR_INVALID_ARG
+    assert q(FAKE, _abi.SA_BF16, 0, 64, 128, None, None, None) == _abi.SA_OK  # nothing to do
+
+
+def new_tokens(**kw):
+    t = _abi.SaNewTokens(n_new=2, seq=FAKE, pos=FAKE, in_dtype=_abi.SA_BF16, k_index=FAKE,
+                         kv=FAKE)
+    for k, v in kw.items():
+        setattr(t, k, v)
+    return t
+
+
+@pytest.mark.parametrize("cache,tokens,ws,expect", [
+    ({"page_table": None}, {}, FAKE, _abi.SA_ERR_INVALID_ARG),
+    ({}, {"n_new": -1}, FAKE, _abi.SA_ERR_INVALID_ARG),
+    ({}, {"in_dtype": _abi.SA_E4M3}, FAKE, _abi.SA_ERR_UNSUPPORTED),
+    ({}, {"seq": None}, FAKE, _abi.SA_ERR_INVALID_ARG),
+    ({}, {"kv": FAKE + 2}, FAKE, _abi.SA_ERR_INVALID_ARG),            # misaligned input
+    ({}, {}, None, _abi.SA_ERR_WORKSPACE),
+    ({}, {}, FAKE + 64, _abi.SA_ERR_WORKSPACE),                        # not 256-aligned
+    # e4m3 latent: only one-token scale tiles can take a new token
+    ({**FP8_KV}, {}, FAKE, _abi.SA_ERR_UNSUPPORTED),
+    ({**FP8_KV, "kv_scale_tokens": 16, "kv_scale_dims": 128}, {}, FAKE,
+     _abi.SA_ERR_UNSUPPORTED),
+])
+def test_append_tokens_checks_arguments_before_launch(L, cache, tokens, ws, expect):
+    c, t = good_cache(**cache), new_tokens(**tokens)
+    assert L.sa_append_tokens(ctypes.byref(c), ctypes.byref(t), ws, 1 << 20, None) == expect
+    if tokens == {"n_new": -1}:
+        assert L.sa_append_tokens(ctypes.byref(c), None, FAKE, 1 << 20, None) == \
+            _abi.SA_ERR_INVALID_ARG
+
+
+def test_append_workspace_needs_no_query(L):
+    c = good_cache()
+    assert L.sa_workspace_size(ctypes.byref(c), None, 0, _abi.SA_WS_APPEND) == 256
+    assert L.sa_workspace_size(ctypes.byref(good_cache(page_size=16)), None, 0,
+                               _abi.SA_WS_APPEND) == 0

@@ -62,3 +62,18 @@ def test_prefill_is_reported_against_the_tensor_pipe():
     assert np.isclose(r["achieved"], fl["indexer"] / 2e-3 / 1e12)
     r = bench.roofline(wl, "attention", 2.0, bench.algorithmic_bytes(wl, idx), fl)
     assert np.isclose(r["peak"], bf16)
+
+
+def test_input_prep_bytes():
+    import dataclasses
+    sp = dataclasses.replace(W.spec("decode_b8_8k"), batch=2, seq_len=("fixed", 128))
+    wl = W.make_workload(sp)
+    n, h, d, D = wl.n_q, sp.h_index, sp.d_index, sp.d_latent + sp.d_rope
+    q = n * h * d * 3 + n * h * 4
+    keys = n * (3 * d + 4)
+    assert bench.input_prep_bytes(wl, False) == q + keys
+    assert bench.input_prep_bytes(wl, True) == q + keys + n * (D * 2 + D * 2)
+    sp8 = dataclasses.replace(sp, kv_dtype="e4m3", kv_scale_tile=(1, 128))
+    wl8 = W.make_workload(sp8)
+    stored = sp.d_latent + 2 * sp.d_rope + 4 * (sp.d_latent // 128)
+    assert bench.input_prep_bytes(wl8, True) == q + keys + n * (D * 2 + stored)
