@@ -23,12 +23,15 @@ from tests import parity
 pytestmark = pytest.mark.gpu
 
 
-def _inputs(rng, shape, dtype):
-    """Random values with a spread of magnitudes; (torch tensor on the GPU, the
-    exact fp32 values the kernel sees)."""
-    x = (rng.standard_normal(shape) * np.exp2(rng.uniform(-6, 6, shape[:-1] + (1,)))) \
-        .astype(np.float32)
-    x.reshape(-1, shape[-1])[0] = 0.0                    # an all-zero row
+def _inputs(rng, shape, dtype, spread=True):
+    """Random values, rows scaled over 2^-6..2^6 when `spread` (else N(0,1), the
+    workloads' distribution), the first row all zero; (torch tensor on the GPU,
+    the exact fp32 values the kernel sees)."""
+    x = rng.standard_normal(shape)
+    if spread:
+        x = x * np.exp2(rng.uniform(-6, 6, shape[:-1] + (1,)))
+    x = x.astype(np.float32)
+    x.reshape(-1, shape[-1])[0] = 0.0
     t = torch.from_numpy(x)
     if dtype == "bf16":
         t = t.to(torch.bfloat16)
@@ -176,9 +179,12 @@ def test_prepared_decode_step_matches_oracle():
     rng = np.random.default_rng(36)
     seq = np.arange(sp.batch, dtype=np.int32)
     pos = (wl.seq_len - 1).astype(np.int32)
-    k_t, k_exact = _inputs(rng, (sp.batch, sp.d_index), "bf16")
-    kv_t, kv_exact = _inputs(rng, (sp.batch, sp.d_latent + sp.d_rope), "bf16")
-    qi_t, qi_exact = _inputs(rng, (wl.n_q, sp.h_index, sp.d_index), "bf16")
+    # N(0,1) like the cached rows: the attention tolerances assume outputs of
+    # that size (a row scaled by 2^6 would leave bf16 rounding of the output
+    # alone above 2e-2)
+    k_t, k_exact = _inputs(rng, (sp.batch, sp.d_index), "bf16", spread=False)
+    kv_t, kv_exact = _inputs(rng, (sp.batch, sp.d_latent + sp.d_rope), "bf16", spread=False)
+    qi_t, qi_exact = _inputs(rng, (wl.n_q, sp.h_index, sp.d_index), "bf16", spread=False)
     ws = api.append_tokens(cache, torch.from_numpy(seq).cuda(), torch.from_numpy(pos).cuda(),
                            k_index=k_t, kv=kv_t)
     assert api.device_status(ws) == (_abi.SA_OK, 0)
