@@ -12,8 +12,8 @@ indexer and the sparse attention kernel -- "Optimizing Next-Gen LLM Inference"
 
 * ``page_table[b, i]`` is the physical page holding tokens ``64*i .. 64*i+63``
   of sequence ``b``; entries past the sequence end are -1.
-* index keys ``k_index[P, 64, d_index]`` (fp32, or e4m3 codes with one fp32
-  scale per token in ``k_index_scale[P, 64]``);
+* index keys ``k_index[P, 64, d_index]`` (fp32, bf16, or e4m3 codes with one
+  fp32 scale per token in ``k_index_scale[P, 64]``);
 * MLA latent rows ``kv[P, 64, d_latent + d_rope]`` (fp32 or bf16), or for the
   FP8 cache ``kv[P, 64, d_latent]`` e4m3 codes, ``kv_scale[P, 64 / ts, d_latent / td]``
   (one fp32 scale per tile of ts tokens x td latent dims of a page; the default
@@ -55,7 +55,7 @@ class WorkloadSpec:
     queries: tuple = ("decode",)   # ("decode",) or ("prefill", first_pos, count)
     h_index: int = 64
     d_index: int = 128
-    index_dtype: str = "e4m3"      # "e4m3" or "f32"
+    index_dtype: str = "e4m3"      # "e4m3", "bf16" or "f32"
     top_k: int = 2048
     heads: int = 128
     d_latent: int = 512
@@ -118,7 +118,12 @@ CONFIGS = (TINY, DECODE_B8_8K, DECODE_B64_16K_32K, PREFILL_4096Q_64K,
 PROFILE_B64_16K = WorkloadSpec(
     name="profile_decode_b64_16k", seed=3, batch=64, seq_len=("fixed", 16384))
 
-EXTRA = (PROFILE_B64_16K,)
+# the headline decode with the indexer's BF16 path (unquantised query and keys)
+DECODE_B64_BF16_INDEX = WorkloadSpec(
+    name="decode_b64_16k_32k_bf16_index", seed=2, batch=64, seq_len=("uniform", 16384, 32768),
+    keys=("planted", 0.05, 3.0), index_dtype="bf16")
+
+EXTRA = (PROFILE_B64_16K, DECODE_B64_BF16_INDEX)
 
 
 def spec(which) -> WorkloadSpec:
@@ -144,9 +149,9 @@ class Workload:
     num_pages: int
     q_seq: np.ndarray            # int32 [n_q]
     q_pos: np.ndarray            # int32 [n_q]; visible length is q_pos + 1
-    k_index: np.ndarray          # f32 or uint8 (e4m3) [P, ps, d_index]
+    k_index: np.ndarray          # f32, uint16 (bf16) or uint8 (e4m3) [P, ps, d_index]
     k_index_scale: Optional[np.ndarray]  # f32 [P, ps]
-    q_index: np.ndarray          # f32 or uint8 (e4m3) [n_q, h_index, d_index]
+    q_index: np.ndarray          # f32, uint16 (bf16) or uint8 (e4m3) [n_q, h_index, d_index]
     q_index_scale: Optional[np.ndarray]  # f32 [n_q, h_index]
     w: np.ndarray                # f32 [n_q, h_index]
     kv: np.ndarray               # f32/uint16(bf16) [P, ps, d_qk] or uint8 [P, ps, d_latent]
@@ -284,6 +289,8 @@ def make_workload(sp: WorkloadSpec) -> Workload:
     w = (_normal(rng, (n_q, H_I)) / np.float32(math.sqrt(H_I))).astype(np.float32)
     if sp.index_dtype == "e4m3":
         q_index, q_index_scale = quantize_rows_e4m3(qi)
+    elif sp.index_dtype == "bf16":
+        q_index, q_index_scale = to_bf16_bits(qi), None
     elif sp.index_dtype == "f32":
         q_index, q_index_scale = qi, None
     else:
@@ -294,6 +301,9 @@ def make_workload(sp: WorkloadSpec) -> Workload:
     if sp.index_dtype == "e4m3":
         k_index = np.full((rows, d_I), E4M3_NAN, dtype=np.uint8)
         k_index_scale = np.full((rows,), np.nan, dtype=np.float32)
+    elif sp.index_dtype == "bf16":
+        k_index = np.full((rows, d_I), BF16_NAN, dtype=np.uint16)
+        k_index_scale = None
     else:
         k_index = np.full((rows, d_I), np.nan, dtype=np.float32)
         k_index_scale = None
@@ -316,6 +326,8 @@ def make_workload(sp: WorkloadSpec) -> Workload:
             if sp.index_dtype == "e4m3":
                 qdeq = torch.from_numpy(q_index[t]).view(torch.float8_e4m3fn).float().numpy()
                 qdeq = qdeq * q_index_scale[t][:, None]
+            elif sp.index_dtype == "bf16":
+                qdeq = (q_index[t].astype(np.uint32) << 16).view(np.float32)
             else:
                 qdeq = q_index[t]
             u = (np.maximum(w[t], 0.0)[:, None].astype(np.float64) * qdeq).sum(axis=0)
@@ -350,6 +362,8 @@ def make_workload(sp: WorkloadSpec) -> Workload:
                 codes, sc = quantize_rows_e4m3(k)
                 k_index[dst] = codes
                 k_index_scale[dst] = sc
+            elif sp.index_dtype == "bf16":
+                k_index[dst] = to_bf16_bits(k)
             else:
                 k_index[dst] = k
     k_index = k_index.reshape(num_pages, ps, d_I)

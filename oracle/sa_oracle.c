@@ -171,11 +171,11 @@ typedef struct {
     int32_t n_q;
     const int32_t *q_seq, *q_pos;
     int32_t h_index, d_index;
-    int32_t q_dtype;           /* OR_F32 or OR_E4M3 */
+    int32_t q_dtype;           /* OR_F32, OR_BF16 or OR_E4M3 */
     const void *q_index;       /* [n_q, h_index, d_index] */
     const float *q_index_scale;/* [n_q, h_index] for e4m3 */
     const float *w;            /* [n_q, h_index] */
-    int32_t k_dtype;           /* OR_F32 or OR_E4M3 */
+    int32_t k_dtype;           /* OR_F32, OR_BF16 or OR_E4M3 */
     const void *k_index;       /* [rows, d_index] */
     const float *k_index_scale;/* [rows] for e4m3 */
     pages_t pg;
@@ -247,7 +247,10 @@ int oracle_index_scores(int32_t n_q, const int32_t *q_seq, const int32_t *q_pos,
 {
     if (n_q < 0 || h_index <= 0 || d_index <= 0 || page_size <= 0 || !scores)
         return OR_BAD_ARG;
-    if ((q_dtype != OR_F32 && q_dtype != OR_E4M3) || (k_dtype != OR_F32 && k_dtype != OR_E4M3))
+    /* the indexer's BF16 path ("Optimizing Next-Gen LLM Inference" §3.1: a BF16
+     * path next to the quantised one) reads unscaled bf16 values */
+    if ((q_dtype != OR_F32 && q_dtype != OR_BF16 && q_dtype != OR_E4M3) ||
+        (k_dtype != OR_F32 && k_dtype != OR_BF16 && k_dtype != OR_E4M3))
         return OR_BAD_ARG;
     int64_t maxV = 0;
     for (int32_t t = 0; t < n_q; t++) {

@@ -130,7 +130,7 @@ def test_bf16_decode_matches_torch():
 
 # --------------------------------------------------------- indexer score ---
 
-@pytest.mark.parametrize("index_dtype", ["f32", "e4m3"])
+@pytest.mark.parametrize("index_dtype", ["f32", "bf16", "e4m3"])
 def test_scores_match_brute_force(index_dtype):
     wl = W.make_workload(small_spec(index_dtype=index_dtype))
     got = oracle.index_scores(wl)
