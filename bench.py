@@ -92,16 +92,18 @@ def roofline(wl, name: str, ms: float, nbytes: dict, flops: dict) -> dict:
     and selected row once: HBM-bound, algorithmic bytes over the measured copy
     bandwidth.  Chunked prefill (many queries of one sequence) reuses keys and rows
     from L2, so the tensor pipe bounds it: algorithmic flops over the dtype's
-    peak (e4m3 = 2 x the measured bf16 GEMM, the nominal fp8:bf16 ratio)."""
+    peak (e4m3 = 2 x the measured bf16 GEMM, the nominal fp8:bf16 ratio; the
+    indexer's BF16 path and the attention take the bf16 GEMM's)."""
     hbm, bf16, kind = measured_peaks()
     sp = wl.spec
     shared = wl.n_q > wl.seq_len.shape[0]
     secs = ms / 1e3
-    if shared and name in flops and sp.index_dtype == "e4m3":
-        peak = bf16 * (2.0 if name == "indexer" else 1.0)
+    if shared and name in flops and sp.index_dtype in ("e4m3", "bf16"):
+        fp8 = name == "indexer" and sp.index_dtype == "e4m3"
+        peak = bf16 * (2.0 if fp8 else 1.0)
         achieved = flops[name] / secs / 1e12 if secs > 0 else 0.0
         return {"bound": "tensor", "kernel": name, "achieved": achieved, "peak": peak,
-                "peak_kind": kind + (" (fp8 = 2 x bf16)" if name == "indexer" else " (bf16)"),
+                "peak_kind": kind + (" (fp8 = 2 x bf16)" if fp8 else " (bf16)"),
                 "unit": "TFLOP/s", "frac": achieved / peak}
     achieved = nbytes[name] / secs / 1e9 if secs > 0 else 0.0
     return {"bound": "hbm", "kernel": name, "achieved": achieved, "peak": hbm,
@@ -113,7 +115,7 @@ def algorithmic_bytes(wl, idx: np.ndarray) -> dict:
     indexer keys + key scales + selected KV rows + outputs)."""
     sp = wl.spec
     V = wl.visible.astype(np.int64)
-    key_b = sp.d_index * (1 if sp.index_dtype == "e4m3" else 4)
+    key_b = sp.d_index * {"e4m3": 1, "bf16": 2, "f32": 4}[sp.index_dtype]
     scale_b = 4 if sp.index_dtype == "e4m3" else 0
     indexer = int((V * (key_b + scale_b)).sum())
     n_sel = np.minimum(V, sp.top_k)
@@ -521,11 +523,12 @@ def run_ours(args, rank: int, world: int, dist):
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "e4m3+bf16", "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None, "dtype": f"{sp.index_dtype}+{sp.kv_dtype}", "data": "synthetic",
         "config": {
             "workload": sp.name, "batch": int(wl.seq_len.shape[0]), "queries_per_gpu": wl.n_q,
             "context_mean": float(wl.seq_len.mean()), "top_k": K, "heads": sp.heads,
-            "index_heads": sp.h_index, "index_dim": sp.d_index, "kv_dtype": sp.kv_dtype,
+            "index_heads": sp.h_index, "index_dim": sp.d_index,
+            "index_dtype": sp.index_dtype, "kv_dtype": sp.kv_dtype,
             "page_size": sp.page_size, "l2": "flushed before every timed step (256 MiB write)",
             "parallelism": f"replicas x{world}"},
         "roofline": dict(roof, traffic=traffic if roof["bound"] == "hbm" else None),

@@ -1,14 +1,18 @@
-// indexer_mma.cu -- FP8 lightning indexer on the 5th-generation tensor cores.
+// indexer_mma.cu -- lightning indexer on the 5th-generation tensor cores.
 //
 // Scores every visible cached position of every query ("Optimizing Next-Gen
-// LLM Inference" §3.1: relevance scoring, head-weight weighting; §4: index keys
-// quantised to 8-bit floats):
+// LLM Inference" §3.1: relevance scoring, head-weight weighting, and its two
+// numerical paths; §4: index keys quantised to 8-bit floats):
 //     I[t,s] = ks[s] * sum_j (w[t,j] * qs[t,j]) * max(0, q8[t,j,:] . k8[s,:])
-// which equals sum_j w * max(0, q_I . k_I) because the scales are positive.
+// which equals sum_j w * max(0, q_I . k_I) because the scales are positive;
+// on the BF16 path ("Inference Acceleration for New Large Model Architectures"
+// §3.1) the query and keys are unscaled bf16 and ks = qs = 1.
 //
 // The contraction of 64 heads x 128 dims against every key is a dense GEMM
 // (M = 128 keys of a two-page tile, N = 64 heads, K = 128), so it runs as
-// tcgen05.mma kind::f8f6f4 (e4m3 x e4m3 -> fp32 in TMEM).  The kernel is
+// tcgen05.mma kind::f8f6f4 (e4m3 x e4m3 -> fp32 in TMEM), or kind::f16 with
+// bf16 operands.  A bf16 key row is 256 bytes, two 128-byte swizzle atoms
+// wide, so its tiles are stored as two 64-column halves.  The kernel is
 // persistent: the tiles of all queries are laid end to end and every CTA takes
 // an equal contiguous share, so short and long contexts balance across SMs.
 // Roles per CTA (192 threads):
@@ -36,21 +40,36 @@ using namespace sm100;
 
 constexpr int kKeys = 128;    // MMA M: keys per tile (two pages)
 constexpr int kHeads = 64;    // MMA N: indexer heads
-constexpr int kDim = 128;     // MMA K: index dimension (bytes of e4m3)
+constexpr int kDim = 128;     // MMA K: index dimension
 constexpr int kStages = 4;
 constexpr int kAcc = 4;       // TMEM accumulators (64 columns each)
 constexpr int kScaleSlots = 8;  // key-scale ring: the epilogue frees these, not the key stages
 constexpr int kEpiGroups = 2;  // epilogue warp groups, alternating tiles
 constexpr int kThreads = 64 + kEpiGroups * 128;
-constexpr uint32_t kPageBytes = 64 * kDim;
-constexpr uint32_t kTileBytes = 2 * kPageBytes;
-constexpr uint32_t kQBytes = kHeads * kDim;
 constexpr uint32_t kTmemCols = kAcc * kHeads;
+constexpr uint32_t kAtom = 128;  // bytes of a row in one 128-byte swizzle atom
 
+// Storage of one index element type.  A row of kDim elements is kChunks
+// 128-byte column chunks; a tile stores chunk c of all 128 keys contiguously
+// (16 KB, page h at + 8 KB * h), the query chunk c of its 64 heads likewise.
+template <bool kBf16>
+struct IxCfg {
+    static constexpr int kElem = kBf16 ? 2 : 1;
+    static constexpr int kChunks = kDim * kElem / kAtom;
+    static constexpr int kChunkElems = kAtom / kElem;              // TMA box width
+    static constexpr uint32_t kPageBytes = 64 * kDim * kElem;
+    static constexpr uint32_t kTileBytes = 2 * kPageBytes;
+    static constexpr uint32_t kQBytes = kHeads * kDim * kElem;
+    static constexpr int kKPerMma = 32 / kElem;                      // K of one instruction
+    static constexpr int kMmas = kDim / kKPerMma;
+    static constexpr int kCtasPerSm = kBf16 ? 1 : 2;
+};
+
+template <bool kBf16>
 struct IndexerSmem {
-    uint8_t keys[kStages][kTileBytes];  // 1024-byte aligned (128-byte swizzle atoms)
+    uint8_t keys[kStages][IxCfg<kBf16>::kTileBytes];  // 1024-byte aligned (swizzle atoms)
     uint32_t hist[kHistBins];              // score-key histogram of the current query
-    uint8_t q[2][kQBytes];                 // 1024-byte aligned like the key stages
+    uint8_t q[2][IxCfg<kBf16>::kQBytes];   // 1024-byte aligned like the key stages
     float wq[kEpiGroups][kHeads];          // head weights x query scales of that query
     float kscale[kScaleSlots][kKeys];   // per-token key scales of the staged pages
     int32_t page_ok[kScaleSlots][2];    // 1 when the staged page id was valid
@@ -64,9 +83,14 @@ struct IndexerSmem {
     int abort;
 };
 
-static_assert(offsetof(IndexerSmem, q) % 1024 == 0, "128-byte-swizzled Q tiles need 1024-byte alignment");
-static_assert(offsetof(IndexerSmem, wq) % 16 == 0, "head weights are read as float4");
-static_assert(2 * (sizeof(IndexerSmem) + 2048) <= 233472, "two CTAs per SM");
+static_assert(offsetof(IndexerSmem<false>, q) % 1024 == 0 &&
+                  offsetof(IndexerSmem<true>, q) % 1024 == 0,
+              "128-byte-swizzled Q tiles need 1024-byte alignment");
+static_assert(offsetof(IndexerSmem<false>, wq) % 16 == 0 &&
+                  offsetof(IndexerSmem<true>, wq) % 16 == 0,
+              "head weights are read as float4");
+static_assert(2 * (sizeof(IndexerSmem<false>) + 2048) <= 233472, "e4m3: two CTAs per SM");
+static_assert(sizeof(IndexerSmem<true>) + 1024 <= 232448, "bf16: one CTA per SM");
 
 struct IndexerArgs {
     PathParams p;
@@ -123,12 +147,14 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volati
     return ok;
 }
 
-__global__ void __launch_bounds__(kThreads, 2)
+template <bool kBf16>
+__global__ void __launch_bounds__(kThreads, IxCfg<kBf16>::kCtasPerSm)
 indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
                    const __grid_constant__ CUtensorMap tm_q, const IndexerArgs a) {
+    using C = IxCfg<kBf16>;
     pdl_wait();
     extern __shared__ uint8_t smem_raw[];
-    IndexerSmem &sm = *reinterpret_cast<IndexerSmem *>(align1024(smem_raw));
+    IndexerSmem<kBf16> &sm = *reinterpret_cast<IndexerSmem<kBf16> *>(align1024(smem_raw));
     const PathParams &p = a.p;
     const int warp = warp_id(), lane = lane_id();
     const int64_t total = p.n_q > 0 ? a.tile_end[p.n_q - 1] : 0;
@@ -219,8 +245,11 @@ indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
                     const int b = c.seg & 1;
                     if (!mbar_wait(&sm.q_empty[b], ((c.seg >> 1) & 1) ^ 1, abort_flag, p.status))
                         break;
-                    mbar_arrive_expect_tx(&sm.q_full[b], kQBytes);
-                    tma_load_2d(sm.q[b], &tm_q, 0, c.t * kHeads, &sm.q_full[b]);
+                    mbar_arrive_expect_tx(&sm.q_full[b], C::kQBytes);
+#pragma unroll
+                    for (int ch = 0; ch < C::kChunks; ++ch)
+                        tma_load_2d(sm.q[b] + ch * (kHeads * kAtom), &tm_q, ch * C::kChunkElems,
+                                    c.t * kHeads, &sm.q_full[b]);
                 }
                 const int stage = n % kStages;
                 // the stage is free once its MMAs and its epilogue are done
@@ -237,19 +266,25 @@ indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
                     const int64_t s = (int64_t)c.i * kKeys + 64 * h;
                     if (s < V && pg[h] >= 0 && pg[h] < p.num_pages) {
                         rows[h] = pg[h] * 64;
-                        bytes += kPageBytes;
+                        bytes += C::kPageBytes;
                     }
                     sm.page_ok[slot][h] = rows[h] >= 0;  // published by the arrive below
                 }
-                mbar_arrive_expect_tx(&sm.sc_full[slot], (bytes / kPageBytes) * 64 * sizeof(float));
+                // the bf16 path has no key scales: the slot then only
+                // publishes the page validity
+                mbar_arrive_expect_tx(&sm.sc_full[slot],
+                                      kBf16 ? 0u : (bytes / C::kPageBytes) * 64 * sizeof(float));
                 mbar_arrive_expect_tx(&sm.full[stage], bytes);
 #pragma unroll
                 for (int h = 0; h < 2; ++h)
                     if (rows[h] >= 0) {
-                        tma_load_2d(sm.keys[stage] + h * kPageBytes, &tm_keys, 0, rows[h],
-                                    &sm.full[stage]);
-                        bulk_load(&sm.kscale[slot][64 * h], p.k_index_scale + rows[h],
-                                  64 * sizeof(float), &sm.sc_full[slot]);
+#pragma unroll
+                        for (int ch = 0; ch < C::kChunks; ++ch)
+                            tma_load_2d(sm.keys[stage] + ch * (kKeys * kAtom) + h * (64 * kAtom),
+                                        &tm_keys, ch * C::kChunkElems, rows[h], &sm.full[stage]);
+                        if (!kBf16)
+                            bulk_load(&sm.kscale[slot][64 * h], p.k_index_scale + rows[h],
+                                      64 * sizeof(float), &sm.sc_full[slot]);
                     }
                 c = nx;
                 seg_start = nx_seg;
@@ -262,7 +297,8 @@ indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
     } else if (warp == 1) {
         // ------------------------------------------------- MMA issuer ---
         if (lane == 0) {
-            constexpr uint32_t idesc = instr_desc(kKeys, kHeads, 0 /*e4m3*/, 0, 0);
+            // kind::f8f6f4 format 0 = e4m3; kind::f16 format 1 = bf16
+            constexpr uint32_t idesc = instr_desc(kKeys, kHeads, kBf16 ? 1 : 0, 0, 0);
             TileCursor c;
             c.init_at(a.tile_end, sm.start_t, sm.start_i, k0, k1);
             bool seg_start = true;
@@ -277,12 +313,21 @@ indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
                     break;
                 if (!mbar_wait(&sm.full[stage], (n / kStages) & 1, abort_flag, p.status)) break;
                 tc_fence_after();
-                const uint64_t adesc = desc_kmajor_sw128(smem_u32(sm.keys[stage]));
-                const uint64_t bdesc = desc_kmajor_sw128(smem_u32(sm.q[c.seg & 1]));
+                const uint32_t keys = smem_u32(sm.keys[stage]);
+                const uint32_t qs = smem_u32(sm.q[c.seg & 1]);
                 const uint32_t d = tmem + acc * kHeads;
+                // 32 bytes of K per instruction: four per 128-byte chunk (the
+                // descriptor address counts 16-byte units)
 #pragma unroll
-                for (int kk = 0; kk < kDim / 32; ++kk)  // 32 bytes of K per instruction
-                    mma_f8(d, adesc + 2 * kk, bdesc + 2 * kk, idesc, kk > 0 ? 1u : 0u);
+                for (int kk = 0; kk < C::kMmas; ++kk) {
+                    const int ch = kk / 4, w = kk % 4;
+                    const uint64_t adesc = desc_kmajor_sw128(keys + ch * (kKeys * kAtom)) + 2 * w;
+                    const uint64_t bdesc = desc_kmajor_sw128(qs + ch * (kHeads * kAtom)) + 2 * w;
+                    if (kBf16)
+                        mma_bf16(d, adesc, bdesc, idesc, kk > 0 ? 1u : 0u);
+                    else
+                        mma_f8(d, adesc, bdesc, idesc, kk > 0 ? 1u : 0u);
+                }
                 mma_commit(&sm.empty[stage]);
                 mma_commit(&sm.acc_full[acc]);
                 seg_start = c.next(a.tile_end);
@@ -337,7 +382,7 @@ indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
                 V = a.vis[c.t];
                 if (et < kHeads)
                     wq[et] = __ldg(p.w + (int64_t)c.t * kHeads + et) *
-                             __ldg(p.q_index_scale + (int64_t)c.t * kHeads + et);
+                             (kBf16 ? 1.f : __ldg(p.q_index_scale + (int64_t)c.t * kHeads + et));
                 named_barrier(bar, 128);
             }
             if ((n & 1) != g) continue;  // the other group's tile
@@ -347,7 +392,7 @@ indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
             if (ok)
                 ok = warp_wait(&sm.sc_full[slot], (n / kScaleSlots) & 1, abort_flag, p.status);
             const bool page_ok = ok && sm.page_ok[slot][row >> 6] != 0;
-            const float kscale = ok ? sm.kscale[slot][row] : 0.f;
+            const float kscale = ok ? (kBf16 ? 1.f : sm.kscale[slot][row]) : 0.f;
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.sc_empty[slot]);
             if (ok && s < V && !page_ok) report(p.status, SA_ERR_DEVICE_FAULT, SA_DETAIL_BAD_PAGE);
@@ -401,27 +446,42 @@ indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
 }  // namespace
 
 bool indexer_mma_supported(const PathParams &p) {
-    return p.index_e4m3 && p.h_index == kHeads && p.d_index == kDim;
+    return (p.index_dtype == SA_E4M3 || p.index_dtype == SA_BF16) && p.h_index == kHeads &&
+           p.d_index == kDim;
 }
+
+namespace {
+
+template <bool kBf16>
+cudaError_t launch_indexer_mma_t(const PathParams &p, const int32_t *vis, const int32_t *tile_end,
+                                 float *scores, int64_t ld, uint32_t *hist, cudaStream_t s) {
+    using C = IxCfg<kBf16>;
+    CUtensorMap tk, tq;
+    if (!encode_tmap_2d(&tk, C::kElem, p.k_index, kDim, (uint64_t)p.num_pages * 64,
+                        kDim * C::kElem, C::kChunkElems, 64, true) ||
+        !encode_tmap_2d(&tq, C::kElem, p.q_index, kDim, (uint64_t)p.n_q * kHeads,
+                        kDim * C::kElem, C::kChunkElems, kHeads, true))
+        return cudaErrorInvalidValue;
+    IndexerArgs a{p, vis, tile_end, scores, ld, hist};
+    const int64_t max_tiles = (int64_t)p.n_q * ceil_div(p.max_visible, kKeys);
+    const int64_t grid = std::min<int64_t>((int64_t)C::kCtasPerSm * num_sms(), max_tiles);
+    const size_t smem = sizeof(IndexerSmem<kBf16>) + 1024;
+    cudaError_t e = cudaFuncSetAttribute(indexer_mma_kernel<kBf16>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    count_launch();
+    return launch_pdl(indexer_mma_kernel<kBf16>, dim3(static_cast<unsigned>(grid)),
+                      dim3(kThreads), smem, s, tk, tq, a);
+}
+
+}  // namespace
 
 cudaError_t launch_indexer_mma(const PathParams &p, const int32_t *vis, const int32_t *tile_end,
                                float *scores, int64_t ld, uint32_t *hist, cudaStream_t s) {
     if (p.n_q == 0) return cudaSuccess;
-    CUtensorMap tk, tq;
-    if (!encode_tmap_2d(&tk, 1, p.k_index, kDim, (uint64_t)p.num_pages * 64, kDim, kDim, 64, true) ||
-        !encode_tmap_2d(&tq, 1, p.q_index, kDim, (uint64_t)p.n_q * kHeads, kDim, kDim, kHeads,
-                        true))
-        return cudaErrorInvalidValue;
-    IndexerArgs a{p, vis, tile_end, scores, ld, hist};
-    const int64_t max_tiles = (int64_t)p.n_q * ceil_div(p.max_visible, kKeys);
-    const int64_t grid = std::min<int64_t>(2 * num_sms(), max_tiles);
-    const size_t smem = sizeof(IndexerSmem) + 1024;
-    cudaError_t e = cudaFuncSetAttribute(indexer_mma_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    count_launch();
-    return launch_pdl(indexer_mma_kernel, dim3(static_cast<unsigned>(grid)), dim3(kThreads), smem,
-                      s, tk, tq, a);
+    return p.index_dtype == SA_BF16
+               ? launch_indexer_mma_t<true>(p, vis, tile_end, scores, ld, hist, s)
+               : launch_indexer_mma_t<false>(p, vis, tile_end, scores, ld, hist, s);
 }
 
 }  // namespace sa

@@ -2,7 +2,8 @@
 //
 // Computes I[t,s] = sum_j w[t,j] * max(0, q_I[t,j,:] . k_I[s,:]) for every
 // visible position ("Optimizing Next-Gen LLM Inference" §3.1, relevance scoring
-// plus head-weight weighting).  With e4m3 inputs the positive per-(token, head)
+// plus head-weight weighting; fp32, the BF16 path or e4m3 inputs).  With e4m3
+// inputs the positive per-(token, head)
 // query scale and per-token key scale factor out of the ReLU:
 //     I[t,s] = ks[s] * sum_j (w[t,j] * qs[t,j]) * max(0, q8[t,j,:] . k8[s,:]).
 // This kernel serves the small fp32 configuration and any shape the tensor-core
@@ -16,9 +17,10 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kHeadBlock = 16;  // head dot products kept in registers at once
 
-template <bool kE4M3>
+template <int kFmt>  // sa_dtype of the index query and keys
 __global__ void __launch_bounds__(kThreads)
 indexer_simt_kernel(const PathParams p, float *__restrict__ scores, int64_t ld) {
+    constexpr bool kE4M3 = kFmt == SA_E4M3, kBF16 = kFmt == SA_BF16;
     pdl_wait();
     pdl_trigger();
     extern __shared__ float smem[];
@@ -31,6 +33,9 @@ indexer_simt_kernel(const PathParams p, float *__restrict__ scores, int64_t ld) 
         if (kE4M3) {
             const uint8_t *qb = static_cast<const uint8_t *>(p.q_index) + (int64_t)t * H * d;
             q_s[i] = e4m3x2_to_float2(qb[i]).x;
+        } else if (kBF16) {
+            q_s[i] = bf16_bits_to_float(
+                static_cast<const uint16_t *>(p.q_index)[(int64_t)t * H * d + i]);
         } else {
             q_s[i] = static_cast<const float *>(p.q_index)[(int64_t)t * H * d + i];
         }
@@ -71,6 +76,19 @@ indexer_simt_kernel(const PathParams p, float *__restrict__ scores, int64_t ld) 
                     k[4 * i + 2] = hi.x;
                     k[4 * i + 3] = hi.y;
                 }
+            } else if (kBF16) {
+                const uint4 *src = reinterpret_cast<const uint4 *>(
+                    static_cast<const uint16_t *>(p.k_index) + row * d + d0);
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const uint4 v = src[i];
+                    const uint32_t words[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        k[8 * i + 2 * j] = __uint_as_float(words[j] << 16);
+                        k[8 * i + 2 * j + 1] = __uint_as_float(words[j] & 0xffff0000u);
+                    }
+                }
             } else {
                 const float4 *src = reinterpret_cast<const float4 *>(
                     static_cast<const float *>(p.k_index) + row * d + d0);
@@ -106,18 +124,16 @@ cudaError_t launch_indexer_simt(const PathParams &p, float *scores, int64_t ld, 
     if (p.n_q == 0 || p.max_visible == 0) return cudaSuccess;
     dim3 grid(static_cast<unsigned>(ceil_div(p.max_visible, kThreads)), p.n_q);
     size_t smem = sizeof(float) * ((size_t)p.h_index * p.d_index + p.h_index);
-    if (p.index_e4m3) {
-        cudaFuncSetAttribute(indexer_simt_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem);
+    auto go = [&](auto kernel) {
+        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+        if (e != cudaSuccess) return e;
         count_launch();
-        return launch_pdl(indexer_simt_kernel<true>, grid, dim3(kThreads), smem, s, p, scores, ld);
-    } else {
-        cudaFuncSetAttribute(indexer_simt_kernel<false>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        count_launch();
-        return launch_pdl(indexer_simt_kernel<false>, grid, dim3(kThreads), smem, s, p, scores,
-                          ld);
-    }
+        return launch_pdl(kernel, grid, dim3(kThreads), smem, s, p, scores, ld);
+    };
+    if (p.index_dtype == SA_E4M3) return go(indexer_simt_kernel<SA_E4M3>);
+    if (p.index_dtype == SA_BF16) return go(indexer_simt_kernel<SA_BF16>);
+    return go(indexer_simt_kernel<SA_F32>);
 }
 
 }  // namespace sa

@@ -43,7 +43,7 @@ struct PathParams {
     const void *k_index;
     const float *k_index_scale;
     int32_t d_index;
-    int32_t index_e4m3;  // 1: e4m3 codes + scales, 0: fp32
+    int32_t index_dtype;  // sa_dtype: SA_E4M3, SA_BF16 (unscaled) or SA_F32
     // latent cache
     const void *kv;
     const void *kv_rope;

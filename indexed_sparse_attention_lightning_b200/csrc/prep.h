@@ -29,7 +29,7 @@ struct AppendParams {
     void *k_index;
     float *k_index_scale;
     int32_t d_index;
-    int32_t index_e4m3;
+    int32_t index_dtype;  // sa_dtype of the pool
     // latent pool
     void *kv;
     void *kv_rope;

@@ -37,7 +37,8 @@ sa_status check_cache(const sa_cache *c) {
     if (c->batch <= 0 || c->max_pages <= 0 || c->num_pages <= 0) return SA_ERR_INVALID_ARG;
     if (!c->page_table || !c->seq_len || !c->k_index || !c->kv) return SA_ERR_INVALID_ARG;
     if (!aligned16(c->k_index) || !aligned16(c->kv)) return SA_ERR_INVALID_ARG;
-    if (c->index_dtype != SA_F32 && c->index_dtype != SA_E4M3) return SA_ERR_UNSUPPORTED;
+    if (c->index_dtype != SA_F32 && c->index_dtype != SA_BF16 && c->index_dtype != SA_E4M3)
+        return SA_ERR_UNSUPPORTED;
     if (c->index_dtype == SA_E4M3 && (!c->k_index_scale || !aligned16(c->k_index_scale)))
         return SA_ERR_INVALID_ARG;
     if (c->d_index <= 0 || c->d_index % 16 != 0) return SA_ERR_INVALID_ARG;
@@ -90,7 +91,7 @@ PathParams make_params(const sa_cache *c, const sa_query *q, void *ws) {
     p.k_index = c->k_index;
     p.k_index_scale = c->k_index_scale;
     p.d_index = c->d_index;
-    p.index_e4m3 = c->index_dtype == SA_E4M3;
+    p.index_dtype = c->index_dtype;
     p.kv = c->kv;
     p.kv_rope = c->kv_rope;
     p.kv_scale = c->kv_scale;
@@ -413,7 +414,7 @@ sa_status sa_append_tokens(const sa_cache *cache, const sa_new_tokens *tokens, v
     p.k_index = const_cast<void *>(cache->k_index);
     p.k_index_scale = const_cast<float *>(cache->k_index_scale);
     p.d_index = cache->d_index;
-    p.index_e4m3 = cache->index_dtype == SA_E4M3;
+    p.index_dtype = cache->index_dtype;
     p.kv = const_cast<void *>(cache->kv);
     p.kv_rope = const_cast<void *>(cache->kv_rope);
     p.kv_scale = const_cast<float *>(cache->kv_scale);

@@ -212,7 +212,7 @@ def append_tokens(pools: dict, layout: dict, seq, pos, k_new=None, kv_new=None):
     pools: ``k_index``, ``k_index_scale``, ``kv``, ``kv_rope``, ``kv_scale`` (numpy
     arrays shaped as the cache stores them; absent entries are None).
     layout: ``page_table`` [batch, max_pages], ``page_size``, ``num_pages``,
-    ``index_dtype`` ("e4m3"/"f32"), ``kv_dtype`` ("e4m3"/"bf16"/"f32"), ``d_latent``,
+    ``index_dtype`` ("e4m3"/"bf16"/"f32"), ``kv_dtype`` ("e4m3"/"bf16"/"f32"), ``d_latent``,
     ``kv_scale_dims`` (latent dims per scale; one token per scale).
     k_new [n, d_index], kv_new [n, d_latent + d_rope]: fp32 values.
     Token i goes to physical row page_table[seq, pos // page_size] * page_size +
@@ -237,6 +237,8 @@ def append_tokens(pools: dict, layout: dict, seq, pos, k_new=None, kv_new=None):
                 codes, sc = quantize_e4m3(k_new[i], k_new.shape[-1])
                 out["k_index"][page, slot] = codes
                 out["k_index_scale"][page, slot] = sc[0]
+            elif layout["index_dtype"] == "bf16":
+                out["k_index"][page, slot] = to_bf16(k_new[i])
             else:
                 out["k_index"][page, slot] = k_new[i]
         if kv_new is not None:

@@ -101,7 +101,7 @@ def decode_call(L, c, q, k=2048, ws=FAKE, ws_bytes=1 << 30, out=FAKE):
     ({"cache": {"page_table": None}}, _abi.SA_ERR_INVALID_ARG),
     ({"cache": {"kv": FAKE + 4}}, _abi.SA_ERR_INVALID_ARG),          # misaligned
     ({"cache": {"page_size": 16}}, _abi.SA_ERR_UNSUPPORTED),
-    ({"cache": {"index_dtype": _abi.SA_BF16}}, _abi.SA_ERR_UNSUPPORTED),
+    ({"cache": {"index_dtype": 7}}, _abi.SA_ERR_UNSUPPORTED),
     ({"cache": {"kv_dtype": 7}}, _abi.SA_ERR_UNSUPPORTED),
     ({"cache": {"num_pages": 0}}, _abi.SA_ERR_INVALID_ARG),
     ({"query": {"n_q": -1}}, _abi.SA_ERR_INVALID_ARG),

@@ -167,6 +167,32 @@ def test_fp8_latent_cache_small(tile, heads):
     parity.check_attention(res["out"], ref_out, "e4m3")
 
 
+@pytest.mark.parametrize("h_index,d_index", [(64, 128), (8, 32)])
+def test_bf16_indexer_path(h_index, d_index):
+    """The indexer's BF16 path (unscaled bf16 query and keys): the tensor-core
+    kernel for 64 heads x 128 dims, the CUDA-core one for other shapes.  bf16
+    products are exact in fp32, so the unfused scores must match the oracle's
+    to fp32 accumulation error."""
+    sp = W.WorkloadSpec(name=f"bf16_index_{h_index}_{d_index}", seed=41, batch=3,
+                        seq_len=("list", (900, 2048, 5000)), index_dtype="bf16",
+                        h_index=h_index, d_index=d_index, keys=("planted", 0.05, 3.0))
+    wl = workload(sp)
+    res = run_fused(wl)
+    assert res["status"] == (_abi.SA_OK, 0)
+    scores = oracle.index_scores(wl)
+    topk = parity.check_topk(res["idx"], scores, wl.visible, sp.top_k)
+    ref_out, ref_lse = oracle.sparse_attn(wl, res["idx"])
+    err = parity.check_attention(res["out"], ref_out, "bf16")
+    parity.check_lse(res["lse"], ref_lse)
+    cache, queries = api.upload(wl)
+    got = api.indexer_score(cache, queries).cpu().numpy()
+    ok = ~np.isnan(scores)
+    rel = float(np.abs(got[ok] - scores[ok]).max() / np.abs(scores[ok]).max())
+    print(f"\nbf16 index {h_index}x{d_index}: score err {rel:.3g} of max|I|, "
+          f"swaps={topk['swaps']} max_abs={err['max_abs']:.3g}")
+    assert rel <= 1e-4
+
+
 # ------------------------------------------------ device-side data errors ---
 
 def test_bad_page_id_is_reported_not_faulted():

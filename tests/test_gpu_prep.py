@@ -101,6 +101,7 @@ def _tokens(wl, rng, bad: bool):
 
 SPECS = [
     ("bf16", "e4m3", (0, 0)),
+    ("bf16", "bf16", (0, 0)),
     ("f32", "f32", (0, 0)),
     ("e4m3", "e4m3", (1, 128)),
     ("e4m3", "e4m3", (1, 16)),
