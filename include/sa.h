@@ -86,7 +86,11 @@ typedef struct sa_cache {
     int32_t page_size;           /* tokens per page (64) */
 
     /* indexer keys */
-    sa_dtype index_dtype;        /* SA_E4M3 (production) or SA_F32 */
+    /* SA_E4M3 (the quantised path) or SA_BF16 (the BF16 path, unscaled): the
+     * indexer's two numerical paths ("Optimizing Next-Gen LLM Inference" §3.1;
+     * "Inference Acceleration for New Large Model Architectures" §3.1); or
+     * SA_F32 */
+    sa_dtype index_dtype;
     const void *k_index;         /* device [num_pages, page_size, d_index] */
     const float *k_index_scale;  /* device [num_pages, page_size] one per token (SA_E4M3 only) */
     int32_t d_index;
