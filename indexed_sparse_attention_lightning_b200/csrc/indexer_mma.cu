@@ -41,7 +41,6 @@ using namespace sm100;
 constexpr int kKeys = 128;    // MMA M: keys per tile (two pages)
 constexpr int kHeads = 64;    // MMA N: indexer heads
 constexpr int kDim = 128;     // MMA K: index dimension
-constexpr int kStages = 4;
 constexpr int kAcc = 4;       // TMEM accumulators (64 columns each)
 constexpr int kScaleSlots = 8;  // key-scale ring: the epilogue frees these, not the key stages
 constexpr int kEpiGroups = 2;  // epilogue warp groups, alternating tiles
@@ -63,17 +62,19 @@ struct IxCfg {
     static constexpr int kKPerMma = 32 / kElem;                      // K of one instruction
     static constexpr int kMmas = kDim / kKPerMma;
     static constexpr int kCtasPerSm = kBf16 ? 1 : 2;
+    // key stages in flight per CTA: 2 x 4 x 16 KB (e4m3) or 5 x 32 KB (bf16) per SM
+    static constexpr int kStages = kBf16 ? 5 : 4;
 };
 
 template <bool kBf16>
 struct IndexerSmem {
-    uint8_t keys[kStages][IxCfg<kBf16>::kTileBytes];  // 1024-byte aligned (swizzle atoms)
+    uint8_t keys[IxCfg<kBf16>::kStages][IxCfg<kBf16>::kTileBytes];  // 1024-byte aligned (swizzle atoms)
     uint32_t hist[kHistBins];              // score-key histogram of the current query
     uint8_t q[2][IxCfg<kBf16>::kQBytes];   // 1024-byte aligned like the key stages
     float wq[kEpiGroups][kHeads];          // head weights x query scales of that query
     float kscale[kScaleSlots][kKeys];   // per-token key scales of the staged pages
     int32_t page_ok[kScaleSlots][2];    // 1 when the staged page id was valid
-    uint64_t full[kStages], empty[kStages];
+    uint64_t full[IxCfg<kBf16>::kStages], empty[IxCfg<kBf16>::kStages];
     uint64_t sc_full[kScaleSlots], sc_empty[kScaleSlots];
     uint64_t acc_full[kAcc], acc_empty[kAcc];
     uint64_t q_full[2], q_empty[2];
@@ -163,7 +164,7 @@ indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
     if (k0 >= k1) return;  // uniform over the CTA, before any allocation
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < C::kStages; ++s) {
             mbar_init(&sm.full[s], 1);
             mbar_init(&sm.empty[s], 1);
         }
@@ -251,9 +252,9 @@ indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
                         tma_load_2d(sm.q[b] + ch * (kHeads * kAtom), &tm_q, ch * C::kChunkElems,
                                     c.t * kHeads, &sm.q_full[b]);
                 }
-                const int stage = n % kStages;
+                const int stage = n % C::kStages;
                 // the stage is free once its MMAs and its epilogue are done
-                if (!mbar_wait(&sm.empty[stage], ((n / kStages) & 1) ^ 1, abort_flag, p.status))
+                if (!mbar_wait(&sm.empty[stage], ((n / C::kStages) & 1) ^ 1, abort_flag, p.status))
                     break;
                 const int slot = n % kScaleSlots;
                 if (!mbar_wait(&sm.sc_empty[slot], ((n / kScaleSlots) & 1) ^ 1, abort_flag,
@@ -308,10 +309,10 @@ indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
                     if (!mbar_wait(&sm.q_full[c.seg & 1], (c.seg >> 1) & 1, abort_flag, p.status))
                         break;
                 }
-                const int stage = n % kStages, acc = n % kAcc;
+                const int stage = n % C::kStages, acc = n % kAcc;
                 if (!mbar_wait(&sm.acc_empty[acc], ((n / kAcc) & 1) ^ 1, abort_flag, p.status))
                     break;
-                if (!mbar_wait(&sm.full[stage], (n / kStages) & 1, abort_flag, p.status)) break;
+                if (!mbar_wait(&sm.full[stage], (n / C::kStages) & 1, abort_flag, p.status)) break;
                 tc_fence_after();
                 const uint32_t keys = smem_u32(sm.keys[stage]);
                 const uint32_t qs = smem_u32(sm.q[c.seg & 1]);

@@ -53,6 +53,37 @@ def test_quantize_index_query_bit_exact(dtype, n_q, h, d):
     assert np.array_equal(codes.cpu().numpy(), want_codes)
 
 
+def test_quantize_index_query_near_rounding_boundaries():
+    """Quotients x / scale within a few fp32 units of an e4m3 rounding midpoint,
+    with scales whose reciprocal is inexact: the codes must still be those of
+    the correctly rounded quotient."""
+    e4 = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).float().numpy()
+    v = np.unique(e4[np.isfinite(e4) & (e4 > 0)]).astype(np.float64)
+    mids = ((v[:-1] + v[1:]) / 2).astype(np.float32)                # exact in fp32
+    rows = []
+    for amax in (447.0, 300.7, 0.0123, 5e-3, 1000.5, 3.3e-7):
+        scale = np.float32(amax) / np.float32(448.0)
+        vals = (mids * scale).astype(np.float32)                  # x / scale ~ midpoint
+        near = [np.nextafter(vals, np.float32(np.inf) if k > 0 else np.float32(-np.inf))
+                for k in (1, -1)]
+        allv = np.concatenate([vals, near[0], near[1], (v.astype(np.float32) * scale)])
+        allv = allv[np.abs(allv) < np.float32(amax)]
+        for c0 in range(0, allv.size, 127):
+            chunk = allv[c0:c0 + 127]
+            row = np.zeros(128, dtype=np.float32)
+            row[0] = amax
+            row[1:1 + chunk.size] = chunk
+            rows.append(row)
+    x = np.stack(rows).astype(np.float32)
+    x[1::2] *= -1.0
+    n = x.shape[0]
+    x = np.concatenate([x, np.zeros(((-n) % 64, 128), np.float32)]).reshape(-1, 64, 128)
+    codes, scales = api.quantize_index_query(torch.from_numpy(x).cuda())
+    want_codes, want_scales = oracle.quantize_index_query(x)
+    assert np.array_equal(scales.cpu().numpy(), want_scales)
+    assert np.array_equal(codes.cpu().numpy(), want_codes)
+
+
 def test_quantize_index_query_empty_is_a_no_op():
     q = torch.empty((0, 64, 128), dtype=torch.bfloat16, device="cuda")
     codes, scales = api.quantize_index_query(q)
