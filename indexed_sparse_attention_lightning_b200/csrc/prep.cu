@@ -31,22 +31,6 @@ __device__ __forceinline__ uint8_t to_e4m3(float x, float scale) {
         __nv_cvt_float_to_fp8(__fdiv_rn(x, scale), __NV_SATFINITE, __NV_E4M3));
 }
 
-// The same code from a multiplication by the reciprocal 1/scale (one rounding
-// each): the product lies within a few fp32 units in the last place of the
-// correctly rounded quotient, and rounding to e4m3 is monotonic, so when the
-// product moved 8 units down and 8 up rounds to one code, the quotient rounds
-// to it as well.  Otherwise an e4m3 rounding boundary is that close and the
-// quotient is taken by division (about once in 10^5 values).
-__device__ __forceinline__ uint8_t to_e4m3_by_recip(float x, float scale, float inv) {
-    const uint32_t y = __float_as_uint(x * inv);
-    const uint32_t sign = y & 0x80000000u, mag = y & 0x7fffffffu;  // |x * inv| <= ~448
-    const float lo = __uint_as_float(sign | (mag > 8u ? mag - 8u : 0u));
-    const float hi = __uint_as_float(sign | (mag + 8u));
-    const uint16_t two = __nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3);
-    if ((two & 0xffu) == (two >> 8)) return static_cast<uint8_t>(two & 0xffu);
-    return to_e4m3(x, scale);
-}
-
 __device__ __forceinline__ float load_value(const void *base, int64_t i, bool bf16) {
     return bf16 ? bf16_bits_to_float(static_cast<const uint16_t *>(base)[i])
                 : static_cast<const float *>(base)[i];
@@ -60,84 +44,62 @@ __device__ __forceinline__ float warp_max(float v) {
 
 // ---------------------------------------------------------------------------
 // Query quantisation.  Rows of d = 32 * C values: lane l holds values
-// [l*C, l*C + C) of a row (one 8- or 16-byte load for bf16, one or two 16-byte
-// loads for fp32) and stores its C codes with one 4- or 8-byte store.  A warp
-// takes 2 KB of rows per pass (8 rows of 128 bf16 values, 4 of 256) and issues
-// all their loads before it reduces any; with four 256-thread CTAs per SM that
-// keeps 64 KB per SM in flight, enough to stream at HBM speed.
+// [l*C, l*C + C) (one 8- or 16-byte load for bf16, one or two 16-byte loads
+// for fp32) and stores its C codes with one 4- or 8-byte store.
 // ---------------------------------------------------------------------------
-constexpr int kQuantCtasPerSm = 4;
-
 template <int C, bool BF16>
-__device__ __forceinline__ void load_row(const void *__restrict__ in, int64_t base, float *v) {
-    if constexpr (BF16) {
-        const uint16_t *src = static_cast<const uint16_t *>(in) + base;
-        uint32_t w[C / 2];
-        if constexpr (C == 4) {
-            const uint2 u = __ldg(reinterpret_cast<const uint2 *>(src));
-            w[0] = u.x, w[1] = u.y;
-        } else {
-            const uint4 u = __ldg(reinterpret_cast<const uint4 *>(src));
-            w[0] = u.x, w[1] = u.y, w[2] = u.z, w[3] = u.w;
-        }
-#pragma unroll
-        for (int j = 0; j < C / 2; j++) {  // little-endian: element 2j is the low half
-            v[2 * j] = __uint_as_float(w[j] << 16);
-            v[2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
-        }
-    } else {
-        const float *src = static_cast<const float *>(in) + base;
-#pragma unroll
-        for (int j = 0; j < C; j += 4) {
-            const float4 f = __ldg(reinterpret_cast<const float4 *>(src + j));
-            v[j] = f.x, v[j + 1] = f.y, v[j + 2] = f.z, v[j + 3] = f.w;
-        }
-    }
-}
-
-template <int C, bool BF16>
-__global__ void __launch_bounds__(256, kQuantCtasPerSm)
-quantize_rows_vec_kernel(const void *__restrict__ in, int64_t n_rows, uint8_t *__restrict__ codes,
-                         float *__restrict__ scales) {
+__global__ void __launch_bounds__(256) quantize_rows_vec_kernel(const void *__restrict__ in,
+                                                                int64_t n_rows,
+                                                                uint8_t *__restrict__ codes,
+                                                                float *__restrict__ scales) {
     static_assert(C == 4 || C == 8, "4 or 8 values per lane");
-    constexpr int kRows = 32 / C;
     const int lane = threadIdx.x & 31;
     const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
-    for (int64_t r0 = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r0 < n_rows;
-         r0 += warps * kRows) {
-        float v[kRows][C];
-#pragma unroll
-        for (int u = 0; u < kRows; u++) {
-            const int64_t r = r0 + u * warps;
-            if (r < n_rows) load_row<C, BF16>(in, r * (32 * C) + (int64_t)lane * C, v[u]);
-        }
-#pragma unroll
-        for (int u = 0; u < kRows; u++) {
-            const int64_t r = r0 + u * warps;
-            if (r >= n_rows) break;  // uniform over the warp
-            float amax = 0.0f;
-#pragma unroll
-            for (int j = 0; j < C; j++) amax = fmaxf(amax, fabsf(v[u][j]));
-            const float scale = fp8_scale(warp_max(amax));
-            const float inv = __frcp_rn(scale);
-            uint32_t packed[C / 4];
-#pragma unroll
-            for (int j = 0; j < C / 4; j++) {
-                packed[j] = 0;
-#pragma unroll
-                for (int b = 0; b < 4; b++)
-                    packed[j] |= static_cast<uint32_t>(to_e4m3_by_recip(v[u][4 * j + b], scale,
-                                                                         inv))
-                                 << (8 * b);
-            }
-            const int64_t base = r * (32 * C) + (int64_t)lane * C;
+    for (int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < n_rows;
+         r += warps) {
+        const int64_t base = r * (32 * C) + (int64_t)lane * C;
+        float v[C];
+        if constexpr (BF16) {
+            const uint16_t *src = static_cast<const uint16_t *>(in) + base;
+            uint32_t w[C / 2];
             if constexpr (C == 4) {
-                *reinterpret_cast<uint32_t *>(codes + base) = packed[0];
+                const uint2 u = __ldg(reinterpret_cast<const uint2 *>(src));
+                w[0] = u.x, w[1] = u.y;
             } else {
-                *reinterpret_cast<uint2 *>(codes + base) = make_uint2(packed[0], packed[1]);
+                const uint4 u = __ldg(reinterpret_cast<const uint4 *>(src));
+                w[0] = u.x, w[1] = u.y, w[2] = u.z, w[3] = u.w;
             }
-            if (lane == 0) scales[r] = scale;
+#pragma unroll
+            for (int j = 0; j < C / 2; j++) {
+                v[2 * j] = __uint_as_float(w[j] << 16);
+                v[2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
+            }
+        } else {
+            const float *src = static_cast<const float *>(in) + base;
+#pragma unroll
+            for (int j = 0; j < C; j += 4) {
+                const float4 f = __ldg(reinterpret_cast<const float4 *>(src + j));
+                v[j] = f.x, v[j + 1] = f.y, v[j + 2] = f.z, v[j + 3] = f.w;
+            }
         }
+        float amax = 0.0f;
+#pragma unroll
+        for (int j = 0; j < C; j++) amax = fmaxf(amax, fabsf(v[j]));
+        const float scale = fp8_scale(warp_max(amax));
+        uint32_t packed[C / 4];
+#pragma unroll
+        for (int j = 0; j < C / 4; j++) {
+            packed[j] = 0;
+#pragma unroll
+            for (int b = 0; b < 4; b++)
+                packed[j] |= static_cast<uint32_t>(to_e4m3(v[4 * j + b], scale)) << (8 * b);
+        }
+        if constexpr (C == 4) {
+            *reinterpret_cast<uint32_t *>(codes + base) = packed[0];
+        } else {
+            *reinterpret_cast<uint2 *>(codes + base) = make_uint2(packed[0], packed[1]);
+        }
+        if (lane == 0) scales[r] = scale;
     }
 }
 
@@ -250,9 +212,8 @@ cudaError_t launch_quantize_rows(const void *in, sa_dtype in_dtype, int64_t n_ro
                                  uint8_t *codes, float *scales, cudaStream_t s) {
     if (n_rows <= 0) return cudaSuccess;
     constexpr int kThreads = 256, kWarps = kThreads / 32;
-    // one resident wave striding over the rows (a warp takes 4 or 8 per pass)
-    const int64_t want = (n_rows + kWarps * 4 - 1) / (kWarps * 4);
-    const int grid = (int)std::min<int64_t>(want, (int64_t)num_sms() * kQuantCtasPerSm);
+    const int64_t want = (n_rows + kWarps - 1) / kWarps;
+    const int grid = (int)std::min<int64_t>(want, (int64_t)num_sms() * 16);
     const bool bf16 = in_dtype == SA_BF16;
     count_launch();
     if (d == 128) {
