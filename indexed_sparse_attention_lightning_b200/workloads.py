@@ -123,7 +123,13 @@ DECODE_B64_BF16_INDEX = WorkloadSpec(
     name="decode_b64_16k_32k_bf16_index", seed=2, batch=64, seq_len=("uniform", 16384, 32768),
     keys=("planted", 0.05, 3.0), index_dtype="bf16")
 
-EXTRA = (PROFILE_B64_16K, DECODE_B64_BF16_INDEX)
+# the 1M FP8 decode with the pages' latent-cache granularity: one scale per
+# token and per 128 latent dims instead of one per page
+DECODE_B2_1M_FP8KV_TILE_1X128 = WorkloadSpec(
+    name="decode_b2_1m_fp8kv_tile_1x128", seed=4, batch=2, seq_len=("fixed", 1048576),
+    kv_dtype="e4m3", keys=("clusters", 16, 4096), kv_scale_tile=(1, 128))
+
+EXTRA = (PROFILE_B64_16K, DECODE_B64_BF16_INDEX, DECODE_B2_1M_FP8KV_TILE_1X128)
 
 
 def spec(which) -> WorkloadSpec:
