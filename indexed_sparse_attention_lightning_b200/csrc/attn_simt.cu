@@ -170,8 +170,9 @@ cudaError_t launch_hg(const PathParams &p, const int32_t *idx, int32_t K, void *
     const int D = p.d_latent + p.d_rope;
     size_t smem = sizeof(float) * ((size_t)HG * D + (size_t)kRows * (D + 1) + HG * kRows + 4 * HG) +
                   sizeof(int64_t) * (kRows + 2);
-    cudaFuncSetAttribute(attn_simt_kernel<HG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)smem);
+    const cudaError_t e = cudaFuncSetAttribute(
+        attn_simt_kernel<HG>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
     dim3 grid(p.heads / HG, p.n_q);
     count_launch();
     return launch_pdl(attn_simt_kernel<HG>, grid, dim3(kThreads), smem, s, p, idx, K, out,

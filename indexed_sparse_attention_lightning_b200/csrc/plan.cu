@@ -2,6 +2,8 @@
 // the inclusive prefix of its 128-key tile count, which the persistent
 // kernels use to split the concatenated tiles of all queries evenly.  The
 // same launch clears the per-call histograms and counters.
+#include <atomic>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -73,17 +75,21 @@ cudaError_t launch_plan(const PathParams &p, int32_t *vis, int32_t *tile_end, in
 }
 
 int num_sms() {
-    static int cached_dev = -1, cached = 0;
+    // one slot per device, safe to read and fill from any host thread (the
+    // value is the same whoever stores it)
+    constexpr int kMaxDevices = 64;
+    static std::atomic<int> cached[kMaxDevices];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 148;
-    if (dev != cached_dev) {
-        int n = 0;
-        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
-            n = 148;
-        cached = n;
-        cached_dev = dev;
+    if (dev >= 0 && dev < kMaxDevices) {
+        const int n = cached[dev].load(std::memory_order_relaxed);
+        if (n > 0) return n;
     }
-    return cached;
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+        n = 148;
+    if (dev >= 0 && dev < kMaxDevices) cached[dev].store(n, std::memory_order_relaxed);
+    return n;
 }
 
 }  // namespace sa
