@@ -185,3 +185,32 @@ def test_append_workspace_needs_no_query(L):
     assert L.sa_workspace_size(ctypes.byref(c), None, 0, _abi.SA_WS_APPEND) == 256
     assert L.sa_workspace_size(ctypes.byref(good_cache(page_size=16)), None, 0,
                                _abi.SA_WS_APPEND) == 0
+
+
+def test_struct_layout_matches_the_header(tmp_path):
+    """The ctypes mirrors have the same size and field offsets as the C structs
+    of include/sa.h, as gcc lays them out."""
+    structs = {"sa_cache": _abi.SaCache, "sa_query": _abi.SaQuery,
+               "sa_new_tokens": _abi.SaNewTokens}
+    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "sa.h"', 'int main(void) {']
+    for cname, py in structs.items():
+        lines.append(f'    printf("{cname} size %zu\\n", sizeof({cname}));')
+        for fname, _ in py._fields_:
+            lines.append(f'    printf("{cname} {fname} %zu\\n", offsetof({cname}, {fname}));')
+    lines += ['    return 0;', '}']
+    src = tmp_path / "layout.c"
+    exe = tmp_path / "layout"
+    src.write_text("\n".join(lines) + "\n")
+    include = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                           "include")
+    import subprocess
+    subprocess.run(["gcc", "-std=c11", "-I", include, str(src), "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout
+    seen = {}
+    for line in out.splitlines():
+        cname, field, value = line.split()
+        seen[(cname, field)] = int(value)
+    for cname, py in structs.items():
+        assert seen[(cname, "size")] == ctypes.sizeof(py), cname
+        for fname, _ in py._fields_:
+            assert seen[(cname, fname)] == getattr(py, fname).offset, (cname, fname)
