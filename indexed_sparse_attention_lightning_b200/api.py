@@ -34,6 +34,36 @@ def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
     return None if t is None else t.data_ptr()
 
 
+def _need(t, name: str, dtype=None, shape=None, optional: bool = False) -> None:
+    """Marshalling precondition: a contiguous CUDA tensor (of `dtype` and `shape`
+    when given).  The library reads raw pointers, so a host tensor, a strided
+    view or an int64 index tensor would be misread; refuse them here."""
+    if t is None:
+        if optional:
+            return
+        raise SaError(_abi.SA_ERR_INVALID_ARG, f"{name} is required")
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise SaError(_abi.SA_ERR_INVALID_ARG, f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise SaError(_abi.SA_ERR_INVALID_ARG, f"{name} must be contiguous")
+    if dtype is not None and t.dtype not in (dtype if isinstance(dtype, tuple) else (dtype,)):
+        raise SaError(_abi.SA_ERR_INVALID_ARG, f"{name} has dtype {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise SaError(_abi.SA_ERR_INVALID_ARG, f"{name} has shape {tuple(t.shape)}, "
+                                               f"expected {tuple(shape)}")
+
+
+def _need_rows(t, name: str, n_rows: int, min_cols: int) -> None:
+    """A CUDA fp32 matrix whose rows may be padded (unit column stride)."""
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise SaError(_abi.SA_ERR_INVALID_ARG, f"{name} must be a CUDA tensor")
+    if t.dtype != torch.float32 or t.dim() != 2 or t.stride(1) != 1:
+        raise SaError(_abi.SA_ERR_INVALID_ARG, f"{name} must be a float32 matrix with unit "
+                                               "column stride")
+    if t.shape[0] != n_rows or t.shape[1] < min_cols:
+        raise SaError(_abi.SA_ERR_INVALID_ARG, f"{name} has shape {tuple(t.shape)}")
+
+
 def _stream(stream) -> int:
     if stream is None:
         stream = torch.cuda.current_stream()
@@ -61,6 +91,10 @@ class DeviceCache:
     kv_scale_tile: tuple = (0, 0)   # (tokens, dims) per e4m3 scale; (0, 0): one per page
 
     def struct(self) -> SaCache:
+        _need(self.page_table, "page_table", torch.int32)
+        _need(self.seq_len, "seq_len", torch.int32)
+        for name in ("k_index", "k_index_scale", "kv", "kv_rope", "kv_scale"):
+            _need(getattr(self, name), name, optional=True)
         return SaCache(
             page_table=_ptr(self.page_table), seq_len=_ptr(self.seq_len),
             batch=self.page_table.shape[0], max_pages=self.page_table.shape[1],
@@ -93,6 +127,10 @@ class DeviceQueries:
         return int(self.q_seq.shape[0])
 
     def struct(self) -> SaQuery:
+        _need(self.q_seq, "q_seq", torch.int32)
+        _need(self.q_pos, "q_pos", torch.int32)
+        for name in ("q_index", "q_index_scale", "w", "q"):
+            _need(getattr(self, name), name, optional=True)
         return SaQuery(
             n_q=self.n_q, q_seq=_ptr(self.q_seq), q_pos=_ptr(self.q_pos),
             max_visible=self.max_visible, q_index=_ptr(self.q_index),
@@ -179,6 +217,8 @@ def indexer_score(cache: DeviceCache, queries: DeviceQueries, scores=None, ws=No
                             dtype=torch.float32, device=dev)
     if ws is None:
         ws = workspace(workspace_size(cache, queries, 1, _abi.SA_WS_INDEXER), dev)
+    _need_rows(scores, "scores", queries.n_q, queries.max_visible)
+    _need(ws, "ws")
     c, q = cache.struct(), queries.struct()
     check(_abi.lib().sa_indexer_score(ctypes.byref(c), ctypes.byref(q), _ptr(scores),
                                       scores.stride(0), _ptr(ws), ws.numel(), _stream(stream)),
@@ -193,6 +233,10 @@ def topk(scores: torch.Tensor, valid_len: torch.Tensor, top_k: int, max_valid: i
         idx = torch.empty((n_q, top_k), dtype=torch.int32, device=scores.device)
     if ws is None:
         ws = workspace(256, scores.device)
+    _need_rows(scores, "scores", n_q, max_valid)
+    _need(valid_len, "valid_len", torch.int32, (n_q,))
+    _need(idx, "idx", torch.int32, (n_q, top_k))
+    _need(ws, "ws")
     check(_abi.lib().sa_topk(_ptr(scores), scores.stride(0), _ptr(valid_len), n_q, max_valid,
                              top_k, _ptr(idx), _ptr(ws), ws.numel(), _stream(stream)),
           "sa_topk")
@@ -201,11 +245,13 @@ def topk(scores: torch.Tensor, valid_len: torch.Tensor, top_k: int, max_valid: i
 
 def _outputs(queries: DeviceQueries, d_latent: int, out, lse, out_dtype: str):
     dev = queries.q_seq.device
+    dt = torch.bfloat16 if out_dtype == "bf16" else torch.float32
     if out is None:
-        dt = torch.bfloat16 if out_dtype == "bf16" else torch.float32
         out = torch.empty((queries.n_q, queries.heads, d_latent), dtype=dt, device=dev)
     if lse is None:
         lse = torch.empty((queries.n_q, queries.heads), dtype=torch.float32, device=dev)
+    _need(out, "out", dt, (queries.n_q, queries.heads, d_latent))
+    _need(lse, "lse", torch.float32, (queries.n_q, queries.heads))
     return out, lse
 
 
@@ -214,6 +260,8 @@ def sparse_mla_attn(cache: DeviceCache, queries: DeviceQueries, idx: torch.Tenso
     out, lse = _outputs(queries, cache.d_latent, out, lse, out_dtype)
     if ws is None:
         ws = workspace(workspace_size(cache, queries, top_k, _abi.SA_WS_ATTN), idx.device)
+    _need(idx, "idx", torch.int32, (queries.n_q, top_k))
+    _need(ws, "ws")
     c, q = cache.struct(), queries.struct()
     check(_abi.lib().sa_sparse_mla_attn(ctypes.byref(c), ctypes.byref(q), _ptr(idx), top_k,
                                         _ptr(out), _abi.DTYPES[out_dtype], _ptr(lse), _ptr(ws),
@@ -232,6 +280,8 @@ def decode(cache: DeviceCache, queries: DeviceQueries, top_k: int, out=None, lse
     if ws is None:
         ws = workspace(workspace_size(cache, queries, top_k, _abi.SA_WS_DECODE),
                        queries.q_seq.device)
+    _need(idx, "idx", torch.int32, (queries.n_q, top_k), optional=True)
+    _need(ws, "ws")
     c, q = cache.struct(), queries.struct()
     args = (ctypes.byref(c), ctypes.byref(q), top_k, _ptr(idx), _ptr(out),
             _abi.DTYPES[out_dtype], _ptr(lse), _ptr(ws), ws.numel(), _stream(stream))
@@ -262,12 +312,14 @@ def _in_dtype(t: torch.Tensor) -> int:
 def quantize_index_query(q: torch.Tensor, out=None, scale=None, stream=None):
     """Indexer query [n_q, h_index, d_index] (bfloat16 or float32) -> (e4m3 codes
     uint8 [n_q, h_index, d_index], fp32 scales [n_q, h_index])."""
-    q = q.contiguous()
+    _need(q, "q", (torch.bfloat16, torch.float32))
     n_q, h, d = q.shape
     if out is None:
         out = torch.empty((n_q, h, d), dtype=torch.uint8, device=q.device)
     if scale is None:
         scale = torch.empty((n_q, h), dtype=torch.float32, device=q.device)
+    _need(out, "out", torch.uint8, (n_q, h, d))
+    _need(scale, "scale", torch.float32, (n_q, h))
     check(_abi.lib().sa_quantize_index_query(_ptr(q), _in_dtype(q), n_q, h, d, _ptr(out),
                                              _ptr(scale), _stream(stream)),
           "sa_quantize_index_query")
@@ -284,8 +336,13 @@ def append_tokens(cache: DeviceCache, seq: torch.Tensor, pos: torch.Tensor,
     ins = [t for t in (k_index, kv) if t is not None]
     if len({t.dtype for t in ins}) > 1:
         raise SaError(_abi.SA_ERR_INVALID_ARG, "append_tokens: k_index and kv dtypes differ")
-    k_index = None if k_index is None else k_index.contiguous()
-    kv = None if kv is None else kv.contiguous()
+    n_new = int(seq.numel())
+    _need(seq, "seq", torch.int32, (n_new,))
+    _need(pos, "pos", torch.int32, (n_new,))
+    _need(k_index, "k_index", (torch.bfloat16, torch.float32), (n_new, cache.d_index),
+          optional=True)
+    _need(kv, "kv", (torch.bfloat16, torch.float32), (n_new, cache.d_latent + cache.d_rope),
+          optional=True)
     dt = _in_dtype(ins[0]) if ins else _abi.SA_BF16
     c = cache.struct()
     if ws is None:
@@ -293,7 +350,8 @@ def append_tokens(cache: DeviceCache, seq: torch.Tensor, pos: torch.Tensor,
         if n == 0:
             raise SaError(_abi.SA_ERR_INVALID_ARG, "sa_workspace_size")
         ws = workspace(n, seq.device)
-    t = SaNewTokens(n_new=int(seq.numel()), seq=_ptr(seq), pos=_ptr(pos), in_dtype=dt,
+    _need(ws, "ws")
+    t = SaNewTokens(n_new=n_new, seq=_ptr(seq), pos=_ptr(pos), in_dtype=dt,
                     k_index=_ptr(k_index), kv=_ptr(kv))
     check(_abi.lib().sa_append_tokens(ctypes.byref(c), ctypes.byref(t), _ptr(ws), ws.numel(),
                                       _stream(stream)),

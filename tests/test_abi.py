@@ -5,6 +5,7 @@ import os
 import re
 
 import pytest
+import torch
 
 from indexed_sparse_attention_lightning_b200 import _abi, build
 
@@ -214,3 +215,39 @@ def test_struct_layout_matches_the_header(tmp_path):
         assert seen[(cname, "size")] == ctypes.sizeof(py), cname
         for fname, _ in py._fields_:
             assert seen[(cname, fname)] == getattr(py, fname).offset, (cname, fname)
+
+
+class _OnDevice(torch.Tensor):
+    """A host tensor that reports itself as a CUDA tensor, to exercise the
+    binding's dtype, shape and layout checks without a GPU (never passed on)."""
+
+    @property
+    def is_cuda(self):
+        return True
+
+
+def test_binding_refuses_tensors_it_would_misread():
+    from indexed_sparse_attention_lightning_b200 import api
+    need = api._need
+    with pytest.raises(_abi.SaError, match="CUDA tensor"):
+        need(torch.zeros(4, dtype=torch.int32), "seq", torch.int32)
+    dev = lambda t: t.as_subclass(_OnDevice)  # noqa: E731
+    need(dev(torch.zeros(4, dtype=torch.int32)), "seq", torch.int32, (4,))
+    with pytest.raises(_abi.SaError, match="dtype"):
+        need(dev(torch.zeros(4, dtype=torch.int64)), "seq", torch.int32)
+    with pytest.raises(_abi.SaError, match="shape"):
+        need(dev(torch.zeros(5, dtype=torch.int32)), "seq", torch.int32, (4,))
+    with pytest.raises(_abi.SaError, match="contiguous"):
+        need(dev(torch.zeros((4, 6), dtype=torch.float32)[:, ::2]), "x")
+    with pytest.raises(_abi.SaError, match="required"):
+        need(None, "x")
+    need(None, "x", optional=True)
+    # score matrices may have padded rows but need unit column stride
+    api._need_rows(dev(torch.zeros((3, 10), dtype=torch.float32)[:, :7]), "scores", 3, 7)
+    with pytest.raises(_abi.SaError):
+        api._need_rows(dev(torch.zeros((3, 10), dtype=torch.float32)[:, ::2]), "scores", 3, 5)
+    with pytest.raises(_abi.SaError):
+        api._need_rows(dev(torch.zeros((3, 10), dtype=torch.float32)), "scores", 3, 11)
+    # the entry points check before they reach the library
+    with pytest.raises(_abi.SaError, match="CUDA tensor"):
+        api.quantize_index_query(torch.zeros((2, 64, 128), dtype=torch.bfloat16))
