@@ -15,18 +15,21 @@
 // wide, so its tiles are stored as two 64-column halves.  The kernel is
 // persistent: the tiles of all queries are laid end to end and every CTA takes
 // an equal contiguous share, so short and long contexts balance across SMs.
-// Roles per CTA (192 threads):
-//   warp 0     TMA producer: key pages (8 KB each, 128-byte swizzle) straight
-//              from the paged cache into a 4-stage ring together with their
-//              per-token scales (bulk copy), and the query's 64x128 e4m3 block
-//              when the query changes;
-//   warp 1     one thread issues the MMAs and commits them to mbarriers;
-//   warps 2-5  epilogue: each thread owns one key row of the tile, reads its
-//              64 head scores from TMEM (tcgen05.ld), applies ReLU, the head
-//              weights and the staged key scale, and writes one fp32 score;
-//              for the fused top-K it also counts the score's 12-bit radix
-//              bucket in a shared-memory histogram per query, which is added
-//              to the query's global histogram when the CTA leaves the query.
+// Roles per CTA (320 threads; two CTAs per SM for e4m3, one for bf16):
+//   warp 0     TMA producer: key pages (8 KB e4m3, or two 8 KB halves bf16,
+//              128-byte swizzle) straight from the paged cache into a 4-stage
+//              ring, with their per-token scales (bulk copy, e4m3 only) in a
+//              ring of their own, and the query's 64x128 block when the query
+//              changes; page-table entries are read one tile ahead;
+//   warp 1     one thread issues the MMAs into four TMEM accumulators and
+//              commits them to mbarriers;
+//   warps 2-9  epilogue, two groups of four warps taking alternate tiles: each
+//              thread owns one key row of the tile, reads its 64 head scores
+//              from TMEM (tcgen05.ld), applies ReLU, the head weights and the
+//              staged key scale, and writes one fp32 score; for the fused top-K
+//              it also counts the score's 12-bit radix bucket in a shared-memory
+//              histogram per query, which is added to the query's global
+//              histogram when the CTA leaves the query.
 // Every wait is bounded; a timeout is reported in the workspace status word.
 #include <cstddef>
 
