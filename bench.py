@@ -245,6 +245,18 @@ def time_oracle(wl, budget_s: float):
     return done, spent
 
 
+def workload_config(sp, wl, world: int) -> dict:
+    """The bench line's `config`: the workload by name and its sizes (both arms)."""
+    return {
+        "workload": sp.name, "batch": int(wl.seq_len.shape[0]), "queries_per_gpu": wl.n_q,
+        "context_mean": float(wl.seq_len.mean()), "top_k": sp.top_k, "heads": sp.heads,
+        "index_heads": sp.h_index, "index_dim": sp.d_index,
+        "index_dtype": sp.index_dtype, "kv_dtype": sp.kv_dtype,
+        "page_size": sp.page_size,
+        "l2": "flushed before every timed step (256 MiB written, then read back)",
+        "parallelism": f"replicas x{world}"}
+
+
 def run_reference(args, rank: int, world: int):
     if rank != 0:
         return 0
@@ -270,7 +282,9 @@ def run_reference(args, rank: int, world: int):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": wl.spec.name, "sample": "1 query per step, rotating"},
+        "config": dict(workload_config(wl.spec, wl, world),
+                       l2="host memory (the oracle runs on the CPU)",
+                       sample="1 query of the workload per step, rotating"),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": "1 query of the workload per step (fp64 oracle, all steps)"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -536,13 +550,7 @@ def run_ours(args, rank: int, world: int, dist):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": f"{sp.index_dtype}+{sp.kv_dtype}", "data": "synthetic",
-        "config": {
-            "workload": sp.name, "batch": int(wl.seq_len.shape[0]), "queries_per_gpu": wl.n_q,
-            "context_mean": float(wl.seq_len.mean()), "top_k": K, "heads": sp.heads,
-            "index_heads": sp.h_index, "index_dim": sp.d_index,
-            "index_dtype": sp.index_dtype, "kv_dtype": sp.kv_dtype,
-            "page_size": sp.page_size, "l2": "flushed before every timed step (256 MiB written, then read back)",
-            "parallelism": f"replicas x{world}"},
+        "config": workload_config(sp, wl, world),
         "roofline": dict(roof, traffic=traffic if roof["bound"] == "hbm" else None),
         "path_hbm": {"bytes_per_step": nbytes["total"], "achieved_gbs": step_gbs,
                      "frac_of_measured": step_gbs / peak, "frac_of_8tbs": step_gbs / SPEC_HBM_GBS},

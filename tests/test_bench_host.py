@@ -77,3 +77,29 @@ def test_input_prep_bytes():
     wl8 = W.make_workload(sp8)
     stored = sp.d_latent + 2 * sp.d_rope + 4 * (sp.d_latent // 128)
     assert bench.input_prep_bytes(wl8, True) == q + keys + n * (D * 2 + stored)
+
+
+def test_reference_arm_prints_one_contract_line():
+    """`bench.py --impl reference` times the oracle on the host and prints one
+    JSON line with the same metric and workload config as the GPU arm."""
+    import json
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference",
+                        "--workload", "tiny_decode_b1_1k_fp32", "--steps", "2", "--warmup", "1"],
+                       capture_output=True, text=True, timeout=300, check=True)
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["metric"] == bench.METRIC and d["unit"] == bench.UNIT
+    assert d["higher_is_better"] is True and d["steps"] == 2 and d["warmup"] == 1
+    assert d["value"] > 0 and d["cpu_baseline"]["value"] == d["value"]
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["e2e"] == {"value": d["value"], "unit": bench.UNIT, "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
+    wl = W.make_workload(W.spec("tiny_decode_b1_1k_fp32"))
+    ours = bench.workload_config(wl.spec, wl, 1)
+    assert {k: v for k, v in d["config"].items() if k not in ("l2", "sample")} == \
+        {k: v for k, v in ours.items() if k != "l2"}
