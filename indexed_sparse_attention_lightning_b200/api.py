@@ -158,6 +158,9 @@ class DeviceQueries:
 def upload(wl, device="cuda") -> tuple[DeviceCache, DeviceQueries]:
     """Place a workload (numpy arrays) on the device."""
     sp = wl.spec
+    if getattr(sp, "index_scale_group", 0):
+        raise SaError(_abi.SA_ERR_UNSUPPORTED,
+                      "upload: index scales per group of values have no kernel in this library")
     cache = DeviceCache(
         page_table=_t(wl.page_table, device), seq_len=_t(wl.seq_len, device),
         num_pages=int(wl.num_pages), index_dtype=sp.index_dtype,

@@ -13,7 +13,8 @@ indexer and the sparse attention kernel -- "Optimizing Next-Gen LLM Inference"
 * ``page_table[b, i]`` is the physical page holding tokens ``64*i .. 64*i+63``
   of sequence ``b``; entries past the sequence end are -1.
 * index keys ``k_index[P, 64, d_index]`` (fp32, bf16, or e4m3 codes with one
-  fp32 scale per token in ``k_index_scale[P, 64]``);
+  fp32 scale per token in ``k_index_scale[P, 64]``, or one per group of values
+  in ``k_index_scale[P, 64, d_index / group]``);
 * MLA latent rows ``kv[P, 64, d_latent + d_rope]`` (fp32 or bf16), or for the
   FP8 cache ``kv[P, 64, d_latent]`` e4m3 codes, ``kv_scale[P, 64 / ts, d_latent / td]``
   (one fp32 scale per tile of ts tokens x td latent dims of a page; the default
@@ -56,6 +57,9 @@ class WorkloadSpec:
     h_index: int = 64
     d_index: int = 128
     index_dtype: str = "e4m3"      # "e4m3", "bf16" or "f32"
+    # e4m3 index scales: 0 = one per key row and one per (query, head) row; g = one
+    # per g consecutive values of a row (the pages' group-32 quantisation)
+    index_scale_group: int = 0
     top_k: int = 2048
     heads: int = 128
     d_latent: int = 512
@@ -156,9 +160,9 @@ class Workload:
     q_seq: np.ndarray            # int32 [n_q]
     q_pos: np.ndarray            # int32 [n_q]; visible length is q_pos + 1
     k_index: np.ndarray          # f32, uint16 (bf16) or uint8 (e4m3) [P, ps, d_index]
-    k_index_scale: Optional[np.ndarray]  # f32 [P, ps]
+    k_index_scale: Optional[np.ndarray]  # f32 [P, ps] (or [P, ps, d_index / group])
     q_index: np.ndarray          # f32, uint16 (bf16) or uint8 (e4m3) [n_q, h_index, d_index]
-    q_index_scale: Optional[np.ndarray]  # f32 [n_q, h_index]
+    q_index_scale: Optional[np.ndarray]  # f32 [n_q, h_index] (or [n_q, h_index, d_index / group])
     w: np.ndarray                # f32 [n_q, h_index]
     kv: np.ndarray               # f32/uint16(bf16) [P, ps, d_qk] or uint8 [P, ps, d_latent]
     kv_rope: Optional[np.ndarray]  # uint16 (bf16) [P, ps, d_rope] for the e4m3 cache
@@ -212,6 +216,18 @@ def quantize_rows_e4m3(x: np.ndarray):
     amax = np.abs(x).max(axis=-1)
     scale = amax_scale(amax)
     return to_e4m3_codes(x / scale[..., None]), scale
+
+
+def quantize_groups_e4m3(x: np.ndarray, group: int):
+    """One scale per `group` consecutive values of the last axis: returns
+    (codes uint8 like x, scale f32 [..., last / group])."""
+    g = x.reshape(x.shape[:-1] + (x.shape[-1] // group, group))
+    codes, scale = quantize_rows_e4m3(g)
+    return codes.reshape(x.shape), scale
+
+
+def _quantize_index(x: np.ndarray, group: int):
+    return quantize_groups_e4m3(x, group) if group > 0 else quantize_rows_e4m3(x)
 
 
 # ----------------------------------------------------------------------------
@@ -293,8 +309,10 @@ def make_workload(sp: WorkloadSpec) -> Workload:
     # indexer queries and head weights
     qi = _normal(rng, (n_q, H_I, d_I))
     w = (_normal(rng, (n_q, H_I)) / np.float32(math.sqrt(H_I))).astype(np.float32)
+    if sp.index_scale_group and (sp.index_dtype != "e4m3" or d_I % sp.index_scale_group):
+        raise ValueError("group scales need e4m3 index data and a group dividing d_index")
     if sp.index_dtype == "e4m3":
-        q_index, q_index_scale = quantize_rows_e4m3(qi)
+        q_index, q_index_scale = _quantize_index(qi, sp.index_scale_group)
     elif sp.index_dtype == "bf16":
         q_index, q_index_scale = to_bf16_bits(qi), None
     elif sp.index_dtype == "f32":
@@ -306,7 +324,9 @@ def make_workload(sp: WorkloadSpec) -> Workload:
     rows = num_pages * ps
     if sp.index_dtype == "e4m3":
         k_index = np.full((rows, d_I), E4M3_NAN, dtype=np.uint8)
-        k_index_scale = np.full((rows,), np.nan, dtype=np.float32)
+        k_index_scale = np.full((rows,) + ((d_I // sp.index_scale_group,)
+                                           if sp.index_scale_group else ()),
+                                np.nan, dtype=np.float32)
     elif sp.index_dtype == "bf16":
         k_index = np.full((rows, d_I), BF16_NAN, dtype=np.uint16)
         k_index_scale = None
@@ -331,7 +351,9 @@ def make_workload(sp: WorkloadSpec) -> Workload:
             t = int(qb[-1])
             if sp.index_dtype == "e4m3":
                 qdeq = torch.from_numpy(q_index[t]).view(torch.float8_e4m3fn).float().numpy()
-                qdeq = qdeq * q_index_scale[t][:, None]
+                sc = q_index_scale[t]
+                qdeq = qdeq * (np.repeat(sc, sp.index_scale_group, axis=-1)
+                               if sp.index_scale_group else sc[:, None])
             elif sp.index_dtype == "bf16":
                 qdeq = (q_index[t].astype(np.uint32) << 16).view(np.float32)
             else:
@@ -365,7 +387,7 @@ def make_workload(sp: WorkloadSpec) -> Workload:
                                             / np.float32(math.sqrt(2.0)))
             dst = _phys_rows(pt, c0, c1, ps)
             if sp.index_dtype == "e4m3":
-                codes, sc = quantize_rows_e4m3(k)
+                codes, sc = _quantize_index(k, sp.index_scale_group)
                 k_index[dst] = codes
                 k_index_scale[dst] = sc
             elif sp.index_dtype == "bf16":
@@ -374,7 +396,7 @@ def make_workload(sp: WorkloadSpec) -> Workload:
                 k_index[dst] = k
     k_index = k_index.reshape(num_pages, ps, d_I)
     if k_index_scale is not None:
-        k_index_scale = k_index_scale.reshape(num_pages, ps)
+        k_index_scale = k_index_scale.reshape((num_pages, ps) + k_index_scale.shape[1:])
 
     # MLA latent cache
     D, dl, dr = sp.d_qk, sp.d_latent, sp.d_rope

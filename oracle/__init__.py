@@ -51,7 +51,7 @@ def _load():
         P, I32, I64, D = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_double
         lib.oracle_decode.argtypes = [ctypes.c_int, P, P, I64]
         lib.oracle_decode.restype = None
-        lib.oracle_index_scores.argtypes = [I32, P, P, I32, I32, I32, P, P, P, I32, P, P,
+        lib.oracle_index_scores.argtypes = [I32, P, P, I32, I32, I32, I32, P, P, P, I32, P, P,
                                             P, I32, I32, I32, P, I64, ctypes.c_int]
         lib.oracle_index_scores.restype = ctypes.c_int
         lib.oracle_topk.argtypes = [I32, P, I64, P, I32, P]
@@ -116,6 +116,7 @@ def index_scores(wl, nthreads: int | None = None) -> np.ndarray:
     pt = _c(wl.page_table, np.int32)
     rc = _load().oracle_index_scores(
         n_q, _ptr(q_seq), _ptr(q_pos), wl.spec.h_index, wl.spec.d_index,
+        getattr(wl.spec, "index_scale_group", 0),
         dt, _ptr(qi), _ptr(qs), _ptr(w), dt, _ptr(ki), _ptr(ks),
         _ptr(pt), pt.shape[1], wl.spec.page_size, wl.num_pages,
         _ptr(scores), ld, nthreads or threads())

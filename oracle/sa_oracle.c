@@ -171,13 +171,14 @@ typedef struct {
     int32_t n_q;
     const int32_t *q_seq, *q_pos;
     int32_t h_index, d_index;
+    int32_t scale_group;       /* e4m3 scale granularity: 0 = one per row, g = one per g values */
     int32_t q_dtype;           /* OR_F32, OR_BF16 or OR_E4M3 */
     const void *q_index;       /* [n_q, h_index, d_index] */
-    const float *q_index_scale;/* [n_q, h_index] for e4m3 */
+    const float *q_index_scale;/* [n_q, h_index, d_index / g] (g = d_index when 0) for e4m3 */
     const float *w;            /* [n_q, h_index] */
     int32_t k_dtype;           /* OR_F32, OR_BF16 or OR_E4M3 */
     const void *k_index;       /* [rows, d_index] */
-    const float *k_index_scale;/* [rows] for e4m3 */
+    const float *k_index_scale;/* [rows, d_index / g] for e4m3 */
     pages_t pg;
     double *scores;
     int64_t ld;
@@ -195,6 +196,8 @@ static int score_item(pool_t *p, int64_t item)
     if (s0 >= s1)
         return OR_OK;
     const int H = c->h_index, d = c->d_index;
+    const int g = c->scale_group > 0 ? c->scale_group : d;   /* values per scale */
+    const int ng = d / g;                                     /* scales per row */
     double *q = malloc(sizeof(double) * (size_t)H * d);
     double *k = malloc(sizeof(double) * (size_t)d);
     if (!q || !k) {
@@ -203,11 +206,12 @@ static int score_item(pool_t *p, int64_t item)
         return OR_NO_MEMORY;
     }
     /* dequantised indexer query q_I[t] */
-    for (int j = 0; j < H; j++) {
-        double qs = c->q_dtype == OR_E4M3 ? (double)c->q_index_scale[t * H + j] : 1.0;
-        for (int i = 0; i < d; i++)
+    for (int j = 0; j < H; j++)
+        for (int i = 0; i < d; i++) {
+            double qs = c->q_dtype == OR_E4M3
+                            ? (double)c->q_index_scale[(t * H + j) * (int64_t)ng + i / g] : 1.0;
             q[j * d + i] = element(c->q_dtype, c->q_index, (t * H + j) * (int64_t)d + i) * qs;
-    }
+        }
     int rc = OR_OK;
     for (int64_t s = s0; s < s1 && rc == OR_OK; s++) {
         int64_t row = phys_row(&c->pg, c->q_seq[t], s);
@@ -215,8 +219,8 @@ static int score_item(pool_t *p, int64_t item)
             rc = OR_BAD_PAGE;
             break;
         }
-        double ks = c->k_dtype == OR_E4M3 ? (double)c->k_index_scale[row] : 1.0;
         for (int i = 0; i < d; i++) {
+            double ks = c->k_dtype == OR_E4M3 ? (double)c->k_index_scale[row * ng + i / g] : 1.0;
             k[i] = element(c->k_dtype, c->k_index, row * d + i) * ks;
             if (isnan(k[i]))
                 rc = OR_NAN;     /* a poisoned (never written) slot was read */
@@ -238,7 +242,7 @@ static int score_item(pool_t *p, int64_t item)
 }
 
 int oracle_index_scores(int32_t n_q, const int32_t *q_seq, const int32_t *q_pos,
-                        int32_t h_index, int32_t d_index,
+                        int32_t h_index, int32_t d_index, int32_t scale_group,
                         int32_t q_dtype, const void *q_index, const float *q_index_scale,
                         const float *w,
                         int32_t k_dtype, const void *k_index, const float *k_index_scale,
@@ -246,6 +250,11 @@ int oracle_index_scores(int32_t n_q, const int32_t *q_seq, const int32_t *q_pos,
                         int32_t num_pages, double *scores, int64_t ld, int nthreads)
 {
     if (n_q < 0 || h_index <= 0 || d_index <= 0 || page_size <= 0 || !scores)
+        return OR_BAD_ARG;
+    /* one scale per row (the spec form), or one per group of scale_group
+     * values (the pages' group-32 scales, "Inference Acceleration for New Large
+     * Model Architectures" §4.1; "Optimizing Next-Gen LLM Inference" §4 table) */
+    if (scale_group < 0 || (scale_group > 0 && d_index % scale_group != 0))
         return OR_BAD_ARG;
     /* the indexer's BF16 path ("Optimizing Next-Gen LLM Inference" §3.1: a BF16
      * path next to the quantised one) reads unscaled bf16 values */
@@ -260,7 +269,8 @@ int oracle_index_scores(int32_t n_q, const int32_t *q_seq, const int32_t *q_pos,
         if (V > maxV)
             maxV = V;
     }
-    score_ctx c = { n_q, q_seq, q_pos, h_index, d_index, q_dtype, q_index, q_index_scale, w,
+    score_ctx c = { n_q, q_seq, q_pos, h_index, d_index, scale_group, q_dtype, q_index,
+                    q_index_scale, w,
                     k_dtype, k_index, k_index_scale,
                     { page_table, max_pages, page_size, num_pages }, scores, ld, 4096, 0 };
     c.chunks_per_query = (maxV + c.chunk - 1) / c.chunk;

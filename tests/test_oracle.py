@@ -44,9 +44,11 @@ def np_rows(wl, b, positions):
 
 def np_index_keys(wl, b, V):
     rows = np_rows(wl, b, np.arange(V))
-    k = np_values(wl.spec.index_dtype, wl.k_index.reshape(-1, wl.spec.d_index)[rows])
+    d = wl.spec.d_index
+    k = np_values(wl.spec.index_dtype, wl.k_index.reshape(-1, d)[rows])
     if wl.k_index_scale is not None:
-        k = k * wl.k_index_scale.reshape(-1)[rows][:, None].astype(np.float64)
+        per_row = wl.k_index_scale.reshape(wl.k_index.shape[0] * wl.k_index.shape[1], -1)[rows]
+        k = k * (np.repeat(per_row, d // per_row.shape[1], axis=1))
     return k
 
 
@@ -57,7 +59,8 @@ def np_scores(wl):
         k = np_index_keys(wl, int(wl.q_seq[t]), V)
         q = np_values(wl.spec.index_dtype, wl.q_index[t])
         if wl.q_index_scale is not None:
-            q = q * wl.q_index_scale[t][:, None].astype(np.float64)
+            qs = wl.q_index_scale[t].reshape(wl.spec.h_index, -1).astype(np.float64)
+            q = q * np.repeat(qs, wl.spec.d_index // qs.shape[1], axis=1)
         dots = np.einsum("sd,jd->sj", k, q)
         out[t, :V] = np.maximum(dots, 0.0) @ wl.w[t].astype(np.float64)
     return out
@@ -130,9 +133,12 @@ def test_bf16_decode_matches_torch():
 
 # --------------------------------------------------------- indexer score ---
 
-@pytest.mark.parametrize("index_dtype", ["f32", "bf16", "e4m3"])
-def test_scores_match_brute_force(index_dtype):
-    wl = W.make_workload(small_spec(index_dtype=index_dtype))
+@pytest.mark.parametrize("index_dtype,group", [("f32", 0), ("bf16", 0), ("e4m3", 0),
+                                               ("e4m3", 8)])
+def test_scores_match_brute_force(index_dtype, group):
+    """group > 0: one e4m3 scale per `group` values of the query and key rows
+    (the pages' group-wise index quantisation, here 8 of 16 dims)."""
+    wl = W.make_workload(small_spec(index_dtype=index_dtype, index_scale_group=group))
     got = oracle.index_scores(wl)
     ref = np_scores(wl)
     assert np.array_equal(np.isnan(got), np.isnan(ref))
