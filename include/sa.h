@@ -58,7 +58,7 @@ extern "C" {
 typedef enum sa_status {
     SA_OK = 0,
     SA_ERR_INVALID_ARG = 1,   /* shape, dtype, pointer or size rejected on the host */
-    SA_ERR_UNSUPPORTED = 2,   /* valid combination this build does not implement */
+    SA_ERR_UNSUPPORTED = 2,   /* valid combination the library does not implement */
     SA_ERR_WORKSPACE = 3,     /* workspace missing or smaller than sa_workspace_size() */
     SA_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed */
     SA_ERR_DEVICE_FAULT = 5,  /* bad data detected on the device (see detail code) */

@@ -251,7 +251,7 @@ int oracle_index_scores(int32_t n_q, const int32_t *q_seq, const int32_t *q_pos,
 {
     if (n_q < 0 || h_index <= 0 || d_index <= 0 || page_size <= 0 || !scores)
         return OR_BAD_ARG;
-    /* one scale per row (the spec form), or one per group of scale_group
+    /* one scale per key row and per (query, head) row, or one per group of scale_group
      * values (the pages' group-32 scales, "Inference Acceleration for New Large
      * Model Architectures" §4.1; "Optimizing Next-Gen LLM Inference" §4 table) */
     if (scale_group < 0 || (scale_group > 0 && d_index % scale_group != 0))
