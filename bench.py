@@ -580,7 +580,9 @@ def main():
         import torch
         import torch.distributed as dist
         torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+        # short enough that ranks waiting on a lost peer fail instead of hanging,
+        # long enough for every rank to draw its inputs before the first barrier
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     try:
         return run_ours(args, rank, world, dist)
     finally:
