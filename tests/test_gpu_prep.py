@@ -200,6 +200,23 @@ def test_append_reports_a_bad_page_and_writes_the_rest():
     assert api.device_status(ws) == (_abi.SA_OK, 0)
 
 
+def test_append_of_no_tokens_is_a_no_op():
+    sp = W.WorkloadSpec(name="append_none", seed=37, batch=2, seq_len=("list", (100, 200)),
+                        h_index=8, heads=16)
+    wl = W.make_workload(sp)
+    cache, _ = api.upload(wl)
+    before = _cache_arrays(cache)
+    none = torch.empty(0, dtype=torch.int32, device="cuda")
+    ws = api.append_tokens(cache, none, none,
+                           k_index=torch.empty((0, sp.d_index), dtype=torch.bfloat16,
+                                               device="cuda"))
+    assert api.device_status(ws) == (_abi.SA_OK, 0)
+    after = _cache_arrays(cache)
+    for k, a in before.items():
+        if a is not None:
+            assert np.array_equal(_bits(after[k]), _bits(a)), k
+
+
 def test_prepared_decode_step_matches_oracle():
     """Append each sequence's new token at its last position, quantise the
     step's indexer query, then decode: the GPU and the oracle agree on the
