@@ -103,3 +103,24 @@ def test_reference_arm_prints_one_contract_line():
     ours = bench.workload_config(wl.spec, wl, 1)
     assert {k: v for k, v in d["config"].items() if k not in ("l2", "sample")} == \
         {k: v for k, v in ours.items() if k != "l2"}
+
+
+def test_end_to_end_copy_accounting():
+    """The end-to-end leg copies every query input of a step and counts its bytes:
+    the count equals the bytes of the workload's query arrays, and the copy
+    lands them bit for bit (host buffers standing in for the device here)."""
+    import dataclasses
+    import torch
+    from indexed_sparse_attention_lightning_b200 import api
+    wl = W.make_workload(dataclasses.replace(W.spec("decode_b8_8k"), batch=3,
+                                             seq_len=("fixed", 300)))
+    host = api.host_queries(wl, pin=False)
+    want = sum(getattr(wl, k).nbytes for k in ("q_seq", "q_pos", "q_index", "q_index_scale",
+                                               "w", "q"))
+    _, queries = api.upload(wl, "cpu")
+    dst = dataclasses.replace(queries, **{k: torch.zeros_like(v)
+                                          for k, v in queries.tensors().items() if v is not None})
+    assert dst.copy_from(host, non_blocking=False) == want
+    for k, v in queries.tensors().items():
+        if v is not None:
+            assert torch.equal(getattr(dst, k), v), k
