@@ -7,13 +7,17 @@ three steps of the path).  Prints ONE JSON line (rank 0):
   value     query-tokens/s over all ranks, device time (CUDA events), inputs
             resident in HBM, L2 flushed before every timed step (a 256 MiB
             buffer written, then read back, outside the timed region);
-  e2e       the same metric through the public API with host buffers: pinned
-            host -> device copy of the step's queries, the call, device -> host
-            copy of the outputs, all inside the timed region (there the 256 MiB
-            write that flushes L2 sits inside the timed region too);
+  e2e       the same metric through the public API with host buffers, as a
+            serving loop runs a step: pinned host -> device copy of the step's
+            inputs (queries in the projection's format and each query's new
+            token), quantisation of the indexer query, append of the new tokens,
+            the decode, device -> host copy of the outputs, all inside the
+            timed region (steps pipelined over three streams, no L2 flush);
   roofline  the dominant phase's algorithmic bytes / its event-timed duration
             against the measured HBM copy bandwidth;
-  cpu_baseline  the fp64 oracle on a bounded sample, on this host's cores.
+  cpu_baseline  the fp64 oracle on a bounded sample, on this host's cores;
+  other_configs the other configurations, each device-timed the same way in
+            the same run (step, phases, path bytes, roofline, clocks).
 
 ``--impl reference`` times the fp64 oracle instead (rank 0 only).
 Multi-GPU (torchrun): every rank decodes its own batch (seeded per rank), no
@@ -53,6 +57,8 @@ def parse():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="time only --workload (skip the other configurations)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target CPU time of the oracle baseline sample")
     return ap.parse_args()
@@ -394,16 +400,65 @@ def time_input_prep(args, wl, cache, dev, flush):
                     "per query appended at its position"}
 
 
-def run_ours(args, rank: int, world: int, dist):
+def serving_inputs(wl) -> dict:
+    """Host arrays a serving step starts from, for the end-to-end leg: the query
+    tokens' sequence, position, head weights and attention query as in the
+    workload; the indexer query as the projection would hand it over (for an
+    e4m3 index cache in bf16 -- the e4m3 codes times their scales, so that
+    quantising it again on the device gives back the workload's query up to
+    the bf16 rounding of those products -- as
+    ``q_index_in``; otherwise in the cache's own format as ``q_index``); and
+    each query's own token -- index key and latent row, the values already
+    cached at its position -- to be appended at that position
+    (``k_new``/``kv_new``, None where the pool takes no single tokens: a bf16
+    index pool, or a latent cache with one scale per page)."""
+    import torch
+    sp = wl.spec
+    out = {k: torch.from_numpy(getattr(wl, k)) for k in ("q_seq", "q_pos", "w", "q")}
+    ps = sp.page_size
+    rows = (wl.page_table[wl.q_seq, wl.q_pos // ps].astype(np.int64) * ps + wl.q_pos % ps)
+    out["k_new"] = out["kv_new"] = None
+    if sp.index_dtype == "e4m3":
+        qi = torch.from_numpy(wl.q_index).view(torch.float8_e4m3fn).float()
+        out["q_index_in"] = (qi * torch.from_numpy(wl.q_index_scale)[..., None]).bfloat16()
+        k = torch.from_numpy(wl.k_index.reshape(-1, sp.d_index)[rows]).view(torch.float8_e4m3fn)
+        k = k.float() * torch.from_numpy(wl.k_index_scale.reshape(-1)[rows])[:, None]
+        out["k_new"] = k.bfloat16()
+    else:
+        out["q_index"] = torch.from_numpy(wl.q_index)
+        if sp.index_dtype == "f32":
+            out["k_new"] = torch.from_numpy(wl.k_index.reshape(-1, sp.d_index)[rows])
+    if sp.kv_dtype == "f32":
+        out["kv_new"] = torch.from_numpy(wl.kv.reshape(-1, sp.d_qk)[rows])
+    elif sp.kv_dtype == "bf16":
+        kv = torch.from_numpy(wl.kv.reshape(-1, sp.d_qk)[rows].view(np.int16))
+        out["kv_new"] = kv.view(torch.bfloat16)
+    elif sp.kv_tile[0] == 1:
+        st, sd = sp.kv_tile
+        codes = torch.from_numpy(wl.kv.reshape(-1, sp.d_latent)[rows]).view(torch.float8_e4m3fn)
+        sc = wl.kv_scale.reshape(wl.num_pages, ps // st, sp.d_latent // sd)
+        sc = sc[rows // ps, (rows % ps) // st]                       # [n_q, d_latent / sd]
+        lat = codes.float() * torch.from_numpy(np.repeat(sc, sd, axis=1))
+        rope = torch.from_numpy(wl.kv_rope.reshape(-1, sp.d_rope)[rows].view(np.int16))
+        out["kv_new"] = torch.cat([lat.bfloat16(), rope.view(torch.bfloat16)], dim=1)
+    ins = [t for t in (out["k_new"], out["kv_new"]) if t is not None]
+    if len({t.dtype for t in ins}) > 1:  # the append takes one input dtype
+        out["k_new"] = out["k_new"].to(out["kv_new"].dtype)
+    return out
+
+
+def serving_bytes(inp: dict) -> int:
+    """Host -> device bytes of one serving step's inputs."""
+    return sum(v.numel() * v.element_size() for v in inp.values() if v is not None)
+
+
+def measure_decode(args, wl, dev, dist=None):
+    """Device-timed fused decode on one workload: the timed steps (L2 flushed
+    before each), then the same steps again with events between the phases.
+    Returns the step time, phase times, launches, clocks and the accounting."""
     import torch
     from indexed_sparse_attention_lightning_b200 import _abi, api
-    from indexed_sparse_attention_lightning_b200 import workloads as W
-
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    sp = rank_spec(W.spec(args.workload), rank)
-    wl = W.make_workload(sp)
+    sp = wl.spec
     cache, queries = api.upload(wl, dev)
     K = sp.top_k
     odt = "f32" if sp.kv_dtype == "f32" else "bf16"
@@ -423,7 +478,7 @@ def run_ours(args, rank: int, world: int, dist):
     torch.cuda.synchronize()
     st = api.device_status(ws)
     if st[0] != _abi.SA_OK:
-        raise RuntimeError(f"device status after warm-up: {st}")
+        raise RuntimeError(f"{sp.name}: device status after warm-up: {st}")
     idx_host = idx.cpu().numpy()
     nbytes = algorithmic_bytes(wl, idx_host)
 
@@ -436,7 +491,7 @@ def run_ours(args, rank: int, world: int, dist):
         dist.barrier()
     torch.cuda.synchronize()
     launches0 = _abi.lib().sa_kernel_launches()
-    with ClockSampler(local) as clocks:
+    with ClockSampler(dev.index or 0) as clocks:
         for k in range(args.steps):
             flush_l2(flush)
             outer[k][0].record(stream)
@@ -458,79 +513,167 @@ def run_ours(args, rank: int, world: int, dist):
                 for i in range(n_phase)]
     st = api.device_status(ws)
     if st[0] != _abi.SA_OK:
-        raise RuntimeError(f"device status after timing: {st}")
+        raise RuntimeError(f"{sp.name}: device status after timing: {st}")
+    return {"total_ms": total_ms, "phase_ms": phase_ms, "launches": int(launches),
+            "clocks": clocks.summary(), "nbytes": nbytes, "idx_host": idx_host,
+            "cache": cache, "queries": queries, "ws": ws, "idx": idx, "out": out, "lse": lse,
+            "flush": flush, "odt": odt}
 
-    # end to end through the public API with host buffers: every step copies
-    # its inputs from pinned host memory and reads its output back.  Steps are
-    # pipelined the way a serving loop runs them -- the copies of one step
-    # overlap the compute of its neighbours (copy-in stream, compute stream,
-    # copy-out stream; inputs and outputs double-buffered) -- and the time
-    # runs from the first copy-in to the last copy-out.
-    e2e = None
-    if not args.no_e2e:
-        import dataclasses as _dc
-        host_in = api.host_queries(wl, pin=True)
-        comp = stream
-        s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
-        qbuf = [queries, _dc.replace(queries, **{k: torch.empty_like(v)
-                                                 for k, v in queries.tensors().items()
-                                                 if v is not None})]
-        obuf = [(out, lse), (torch.empty_like(out), torch.empty_like(lse))]
-        hout = [(torch.empty(out.shape, dtype=out.dtype, pin_memory=True),
-                 torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)) for _ in range(2)]
 
-        def pipelined(n):
-            if n <= 0:
-                return 0.0, 0
-            in_done = [torch.cuda.Event() for _ in range(n)]
-            comp_done = [torch.cuda.Event() for _ in range(n)]
-            out_done = [torch.cuda.Event() for _ in range(n)]
-            t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            h2d = 0
-            t0.record(s_in)
-            for k in range(n):
-                b = k % 2
-                with torch.cuda.stream(s_in):
-                    if k >= 2:
-                        s_in.wait_event(comp_done[k - 2])  # buffer b no longer read
-                    h2d = qbuf[b].copy_from(host_in, non_blocking=True)
-                    in_done[k].record(s_in)
-                comp.wait_event(in_done[k])
+def summarise(wl, m: dict, n_q_all: float, total_ms: float, steps: int) -> dict:
+    """The per-workload figures of a bench line."""
+    from indexed_sparse_attention_lightning_b200 import _abi
+    ms_per_step = total_ms / steps
+    peak, _, _ = measured_peaks()
+    phase_ms = m["phase_ms"]
+    dom = int(np.argmax(phase_ms))
+    dom_name = _abi.DECODE_PHASES[dom]
+    roof = roofline(wl, dom_name, phase_ms[dom], m["nbytes"],
+                    algorithmic_flops(wl, m["idx_host"]))
+    step_gbs = m["nbytes"]["total"] / (ms_per_step / 1e3) / 1e9
+    return {
+        "value": n_q_all * steps / (total_ms / 1e3), "ms_per_step": ms_per_step,
+        "roofline": roof,
+        "path_hbm": {"bytes_per_step": m["nbytes"]["total"], "achieved_gbs": step_gbs,
+                     "frac_of_measured": step_gbs / peak, "frac_of_8tbs": step_gbs / SPEC_HBM_GBS},
+        "phases_ms": dict(zip(_abi.DECODE_PHASES, phase_ms)),
+        "gpu_launches": m["launches"],
+        "clocks": m["clocks"],
+    }
+
+
+def time_e2e(args, wl, m: dict, dev):
+    """End to end through the public API with host buffers: every step copies
+    its inputs from pinned host memory -- the bf16 indexer query, head weights,
+    attention query, sequence and position of each query, and each query's own
+    new token -- then quantises the indexer query, appends the new tokens to
+    the paged caches and decodes (all on the device), and reads the output and
+    lse back.  Steps are pipelined the way a serving loop runs them -- the
+    copies of one step overlap the compute of its neighbours (copy-in stream,
+    compute stream, copy-out stream; inputs and outputs double-buffered) -- and
+    the time runs from the first copy-in to the last copy-out.  No L2 flush
+    runs inside this loop: a serving loop has none."""
+    import torch
+    from indexed_sparse_attention_lightning_b200 import api
+    sp = wl.spec
+    cache, queries, ws, idx = m["cache"], m["queries"], m["ws"], m["idx"]
+    out, lse, odt = m["out"], m["lse"], m["odt"]
+    host = {k: (v.pin_memory() if v is not None else None)
+            for k, v in serving_inputs(wl).items()}
+    comp = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+
+    def dev_set():
+        d = {k: (torch.empty_like(v, device=dev) if v is not None else None)
+             for k, v in host.items()}
+        q = dataclasses.replace(
+            queries, q_seq=d["q_seq"], q_pos=d["q_pos"], w=d["w"], q=d["q"],
+            q_index=d.get("q_index", torch.empty_like(queries.q_index)),
+            q_index_scale=(None if queries.q_index_scale is None
+                           else torch.empty_like(queries.q_index_scale)))
+        return d, q
+
+    bufs = [dev_set(), dev_set()]
+    obuf = [(out, lse), (torch.empty_like(out), torch.empty_like(lse))]
+    hout = [(torch.empty(out.shape, dtype=out.dtype, pin_memory=True),
+             torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)) for _ in range(2)]
+    aws = api.workspace(256, dev)
+
+    def pipelined(n):
+        if n <= 0:
+            return 0.0
+        in_done = [torch.cuda.Event() for _ in range(n)]
+        comp_done = [torch.cuda.Event() for _ in range(n)]
+        out_done = [torch.cuda.Event() for _ in range(n)]
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(s_in)
+        for k in range(n):
+            b = k % 2
+            d, q = bufs[b]
+            with torch.cuda.stream(s_in):
                 if k >= 2:
-                    comp.wait_event(out_done[k - 2])  # output b has been read back
-                flush.zero_()
-                api.decode(cache, qbuf[b], K, out=obuf[b][0], lse=obuf[b][1], idx=idx,
-                           out_dtype=odt, ws=ws)
-                comp_done[k].record(comp)
-                with torch.cuda.stream(s_out):
-                    s_out.wait_event(comp_done[k])
-                    hout[b][0].copy_(obuf[b][0], non_blocking=True)
-                    hout[b][1].copy_(obuf[b][1], non_blocking=True)
-                    out_done[k].record(s_out)
-            s_out.wait_event(out_done[n - 1])
-            t1.record(s_out)
-            torch.cuda.synchronize()
-            return t0.elapsed_time(t1), h2d
+                    s_in.wait_event(comp_done[k - 2])  # buffer b no longer read
+                for key, v in host.items():
+                    if v is not None:
+                        d[key].copy_(v, non_blocking=True)
+                in_done[k].record(s_in)
+            comp.wait_event(in_done[k])
+            if k >= 2:
+                comp.wait_event(out_done[k - 2])  # output b has been read back
+            if "q_index_in" in d:
+                api.quantize_index_query(d["q_index_in"], out=q.q_index,
+                                         scale=q.q_index_scale)
+            if d["k_new"] is not None or d["kv_new"] is not None:
+                api.append_tokens(cache, d["q_seq"], d["q_pos"], k_index=d["k_new"],
+                                  kv=d["kv_new"], ws=aws)
+            api.decode(cache, q, sp.top_k, out=obuf[b][0], lse=obuf[b][1], idx=idx,
+                       out_dtype=odt, ws=ws)
+            comp_done[k].record(comp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(comp_done[k])
+                hout[b][0].copy_(obuf[b][0], non_blocking=True)
+                hout[b][1].copy_(obuf[b][1], non_blocking=True)
+                out_done[k].record(s_out)
+        s_out.wait_event(out_done[n - 1])
+        t1.record(s_out)
+        torch.cuda.synchronize()
+        return t0.elapsed_time(t1)
 
-        pipelined(args.warmup)
-        e2e_total, h2d = pipelined(args.steps)
-        d2h = out.numel() * out.element_size() + lse.numel() * lse.element_size()
-        e2e = {"ms_per_step": e2e_total / args.steps, "h2d": h2d, "d2h": d2h}
+    pipelined(args.warmup)
+    total = pipelined(args.steps)
+    st = api.device_status(aws)
+    if st[0] != 0:
+        raise RuntimeError(f"device status after the end-to-end appends: {st}")
+    d2h = out.numel() * out.element_size() + lse.numel() * lse.element_size()
+    return {"ms_per_step": total / args.steps, "h2d": serving_bytes(host), "d2h": d2h,
+            "appends_keys": host["k_new"] is not None,
+            "appends_latent": host["kv_new"] is not None}
 
-    prep = time_input_prep(args, wl, cache, dev, flush)
 
+def other_workloads(args, dev) -> dict:
+    """The other configurations, each timed like the headline in the same run
+    (device time, L2 flushed before every step; no end-to-end or CPU leg)."""
+    import torch
+    from indexed_sparse_attention_lightning_b200 import workloads as W
+    res = {}
+    for sp in W.CONFIGS:
+        if sp.name == args.workload:
+            continue
+        wl = W.make_workload(sp)
+        m = measure_decode(args, wl, dev)
+        r = summarise(wl, m, wl.n_q, m["total_ms"], args.steps)
+        r["config"] = workload_config(sp, wl, 1)
+        res[sp.name] = r
+        del m, wl
+        torch.cuda.empty_cache()
+    return res
+
+
+def run_ours(args, rank: int, world: int, dist):
+    import torch
+    from indexed_sparse_attention_lightning_b200 import workloads as W
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    sp = rank_spec(W.spec(args.workload), rank)
+    wl = W.make_workload(sp)
+    m = measure_decode(args, wl, dev, dist)
+    e2e = None if args.no_e2e else time_e2e(args, wl, m, dev)
+    prep = time_input_prep(args, wl, m["cache"], dev, m["flush"])
     total_ms, e2e_step_ms, n_q_all = reduce_over_ranks(
-        dist, dev, total_ms, e2e["ms_per_step"] if e2e else 0.0, wl.n_q)
+        dist, dev, m["total_ms"], e2e["ms_per_step"] if e2e else 0.0, wl.n_q)
+    extra = None
+    if world == 1 and not args.no_extra:
+        del m["cache"], m["queries"], m["ws"], m["out"], m["lse"], m["idx"], m["flush"]
+        torch.cuda.empty_cache()
+        extra = other_workloads(args, dev)
     if rank != 0:
         return 0
 
-    ms_per_step = total_ms / args.steps
-    value = n_q_all * args.steps / (total_ms / 1e3)
-    peak, _, peak_kind = measured_peaks()
-    dom = int(np.argmax(phase_ms))
-    dom_name = _abi.DECODE_PHASES[dom]
-    roof = roofline(wl, dom_name, phase_ms[dom], nbytes, algorithmic_flops(wl, idx_host))
-    step_gbs = nbytes["total"] / (ms_per_step / 1e3) / 1e9
+    summ = summarise(wl, m, n_q_all, total_ms, args.steps)
+    roof = summ["roofline"]
+    dom_name = roof["kernel"]
     csrc = "indexed_sparse_attention_lightning_b200/csrc/"
     shared = [csrc + f for f in ("common.cuh", "sm100.cuh", "internal.h")]
     kernel_src = {"indexer": [csrc + "indexer_mma.cu", csrc + "plan.cu"] + shared,
@@ -547,22 +690,29 @@ def run_ours(args, rank: int, world: int, dist):
                          f"top-K, attention), {spent:.1f} s"}
 
     line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": f"{sp.index_dtype}+{sp.kv_dtype}", "data": "synthetic",
+        "metric": METRIC, "value": summ["value"], "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": summ["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": f"{sp.index_dtype}+{sp.kv_dtype}", "data": "synthetic",
         "config": workload_config(sp, wl, world),
         "roofline": dict(roof, traffic=traffic if roof["bound"] == "hbm" else None),
-        "path_hbm": {"bytes_per_step": nbytes["total"], "achieved_gbs": step_gbs,
-                     "frac_of_measured": step_gbs / peak, "frac_of_8tbs": step_gbs / SPEC_HBM_GBS},
-        "phases_ms": dict(zip(_abi.DECODE_PHASES, phase_ms)),
-        "gpu_launches": int(launches),
-        "clocks": clocks.summary(),
+        "path_hbm": summ["path_hbm"],
+        "phases_ms": summ["phases_ms"],
+        "gpu_launches": summ["gpu_launches"],
+        "clocks": summ["clocks"],
         "cpu_baseline": cpu,
         "input_prep": prep,
     }
     if e2e:
         line["e2e"] = {"value": n_q_all / (e2e_step_ms / 1e3), "unit": UNIT,
-                       "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]}
+                       "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
+                       "what": "pinned host inputs -> quantise the indexer query, append each "
+                               "query's new token (index key: %s, latent row: %s), decode -> "
+                               "output and lse to the host; pipelined over three streams"
+                               % ("yes" if e2e["appends_keys"] else "no",
+                                  "yes" if e2e["appends_latent"] else "no")}
+    if extra is not None:
+        line["other_configs"] = extra
     print(json.dumps(line), flush=True)
     return 0
 

@@ -224,14 +224,22 @@ SA_API sa_status sa_decode_traced(const sa_cache *cache, const sa_query *query, 
  *    SA_WS_DECODE) > SA_NOALLOC_SCRATCH_BYTES) return SA_ERR_WORKSPACE and
  *    launch nothing.
  *  - The first call on a device looks the array's address up with that
- *    device current; make it before any stream capture.
+ *    device current; make it before any stream capture.  The address is
+ *    kept per device and CUDA context, so a call after cudaDeviceReset looks
+ *    it up again (that call, too, belongs before any capture).
  *  - All calls on a device share the array: calls whose GPU work overlaps
  *    race and must not be issued.  The device status word of these calls
- *    lives in the array and is not readable through sa_device_status(). */
+ *    lives in the array: read it with sa_noalloc_status(). */
 #define SA_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
 SA_API sa_status sa_decode_noalloc(const sa_cache *cache, const sa_query *query, int32_t top_k,
                                    int32_t *idx_out, void *out, sa_dtype out_dtype, float *lse,
                                    void *stream);
+
+/* Device-side status of the most recent sa_decode_noalloc call on the current
+ * device: what sa_device_status reports for a workspace, read from the status
+ * word at the start of the static array.  Synchronises `stream`; allocates
+ * nothing.  *detail (may be NULL) receives an SA_DETAIL_* code. */
+SA_API sa_status sa_noalloc_status(void *stream, int32_t *detail);
 
 /* ---- Input preparation -------------------------------------------------
  * Before the indexer runs, the query is quantised and the step's new tokens
@@ -279,7 +287,12 @@ typedef struct sa_new_tokens {
  *    the others to be requantised, so other tiles return SA_ERR_UNSUPPORTED.
  * The pools named by `cache` (k_index, k_index_scale, kv, kv_rope, kv_scale)
  * are written in place and must be writable device memory; seq_len is neither
- * read nor changed (the caller advances it).  Tokens must not share a row.
+ * read nor changed (the caller advances it), so a position is not checked
+ * against it: appending at seq_len[seq] before advancing it is the normal use.
+ * Tokens must not share a row: two tokens with the same (seq, pos), or whose
+ * page-table entries point at the same page, are written by two CTAs at once,
+ * and the row may end up with codes of one token and the scale of the other.
+ * The call does not detect such a batch.
  * A token whose sequence is outside [0, batch), whose position is negative or
  * at or past max_pages * page_size, or whose page-table entry is outside
  * [0, num_pages) is skipped and recorded in the workspace status word

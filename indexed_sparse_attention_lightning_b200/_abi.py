@@ -22,7 +22,8 @@ DTYPES = {"f32": SA_F32, "bf16": SA_BF16, "e4m3": SA_E4M3}
 
 # every symbol include/sa.h declares
 EXPORTS = ("sa_workspace_size", "sa_indexer_score", "sa_topk", "sa_sparse_mla_attn",
-           "sa_decode", "sa_decode_traced", "sa_decode_noalloc", "sa_quantize_index_query",
+           "sa_decode", "sa_decode_traced", "sa_decode_noalloc", "sa_noalloc_status",
+           "sa_quantize_index_query",
            "sa_append_tokens", "sa_device_status",
            "sa_kernel_launches", "sa_status_string", "sa_version")
 NOALLOC_SCRATCH_BYTES = 32 << 20
@@ -88,6 +89,8 @@ def lib():
         L.sa_decode_traced.restype = ctypes.c_int
         L.sa_decode_noalloc.argtypes = [CP, QP, _I32, _P, _P, ctypes.c_int, _P, _P]
         L.sa_decode_noalloc.restype = ctypes.c_int
+        L.sa_noalloc_status.argtypes = [_P, ctypes.POINTER(_I32)]
+        L.sa_noalloc_status.restype = ctypes.c_int
         L.sa_quantize_index_query.argtypes = [_P, ctypes.c_int, _I32, _I32, _I32, _P, _P, _P]
         L.sa_quantize_index_query.restype = ctypes.c_int
         L.sa_append_tokens.argtypes = [CP, ctypes.POINTER(SaNewTokens), _P, _SZ, _P]

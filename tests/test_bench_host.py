@@ -124,3 +124,31 @@ def test_end_to_end_copy_accounting():
     for k, v in queries.tensors().items():
         if v is not None:
             assert torch.equal(getattr(dst, k), v), k
+
+
+def test_serving_inputs_are_the_cached_tokens_and_their_bytes_are_counted():
+    """The end-to-end leg's host inputs: each query's new token is the row
+    already cached at its position (so appending it keeps the cache), the
+    indexer query is handed over in bf16 for the e4m3 cache, and the bytes
+    copied per step are exactly those of the arrays."""
+    import dataclasses
+    import torch
+    wl = W.make_workload(dataclasses.replace(W.spec("decode_b8_8k"), batch=3,
+                                             seq_len=("list", (300, 77, 129))))
+    inp = bench.serving_inputs(wl)
+    sp = wl.spec
+    rows = wl.page_table[wl.q_seq, wl.q_pos // 64].astype(np.int64) * 64 + wl.q_pos % 64
+    kv = wl.kv.reshape(-1, sp.d_qk)[rows]
+    assert np.array_equal(inp["kv_new"].view(torch.int16).numpy().view(np.uint16), kv)
+    k = torch.from_numpy(wl.k_index.reshape(-1, sp.d_index)[rows]).view(torch.float8_e4m3fn)
+    want = (k.float() * torch.from_numpy(wl.k_index_scale.reshape(-1)[rows])[:, None]).bfloat16()
+    assert torch.equal(inp["k_new"], want)
+    assert inp["q_index_in"].dtype == torch.bfloat16
+    assert inp["q_index_in"].shape == (wl.n_q, sp.h_index, sp.d_index)
+    n = sum(a.nbytes for a in (wl.q_seq, wl.q_pos, wl.w, wl.q))
+    n += wl.n_q * (sp.h_index * sp.d_index + sp.d_index + sp.d_qk) * 2
+    assert bench.serving_bytes(inp) == n
+    # a latent cache with one scale per page takes no single tokens
+    wl8 = W.make_workload(dataclasses.replace(W.spec("decode_b2_1m_fp8kv_clustered"), batch=1,
+                                              seq_len=("fixed", 70000)))
+    assert bench.serving_inputs(wl8)["kv_new"] is None

@@ -51,6 +51,29 @@ def test_noalloc_matches_workspace_decode_on_consecutive_calls():
         parity.check_lse(lse.cpu().numpy(), ref_lse.cpu().numpy())
 
 
+def _noalloc_status():
+    detail = ctypes.c_int32(-1)
+    st = _abi.lib().sa_noalloc_status(torch.cuda.current_stream().cuda_stream,
+                                      ctypes.byref(detail))
+    return st, detail.value
+
+
+def test_noalloc_reports_bad_data_through_its_status_reader():
+    """A bad page id (host-side input, checked by the kernels) must show up in
+    the static array's status word, and a clean call must clear it again."""
+    wl = W.make_workload(W.DECODE_B8_8K)
+    K = wl.spec.top_k
+    cache, queries = api.upload(wl)
+    idx = torch.empty((wl.n_q, K), dtype=torch.int32, device="cuda")
+    out, lse = api._outputs(queries, wl.spec.d_latent, None, None, "bf16")
+    cache.page_table[3, 5] = wl.num_pages + 3
+    assert _noalloc(cache, queries, K, idx, out, lse) == _abi.SA_OK
+    assert _noalloc_status() == (_abi.SA_ERR_DEVICE_FAULT, _abi.SA_DETAIL_BAD_PAGE)
+    cache.page_table[3, 5] = int(wl.page_table[3, 5])
+    assert _noalloc(cache, queries, K, idx, out, lse) == _abi.SA_OK
+    assert _noalloc_status() == (_abi.SA_OK, 0)
+
+
 def test_noalloc_rejects_requests_beyond_its_scratch():
     wl = W.make_workload(W.DECODE_B8_8K)
     cache, queries = api.upload(wl)
