@@ -314,6 +314,64 @@ topk_collect_kernel(const float *__restrict__ scores, int64_t ld, const int32_t 
     }
 }
 
+// Marks in `bits` (by position) the `need` largest of the n_cand composite
+// candidate keys cs[] -- order-preserving score key in the high word, inverted
+// position in the low word, so all distinct and ties go to the lower position --
+// which all share their top kHistBits bits (the threshold bucket `bstar`).
+// Radix passes of 10-bit digits below the bucket bits find the need-th
+// largest key, stopping as soon as a whole digit bin is taken (normally after
+// two passes); the bucket bits themselves are never counted, so no pass piles
+// every candidate onto one histogram bin.  1 <= need <= n_cand.  All threads
+// of the block call it; dh holds 1024 counters.
+__device__ void mark_top_candidates(const uint64_t *cs, int n_cand, int need, int bstar,
+                                    uint32_t *bits, unsigned *dh, int *warp_sums) {
+    __shared__ int sel_digit_s, sel_above_s, sel_count_s;
+    const int tid = threadIdx.x;
+    uint64_t prefix = static_cast<uint64_t>(bstar) << (64 - kHistBits);
+    uint64_t mask = ~0ull << (64 - kHistBits);
+    int remaining = need, tot;
+    int shift = 64 - kHistBits - 10, width = 10;
+    for (;;) {
+        const uint64_t dmask = (1ull << width) - 1;
+        dh[tid] = 0;
+        __syncthreads();
+        for (int i = tid; i < n_cand; i += kThreads) {
+            const uint64_t k = cs[i];
+            if ((k & mask) == prefix) atomicAdd(&dh[(k >> shift) & dmask], 1u);
+        }
+        __syncthreads();
+        const int d = 1023 - tid;  // digits in descending order
+        const int cd = static_cast<int>(dh[d]);
+        const int ex = block_exclusive_prefix(cd, warp_sums, &tot);
+        if (ex < remaining && ex + cd >= remaining) {
+            sel_digit_s = d;
+            sel_above_s = ex;
+            sel_count_s = cd;
+        }
+        __syncthreads();
+        prefix |= static_cast<uint64_t>(sel_digit_s) << shift;
+        mask |= dmask << shift;
+        remaining -= sel_above_s;
+        const bool whole = remaining == sel_count_s;
+        __syncthreads();
+        if (whole || shift == 0) break;
+        if (shift >= 10) {
+            shift -= 10;
+        } else {
+            width = shift;
+            shift = 0;
+        }
+    }
+    // exactly `need` candidates satisfy (k & mask) >= prefix
+    for (int i = tid; i < n_cand; i += kThreads) {
+        const uint64_t k = cs[i];
+        if ((k & mask) >= prefix) {
+            const uint32_t pos = 0xFFFFFFFFu - static_cast<uint32_t>(k);
+            atomicOr(&bits[pos >> 5], 1u << (pos & 31));
+        }
+    }
+}
+
 // Writes the selected positions (bits set in `bits`, `words` words) to out in
 // ascending order, -1 after them, and -- when rows != null -- their physical
 // cache rows (compact_rows layout, tile 64) and count.  Positions first (each
@@ -390,9 +448,8 @@ topk_finalize_kernel(const float *__restrict__ scores, int64_t ld, const int32_t
     pdl_wait();
     pdl_trigger();
     extern __shared__ uint64_t fin_smem[];
-    __shared__ unsigned hist[256];
+    __shared__ unsigned dh[1024];
     __shared__ int warp_sums[33];
-    __shared__ unsigned sel_digit, sel_above;
     const int t = blockIdx.x;
     const int32_t V = vis[t];
     int32_t *out = idx + (int64_t)t * top_k;
@@ -417,58 +474,10 @@ topk_finalize_kernel(const float *__restrict__ scores, int64_t ld, const int32_t
     const int words = (V + 31) / 32;
     for (int w = threadIdx.x; w < words; w += kThreads) bits[w] = 0;
     __syncthreads();
-    // the need-th largest 64-bit candidate key (all distinct: the low word
-    // holds the inverted position), by 8-bit radix passes from the top
-    uint64_t prefix = 0, mask = 0;
-    unsigned remaining = need;
-    const int lane = threadIdx.x & 31;
-    for (int pass = 0; pass < 8; ++pass) {
-        const int shift = 56 - 8 * pass;
-        for (int i = threadIdx.x; i < 256; i += kThreads) hist[i] = 0;
-        __syncthreads();
-        for (int i = threadIdx.x; i < n_cand; i += kThreads) {
-            const uint64_t k = cs[i];
-            if ((k & mask) == prefix) atomicAdd(&hist[(k >> shift) & 255u], 1u);
-        }
-        __syncthreads();
-        if (threadIdx.x < 32) {
-            unsigned c[8], lane_sum = 0;
-#pragma unroll
-            for (int b = 0; b < 8; ++b) {
-                c[b] = hist[8 * lane + b];
-                lane_sum += c[b];
-            }
-            unsigned suffix = lane_sum;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                unsigned n = __shfl_down_sync(0xffffffffu, suffix, o);
-                if (lane + o < 32) suffix += n;
-            }
-            const unsigned above_lane = suffix - lane_sum;
-            if (above_lane < remaining && remaining <= suffix) {
-                unsigned acc = above_lane;
-                for (int b = 7; b >= 0; --b) {
-                    if (acc + c[b] >= remaining) {
-                        sel_digit = 8 * lane + b;
-                        sel_above = acc;
-                        break;
-                    }
-                    acc += c[b];
-                }
-            }
-        }
-        __syncthreads();
-        prefix |= static_cast<uint64_t>(sel_digit) << shift;
-        mask |= static_cast<uint64_t>(255u) << shift;
-        remaining -= sel_above;
-        __syncthreads();
-    }
-    // keys are distinct, so exactly `need` candidates are >= prefix
-    for (int i = threadIdx.x; i < n_cand; i += kThreads)
-        if (cs[i] >= prefix) {
-            const uint32_t pos = 0xFFFFFFFFu - static_cast<uint32_t>(cs[i]);
-            atomicOr(&bits[pos >> 5], 1u << (pos & 31));
-        }
+    // the need largest candidates (all in the threshold bucket, whose bits
+    // every candidate key carries on top)
+    mark_top_candidates(cs, n_cand, need, static_cast<int>(cs[0] >> (64 - kHistBits)), bits,
+                        dh, warp_sums);
     const int32_t *st = sel + (int64_t)t * top_k;
     for (int i = threadIdx.x; i < n_sel; i += kThreads) {
         const uint32_t pos = static_cast<uint32_t>(st[i]);
@@ -504,7 +513,7 @@ topk_single_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *
     uint32_t *bits = reinterpret_cast<uint32_t *>(single_smem + kSingleCap);  // [V / 32]
     __shared__ unsigned dh[1024];
     __shared__ int warp_sums[33];
-    __shared__ int n_cand_s, bstar_s, above_s, sel_digit_s, sel_above_s, sel_count_s;
+    __shared__ int n_cand_s, bstar_s, above_s;
     const int t = blockIdx.x, tid = threadIdx.x, lane = tid & 31;
     const int32_t V = vis[t];
     int32_t *out = idx + (int64_t)t * top_k;
@@ -619,52 +628,7 @@ topk_single_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *
         }
         return;
     }
-    // the need-th largest composite key among the candidates: digits of 10
-    // bits below the fixed bucket bits, stopping once a whole digit bin is taken
-    const int n_cand = n_cand_s;
-    uint64_t prefix = static_cast<uint64_t>(bstar) << (64 - kHistBits);
-    uint64_t mask = ~0ull << (64 - kHistBits);
-    int remaining = need;
-    int shift = 64 - kHistBits - 10, width = 10;
-    for (;;) {
-        const uint64_t dmask = (1ull << width) - 1;
-        dh[tid] = 0;
-        __syncthreads();
-        for (int i = tid; i < n_cand; i += kThreads) {
-            const uint64_t k = cs[i];
-            if ((k & mask) == prefix) atomicAdd(&dh[(k >> shift) & dmask], 1u);
-        }
-        __syncthreads();
-        const int d = 1023 - tid;  // digits in descending order
-        const int cd = static_cast<int>(dh[d]);
-        const int ex = block_exclusive_prefix(cd, warp_sums, &tot);
-        if (ex < remaining && ex + cd >= remaining) {
-            sel_digit_s = d;
-            sel_above_s = ex;
-            sel_count_s = cd;
-        }
-        __syncthreads();
-        prefix |= static_cast<uint64_t>(sel_digit_s) << shift;
-        mask |= dmask << shift;
-        remaining -= sel_above_s;
-        const bool whole = remaining == sel_count_s;
-        __syncthreads();
-        if (whole || shift == 0) break;
-        if (shift >= 10) {
-            shift -= 10;
-        } else {
-            width = shift;
-            shift = 0;
-        }
-    }
-    // exactly `need` candidates satisfy (k & mask) >= prefix
-    for (int i = tid; i < n_cand; i += kThreads) {
-        const uint64_t k = cs[i];
-        if ((k & mask) >= prefix) {
-            const uint32_t pos = 0xFFFFFFFFu - static_cast<uint32_t>(k);
-            atomicOr(&bits[pos >> 5], 1u << (pos & 31));
-        }
-    }
+    mark_top_candidates(cs, n_cand_s, need, bstar, bits, dh, warp_sums);
     __syncthreads();
     emit_selection(bits, words, top_k, out, p, t, rows, nv_out, warp_sums);
 }
