@@ -14,7 +14,9 @@ indexer and the sparse attention kernel -- "Optimizing Next-Gen LLM Inference"
   of sequence ``b``; entries past the sequence end are -1.
 * index keys ``k_index[P, 64, d_index]`` (fp32, bf16, or e4m3 codes with one
   fp32 scale per token in ``k_index_scale[P, 64]``, or one per group of values
-  in ``k_index_scale[P, 64, d_index / group]``);
+  in ``k_index_scale[P, 64, d_index / group]``; or MXFP8: e4m3 codes with one
+  E8M0 scale byte per 32 values in ``k_index_scale[P, 64, d_index / 32]``,
+  uint8);
 * MLA latent rows ``kv[P, 64, d_latent + d_rope]`` (fp32 or bf16), or for the
   FP8 cache ``kv[P, 64, d_latent]`` e4m3 codes, ``kv_scale[P, 64 / ts, d_latent / td]``
   (one fp32 scale per tile of ts tokens x td latent dims of a page; the default
@@ -25,6 +27,11 @@ that any read outside the visible range shows up as NaN in a result.
 
 Quantisation rule (inputs arrive already quantised): ``scale = amax / 448``
 (1 when amax is 0), ``code = RNE(x / scale)`` saturated to +-448 in e4m3fn.
+MXFP8 (OCP MX rule, power-of-two scales): per group of 32 values
+``scale = 2^(floor(log2 amax) - 8)`` (8 = the exponent of e4m3's largest
+value), stored as the E8M0 byte ``127 + floor(log2 amax) - 8``; codes as above
+(values that land in [448, 512) of the scale saturate to 448); an all-zero
+group stores byte 127 (scale 1).
 """
 from __future__ import annotations
 
@@ -56,7 +63,7 @@ class WorkloadSpec:
     queries: tuple = ("decode",)   # ("decode",) or ("prefill", first_pos, count)
     h_index: int = 64
     d_index: int = 128
-    index_dtype: str = "e4m3"      # "e4m3", "bf16" or "f32"
+    index_dtype: str = "e4m3"      # "e4m3", "mxfp8", "bf16" or "f32"
     # e4m3 index scales: 0 = one per key row and one per (query, head) row; g = one
     # per g consecutive values of a row (the pages' group-32 quantisation)
     index_scale_group: int = 0
@@ -133,7 +140,14 @@ DECODE_B2_1M_FP8KV_TILE_1X128 = WorkloadSpec(
     name="decode_b2_1m_fp8kv_tile_1x128", seed=4, batch=2, seq_len=("fixed", 1048576),
     kv_dtype="e4m3", keys=("clusters", 16, 4096), kv_scale_tile=(1, 128))
 
-EXTRA = (PROFILE_B64_16K, DECODE_B64_BF16_INDEX, DECODE_B2_1M_FP8KV_TILE_1X128)
+# the headline decode with the pages' MXFP8 index path: e4m3 index query and
+# keys with one power-of-two (E8M0) scale per 32 values
+DECODE_B64_MXFP8_INDEX = WorkloadSpec(
+    name="decode_b64_16k_32k_mxfp8_index", seed=2, batch=64, seq_len=("uniform", 16384, 32768),
+    keys=("planted", 0.05, 3.0), index_dtype="mxfp8")
+
+EXTRA = (PROFILE_B64_16K, DECODE_B64_BF16_INDEX, DECODE_B2_1M_FP8KV_TILE_1X128,
+         DECODE_B64_MXFP8_INDEX)
 
 
 def spec(which) -> WorkloadSpec:
@@ -226,7 +240,32 @@ def quantize_groups_e4m3(x: np.ndarray, group: int):
     return codes.reshape(x.shape), scale
 
 
-def _quantize_index(x: np.ndarray, group: int):
+MX_GROUP = 32
+
+
+def quantize_mxfp8(x: np.ndarray):
+    """OCP MX quantisation of groups of 32 values of the last axis: returns
+    (e4m3 codes uint8 like x, E8M0 scale bytes uint8 [..., last / 32])."""
+    g = x.reshape(x.shape[:-1] + (x.shape[-1] // MX_GROUP, MX_GROUP)).astype(np.float32)
+    amax = np.abs(g).max(axis=-1)
+    _, ex = np.frexp(amax)                      # amax = m * 2^ex, m in [0.5, 1)
+    e = np.where(amax > 0, ex.astype(np.int64) - 1 - 8, 0)  # floor(log2 amax) - 8
+    byte = np.clip(e + 127, 0, 254).astype(np.uint8)
+    scale = np.ldexp(np.float32(1.0), byte.astype(np.int64) - 127).astype(np.float32)
+    codes = to_e4m3_codes(g / scale[..., None])
+    return codes.reshape(x.shape), byte
+
+
+def e8m0_value(byte: np.ndarray) -> np.ndarray:
+    """E8M0 bytes -> their fp32 values 2^(b - 127) (255 -> NaN); storage decode only."""
+    b = np.asarray(byte).astype(np.int64)
+    v = np.ldexp(np.float64(1.0), b - 127)
+    return np.where(b == 255, np.nan, v).astype(np.float32)
+
+
+def _quantize_index(x: np.ndarray, group: int, mx: bool = False):
+    if mx:
+        return quantize_mxfp8(x)
     return quantize_groups_e4m3(x, group) if group > 0 else quantize_rows_e4m3(x)
 
 
@@ -313,6 +352,10 @@ def make_workload(sp: WorkloadSpec) -> Workload:
         raise ValueError("group scales need e4m3 index data and a group dividing d_index")
     if sp.index_dtype == "e4m3":
         q_index, q_index_scale = _quantize_index(qi, sp.index_scale_group)
+    elif sp.index_dtype == "mxfp8":
+        if d_I % MX_GROUP or sp.index_scale_group:
+            raise ValueError("MXFP8 needs d_index a multiple of 32 and no other scale group")
+        q_index, q_index_scale = quantize_mxfp8(qi)
     elif sp.index_dtype == "bf16":
         q_index, q_index_scale = to_bf16_bits(qi), None
     elif sp.index_dtype == "f32":
@@ -327,6 +370,9 @@ def make_workload(sp: WorkloadSpec) -> Workload:
         k_index_scale = np.full((rows,) + ((d_I // sp.index_scale_group,)
                                            if sp.index_scale_group else ()),
                                 np.nan, dtype=np.float32)
+    elif sp.index_dtype == "mxfp8":
+        k_index = np.full((rows, d_I), E4M3_NAN, dtype=np.uint8)
+        k_index_scale = np.full((rows, d_I // MX_GROUP), 255, dtype=np.uint8)  # NaN scale
     elif sp.index_dtype == "bf16":
         k_index = np.full((rows, d_I), BF16_NAN, dtype=np.uint16)
         k_index_scale = None
@@ -349,11 +395,14 @@ def make_workload(sp: WorkloadSpec) -> Workload:
             if qb.size == 0:
                 raise ValueError("planted keys need a query on the sequence")
             t = int(qb[-1])
-            if sp.index_dtype == "e4m3":
+            if sp.index_dtype in ("e4m3", "mxfp8"):
                 qdeq = torch.from_numpy(q_index[t]).view(torch.float8_e4m3fn).float().numpy()
-                sc = q_index_scale[t]
-                qdeq = qdeq * (np.repeat(sc, sp.index_scale_group, axis=-1)
-                               if sp.index_scale_group else sc[:, None])
+                if sp.index_dtype == "mxfp8":
+                    qdeq = qdeq * np.repeat(e8m0_value(q_index_scale[t]), MX_GROUP, axis=-1)
+                else:
+                    sc = q_index_scale[t]
+                    qdeq = qdeq * (np.repeat(sc, sp.index_scale_group, axis=-1)
+                                   if sp.index_scale_group else sc[:, None])
             elif sp.index_dtype == "bf16":
                 qdeq = (q_index[t].astype(np.uint32) << 16).view(np.float32)
             else:
@@ -386,8 +435,8 @@ def make_workload(sp: WorkloadSpec) -> Workload:
                         k[a - c0:e - c0] = ((centers[ci][None, :] + k[a - c0:e - c0])
                                             / np.float32(math.sqrt(2.0)))
             dst = _phys_rows(pt, c0, c1, ps)
-            if sp.index_dtype == "e4m3":
-                codes, sc = _quantize_index(k, sp.index_scale_group)
+            if sp.index_dtype in ("e4m3", "mxfp8"):
+                codes, sc = _quantize_index(k, sp.index_scale_group, sp.index_dtype == "mxfp8")
                 k_index[dst] = codes
                 k_index_scale[dst] = sc
             elif sp.index_dtype == "bf16":
@@ -476,6 +525,41 @@ def permute_pages(wl: Workload, seed: int) -> Workload:
     return dataclasses.replace(
         wl, page_table=pt, k_index=move(wl.k_index), k_index_scale=move(wl.k_index_scale),
         kv=move(wl.kv), kv_rope=move(wl.kv_rope), kv_scale=move(wl.kv_scale))
+
+
+def shard_workload(wl: Workload, lo, hi) -> Workload:
+    """The cache one rank of a context-parallel group holds: positions
+    [lo[b], hi[b]) of every sequence (page-aligned lo), as local positions
+    0 .. hi - lo - 1, in pools of its own holding only those pages (renumbered
+    in the order of their logical positions) plus the unused poisoned pages;
+    each decode query sits at its shard's last local position."""
+    ps = wl.spec.page_size
+    lo, hi = np.asarray(lo, np.int64), np.asarray(hi, np.int64)
+    if np.any(lo % ps) or np.any(hi <= lo):
+        raise ValueError("shards start on a page and hold at least one position")
+    if wl.spec.queries[0] != "decode":
+        raise ValueError("context-parallel shards serve decode queries")
+    B = wl.seq_len.shape[0]
+    n_pg = (hi - lo + ps - 1) // ps
+    pages = [wl.page_table[b, lo[b] // ps: lo[b] // ps + n_pg[b]].astype(np.int64)
+             for b in range(B)]
+    keep = np.concatenate(pages + [np.setdiff1d(np.arange(wl.num_pages),
+                                                wl.page_table[wl.page_table >= 0])])
+    new_id = np.full(wl.num_pages, -1, np.int64)
+    new_id[keep] = np.arange(keep.size)
+    pt = np.full((B, int(n_pg.max())), -1, dtype=np.int32)
+    for b in range(B):
+        pt[b, :n_pg[b]] = new_id[pages[b]]
+
+    def take(a):
+        return None if a is None else np.ascontiguousarray(a[keep])
+
+    lens = (hi - lo).astype(np.int32)
+    return dataclasses.replace(
+        wl, seq_len=lens, page_table=pt, num_pages=int(keep.size),
+        q_pos=(lens[wl.q_seq] - 1).astype(np.int32),
+        k_index=take(wl.k_index), k_index_scale=take(wl.k_index_scale), kv=take(wl.kv),
+        kv_rope=take(wl.kv_rope), kv_scale=take(wl.kv_scale), planted={}, clusters={})
 
 
 def subset_queries(wl: Workload, rows) -> Workload:

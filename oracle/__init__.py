@@ -66,6 +66,8 @@ def _load():
         lib.oracle_e4m3_encode.restype = ctypes.c_int
         lib.oracle_to_bf16.argtypes = [I64, P, P]
         lib.oracle_to_bf16.restype = ctypes.c_int
+        lib.oracle_e8m0_decode.argtypes = [I64, P, P]
+        lib.oracle_e8m0_decode.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -98,25 +100,42 @@ def decode(dtype: str, codes: np.ndarray) -> np.ndarray:
     return out
 
 
+MX_GROUP = 32  # values per E8M0 scale in the MXFP8 format
+
+
+def e8m0_decode(b: np.ndarray) -> np.ndarray:
+    """E8M0 scale bytes -> fp32 values 2^(b - 127) (255 -> NaN), exactly."""
+    b = np.ascontiguousarray(b, dtype=np.uint8)
+    out = np.empty(b.shape, dtype=np.float32)
+    _check(_load().oracle_e8m0_decode(b.size, _ptr(b), _ptr(out)), "e8m0_decode")
+    return out
+
+
 def _index_dtype(wl):
     return wl.spec.index_dtype
 
 
 def index_scores(wl, nthreads: int | None = None) -> np.ndarray:
-    """I[t, s] for s < V_t (float64 [n_q, max V]; NaN past each V_t)."""
+    """I[t, s] for s < V_t (float64 [n_q, max V]; NaN past each V_t).  MXFP8
+    inputs (e4m3 codes, one E8M0 byte per 32 values) are scored as e4m3 codes
+    with those group scales decoded to fp32 (exact: powers of two)."""
     n_q = wl.n_q
     ld = max(1, wl.max_visible)
     scores = np.full((n_q, ld), np.nan, dtype=np.float64)
-    dt = _DT[_index_dtype(wl)]
+    mx = _index_dtype(wl) == "mxfp8"
+    dt = _DT["e4m3" if mx else _index_dtype(wl)]
+    group = MX_GROUP if mx else getattr(wl.spec, "index_scale_group", 0)
     qi = np.ascontiguousarray(wl.q_index)
     ki = np.ascontiguousarray(wl.k_index)
-    qs, ks = _c(wl.q_index_scale, np.float32), _c(wl.k_index_scale, np.float32)
+    if mx:
+        qs, ks = e8m0_decode(wl.q_index_scale), e8m0_decode(wl.k_index_scale)
+    else:
+        qs, ks = _c(wl.q_index_scale, np.float32), _c(wl.k_index_scale, np.float32)
     w = _c(wl.w, np.float32)
     q_seq, q_pos = _c(wl.q_seq, np.int32), _c(wl.q_pos, np.int32)
     pt = _c(wl.page_table, np.int32)
     rc = _load().oracle_index_scores(
-        n_q, _ptr(q_seq), _ptr(q_pos), wl.spec.h_index, wl.spec.d_index,
-        getattr(wl.spec, "index_scale_group", 0),
+        n_q, _ptr(q_seq), _ptr(q_pos), wl.spec.h_index, wl.spec.d_index, group,
         dt, _ptr(qi), _ptr(qs), _ptr(w), dt, _ptr(ki), _ptr(ks),
         _ptr(pt), pt.shape[1], wl.spec.page_size, wl.num_pages,
         _ptr(scores), ld, nthreads or threads())

@@ -602,3 +602,16 @@ int oracle_e4m3_encode(int64_t n, const float *x, uint8_t *codes)
     }
     return OR_OK;
 }
+
+/* E8M0 scale bytes (the shared scale of the OCP MX formats, which "Long-Context
+ * LLM Inference Optimization" names for the index query and keys: MXFP8, one
+ * scale per group of 32 values) -> their values as fp32: byte b stands for
+ * 2^(b - 127), exactly representable for every b in [0, 254]; 255 is NaN. */
+int oracle_e8m0_decode(int64_t n, const uint8_t *bytes, float *out)
+{
+    if (n < 0 || (n > 0 && (!bytes || !out)))
+        return OR_BAD_ARG;
+    for (int64_t i = 0; i < n; i++)
+        out[i] = bytes[i] == 255 ? (float)NAN : (float)ldexp(1.0, (int)bytes[i] - 127);
+    return OR_OK;
+}

@@ -31,9 +31,16 @@ def np_values(dtype, a):
         return a.astype(np.float64)
     if dtype == "bf16":
         return (a.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
-    if dtype == "e4m3":
+    if dtype in ("e4m3", "mxfp8"):
         return torch.from_numpy(np.ascontiguousarray(a)).view(torch.float8_e4m3fn).double().numpy()
     raise ValueError(dtype)
+
+
+def np_scales(dtype, a):
+    """Scale values: fp32 as stored, or E8M0 bytes (MXFP8) through torch's decoder."""
+    if dtype == "mxfp8":
+        return torch.from_numpy(np.ascontiguousarray(a)).view(torch.float8_e8m0fnu).double().numpy()
+    return np.asarray(a).astype(np.float64)
 
 
 def np_rows(wl, b, positions):
@@ -48,6 +55,7 @@ def np_index_keys(wl, b, V):
     k = np_values(wl.spec.index_dtype, wl.k_index.reshape(-1, d)[rows])
     if wl.k_index_scale is not None:
         per_row = wl.k_index_scale.reshape(wl.k_index.shape[0] * wl.k_index.shape[1], -1)[rows]
+        per_row = np_scales(wl.spec.index_dtype, per_row)
         k = k * (np.repeat(per_row, d // per_row.shape[1], axis=1))
     return k
 
@@ -59,7 +67,7 @@ def np_scores(wl):
         k = np_index_keys(wl, int(wl.q_seq[t]), V)
         q = np_values(wl.spec.index_dtype, wl.q_index[t])
         if wl.q_index_scale is not None:
-            qs = wl.q_index_scale[t].reshape(wl.spec.h_index, -1).astype(np.float64)
+            qs = np_scales(wl.spec.index_dtype, wl.q_index_scale[t].reshape(wl.spec.h_index, -1))
             q = q * np.repeat(qs, wl.spec.d_index // qs.shape[1], axis=1)
         dots = np.einsum("sd,jd->sj", k, q)
         out[t, :V] = np.maximum(dots, 0.0) @ wl.w[t].astype(np.float64)
@@ -119,6 +127,38 @@ def test_e4m3_decode_matches_torch_for_every_code():
     assert ours[0x7E] == 448.0 and ours[0x01] == 2.0 ** -9
 
 
+def test_e8m0_decode_matches_torch_for_every_byte():
+    """The MXFP8 scale bytes: b -> 2^(b - 127), 255 -> NaN (torch's float8_e8m0fnu)."""
+    b = np.arange(256, dtype=np.uint8)
+    ours = oracle.e8m0_decode(b).astype(np.float64)
+    ref = torch.from_numpy(b).view(torch.float8_e8m0fnu).double().numpy()
+    assert np.array_equal(np.isnan(ours), np.isnan(ref)) and np.isnan(ours[255])
+    assert np.array_equal(ours[:255], ref[:255])
+    assert ours[127] == 1.0 and ours[0] == 2.0 ** -127 and ours[254] == 2.0 ** 127
+
+
+def test_mxfp8_inputs_follow_the_mx_scale_rule():
+    """The input generator's MXFP8 groups: every scale is the power of two
+    2^(floor(log2 amax) - 8), so the group's largest value lands in [256, 512)
+    times the scale (saturated to 448), and every value is within half an e4m3
+    step (or the saturation) of its input."""
+    rng = np.random.default_rng(3)
+    x = (rng.standard_normal((40, 64)) * np.exp(rng.uniform(-20, 20, (40, 1)))).astype(np.float32)
+    x[5, :32] = 0.0
+    codes, b = W.quantize_mxfp8(x)
+    sc = np_scales("mxfp8", b)
+    g = x.reshape(40, 2, 32).astype(np.float64)
+    amax = np.abs(g).max(axis=2)
+    nz = amax > 0
+    assert np.all(np.floor(np.log2(amax[nz])) - 8 == np.log2(sc[nz]))
+    assert b[5, 0] == 127
+    deq = np_values("e4m3", codes).reshape(40, 2, 32) * sc[..., None]
+    top = np.abs(deq).max(axis=2)[nz] / sc[nz]
+    assert np.all((top >= 256) & (top <= 448))
+    err = np.abs(deq - g) / sc[..., None]
+    assert np.all((err <= 16) | (np.abs(g) / sc[..., None] >= 448))
+
+
 def test_bf16_decode_matches_torch():
     rng = np.random.default_rng(0)
     bits = rng.integers(0, 1 << 16, size=4096, dtype=np.uint16)
@@ -134,11 +174,14 @@ def test_bf16_decode_matches_torch():
 # --------------------------------------------------------- indexer score ---
 
 @pytest.mark.parametrize("index_dtype,group", [("f32", 0), ("bf16", 0), ("e4m3", 0),
-                                               ("e4m3", 8)])
+                                               ("e4m3", 8), ("mxfp8", 0)])
 def test_scores_match_brute_force(index_dtype, group):
     """group > 0: one e4m3 scale per `group` values of the query and key rows
-    (the pages' group-wise index quantisation, here 8 of 16 dims)."""
-    wl = W.make_workload(small_spec(index_dtype=index_dtype, index_scale_group=group))
+    (the pages' group-wise index quantisation, here 8 of 16 dims); mxfp8: one
+    E8M0 scale per 32 values (MXFP8, 64 dims)."""
+    d = 64 if index_dtype == "mxfp8" else 16
+    wl = W.make_workload(small_spec(index_dtype=index_dtype, index_scale_group=group,
+                                    d_index=d))
     got = oracle.index_scores(wl)
     ref = np_scores(wl)
     assert np.array_equal(np.isnan(got), np.isnan(ref))
