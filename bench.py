@@ -123,8 +123,9 @@ def algorithmic_bytes(wl, idx: np.ndarray) -> dict:
     indexer keys + key scales + selected KV rows + outputs)."""
     sp = wl.spec
     V = wl.visible.astype(np.int64)
-    key_b = sp.d_index * {"e4m3": 1, "bf16": 2, "f32": 4}[sp.index_dtype]
-    scale_b = 4 if sp.index_dtype == "e4m3" else 0
+    key_b = sp.d_index * {"e4m3": 1, "mxfp8": 1, "bf16": 2, "f32": 4}[sp.index_dtype]
+    # one fp32 scale per key, or one E8M0 byte per 32 values (MXFP8)
+    scale_b = {"e4m3": 4, "mxfp8": sp.d_index // 32}.get(sp.index_dtype, 0)
     indexer = int((V * (key_b + scale_b)).sum())
     n_sel = np.minimum(V, sp.top_k)
     if sp.kv_dtype == "e4m3":
@@ -426,6 +427,8 @@ def serving_inputs(wl) -> dict:
         out["k_new"] = k.bfloat16()
     else:
         out["q_index"] = torch.from_numpy(wl.q_index)
+        if wl.q_index_scale is not None:  # MXFP8: the quantised query and its scale bytes
+            out["q_index_scale"] = torch.from_numpy(wl.q_index_scale)
         if sp.index_dtype == "f32":
             out["k_new"] = torch.from_numpy(wl.k_index.reshape(-1, sp.d_index)[rows])
     if sp.kv_dtype == "f32":
@@ -569,8 +572,9 @@ def time_e2e(args, wl, m: dict, dev):
         q = dataclasses.replace(
             queries, q_seq=d["q_seq"], q_pos=d["q_pos"], w=d["w"], q=d["q"],
             q_index=d.get("q_index", torch.empty_like(queries.q_index)),
-            q_index_scale=(None if queries.q_index_scale is None
-                           else torch.empty_like(queries.q_index_scale)))
+            q_index_scale=d.get("q_index_scale",
+                                None if queries.q_index_scale is None
+                                else torch.empty_like(queries.q_index_scale)))
         return d, q
 
     bufs = [dev_set(), dev_set()]

@@ -68,7 +68,10 @@ typedef enum sa_status {
 typedef enum sa_dtype {
     SA_F32 = 0,
     SA_BF16 = 1,
-    SA_E4M3 = 2               /* OCP e4m3fn code bytes, always paired with fp32 scales */
+    SA_E4M3 = 2,              /* OCP e4m3fn code bytes, always paired with fp32 scales */
+    SA_MXFP8 = 3              /* index query and keys only: e4m3fn code bytes with one E8M0
+                               * scale byte per 32 consecutive values (the OCP MX format:
+                               * scale = 2^(byte - 127); byte 255 is NaN) */
 } sa_dtype;
 
 /* Paged caches of one attention layer.
@@ -89,10 +92,15 @@ typedef struct sa_cache {
     /* SA_E4M3 (the quantised path) or SA_BF16 (the BF16 path, unscaled): the
      * indexer's two numerical paths ("Optimizing Next-Gen LLM Inference" §3.1;
      * "Inference Acceleration for New Large Model Architectures" §3.1); or
+     * SA_MXFP8, the pages' group-wise quantisation with one scale per 32
+     * values ("Inference Acceleration for New Large Model Architectures" §4.1;
+     * "Long-Context LLM Inference Optimization", Layered Quantization); or
      * SA_F32 */
     sa_dtype index_dtype;
     const void *k_index;         /* device [num_pages, page_size, d_index] */
-    const float *k_index_scale;  /* device [num_pages, page_size] one per token (SA_E4M3 only) */
+    const float *k_index_scale;  /* device SA_E4M3: fp32 [num_pages, page_size], one per token;
+                                  * SA_MXFP8: E8M0 bytes [num_pages, page_size, d_index / 32]
+                                  * (pass the byte array's address); NULL otherwise */
     int32_t d_index;
 
     /* MLA latent KV rows */
@@ -128,7 +136,8 @@ typedef struct sa_query {
 
     /* indexer query, same dtype as the cache's index keys */
     const void *q_index;         /* device [n_q, h_index, d_index] */
-    const float *q_index_scale;  /* device [n_q, h_index] one per (token, head) (SA_E4M3 only) */
+    const float *q_index_scale;  /* device SA_E4M3: fp32 [n_q, h_index], one per (token, head);
+                                  * SA_MXFP8: E8M0 bytes [n_q, h_index, d_index / 32] */
     const float *w;              /* device [n_q, h_index] head weights */
     int32_t h_index;
 
@@ -240,6 +249,57 @@ SA_API sa_status sa_decode_noalloc(const sa_cache *cache, const sa_query *query,
  * word at the start of the static array.  Synchronises `stream`; allocates
  * nothing.  *detail (may be NULL) receives an SA_DETAIL_* code. */
 SA_API sa_status sa_noalloc_status(void *stream, int32_t *detail);
+
+/* ---- Context parallelism across GPUs -------------------------------------
+ * One long sequence split along its context over G GPUs ("Inference
+ * Acceleration for New Large Model Architectures" §5.1-5.2: each device
+ * handles a contiguous portion of the sequence; "Long-Context LLM Inference
+ * Optimization", Distributed Scaling).  Rank r holds positions
+ * [lo_r, hi_r) of each sequence in its own paged caches, as local positions
+ * 0 .. hi_r - lo_r - 1, with lo_0 = 0 and hi_r = lo_{r+1}.  A decode step:
+ *   1. sa_local_candidates on every rank (its shard, its query positions
+ *      clamped to the shard: the last local position for decode);
+ *   2. all-gather of the candidates (the caller's collective) into
+ *      [G, n_q, top_k], rank-major;
+ *   3. sa_merge_candidates on every rank: the same global top-K everywhere,
+ *      and the part this rank holds, as local positions;
+ *   4. sa_sparse_mla_attn on every rank over its local part, fp32 output;
+ *   5. all-gather of those outputs and lse into [G, n_q, heads, d] / [G, n_q,
+ *      heads]; 6. sa_combine_partials.
+ * Positions selected match the single-GPU sa_decode exactly (the scores of a
+ * position do not depend on the shard); the output differs by the rounding
+ * of the merge. */
+
+/* Step 1: this rank's top_k by the fused indexer + top-K, as
+ * cand_score (device fp32 [n_q, top_k]) and cand_pos (device int32 [n_q,
+ * top_k]) = local position + position_offset[t] (device int32 [n_q]: the
+ * shard's lo for query t's sequence), ascending, padded with (-inf, -1).
+ * Workspace as for sa_decode (SA_WS_DECODE). */
+SA_API sa_status sa_local_candidates(const sa_cache *cache, const sa_query *query, int32_t top_k,
+                                     const int32_t *position_offset, float *cand_score,
+                                     int32_t *cand_pos, void *workspace, size_t workspace_bytes,
+                                     void *stream);
+
+/* Step 3: cand_score / cand_pos are device [n_ranks, n_q, top_k] as step 1
+ * wrote them on each rank, rank r's block r-th.  Per query the top_k
+ * candidates by score (ties to the lower position; padding last) go to
+ * idx_global (device int32 [n_q, top_k], ascending, -1 padded); idx_local
+ * (same shape) holds position - pos_lo[t] where pos_lo[t] <= position <
+ * pos_hi[t] (device int32 [n_q]: this rank's shard of query t's sequence),
+ * else -1.  n_ranks * top_k <= 24576.  No workspace. */
+SA_API sa_status sa_merge_candidates(const float *cand_score, const int32_t *cand_pos,
+                                     int32_t n_ranks, int32_t n_q, int32_t top_k,
+                                     const int32_t *pos_lo, const int32_t *pos_hi,
+                                     int32_t *idx_global, int32_t *idx_local, void *stream);
+
+/* Step 6: o_part device fp32 [n_parts, n_q, heads, d], lse_part device fp32
+ * [n_parts, n_q, heads] (natural log; -inf for a part with no selected row)
+ * -> out [n_q, heads, d] in out_dtype (SA_BF16 or SA_F32) and lse [n_q,
+ * heads] (may be NULL): out = sum_r exp(lse_r - lse) o_r, lse = log sum_r
+ * exp(lse_r).  n_parts <= 256.  No workspace. */
+SA_API sa_status sa_combine_partials(const float *o_part, const float *lse_part, int32_t n_parts,
+                                     int32_t n_q, int32_t heads, int32_t d, void *out,
+                                     sa_dtype out_dtype, float *lse, void *stream);
 
 /* ---- Input preparation -------------------------------------------------
  * Before the indexer runs, the query is quantised and the step's new tokens

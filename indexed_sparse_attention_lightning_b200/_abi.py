@@ -13,16 +13,17 @@ LIB_PATH = os.path.join(_HERE, "libsa.so")
 
 SA_OK, SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED, SA_ERR_WORKSPACE, SA_ERR_CUDA, \
     SA_ERR_DEVICE_FAULT, SA_ERR_TIMEOUT = range(7)
-SA_F32, SA_BF16, SA_E4M3 = 0, 1, 2
+SA_F32, SA_BF16, SA_E4M3, SA_MXFP8 = 0, 1, 2, 3
 SA_WS_INDEXER, SA_WS_TOPK, SA_WS_ATTN, SA_WS_DECODE, SA_WS_APPEND = 1, 2, 4, 8, 16
 SA_DETAIL_NONE, SA_DETAIL_BAD_PAGE, SA_DETAIL_BAD_POSITION, SA_DETAIL_BAD_INDEX, \
     SA_DETAIL_WAIT_TIMEOUT = range(5)
 
-DTYPES = {"f32": SA_F32, "bf16": SA_BF16, "e4m3": SA_E4M3}
+DTYPES = {"f32": SA_F32, "bf16": SA_BF16, "e4m3": SA_E4M3, "mxfp8": SA_MXFP8}
 
 # every symbol include/sa.h declares
 EXPORTS = ("sa_workspace_size", "sa_indexer_score", "sa_topk", "sa_sparse_mla_attn",
            "sa_decode", "sa_decode_traced", "sa_decode_noalloc", "sa_noalloc_status",
+           "sa_local_candidates", "sa_merge_candidates", "sa_combine_partials",
            "sa_quantize_index_query",
            "sa_append_tokens", "sa_device_status",
            "sa_kernel_launches", "sa_status_string", "sa_version")
@@ -91,6 +92,13 @@ def lib():
         L.sa_decode_noalloc.restype = ctypes.c_int
         L.sa_noalloc_status.argtypes = [_P, ctypes.POINTER(_I32)]
         L.sa_noalloc_status.restype = ctypes.c_int
+        L.sa_local_candidates.argtypes = [CP, QP, _I32, _P, _P, _P, _P, _SZ, _P]
+        L.sa_local_candidates.restype = ctypes.c_int
+        L.sa_merge_candidates.argtypes = [_P, _P, _I32, _I32, _I32, _P, _P, _P, _P, _P]
+        L.sa_merge_candidates.restype = ctypes.c_int
+        L.sa_combine_partials.argtypes = [_P, _P, _I32, _I32, _I32, _I32, _P, ctypes.c_int, _P,
+                                          _P]
+        L.sa_combine_partials.restype = ctypes.c_int
         L.sa_quantize_index_query.argtypes = [_P, ctypes.c_int, _I32, _I32, _I32, _P, _P, _P]
         L.sa_quantize_index_query.restype = ctypes.c_int
         L.sa_append_tokens.argtypes = [CP, ctypes.POINTER(SaNewTokens), _P, _SZ, _P]

@@ -160,7 +160,8 @@ def upload(wl, device="cuda") -> tuple[DeviceCache, DeviceQueries]:
     sp = wl.spec
     if getattr(sp, "index_scale_group", 0):
         raise SaError(_abi.SA_ERR_UNSUPPORTED,
-                      "upload: index scales per group of values have no kernel in this library")
+                      "upload: fp32 index scales per group of values have no kernel in this "
+                      "library (its group-scaled index format is MXFP8: E8M0 scales per 32)")
     cache = DeviceCache(
         page_table=_t(wl.page_table, device), seq_len=_t(wl.seq_len, device),
         num_pages=int(wl.num_pages), index_dtype=sp.index_dtype,
@@ -299,6 +300,77 @@ def decode(cache: DeviceCache, queries: DeviceQueries, top_k: int, out=None, lse
         handles = (ctypes.c_void_p * len(phase_events))(*[e.cuda_event for e in phase_events])
         check(_abi.lib().sa_decode_traced(*args, handles), "sa_decode_traced")
     return out, lse, idx
+
+
+# -------------------------------------------- context-parallel decode steps ---
+
+def local_candidates(cache: DeviceCache, queries: DeviceQueries, top_k: int,
+                     offset: torch.Tensor, score=None, pos=None, ws=None, stream=None):
+    """This GPU's top_k of its context shard as (score fp32, position + offset
+    int32), both [n_q, top_k], ascending positions, (-inf, -1) padding."""
+    dev = queries.q_seq.device
+    n_q = queries.n_q
+    if score is None:
+        score = torch.empty((n_q, top_k), dtype=torch.float32, device=dev)
+    if pos is None:
+        pos = torch.empty((n_q, top_k), dtype=torch.int32, device=dev)
+    if ws is None:
+        ws = workspace(workspace_size(cache, queries, top_k, _abi.SA_WS_DECODE), dev)
+    _need(offset, "offset", torch.int32, (n_q,))
+    _need(score, "score", torch.float32, (n_q, top_k))
+    _need(pos, "pos", torch.int32, (n_q, top_k))
+    _need(ws, "ws")
+    c, q = cache.struct(), queries.struct()
+    check(_abi.lib().sa_local_candidates(ctypes.byref(c), ctypes.byref(q), top_k, _ptr(offset),
+                                         _ptr(score), _ptr(pos), _ptr(ws), ws.numel(),
+                                         _stream(stream)),
+          "sa_local_candidates")
+    return score, pos, ws
+
+
+def merge_candidates(score: torch.Tensor, pos: torch.Tensor, top_k: int, lo: torch.Tensor,
+                     hi: torch.Tensor, idx_global=None, idx_local=None, stream=None):
+    """All ranks' candidates [n_ranks, n_q, top_k] -> (global top-K positions,
+    the ones in [lo, hi) as local positions), both int32 [n_q, top_k]."""
+    n_ranks, n_q, k = score.shape
+    if k != top_k:
+        raise SaError(_abi.SA_ERR_INVALID_ARG, "merge_candidates: candidate rows of top_k")
+    _need(score, "score", torch.float32, (n_ranks, n_q, top_k))
+    _need(pos, "pos", torch.int32, (n_ranks, n_q, top_k))
+    _need(lo, "lo", torch.int32, (n_q,))
+    _need(hi, "hi", torch.int32, (n_q,))
+    if idx_global is None:
+        idx_global = torch.empty((n_q, top_k), dtype=torch.int32, device=score.device)
+    if idx_local is None:
+        idx_local = torch.empty((n_q, top_k), dtype=torch.int32, device=score.device)
+    _need(idx_global, "idx_global", torch.int32, (n_q, top_k))
+    _need(idx_local, "idx_local", torch.int32, (n_q, top_k))
+    check(_abi.lib().sa_merge_candidates(_ptr(score), _ptr(pos), n_ranks, n_q, top_k, _ptr(lo),
+                                         _ptr(hi), _ptr(idx_global), _ptr(idx_local),
+                                         _stream(stream)),
+          "sa_merge_candidates")
+    return idx_global, idx_local
+
+
+def combine_partials(o_part: torch.Tensor, lse_part: torch.Tensor, out=None, lse=None,
+                     out_dtype: str = "bf16", stream=None):
+    """Partial outputs [n_parts, n_q, heads, d] (fp32) with their lse [n_parts,
+    n_q, heads] -> (out [n_q, heads, d], lse [n_q, heads])."""
+    n_parts, n_q, heads, d = o_part.shape
+    _need(o_part, "o_part", torch.float32, (n_parts, n_q, heads, d))
+    _need(lse_part, "lse_part", torch.float32, (n_parts, n_q, heads))
+    dt = torch.bfloat16 if out_dtype == "bf16" else torch.float32
+    if out is None:
+        out = torch.empty((n_q, heads, d), dtype=dt, device=o_part.device)
+    if lse is None:
+        lse = torch.empty((n_q, heads), dtype=torch.float32, device=o_part.device)
+    _need(out, "out", dt, (n_q, heads, d))
+    _need(lse, "lse", torch.float32, (n_q, heads))
+    check(_abi.lib().sa_combine_partials(_ptr(o_part), _ptr(lse_part), n_parts, n_q, heads, d,
+                                         _ptr(out), _abi.DTYPES[out_dtype], _ptr(lse),
+                                         _stream(stream)),
+          "sa_combine_partials")
+    return out, lse
 
 
 # ------------------------------------------------------- input preparation ---

@@ -39,6 +39,12 @@ __device__ __forceinline__ float2 e4m3x2_to_float2(uint16_t two) {
     return __half22float2(hh);
 }
 
+// E8M0 scale byte (OCP MX) -> its value 2^(b - 127), exactly; 255 is NaN.
+__device__ __forceinline__ float e8m0_to_float(uint32_t b) {
+    if (b == 255u) return __int_as_float(0x7FC00000);
+    return b == 0u ? __int_as_float(0x00400000) : __int_as_float(static_cast<int>(b << 23));
+}
+
 // ---------------------------------------------------------------------------
 // Order-preserving map float -> uint32: a > b as floats (no NaN) iff
 // key(a) > key(b) as unsigned integers, and a == b iff the keys are equal.

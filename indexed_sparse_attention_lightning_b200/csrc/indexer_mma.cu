@@ -6,7 +6,14 @@
 //     I[t,s] = ks[s] * sum_j (w[t,j] * qs[t,j]) * max(0, q8[t,j,:] . k8[s,:])
 // which equals sum_j w * max(0, q_I . k_I) because the scales are positive;
 // on the BF16 path ("Inference Acceleration for New Large Model Architectures"
-// §3.1) the query and keys are unscaled bf16 and ks = qs = 1.
+// §3.1) the query and keys are unscaled bf16 and ks = qs = 1.  On the MXFP8
+// path (the index query and keys with one power-of-two scale per group of 32
+// values: "Long-Context LLM Inference Optimization", Layered Quantization;
+// "Inference Acceleration for New Large Model Architectures" §4.1) the group
+// scales cannot leave the ReLU -- they differ inside one dot product -- so the
+// tensor cores apply them: tcgen05.mma kind::mxf8f6f4.block_scale multiplies
+// each 32-wide slice of a key row and of a query row by its E8M0 scale inside
+// the MMA, and the epilogue sees q_I . k_I directly.
 //
 // The contraction of 64 heads x 128 dims against every key is a dense GEMM
 // (M = 128 keys of a two-page tile, N = 64 heads, K = 128), so it runs as
@@ -44,18 +51,31 @@ using namespace sm100;
 constexpr int kKeys = 128;    // MMA M: keys per tile (two pages)
 constexpr int kHeads = 64;    // MMA N: indexer heads
 constexpr int kDim = 128;     // MMA K: index dimension
-constexpr int kAcc = 4;       // TMEM accumulators (64 columns each)
 constexpr int kScaleSlots = 8;  // key-scale ring: the epilogue frees these, not the key stages
 constexpr int kEpiGroups = 2;  // epilogue warp groups, alternating tiles
 constexpr int kThreads = 64 + kEpiGroups * 128;
-constexpr uint32_t kTmemCols = kAcc * kHeads;
+constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kAtom = 128;  // bytes of a row in one 128-byte swizzle atom
+
+// Numerical paths: e4m3 codes with one fp32 scale per key and per (query,
+// head); unscaled bf16; e4m3 codes with one E8M0 scale byte per 32 values.
+enum IxMode : int { kModeE4m3 = 0, kModeBf16 = 1, kModeMx = 2 };
+
+// MXFP8 scale factors in tensor memory (columns past the accumulators): the
+// block-scaled MMA reads the scale of row r of a 128-row operand for K-block
+// kb from lane r % 32 (of every 32-lane subpartition), column r / 32, byte kb
+// -- the layout tcgen05.cp 32x128b.warpx4 produces from 32 rows of 16 bytes.
+constexpr uint32_t kMxGroup = 32;
+constexpr uint32_t kColSfa = 192;  // key scales: 4 columns per accumulator in flight
+constexpr uint32_t kColSfb = 208;  // query scales: 4 columns per query buffer
 
 // Storage of one index element type.  A row of kDim elements is kChunks
 // 128-byte column chunks; a tile stores chunk c of all 128 keys contiguously
 // (16 KB, page h at + 8 KB * h), the query chunk c of its 64 heads likewise.
-template <bool kBf16>
+template <int kMode>
 struct IxCfg {
+    static constexpr bool kBf16 = kMode == kModeBf16;
+    static constexpr bool kMx = kMode == kModeMx;
     static constexpr int kElem = kBf16 ? 2 : 1;
     static constexpr int kChunks = kDim * kElem / kAtom;
     static constexpr int kChunkElems = kAtom / kElem;              // TMA box width
@@ -68,19 +88,29 @@ struct IxCfg {
     // key stages in flight per CTA: 2 x 4 x 16 KB (e4m3) or 4 x 32 KB (bf16) per SM
     // (a fifth bf16 stage measured no faster)
     static constexpr int kStages = 4;
+    // TMEM accumulators (64 columns each); MXFP8 keeps three, leaving room
+    // for the scale factors
+    static constexpr int kAcc = kMx ? 3 : 4;
 };
 
-template <bool kBf16>
+template <int kMode>
 struct IndexerSmem {
-    uint8_t keys[IxCfg<kBf16>::kStages][IxCfg<kBf16>::kTileBytes];  // 1024-byte aligned (swizzle atoms)
+    uint8_t keys[IxCfg<kMode>::kStages][IxCfg<kMode>::kTileBytes];  // 1024-byte aligned (swizzle atoms)
     uint32_t hist[kHistBins];              // score-key histogram of the current query
-    uint8_t q[2][IxCfg<kBf16>::kQBytes];   // 1024-byte aligned like the key stages
+    uint8_t q[2][IxCfg<kMode>::kQBytes];   // 1024-byte aligned like the key stages
     float wq[kEpiGroups][kHeads];          // head weights x query scales of that query
-    float kscale[kScaleSlots][kKeys];   // per-token key scales of the staged pages
+    // key scales of the staged pages: one fp32 per key (e4m3), or four E8M0
+    // bytes per key (MXFP8), 512 bytes a slot either way
+    alignas(16) float kscale[kScaleSlots][kKeys];
     int32_t page_ok[kScaleSlots][2];    // 1 when the staged page id was valid
-    uint64_t full[IxCfg<kBf16>::kStages], empty[IxCfg<kBf16>::kStages];
+    // MXFP8: query scale bytes as loaded, and both operands' scales in the
+    // 32 x 16-byte row order the copy into tensor memory takes
+    alignas(16) uint8_t q_sf[2][kHeads * (kDim / kMxGroup)];
+    alignas(128) uint8_t sfa[4][512];
+    alignas(128) uint8_t sfb[2][512];
+    uint64_t full[IxCfg<kMode>::kStages], empty[IxCfg<kMode>::kStages];
     uint64_t sc_full[kScaleSlots], sc_empty[kScaleSlots];
-    uint64_t acc_full[kAcc], acc_empty[kAcc];
+    uint64_t acc_full[IxCfg<kMode>::kAcc], acc_empty[IxCfg<kMode>::kAcc];
     uint64_t q_full[2], q_empty[2];
     uint64_t done;
     uint32_t tmem_base;
@@ -88,14 +118,19 @@ struct IndexerSmem {
     int abort;
 };
 
-static_assert(offsetof(IndexerSmem<false>, q) % 1024 == 0 &&
-                  offsetof(IndexerSmem<true>, q) % 1024 == 0,
+static_assert(offsetof(IndexerSmem<kModeE4m3>, q) % 1024 == 0 &&
+                  offsetof(IndexerSmem<kModeBf16>, q) % 1024 == 0 &&
+                  offsetof(IndexerSmem<kModeMx>, q) % 1024 == 0,
               "128-byte-swizzled Q tiles need 1024-byte alignment");
-static_assert(offsetof(IndexerSmem<false>, wq) % 16 == 0 &&
-                  offsetof(IndexerSmem<true>, wq) % 16 == 0,
+static_assert(offsetof(IndexerSmem<kModeE4m3>, wq) % 16 == 0 &&
+                  offsetof(IndexerSmem<kModeBf16>, wq) % 16 == 0,
               "head weights are read as float4");
-static_assert(2 * (sizeof(IndexerSmem<false>) + 2048) <= 233472, "e4m3: two CTAs per SM");
-static_assert(sizeof(IndexerSmem<true>) + 1024 <= 232448, "bf16: one CTA per SM");
+static_assert(2 * (sizeof(IndexerSmem<kModeE4m3>) + 2048) <= 233472, "e4m3: two CTAs per SM");
+static_assert(2 * (sizeof(IndexerSmem<kModeMx>) + 2048) <= 233472, "mxfp8: two CTAs per SM");
+static_assert(sizeof(IndexerSmem<kModeBf16>) + 1024 <= 232448, "bf16: one CTA per SM");
+static_assert(IxCfg<kModeMx>::kAcc * kHeads <= kColSfa && kColSfa + 4 * 4 <= kColSfb &&
+                  kColSfb + 2 * 4 <= kTmemCols,
+              "MXFP8 scale columns sit past the accumulators");
 
 struct IndexerArgs {
     PathParams p;
@@ -152,14 +187,48 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volati
     return ok;
 }
 
-template <bool kBf16>
-__global__ void __launch_bounds__(kThreads, IxCfg<kBf16>::kCtasPerSm)
+// Copy a 32-row x 16-byte shared-memory matrix (rows 16 bytes apart) into
+// tensor memory lanes 0-31 of every subpartition, four 32-bit columns.
+__device__ __forceinline__ void tmem_cp_32x128b(uint32_t taddr, const void *smem) {
+    // no-swizzle K-major descriptor: 8-row core matrices of 16-byte rows, 128
+    // bytes apart (one core matrix wide in K)
+    const uint32_t a = smem_u32(smem);
+    const uint64_t desc = (uint64_t)((a >> 4) & 0x3FFFu) | ((uint64_t)(128 >> 4) << 16) |
+                          ((uint64_t)(128 >> 4) << 32) | ((uint64_t)1 << 46);
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(desc)
+                 : "memory");
+}
+
+// D (+)= (A x its block scales) (B x its block scales)^T, e4m3 operands with
+// one E8M0 scale per 32 K-values; sfa / sfb are tensor-memory addresses with
+// the scale byte (the K-block) in their top two bits.
+__device__ __forceinline__ void mma_mxf8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                         uint32_t idesc, uint32_t sfa, uint32_t sfb,
+                                         uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+        : "memory");
+}
+
+// Instruction descriptor of the block-scaled MMA: e4m3 x e4m3, fp32
+// accumulation, E8M0 scales; scale byte `kb` of both operands.
+__host__ __device__ constexpr uint32_t mx_instr_desc(uint32_t m, uint32_t n, uint32_t kb) {
+    return (kb << 4) | ((n >> 3) << 17) | (1u << 23) | ((m >> 4) << 24) | (kb << 29);
+}
+
+template <int kMode>
+__global__ void __launch_bounds__(kThreads, IxCfg<kMode>::kCtasPerSm)
 indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
                    const __grid_constant__ CUtensorMap tm_q, const IndexerArgs a) {
-    using C = IxCfg<kBf16>;
+    using C = IxCfg<kMode>;
+    constexpr bool kBf16 = C::kBf16, kMx = C::kMx;
+    constexpr int kAcc = C::kAcc;
     pdl_wait();
     extern __shared__ uint8_t smem_raw[];
-    IndexerSmem<kBf16> &sm = *reinterpret_cast<IndexerSmem<kBf16> *>(align1024(smem_raw));
+    IndexerSmem<kMode> &sm = *reinterpret_cast<IndexerSmem<kMode> *>(align1024(smem_raw));
     const PathParams &p = a.p;
     const int warp = warp_id(), lane = lane_id();
     const int64_t total = p.n_q > 0 ? a.tile_end[p.n_q - 1] : 0;
@@ -174,7 +243,9 @@ indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
         }
         for (int s = 0; s < kScaleSlots; ++s) {
             mbar_init(&sm.sc_full[s], 1);
-            mbar_init(&sm.sc_empty[s], 4);
+            // the epilogue group's four warps (and the MMA warp, which reads
+            // the MXFP8 scale bytes)
+            mbar_init(&sm.sc_empty[s], kMx ? 5 : 4);
         }
         for (int c = 0; c < kAcc; ++c) {
             mbar_init(&sm.acc_full[c], 1);
@@ -250,11 +321,17 @@ indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
                     const int b = c.seg & 1;
                     if (!mbar_wait(&sm.q_empty[b], ((c.seg >> 1) & 1) ^ 1, abort_flag, p.status))
                         break;
-                    mbar_arrive_expect_tx(&sm.q_full[b], C::kQBytes);
+                    constexpr uint32_t kQSfBytes = kHeads * (kDim / kMxGroup);
+                    mbar_arrive_expect_tx(&sm.q_full[b], C::kQBytes + (kMx ? kQSfBytes : 0u));
 #pragma unroll
                     for (int ch = 0; ch < C::kChunks; ++ch)
                         tma_load_2d(sm.q[b] + ch * (kHeads * kAtom), &tm_q, ch * C::kChunkElems,
                                     c.t * kHeads, &sm.q_full[b]);
+                    if (kMx)
+                        bulk_load(sm.q_sf[b],
+                                  reinterpret_cast<const uint8_t *>(p.q_index_scale) +
+                                      (int64_t)c.t * kQSfBytes,
+                                  kQSfBytes, &sm.q_full[b]);
                 }
                 const int stage = n % C::kStages;
                 // the stage is free once its MMAs and its epilogue are done
@@ -287,6 +364,8 @@ indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
                         for (int ch = 0; ch < C::kChunks; ++ch)
                             tma_load_2d(sm.keys[stage] + ch * (kKeys * kAtom) + h * (64 * kAtom),
                                         &tm_keys, ch * C::kChunkElems, rows[h], &sm.full[stage]);
+                        // 256 bytes a page either way: 64 fp32 scales, or 64 x 4
+                        // E8M0 bytes (MXFP8, [num_pages, 64, 4] in memory)
                         if (!kBf16)
                             bulk_load(&sm.kscale[slot][64 * h], p.k_index_scale + rows[h],
                                       64 * sizeof(float), &sm.sc_full[slot]);
@@ -301,7 +380,69 @@ indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
         }
     } else if (warp == 1) {
         // ------------------------------------------------- MMA issuer ---
-        if (lane == 0) {
+        if constexpr (kMx) {
+            // The whole warp: it reorders the scale bytes of each tile (and of
+            // each query) into the 32 x 16-byte rows that tcgen05.cp copies to
+            // tensor memory -- row r holds the four K-block scales of operand
+            // rows r, r + 32, r + 64, r + 96 -- then lane 0 copies them and
+            // issues the four block-scaled MMAs (one per 32-wide K-block).
+            TileCursor c;
+            c.init_at(a.tile_end, sm.start_t, sm.start_i, k0, k1);
+            bool seg_start = true;
+            for (int n = 0; c.valid(); ++n) {
+                const int b = c.seg & 1;
+                if (seg_start) {
+                    if (c.seg > 0 && lane == 0) mma_commit(&sm.q_empty[(c.seg - 1) & 1]);
+                    if (!warp_wait(&sm.q_full[b], (c.seg >> 1) & 1, abort_flag, p.status)) break;
+                    // heads 0-63: row r = heads r and r + 32 (4 bytes each), padded
+                    const uint32_t *qsf = reinterpret_cast<const uint32_t *>(sm.q_sf[b]);
+                    *reinterpret_cast<uint4 *>(sm.sfb[b] + 16 * lane) =
+                        make_uint4(qsf[lane], qsf[lane + 32], 0x7F7F7F7Fu, 0x7F7F7F7Fu);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tc_fence_after();
+                        tmem_cp_32x128b(tmem + kColSfb + 4 * b, sm.sfb[b]);
+                    }
+                }
+                const int stage = n % C::kStages, acc = n % kAcc, slot = n % kScaleSlots;
+                if (!warp_wait(&sm.acc_empty[acc], ((n / kAcc) & 1) ^ 1, abort_flag, p.status))
+                    break;
+                if (!warp_wait(&sm.sc_full[slot], (n / kScaleSlots) & 1, abort_flag, p.status))
+                    break;
+                // keys 0-127 of the tile: row r = keys r, r + 32, r + 64, r + 96
+                const uint32_t *ksf = reinterpret_cast<const uint32_t *>(sm.kscale[slot]);
+                *reinterpret_cast<uint4 *>(sm.sfa[acc] + 16 * lane) =
+                    make_uint4(ksf[lane], ksf[lane + 32], ksf[lane + 64], ksf[lane + 96]);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm.sc_empty[slot]);
+                if (!warp_wait(&sm.full[stage], (n / C::kStages) & 1, abort_flag, p.status)) break;
+                if (lane == 0) {
+                    tc_fence_after();
+                    tmem_cp_32x128b(tmem + kColSfa + 4 * acc, sm.sfa[acc]);
+                    const uint32_t keys = smem_u32(sm.keys[stage]);
+                    const uint32_t qs = smem_u32(sm.q[b]);
+                    const uint32_t d = tmem + acc * kHeads;
+#pragma unroll
+                    for (int kb = 0; kb < 4; ++kb)  // 32 bytes of K (one scale block) each
+                        mma_mxf8(d, desc_kmajor_sw128(keys) + 2 * kb, desc_kmajor_sw128(qs) + 2 * kb,
+                                 mx_instr_desc(kKeys, kHeads, kb),
+                                 (tmem + kColSfa + 4 * acc) | ((uint32_t)kb << 30),
+                                 (tmem + kColSfb + 4 * b) | ((uint32_t)kb << 30), kb > 0 ? 1u : 0u);
+                    mma_commit(&sm.empty[stage]);
+                    mma_commit(&sm.acc_full[acc]);
+                }
+                __syncwarp();
+                seg_start = c.next(a.tile_end);
+            }
+            // every issued MMA has landed before TMEM is released
+            if (lane == 0) {
+                mma_commit(&sm.done);
+                mbar_wait(&sm.done, 0, abort_flag, p.status);
+            }
+            __syncwarp();
+        } else if (lane == 0) {
             // kind::f8f6f4 format 0 = e4m3; kind::f16 format 1 = bf16
             constexpr uint32_t idesc = instr_desc(kKeys, kHeads, kBf16 ? 1 : 0, 0, 0);
             TileCursor c;
@@ -387,7 +528,8 @@ indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
                 V = a.vis[c.t];
                 if (et < kHeads)
                     wq[et] = __ldg(p.w + (int64_t)c.t * kHeads + et) *
-                             (kBf16 ? 1.f : __ldg(p.q_index_scale + (int64_t)c.t * kHeads + et));
+                             ((kBf16 || kMx) ? 1.f
+                                             : __ldg(p.q_index_scale + (int64_t)c.t * kHeads + et));
                 named_barrier(bar, 128);
             }
             if ((n & 1) != g) continue;  // the other group's tile
@@ -397,7 +539,7 @@ indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
             if (ok)
                 ok = warp_wait(&sm.sc_full[slot], (n / kScaleSlots) & 1, abort_flag, p.status);
             const bool page_ok = ok && sm.page_ok[slot][row >> 6] != 0;
-            const float kscale = ok ? (kBf16 ? 1.f : sm.kscale[slot][row]) : 0.f;
+            const float kscale = ok ? ((kBf16 || kMx) ? 1.f : sm.kscale[slot][row]) : 0.f;
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.sc_empty[slot]);
             if (ok && s < V && !page_ok) report(p.status, SA_ERR_DEVICE_FAULT, SA_DETAIL_BAD_PAGE);
@@ -451,16 +593,17 @@ indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
 }  // namespace
 
 bool indexer_mma_supported(const PathParams &p) {
-    return (p.index_dtype == SA_E4M3 || p.index_dtype == SA_BF16) && p.h_index == kHeads &&
-           p.d_index == kDim;
+    return (p.index_dtype == SA_E4M3 || p.index_dtype == SA_BF16 ||
+            p.index_dtype == SA_MXFP8) &&
+           p.h_index == kHeads && p.d_index == kDim;
 }
 
 namespace {
 
-template <bool kBf16>
+template <int kMode>
 cudaError_t launch_indexer_mma_t(const PathParams &p, const int32_t *vis, const int32_t *tile_end,
                                  float *scores, int64_t ld, uint32_t *hist, cudaStream_t s) {
-    using C = IxCfg<kBf16>;
+    using C = IxCfg<kMode>;
     CUtensorMap tk, tq;
     if (!encode_tmap_2d(&tk, C::kElem, p.k_index, kDim, (uint64_t)p.num_pages * 64,
                         kDim * C::kElem, C::kChunkElems, 64, true) ||
@@ -470,12 +613,12 @@ cudaError_t launch_indexer_mma_t(const PathParams &p, const int32_t *vis, const 
     IndexerArgs a{p, vis, tile_end, scores, ld, hist};
     const int64_t max_tiles = (int64_t)p.n_q * ceil_div(p.max_visible, kKeys);
     const int64_t grid = std::min<int64_t>((int64_t)C::kCtasPerSm * num_sms(), max_tiles);
-    const size_t smem = sizeof(IndexerSmem<kBf16>) + 1024;
-    cudaError_t e = cudaFuncSetAttribute(indexer_mma_kernel<kBf16>,
+    const size_t smem = sizeof(IndexerSmem<kMode>) + 1024;
+    cudaError_t e = cudaFuncSetAttribute(indexer_mma_kernel<kMode>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     count_launch();
-    return launch_pdl(indexer_mma_kernel<kBf16>, dim3(static_cast<unsigned>(grid)),
+    return launch_pdl(indexer_mma_kernel<kMode>, dim3(static_cast<unsigned>(grid)),
                       dim3(kThreads), smem, s, tk, tq, a);
 }
 
@@ -484,9 +627,11 @@ cudaError_t launch_indexer_mma_t(const PathParams &p, const int32_t *vis, const 
 cudaError_t launch_indexer_mma(const PathParams &p, const int32_t *vis, const int32_t *tile_end,
                                float *scores, int64_t ld, uint32_t *hist, cudaStream_t s) {
     if (p.n_q == 0) return cudaSuccess;
-    return p.index_dtype == SA_BF16
-               ? launch_indexer_mma_t<true>(p, vis, tile_end, scores, ld, hist, s)
-               : launch_indexer_mma_t<false>(p, vis, tile_end, scores, ld, hist, s);
+    if (p.index_dtype == SA_BF16)
+        return launch_indexer_mma_t<kModeBf16>(p, vis, tile_end, scores, ld, hist, s);
+    if (p.index_dtype == SA_MXFP8)
+        return launch_indexer_mma_t<kModeMx>(p, vis, tile_end, scores, ld, hist, s);
+    return launch_indexer_mma_t<kModeE4m3>(p, vis, tile_end, scores, ld, hist, s);
 }
 
 }  // namespace sa

@@ -6,8 +6,11 @@
 // inputs the positive per-(token, head)
 // query scale and per-token key scale factor out of the ReLU:
 //     I[t,s] = ks[s] * sum_j (w[t,j] * qs[t,j]) * max(0, q8[t,j,:] . k8[s,:]).
-// This kernel serves the small fp32 configuration and any shape the tensor-core
-// indexer does not take; one thread owns one position.
+// With MXFP8 inputs (one E8M0 scale per 32 values) the scales differ inside a
+// dot product, so both sides are dequantised first (exact in fp32: an e4m3
+// value times a power of two).  This kernel serves the small fp32
+// configuration and any shape the tensor-core indexer does not take; one
+// thread owns one position.
 #include "common.cuh"
 #include "internal.h"
 
@@ -20,7 +23,7 @@ constexpr int kHeadBlock = 16;  // head dot products kept in registers at once
 template <int kFmt>  // sa_dtype of the index query and keys
 __global__ void __launch_bounds__(kThreads)
 indexer_simt_kernel(const PathParams p, float *__restrict__ scores, int64_t ld) {
-    constexpr bool kE4M3 = kFmt == SA_E4M3, kBF16 = kFmt == SA_BF16;
+    constexpr bool kE4M3 = kFmt == SA_E4M3, kBF16 = kFmt == SA_BF16, kMX = kFmt == SA_MXFP8;
     pdl_wait();
     pdl_trigger();
     extern __shared__ float smem[];
@@ -30,9 +33,13 @@ indexer_simt_kernel(const PathParams p, float *__restrict__ scores, int64_t ld) 
     const int32_t t = blockIdx.y;
 
     for (int i = threadIdx.x; i < H * d; i += kThreads) {
-        if (kE4M3) {
+        if (kE4M3 || kMX) {
             const uint8_t *qb = static_cast<const uint8_t *>(p.q_index) + (int64_t)t * H * d;
             q_s[i] = e4m3x2_to_float2(qb[i]).x;
+            if (kMX) {  // [n_q, H, d / 32] scale bytes: element i of the row block
+                const uint8_t *qsf = reinterpret_cast<const uint8_t *>(p.q_index_scale);
+                q_s[i] *= e8m0_to_float(qsf[((int64_t)t * H * d + i) / 32]);
+            }
         } else if (kBF16) {
             q_s[i] = bf16_bits_to_float(
                 static_cast<const uint16_t *>(p.q_index)[(int64_t)t * H * d + i]);
@@ -63,7 +70,7 @@ indexer_simt_kernel(const PathParams p, float *__restrict__ scores, int64_t ld) 
         for (int jj = 0; jj < kHeadBlock; ++jj) acc[jj] = 0.f;
         for (int d0 = 0; d0 < d; d0 += 16) {
             float k[16];
-            if (kE4M3) {
+            if (kE4M3 || kMX) {
                 const uint4 raw = *reinterpret_cast<const uint4 *>(
                     static_cast<const uint8_t *>(p.k_index) + row * d + d0);
                 const uint32_t words[4] = {raw.x, raw.y, raw.z, raw.w};
@@ -75,6 +82,12 @@ indexer_simt_kernel(const PathParams p, float *__restrict__ scores, int64_t ld) 
                     k[4 * i + 1] = lo.y;
                     k[4 * i + 2] = hi.x;
                     k[4 * i + 3] = hi.y;
+                }
+                if (kMX) {  // the key's scale for these 16 values (one 32-value group)
+                    const float ks = e8m0_to_float(
+                        reinterpret_cast<const uint8_t *>(p.k_index_scale)[(row * d + d0) / 32]);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) k[i] *= ks;
                 }
             } else if (kBF16) {
                 const uint4 *src = reinterpret_cast<const uint4 *>(
@@ -132,6 +145,7 @@ cudaError_t launch_indexer_simt(const PathParams &p, float *scores, int64_t ld, 
         return launch_pdl(kernel, grid, dim3(kThreads), smem, s, p, scores, ld);
     };
     if (p.index_dtype == SA_E4M3) return go(indexer_simt_kernel<SA_E4M3>);
+    if (p.index_dtype == SA_MXFP8) return go(indexer_simt_kernel<SA_MXFP8>);
     if (p.index_dtype == SA_BF16) return go(indexer_simt_kernel<SA_BF16>);
     return go(indexer_simt_kernel<SA_F32>);
 }

@@ -134,6 +134,20 @@ cudaError_t launch_sfa_mma(const PathParams &p, const int32_t *idx, int32_t top_
                            int32_t out_dtype, float *lse, float *o_part, float *lse_part,
                            cudaStream_t s);
 
+// Context-parallel decode steps (cp.cu).
+int32_t cp_merge_max_candidates();
+int32_t cp_combine_max_parts();
+cudaError_t launch_cand_emit(const float *scores, int64_t ld, const int32_t *idx, int32_t n_q,
+                             int32_t top_k, const int32_t *offset, float *cand_score,
+                             int32_t *cand_pos, cudaStream_t s);
+cudaError_t launch_cp_merge(const float *cand_score, const int32_t *cand_pos, int32_t n_ranks,
+                            int32_t n_q, int32_t top_k, const int32_t *pos_lo,
+                            const int32_t *pos_hi, int32_t *idx_global, int32_t *idx_local,
+                            cudaStream_t s);
+cudaError_t launch_cp_combine(const float *o_part, const float *lse_part, int32_t n_parts,
+                              int64_t rows, int32_t d, void *out, int32_t out_dtype, float *lse,
+                              cudaStream_t s);
+
 }  // namespace sa
 
 // ---- inline device definitions -------------------------------------------

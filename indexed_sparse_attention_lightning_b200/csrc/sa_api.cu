@@ -37,14 +37,16 @@ sa_status check_cache(const sa_cache *c) {
     if (c->batch <= 0 || c->max_pages <= 0 || c->num_pages <= 0) return SA_ERR_INVALID_ARG;
     if (!c->page_table || !c->seq_len || !c->k_index || !c->kv) return SA_ERR_INVALID_ARG;
     if (!aligned16(c->k_index) || !aligned16(c->kv)) return SA_ERR_INVALID_ARG;
-    if (c->index_dtype != SA_F32 && c->index_dtype != SA_BF16 && c->index_dtype != SA_E4M3)
+    if (c->index_dtype != SA_F32 && c->index_dtype != SA_BF16 && c->index_dtype != SA_E4M3 &&
+        c->index_dtype != SA_MXFP8)
         return SA_ERR_UNSUPPORTED;
-    if (c->index_dtype == SA_E4M3 && (!c->k_index_scale || !aligned16(c->k_index_scale)))
-        return SA_ERR_INVALID_ARG;
+    const bool scaled = c->index_dtype == SA_E4M3 || c->index_dtype == SA_MXFP8;
+    if (scaled && (!c->k_index_scale || !aligned16(c->k_index_scale))) return SA_ERR_INVALID_ARG;
     if (c->d_index <= 0 || c->d_index % 16 != 0) return SA_ERR_INVALID_ARG;
+    if (c->index_dtype == SA_MXFP8 && c->d_index % 32 != 0) return SA_ERR_INVALID_ARG;
     if (c->d_index > 256) return SA_ERR_UNSUPPORTED;
     if (c->kv_dtype != SA_F32 && c->kv_dtype != SA_BF16 && c->kv_dtype != SA_E4M3)
-        return SA_ERR_UNSUPPORTED;
+        return SA_ERR_UNSUPPORTED;  // SA_MXFP8 names index data only
     if (c->d_latent <= 0 || c->d_rope < 0) return SA_ERR_INVALID_ARG;
     if (c->d_latent > 512 || c->d_latent + c->d_rope > 1024) return SA_ERR_UNSUPPORTED;
     if (c->kv_dtype == SA_E4M3) {
@@ -71,7 +73,9 @@ sa_status check_query(const sa_query *q, const sa_cache *c, bool need_index, boo
     if (need_index) {
         if (!q->q_index || !q->w || q->h_index <= 0) return SA_ERR_INVALID_ARG;
         if (q->h_index > 128) return SA_ERR_UNSUPPORTED;
-        if (c->index_dtype == SA_E4M3 && !q->q_index_scale) return SA_ERR_INVALID_ARG;
+        if ((c->index_dtype == SA_E4M3 || c->index_dtype == SA_MXFP8) && !q->q_index_scale)
+            return SA_ERR_INVALID_ARG;
+        if (c->index_dtype == SA_MXFP8 && !aligned16(q->q_index_scale)) return SA_ERR_INVALID_ARG;
     }
     if (need_attn) {
         if (!q->q || q->heads <= 0) return SA_ERR_INVALID_ARG;
@@ -295,16 +299,23 @@ sa_status sa_sparse_mla_attn(const sa_cache *cache, const sa_query *query, const
     return run_attention(p, l, false, false, workspace, idx, top_k, out, out_dtype, lse, s);
 }
 
+// Where sa_local_candidates wants the selection: (score, position + offset).
+struct CandOut {
+    const int32_t *offset;  // device [n_q]
+    float *score;
+    int32_t *pos;
+};
+
 static sa_status decode_impl(const sa_cache *cache, const sa_query *query, int32_t top_k,
                              int32_t *idx_out, void *out, sa_dtype out_dtype, float *lse,
                              void *workspace, size_t workspace_bytes, void *stream,
-                             void *const *events) {
+                             void *const *events, const CandOut *cand = nullptr) {
     sa_status st = check_cache(cache);
     if (st != SA_OK) return st;
     if ((st = check_query(query, cache, true, true)) != SA_OK) return st;
     if (top_k <= 0 || top_k > kMaxTopK) return SA_ERR_INVALID_ARG;
     if (out_dtype != SA_BF16 && out_dtype != SA_F32) return SA_ERR_UNSUPPORTED;
-    if (query->n_q > 0 && !out) return SA_ERR_INVALID_ARG;
+    if (query->n_q > 0 && !out && !cand) return SA_ERR_INVALID_ARG;
     const Layout l = make_layout(query, top_k);
     if ((st = check_workspace(workspace, workspace_bytes, l.decode_total)) != SA_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -340,6 +351,9 @@ static sa_status decode_impl(const sa_cache *cache, const sa_query *query, int32
                                                  query->n_q, top_k, idx, p.status, s));
         }
         if (st != SA_OK) return st;
+        if (cand != nullptr)  // this GPU's candidates for a context-parallel merge
+            return cuda_status(launch_cand_emit(scores, l.ld, idx, query->n_q, top_k, cand->offset,
+                                                cand->score, cand->pos, s));
         if ((st = mark(2)) != SA_OK) return st;
         if ((st = run_attention(p, l, true, rows_ready, workspace, idx, top_k, out, out_dtype,
                                 lse, s)) != SA_OK)
@@ -366,6 +380,43 @@ sa_status sa_decode_traced(const sa_cache *cache, const sa_query *query, int32_t
                        workspace_bytes, stream, phase_events);
 }
 
+sa_status sa_local_candidates(const sa_cache *cache, const sa_query *query, int32_t top_k,
+                              const int32_t *position_offset, float *cand_score,
+                              int32_t *cand_pos, void *workspace, size_t workspace_bytes,
+                              void *stream) {
+    if (query != nullptr && query->n_q > 0 && (!cand_score || !cand_pos || !position_offset))
+        return SA_ERR_INVALID_ARG;
+    const CandOut cand{position_offset, cand_score, cand_pos};
+    return decode_impl(cache, query, top_k, nullptr, nullptr, SA_BF16, nullptr, workspace,
+                       workspace_bytes, stream, nullptr, &cand);
+}
+
+sa_status sa_merge_candidates(const float *cand_score, const int32_t *cand_pos, int32_t n_ranks,
+                              int32_t n_q, int32_t top_k, const int32_t *pos_lo,
+                              const int32_t *pos_hi, int32_t *idx_global, int32_t *idx_local,
+                              void *stream) {
+    if (n_ranks <= 0 || n_q < 0 || top_k <= 0) return SA_ERR_INVALID_ARG;
+    if (n_q > kMaxQueries) return SA_ERR_UNSUPPORTED;
+    if ((int64_t)n_ranks * top_k > cp_merge_max_candidates()) return SA_ERR_UNSUPPORTED;
+    if (n_q == 0) return SA_OK;
+    if (!cand_score || !cand_pos || !pos_lo || !pos_hi || !idx_global || !idx_local)
+        return SA_ERR_INVALID_ARG;
+    return cuda_status(launch_cp_merge(cand_score, cand_pos, n_ranks, n_q, top_k, pos_lo, pos_hi,
+                                       idx_global, idx_local, static_cast<cudaStream_t>(stream)));
+}
+
+sa_status sa_combine_partials(const float *o_part, const float *lse_part, int32_t n_parts,
+                              int32_t n_q, int32_t heads, int32_t d, void *out,
+                              sa_dtype out_dtype, float *lse, void *stream) {
+    if (n_parts <= 0 || n_q < 0 || heads <= 0 || d <= 0) return SA_ERR_INVALID_ARG;
+    if (n_parts > cp_combine_max_parts()) return SA_ERR_UNSUPPORTED;
+    if (out_dtype != SA_BF16 && out_dtype != SA_F32) return SA_ERR_UNSUPPORTED;
+    if (n_q == 0) return SA_OK;
+    if (!o_part || !lse_part || !out) return SA_ERR_INVALID_ARG;
+    return cuda_status(launch_cp_combine(o_part, lse_part, n_parts, (int64_t)n_q * heads, d, out,
+                                         out_dtype, lse, static_cast<cudaStream_t>(stream)));
+}
+
 sa_status sa_quantize_index_query(const void *q_in, sa_dtype in_dtype, int32_t n_q,
                                   int32_t h_index, int32_t d_index, void *q_out, float *q_scale,
                                   void *stream) {
@@ -388,6 +439,8 @@ sa_status sa_append_tokens(const sa_cache *cache, const sa_new_tokens *tokens, v
     const bool page_tile = cache->kv_scale_tokens == 0 && cache->kv_scale_dims == 0;
     if (tokens->kv && cache->kv_dtype == SA_E4M3 && (page_tile || cache->kv_scale_tokens != 1))
         return SA_ERR_UNSUPPORTED;  // a scale shared by several tokens cannot take one more
+    if (tokens->k_index && cache->index_dtype == SA_MXFP8)
+        return SA_ERR_UNSUPPORTED;  // no MXFP8 key encoder: such pools are filled by the caller
     if (tokens->n_new > 0) {
         if (!tokens->seq || !tokens->pos) return SA_ERR_INVALID_ARG;
         if ((tokens->k_index && !aligned16(tokens->k_index)) ||

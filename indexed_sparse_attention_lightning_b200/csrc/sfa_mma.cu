@@ -20,7 +20,11 @@
 // columns) on the upper half-lanes: head m's S row is lane 32(m/16) + m%16,
 // its O row that lane + 16, i.e. the same warp.  Each tile's 64 full 1152-byte
 // rows are copied once into a 128-byte-swizzled stage that is the K-major B
-// operand of S and, read MN-major, the B operand of P V.
+// operand of S and, read MN-major, the B operand of P V.  The stage's rope
+// block (the last 64 dims of every row, 8 KB) is read by S only, so once S is
+// done the softmax writes that tile's P (64 heads x 64 keys bf16, also 8 KB)
+// over it: every stage carries its own P, and the softmax of the next tile
+// never waits for P V of this one to release a shared P buffer.
 //
 // Roles (384 threads, one CTA per SM):
 //   warp 0     lane 0 loads Q by TMA (into the third ring stage; this copy
@@ -72,17 +76,20 @@ constexpr int kChunksPerRow = kD * 2 / 16;  // 72 sixteen-byte pieces of a row
 // Stage layout: key k of a tile, 64-dim block b -> byte (k/8)*kGroupBytes +
 // b*1024 + (k%8)*128 (+ the 16-byte swizzle): the S view (K-major, 8-key
 // groups kGroupBytes apart) and the P V view (MN-major, 64-dim atoms 1024
-// bytes apart, 8-key groups kGroupBytes apart) read the same bytes.
+// bytes apart, 8-key groups kGroupBytes apart) read the same bytes.  After S,
+// block 8 (the rope) holds P: head h's 64 keys at (h/8)*kGroupBytes + 8*1024 +
+// (h%8)*128 (+ swizzle), the K-major A operand of P V with 8-head groups
+// kGroupBytes apart.
 constexpr uint32_t kGroupBytes = kBlocks * 1024;             // 9216
 constexpr uint32_t kStageBytes = (kTile / 8) * kGroupBytes;  // 73728
+constexpr uint32_t kPOffset = (kBlocks - 1) * 1024;          // the rope block
 
 struct SfaSmem {
     // ring stage: 8 groups of 8 rows; a group holds the 9 column blocks of its
     // rows, each 8 x 128 bytes with the 128-byte swizzle (see kGroupBytes)
     uint8_t kv[kStages][kStageBytes];
-    uint8_t p[kHeadsCta * 128];                 // P (bf16), K-major, 128-byte swizzle
     uint64_t kv_full[kStages], kv_empty[kStages];
-    uint64_t s_full[2], p_full, o_done, q_full, q_ready;
+    uint64_t s_full[2], p_full[kStages], o_done, q_full, q_ready;
     uint32_t tmem_base;
     int abort;
 };
@@ -162,7 +169,7 @@ sfa_mma_kernel(const __grid_constant__ CUtensorMap tm_q, const SfaArgs a) {
             mbar_init(&sm.kv_empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) mbar_init(&sm.s_full[b], 1);
-        mbar_init(&sm.p_full, 4);  // the four softmax warps
+        for (int s = 0; s < kStages; ++s) mbar_init(&sm.p_full[s], 4);  // the four softmax warps
         mbar_init(&sm.o_done, 1);
         mbar_init(&sm.q_full, 1);
         mbar_init(&sm.q_ready, 4);
@@ -290,9 +297,11 @@ sfa_mma_kernel(const __grid_constant__ CUtensorMap tm_q, const SfaArgs a) {
                 pa[r] = *reinterpret_cast<uint32_t *>(&x);
                 pb[r] = *reinterpret_cast<uint32_t *>(&y);
             }
-            // O and the P buffer belong to P V of the previous tile until it is done
-            if (n > 0 && ok) ok = warp_wait(&sm.o_done, (n - 1) & 1, abort_flag, status);
-            if (ok && __any_sync(0xffffffffu, (grow_a || grow_b) && n > 0)) {
+            // O belongs to P V of the previous tile until it is done: only a
+            // rescale has to wait for it (P goes to this tile's own stage)
+            const bool rescale = __any_sync(0xffffffffu, (grow_a || grow_b) && n > 0);
+            if (rescale && ok) ok = warp_wait(&sm.o_done, (n - 1) & 1, abort_flag, status);
+            if (ok && rescale) {
                 tc_fence_after();
 #pragma unroll 1
                 for (int c = 0; c < 4; ++c) {
@@ -314,9 +323,11 @@ sfa_mma_kernel(const __grid_constant__ CUtensorMap tm_q, const SfaArgs a) {
             l_b = l_b * f_b + lb;
             m_a = mn_a;
             m_b = mn_b;
-            // P rows ha, hb: keys 8r + 2 q4 (+1) -> bytes 16r + 4 q4 of the row
-            uint8_t *row_a = sm.p + ha * 128 + 4 * q4;
-            uint8_t *row_b = sm.p + hb * 128 + 4 * q4;
+            // P rows ha, hb: keys 8r + 2 q4 (+1) -> bytes 16r + 4 q4 of the row,
+            // in the rope block of this tile's stage (S has read it: s_full)
+            uint8_t *pbase = sm.kv[n % kStages] + kPOffset;
+            uint8_t *row_a = pbase + (ha >> 3) * kGroupBytes + (ha & 7) * 128 + 4 * q4;
+            uint8_t *row_b = pbase + (hb >> 3) * kGroupBytes + (hb & 7) * 128 + 4 * q4;
 #pragma unroll
             for (int r = 0; r < 8; ++r) {
                 *reinterpret_cast<uint32_t *>(row_a + ((r ^ (ha & 7)) << 4)) = pa[r];
@@ -325,7 +336,7 @@ sfa_mma_kernel(const __grid_constant__ CUtensorMap tm_q, const SfaArgs a) {
             fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.p_full);
+            if (lane == 0) mbar_arrive(&sm.p_full[n % kStages]);
         }
         if (ok && T > 0) ok = warp_wait(&sm.o_done, (T - 1) & 1, abort_flag, status);
         tc_fence_after();
@@ -517,11 +528,11 @@ sfa_mma_kernel(const __grid_constant__ CUtensorMap tm_q, const SfaArgs a) {
         int ns = 0, np = 0;  // next S and next P V to issue
         // P V(np) needs P of tile np
         auto try_pv = [&]() -> bool {
-            if (!(np < ns && mbar_test(&sm.p_full, np & 1))) return false;
+            const int st = np % kStages;
+            if (!(np < ns && mbar_test(&sm.p_full[st], (np / kStages) & 1))) return false;
             fence_proxy_async_smem();
             tc_fence_after();
-            const int st = np % kStages;
-            const uint64_t ad = desc_kmajor_sw128(smem_u32(sm.p));
+            const uint64_t ad = desc_kmajor_sw128_sbo(smem_u32(sm.kv[st]) + kPOffset, kGroupBytes);
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 const uint32_t vb = smem_u32(sm.kv[st]) + 4 * half * 1024;

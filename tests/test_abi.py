@@ -79,6 +79,23 @@ def test_workspace_size_valid_and_invalid(L):
 FP8_KV = {"kv_dtype": _abi.SA_E4M3, "kv_rope": FAKE, "kv_scale": FAKE}
 
 
+def test_mxfp8_index_argument_checks(L):
+    """MXFP8 index data (one E8M0 byte per 32 values) needs both scale arrays,
+    16-byte aligned, and a dimension that is a whole number of groups; it names
+    index data only, and no key encoder exists for appending to such a pool."""
+    mx = {"index_dtype": _abi.SA_MXFP8}
+    assert ws_size(L, good_cache(**mx), good_query()) > 0
+    assert ws_size(L, good_cache(**mx, d_index=48), good_query()) == 0     # 1.5 groups
+    assert ws_size(L, good_cache(**mx, k_index_scale=None), good_query()) == 0
+    assert ws_size(L, good_cache(**mx), good_query(q_index_scale=None)) == 0
+    assert ws_size(L, good_cache(**mx), good_query(q_index_scale=FAKE + 4)) == 0
+    assert decode_call(L, good_cache(kv_dtype=_abi.SA_MXFP8), good_query()) == \
+        _abi.SA_ERR_UNSUPPORTED
+    t = new_tokens()
+    assert L.sa_append_tokens(ctypes.byref(good_cache(**mx)), ctypes.byref(t), FAKE, 1 << 20,
+                              None) == _abi.SA_ERR_UNSUPPORTED
+
+
 @pytest.mark.parametrize("tile,ok", [
     ((0, 0), True),       # one scale per page
     ((1, 128), True),     # per token and 128 latent dims

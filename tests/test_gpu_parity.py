@@ -196,6 +196,49 @@ def test_bf16_indexer_path(h_index, d_index):
     assert rel <= 1e-4
 
 
+@pytest.mark.parametrize("h_index,d_index", [(64, 128), (8, 64)])
+def test_mxfp8_indexer_path(h_index, d_index):
+    """The pages' MXFP8 index path (e4m3 query and keys, one E8M0 scale per 32
+    values): block-scaled tensor-core MMAs for 64 heads x 128 dims, the
+    CUDA-core kernel for other shapes.  Products of e4m3 values and powers of
+    two are exact in fp32, so the unfused scores must match the oracle's to
+    fp32 accumulation error; the fused decode must pass the top-K window and
+    the attention tolerances."""
+    sp = W.WorkloadSpec(name=f"mxfp8_index_{h_index}_{d_index}", seed=43, batch=4,
+                        seq_len=("list", (130, 900, 2049, 5000)), index_dtype="mxfp8",
+                        h_index=h_index, d_index=d_index, keys=("planted", 0.05, 3.0))
+    wl = workload(sp)
+    res = run_fused(wl)
+    assert res["status"] == (_abi.SA_OK, 0)
+    scores = oracle.index_scores(wl)
+    topk = parity.check_topk(res["idx"], scores, wl.visible, sp.top_k)
+    ref_out, ref_lse = oracle.sparse_attn(wl, res["idx"])
+    err = parity.check_attention(res["out"], ref_out, "bf16")
+    parity.check_lse(res["lse"], ref_lse)
+    cache, queries = api.upload(wl)
+    got = api.indexer_score(cache, queries).cpu().numpy()
+    ok = ~np.isnan(scores)
+    rel = float(np.abs(got[ok] - scores[ok]).max() / np.abs(scores[ok]).max())
+    print(f"\nmxfp8 index {h_index}x{d_index}: score err {rel:.3g} of max|I|, "
+          f"swaps={topk['swaps']} max_abs={err['max_abs']:.3g}")
+    assert rel <= 1e-4
+
+
+def test_mxfp8_headline_decode_matches_oracle():
+    """The headline decode (64 sequences, 16K-32K context, planted keys) with the
+    MXFP8 index path, every query checked: the launch bench.py times for it."""
+    wl = workload(W.DECODE_B64_MXFP8_INDEX)
+    res = run_fused(wl)
+    assert res["status"] == (_abi.SA_OK, 0)
+    scores = oracle.index_scores(wl)
+    topk = parity.check_topk(res["idx"], scores, wl.visible, wl.spec.top_k)
+    ref_out, ref_lse = oracle.sparse_attn(wl, res["idx"])
+    err = parity.check_attention(res["out"], ref_out, "bf16")
+    parity.check_lse(res["lse"], ref_lse)
+    print(f"\nmxfp8 headline: swaps={topk['swaps']} window={topk['worst_window_fraction']:.3g} "
+          f"max_abs={err['max_abs']:.3g} mean_rel={err['mean_rel']:.3g}")
+
+
 # ------------------------------------------------ device-side data errors ---
 
 def test_bad_page_id_is_reported_not_faulted():
