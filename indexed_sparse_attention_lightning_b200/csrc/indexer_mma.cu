@@ -226,6 +226,7 @@ indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
     using C = IxCfg<kMode>;
     constexpr bool kBf16 = C::kBf16, kMx = C::kMx;
     constexpr int kAcc = C::kAcc;
+    static_assert(C::kMmas * C::kKPerMma == kDim, "the MMA K steps cover the index dimension");
     pdl_wait();
     extern __shared__ uint8_t smem_raw[];
     IndexerSmem<kMode> &sm = *reinterpret_cast<IndexerSmem<kMode> *>(align1024(smem_raw));

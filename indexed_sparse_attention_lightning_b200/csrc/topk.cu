@@ -247,6 +247,37 @@ __device__ void threshold_bucket(const uint32_t *__restrict__ h, int32_t K, int 
     *above_out = sa;
 }
 
+// Exclusive prefix of v over the kCollectThreads threads of the block (total
+// through *total).  All threads call it.
+__device__ __forceinline__ int collect_prefix(int v, int *warp_sums, int *total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    constexpr int kWarps = kCollectThreads / 32;
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += n;
+    }
+    if (lane == 31) warp_sums[warp] = incl;
+    __syncthreads();
+    int before = 0, all = 0;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+        const int x = warp_sums[w];
+        before += w < warp ? x : 0;
+        all += x;
+    }
+    __syncthreads();
+    *total = all;
+    return before + incl - v;
+}
+
+// Collects one chunk of a long row: its keys above the threshold bucket into
+// sel (positions) and its keys inside the bucket into cand (composite keys).
+// The chunk's scores are loaded once, all in flight together (each thread
+// 8 x 4 consecutive scores), kept in registers for both the count and the
+// write; one global reservation per list and CTA.
+constexpr int kCollectPer = 8;  // float4 per thread: a chunk of 256 x 32 = 8192 positions
 __global__ void __launch_bounds__(kCollectThreads)
 topk_collect_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *__restrict__ vis,
                     const uint32_t *__restrict__ hist, int32_t top_k, int32_t chunk,
@@ -254,63 +285,73 @@ topk_collect_kernel(const float *__restrict__ scores, int64_t ld, const int32_t 
                     uint64_t *__restrict__ cand, int32_t cap) {
     pdl_wait();
     pdl_trigger();
-    __shared__ int32_t cnt_s[2], base_s[2];
-    const int t = blockIdx.y;
+    __shared__ int warp_sums[kCollectThreads / 32];
+    __shared__ int32_t base_s[2];
+    const int t = blockIdx.y, tid = threadIdx.x;
     const int32_t V = vis[t];
     const int64_t c0 = (int64_t)blockIdx.x * chunk;
     if (V <= top_k || c0 >= V) return;
     const int64_t c1 = min((int64_t)V, c0 + chunk);
+    const float *row = scores + (int64_t)t * ld;
+    float4 xs[kCollectPer];
+#pragma unroll
+    for (int u = 0; u < kCollectPer; ++u) {
+        const int64_t i0 = c0 + 4 * (tid + (int64_t)u * kCollectThreads);
+        if (i0 + 4 <= c1) {
+            xs[u] = *reinterpret_cast<const float4 *>(row + i0);
+        } else {
+            xs[u].x = i0 < c1 ? row[i0] : 0.f;
+            xs[u].y = i0 + 1 < c1 ? row[i0 + 1] : 0.f;
+            xs[u].z = i0 + 2 < c1 ? row[i0 + 2] : 0.f;
+            xs[u].w = i0 + 3 < c1 ? row[i0 + 3] : 0.f;
+        }
+    }
     int bstar;
     uint32_t above;
     threshold_bucket(hist + (int64_t)t * kHistBins, top_k, &bstar, &above);
-    const float *row = scores + (int64_t)t * ld;
-    const int lane = threadIdx.x & 31;
-    const unsigned lt = (1u << lane) - 1u;
-    // pass 1: this chunk's counts, then one global reservation per list
-    if (threadIdx.x < 2) cnt_s[threadIdx.x] = 0;
-    __syncthreads();
-    int32_t nh = 0, ne = 0;
-    for (int64_t i = c0 + threadIdx.x; i < c1; i += kCollectThreads) {
-        const int b = static_cast<int>(order_key(row[i]) >> (32 - kHistBits));
-        nh += b > bstar;
-        ne += b == bstar;
-    }
+    int nh = 0, ne = 0;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        nh += __shfl_xor_sync(0xffffffffu, nh, o);
-        ne += __shfl_xor_sync(0xffffffffu, ne, o);
+    for (int u = 0; u < kCollectPer; ++u) {
+        const int64_t i0 = c0 + 4 * (tid + (int64_t)u * kCollectThreads);
+        const float x[4] = {xs[u].x, xs[u].y, xs[u].z, xs[u].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int b = static_cast<int>(order_key(x[e]) >> (32 - kHistBits));
+            nh += (i0 + e < c1 && b > bstar) ? 1 : 0;
+            ne += (i0 + e < c1 && b == bstar) ? 1 : 0;
+        }
     }
-    if (lane == 0) {
-        atomicAdd(&cnt_s[0], nh);
-        atomicAdd(&cnt_s[1], ne);
+    int tot_h, tot_e;
+    int oh = collect_prefix(nh, warp_sums, &tot_h);
+    int oe = collect_prefix(ne, warp_sums, &tot_e);
+    if (tid == 0) {
+        base_s[0] = tot_h > 0 ? atomicAdd(&counts[2 * t], tot_h) : 0;
+        base_s[1] = tot_e > 0 ? atomicAdd(&counts[2 * t + 1], tot_e) : 0;
     }
     __syncthreads();
-    if (threadIdx.x < 2) {
-        base_s[threadIdx.x] = cnt_s[threadIdx.x] > 0
-                                  ? atomicAdd(&counts[2 * t + threadIdx.x], cnt_s[threadIdx.x])
-                                  : 0;
-        cnt_s[threadIdx.x] = 0;
-    }
-    __syncthreads();
-    // pass 2: write into the reserved ranges (slots from shared-memory counters)
+    oh += base_s[0];
+    oe += base_s[1];
     int32_t *sel_t = sel + (int64_t)t * top_k;
     uint64_t *cand_t = cand + (int64_t)t * cap;
-    for (int64_t base = c0; base < c1; base += kCollectThreads) {
-        const int64_t i = base + threadIdx.x;
-        const uint32_t key = i < c1 ? order_key(row[i]) : 0u;
-        const int b = static_cast<int>(key >> (32 - kHistBits));
-        const bool hi = i < c1 && b > bstar, eq = i < c1 && b == bstar;
-        const unsigned bh = __ballot_sync(0xffffffffu, hi), be = __ballot_sync(0xffffffffu, eq);
-        int32_t oh = 0, oe = 0;
-        if (lane == 0) {
-            if (bh) oh = atomicAdd(&cnt_s[0], __popc(bh));
-            if (be) oe = atomicAdd(&cnt_s[1], __popc(be));
+#pragma unroll
+    for (int u = 0; u < kCollectPer; ++u) {
+        const int64_t i0 = c0 + 4 * (tid + (int64_t)u * kCollectThreads);
+        const float x[4] = {xs[u].x, xs[u].y, xs[u].z, xs[u].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            if (i0 + e >= c1) continue;
+            const uint32_t key = order_key(x[e]);
+            const int b = static_cast<int>(key >> (32 - kHistBits));
+            const int32_t i = static_cast<int32_t>(i0 + e);
+            if (b > bstar) {
+                if (oh < top_k) sel_t[oh] = i;
+                ++oh;
+            } else if (b == bstar) {
+                if (oe < cap)
+                    cand_t[oe] = (static_cast<uint64_t>(key) << 32) | (0xFFFFFFFFu - static_cast<uint32_t>(i));
+                ++oe;
+            }
         }
-        oh = base_s[0] + __shfl_sync(0xffffffffu, oh, 0) + __popc(bh & lt);
-        oe = base_s[1] + __shfl_sync(0xffffffffu, oe, 0) + __popc(be & lt);
-        if (hi && oh < top_k) sel_t[oh] = static_cast<int32_t>(i);
-        if (eq && oe < cap)
-            cand_t[oe] = (static_cast<uint64_t>(key) << 32) | (0xFFFFFFFFu - static_cast<uint32_t>(i));
     }
 }
 
@@ -397,6 +438,7 @@ __device__ void emit_selection(const uint32_t *bits, int words, int32_t top_k, i
     for (int c0 = w0; c0 < w1; c0 += 32) {
         const int w = c0 + lane;
         uint32_t b = w < w1 ? bits[w] : 0u;
+        if (!__any_sync(0xffffffffu, b != 0u)) continue;  // sparse long rows: most chunks empty
         const int c = __popc(b);
         int incl = c;
 #pragma unroll
@@ -594,7 +636,14 @@ topk_single_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *
                     if (valid && b > bstar) above_mask |= 1u << e;
                     if (valid && b == bstar) ++n_eq;
                 }
-                if (above_mask) atomicOr(&bits[i0 >> 5], above_mask << (i0 & 31));
+                // the 8 lanes of a 32-position word combine their 4-bit masks
+                // (lane l holds positions 4l .. 4l + 3 of the warp's 128), and
+                // the group's first lane stores the word: no atomics
+                uint32_t word = above_mask << (4 * (lane & 7));
+                word |= __shfl_xor_sync(0xffffffffu, word, 1);
+                word |= __shfl_xor_sync(0xffffffffu, word, 2);
+                word |= __shfl_xor_sync(0xffffffffu, word, 4);
+                if ((lane & 7) == 0 && i0 < V) bits[i0 >> 5] = word;
                 // warp-aggregated slots for the bucket's keys
                 int incl = n_eq;
 #pragma unroll
@@ -650,6 +699,7 @@ cudaError_t launch_topk_hist(const float *scores, int64_t ld, const int32_t *vis
                           ld, vis, hist, top_k, idx, p, rows, ld_rows, n_valid);
     }
     constexpr int32_t kChunk = 8192;
+    static_assert(kChunk == kCollectThreads * kCollectPer * 4, "one float4 batch per thread");
     const dim3 grid_c(static_cast<unsigned>(ceil_div(std::max(max_valid, 1), kChunk)), n_q);
     count_launch();
     cudaError_t e = launch_pdl(topk_collect_kernel, grid_c, dim3(kCollectThreads), 0, s, scores, ld,
