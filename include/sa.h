@@ -146,6 +146,13 @@ typedef struct sa_query {
     const void *q;               /* device [n_q, heads, d_latent + d_rope] */
     int32_t heads;
     float sm_scale;              /* softmax scale applied to q . kv */
+
+    /* A promise for chunked prefill: queries 4i .. 4i+3 belong to one sequence
+     * (0 or 1: no promise).  With 4 and e4m3 index keys, the indexer scores
+     * each group against every key tile once (the tile shared by the four
+     * queries); a group that breaks the promise is skipped and reported as
+     * SA_DETAIL_BAD_POSITION. */
+    int32_t q_group;
 } sa_query;
 
 /* Which entry point a workspace is sized for. */

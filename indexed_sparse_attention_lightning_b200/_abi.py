@@ -47,7 +47,7 @@ class SaQuery(ctypes.Structure):
     _fields_ = [("n_q", _I32), ("q_seq", _P), ("q_pos", _P), ("max_visible", _I32),
                 ("q_index", _P), ("q_index_scale", _P), ("w", _P), ("h_index", _I32),
                 ("q_dtype", ctypes.c_int), ("q", _P), ("heads", _I32),
-                ("sm_scale", ctypes.c_float)]
+                ("sm_scale", ctypes.c_float), ("q_group", _I32)]
 
 
 class SaNewTokens(ctypes.Structure):

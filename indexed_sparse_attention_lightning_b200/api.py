@@ -121,6 +121,8 @@ class DeviceQueries:
     q: torch.Tensor
     heads: int
     sm_scale: float
+    # chunked prefill: queries 4i .. 4i+3 belong to one sequence (see sa_query.q_group)
+    q_group: int = 1
 
     @property
     def n_q(self) -> int:
@@ -136,7 +138,7 @@ class DeviceQueries:
             max_visible=self.max_visible, q_index=_ptr(self.q_index),
             q_index_scale=_ptr(self.q_index_scale), w=_ptr(self.w), h_index=self.h_index,
             q_dtype=_abi.DTYPES[self.q_dtype], q=_ptr(self.q), heads=self.heads,
-            sm_scale=self.sm_scale)
+            sm_scale=self.sm_scale, q_group=self.q_group)
 
     def tensors(self) -> dict:
         return {"q_seq": self.q_seq, "q_pos": self.q_pos, "q_index": self.q_index,
@@ -173,7 +175,8 @@ def upload(wl, device="cuda") -> tuple[DeviceCache, DeviceQueries]:
         q_seq=_t(wl.q_seq, device), q_pos=_t(wl.q_pos, device), max_visible=wl.max_visible,
         q_index=_t(wl.q_index, device), q_index_scale=_t(wl.q_index_scale, device),
         w=_t(wl.w, device), h_index=sp.h_index, q_dtype=sp.q_dtype, q=_t(wl.q, device),
-        heads=sp.heads, sm_scale=sp.softmax_scale)
+        heads=sp.heads, sm_scale=sp.softmax_scale,
+        q_group=4 if sp.queries[0] == "prefill" else 1)
     return cache, queries
 
 

@@ -18,7 +18,11 @@
 // The contraction of 64 heads x 128 dims against every key is a dense GEMM
 // (M = 128 keys of a two-page tile, N = 64 heads, K = 128), so it runs as
 // tcgen05.mma kind::f8f6f4 (e4m3 x e4m3 -> fp32 in TMEM), or kind::f16 with
-// bf16 operands.  A bf16 key row is 256 bytes, two 128-byte swizzle atoms
+// bf16 operands.  In chunked prefill, consecutive queries of one sequence see
+// (nearly) the same keys ("Inference Acceleration for New Large Model
+// Architectures" §5.2: the causal index load grows with position), so groups
+// of four of them share every key tile: N = 4 x 64 heads, one full-rate
+// M = 128, N = 256 MMA per 32-wide K step, each key tile read once per group.  A bf16 key row is 256 bytes, two 128-byte swizzle atoms
 // wide, so its tiles are stored as two 64-column halves.  The kernel is
 // persistent: the tiles of all queries are laid end to end and every CTA takes
 // an equal contiguous share, so short and long contexts balance across SMs.
@@ -54,7 +58,6 @@ constexpr int kDim = 128;     // MMA K: index dimension
 constexpr int kScaleSlots = 8;  // key-scale ring: the epilogue frees these, not the key stages
 constexpr int kEpiGroups = 2;  // epilogue warp groups, alternating tiles
 constexpr int kThreads = 64 + kEpiGroups * 128;
-constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kAtom = 128;  // bytes of a row in one 128-byte swizzle atom
 
 // Numerical paths: e4m3 codes with one fp32 scale per key and per (query,
@@ -72,7 +75,8 @@ constexpr uint32_t kColSfb = 208;  // query scales: 4 columns per query buffer
 // Storage of one index element type.  A row of kDim elements is kChunks
 // 128-byte column chunks; a tile stores chunk c of all 128 keys contiguously
 // (16 KB, page h at + 8 KB * h), the query chunk c of its 64 heads likewise.
-template <int kMode>
+// kQb: queries sharing each key tile (1, or 4 for chunked prefill, e4m3 only).
+template <int kMode, int kQb = 1>
 struct IxCfg {
     static constexpr bool kBf16 = kMode == kModeBf16;
     static constexpr bool kMx = kMode == kModeMx;
@@ -84,21 +88,24 @@ struct IxCfg {
     static constexpr uint32_t kQBytes = kHeads * kDim * kElem;
     static constexpr int kKPerMma = 32 / kElem;                      // K of one instruction
     static constexpr int kMmas = kDim / kKPerMma;
-    static constexpr int kCtasPerSm = kBf16 ? 1 : 2;
+    static constexpr int kCtasPerSm = (kBf16 || kQb > 1) ? 1 : 2;
+    static constexpr int kN = kHeads * kQb;                            // MMA N
     // key stages in flight per CTA: 2 x 4 x 16 KB (e4m3) or 4 x 32 KB (bf16) per SM
     // (a fifth bf16 stage measured no faster)
     static constexpr int kStages = 4;
-    // TMEM accumulators (64 columns each); MXFP8 keeps three, leaving room
-    // for the scale factors
-    static constexpr int kAcc = kMx ? 3 : 4;
+    // TMEM accumulators (kN columns each); MXFP8 keeps three, leaving room
+    // for the scale factors; query groups keep two of 256 columns
+    static constexpr int kAcc = kMx ? 3 : (kQb > 1 ? 2 : 4);
+    static constexpr uint32_t kTmemCols = kQb > 1 ? 512 : 256;
 };
 
-template <int kMode>
+template <int kMode, int kQb = 1>
 struct IndexerSmem {
-    uint8_t keys[IxCfg<kMode>::kStages][IxCfg<kMode>::kTileBytes];  // 1024-byte aligned (swizzle atoms)
-    uint32_t hist[kHistBins];              // score-key histogram of the current query
-    uint8_t q[2][IxCfg<kMode>::kQBytes];   // 1024-byte aligned like the key stages
-    float wq[kEpiGroups][kHeads];          // head weights x query scales of that query
+    using C = IxCfg<kMode, kQb>;
+    uint8_t keys[C::kStages][C::kTileBytes];  // 1024-byte aligned (swizzle atoms)
+    uint32_t hist[kQb][kHistBins];            // score-key histograms of the current queries
+    uint8_t q[2][kQb * C::kQBytes];           // 1024-byte aligned like the key stages
+    float wq[kEpiGroups][kQb * kHeads];       // head weights x query scales of those queries
     // key scales of the staged pages: one fp32 per key (e4m3), or four E8M0
     // bytes per key (MXFP8), 512 bytes a slot either way
     alignas(16) float kscale[kScaleSlots][kKeys];
@@ -108,20 +115,23 @@ struct IndexerSmem {
     alignas(16) uint8_t q_sf[2][kHeads * (kDim / kMxGroup)];
     alignas(128) uint8_t sfa[4][512];
     alignas(128) uint8_t sfb[2][512];
-    uint64_t full[IxCfg<kMode>::kStages], empty[IxCfg<kMode>::kStages];
+    uint64_t full[C::kStages], empty[C::kStages];
     uint64_t sc_full[kScaleSlots], sc_empty[kScaleSlots];
-    uint64_t acc_full[IxCfg<kMode>::kAcc], acc_empty[IxCfg<kMode>::kAcc];
+    uint64_t acc_full[C::kAcc], acc_empty[C::kAcc];
     uint64_t q_full[2], q_empty[2];
     uint64_t done;
     uint32_t tmem_base;
-    int32_t start_t, start_i;           // this CTA's first tile (query, tile in query)
+    int32_t start_t, start_i;           // this CTA's first tile (query or group, tile in it)
     int abort;
 };
 
+using PrefillSmem = IndexerSmem<kModeE4m3, 4>;
 static_assert(offsetof(IndexerSmem<kModeE4m3>, q) % 1024 == 0 &&
                   offsetof(IndexerSmem<kModeBf16>, q) % 1024 == 0 &&
-                  offsetof(IndexerSmem<kModeMx>, q) % 1024 == 0,
+                  offsetof(IndexerSmem<kModeMx>, q) % 1024 == 0 &&
+                  offsetof(PrefillSmem, q) % 1024 == 0,
               "128-byte-swizzled Q tiles need 1024-byte alignment");
+static_assert(sizeof(PrefillSmem) + 1024 <= 232448, "query groups: one CTA per SM");
 static_assert(offsetof(IndexerSmem<kModeE4m3>, wq) % 16 == 0 &&
                   offsetof(IndexerSmem<kModeBf16>, wq) % 16 == 0,
               "head weights are read as float4");
@@ -129,13 +139,14 @@ static_assert(2 * (sizeof(IndexerSmem<kModeE4m3>) + 2048) <= 233472, "e4m3: two 
 static_assert(2 * (sizeof(IndexerSmem<kModeMx>) + 2048) <= 233472, "mxfp8: two CTAs per SM");
 static_assert(sizeof(IndexerSmem<kModeBf16>) + 1024 <= 232448, "bf16: one CTA per SM");
 static_assert(IxCfg<kModeMx>::kAcc * kHeads <= kColSfa && kColSfa + 4 * 4 <= kColSfb &&
-                  kColSfb + 2 * 4 <= kTmemCols,
+                  kColSfb + 2 * 4 <= IxCfg<kModeMx>::kTmemCols,
               "MXFP8 scale columns sit past the accumulators");
 
 struct IndexerArgs {
     PathParams p;
     const int32_t *vis;       // [n_q] visible length (0 = invalid query)
-    const int32_t *tile_end;  // [n_q] inclusive prefix of ceil(vis / 128)
+    const int32_t *tile_end;  // [n_units] inclusive prefix of the units' tile counts
+    int32_t n_units;          // queries, or groups of kQb queries
     float *scores;
     int64_t ld;
     uint32_t *hist;           // [n_q, kHistBins] (zeroed by the caller) or null
@@ -219,20 +230,22 @@ __host__ __device__ constexpr uint32_t mx_instr_desc(uint32_t m, uint32_t n, uin
     return (kb << 4) | ((n >> 3) << 17) | (1u << 23) | ((m >> 4) << 24) | (kb << 29);
 }
 
-template <int kMode>
-__global__ void __launch_bounds__(kThreads, IxCfg<kMode>::kCtasPerSm)
+template <int kMode, int kQb>
+__global__ void __launch_bounds__(kThreads, IxCfg<kMode, kQb>::kCtasPerSm)
 indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
                    const __grid_constant__ CUtensorMap tm_q, const IndexerArgs a) {
-    using C = IxCfg<kMode>;
+    using C = IxCfg<kMode, kQb>;
     constexpr bool kBf16 = C::kBf16, kMx = C::kMx;
     constexpr int kAcc = C::kAcc;
+    static_assert(kQb == 1 || kMode == kModeE4m3, "query groups: e4m3 keys only");
     static_assert(C::kMmas * C::kKPerMma == kDim, "the MMA K steps cover the index dimension");
     pdl_wait();
     extern __shared__ uint8_t smem_raw[];
-    IndexerSmem<kMode> &sm = *reinterpret_cast<IndexerSmem<kMode> *>(align1024(smem_raw));
+    IndexerSmem<kMode, kQb> &sm =
+        *reinterpret_cast<IndexerSmem<kMode, kQb> *>(align1024(smem_raw));
     const PathParams &p = a.p;
     const int warp = warp_id(), lane = lane_id();
-    const int64_t total = p.n_q > 0 ? a.tile_end[p.n_q - 1] : 0;
+    const int64_t total = a.n_units > 0 ? a.tile_end[a.n_units - 1] : 0;
     const int64_t k0 = total * blockIdx.x / gridDim.x;
     const int64_t k1 = total * (blockIdx.x + 1) / gridDim.x;
     if (k0 >= k1) return;  // uniform over the CTA, before any allocation
@@ -264,7 +277,7 @@ indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
         // this CTA's first tile: the first query t with tile_end[t] > k0, by a
         // 32-way search (a few dependent loads instead of a binary search's
         // dozen), shared with the other roles through shared memory
-        int lo = 0, hi = p.n_q - 1;
+        int lo = 0, hi = a.n_units - 1;
         while (lo < hi) {
             const int step = (hi - lo + 32) / 32;
             const int q = min(hi, lo + (lane + 1) * step - 1);
@@ -277,7 +290,7 @@ indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
             sm.start_t = lo;
             sm.start_i = static_cast<int32_t>(k0 - (lo > 0 ? a.tile_end[lo - 1] : 0));
         }
-        tmem_alloc(&sm.tmem_base, kTmemCols);
+        tmem_alloc(&sm.tmem_base, C::kTmemCols);
     }
     tc_fence_before();
     __syncthreads();
@@ -295,7 +308,15 @@ indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
             TileCursor c;
             c.init_at(a.tile_end, sm.start_t, sm.start_i, k0, k1);
             bool seg_start = true;
-            int32_t seq = p.q_seq[c.t], V = a.vis[c.t];
+            // a unit's keys: its (first) query's sequence, up to its longest query
+            auto unit_vis = [&](int32_t u) {
+                int32_t v = 0;
+#pragma unroll
+                for (int j = 0; j < kQb; ++j)
+                    if (kQb * u + j < p.n_q) v = max(v, a.vis[kQb * u + j]);
+                return v;
+            };
+            int32_t seq = p.q_seq[kQb * c.t], V = unit_vis(c.t);
             int32_t pg[2];
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
@@ -309,8 +330,8 @@ indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
                 int32_t nseq = seq, nV = V, npg[2] = {-1, -1};
                 if (nx.valid()) {
                     if (nx_seg) {
-                        nseq = p.q_seq[nx.t];
-                        nV = a.vis[nx.t];
+                        nseq = p.q_seq[kQb * nx.t];
+                        nV = unit_vis(nx.t);
                     }
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
@@ -323,11 +344,16 @@ indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
                     if (!mbar_wait(&sm.q_empty[b], ((c.seg >> 1) & 1) ^ 1, abort_flag, p.status))
                         break;
                     constexpr uint32_t kQSfBytes = kHeads * (kDim / kMxGroup);
-                    mbar_arrive_expect_tx(&sm.q_full[b], C::kQBytes + (kMx ? kQSfBytes : 0u));
+                    const int nq = min(kQb, p.n_q - kQb * c.t);  // queries of the unit
+                    mbar_arrive_expect_tx(&sm.q_full[b],
+                                          nq * C::kQBytes + (kMx ? kQSfBytes : 0u));
+                    for (int j = 0; j < nq; ++j) {
 #pragma unroll
-                    for (int ch = 0; ch < C::kChunks; ++ch)
-                        tma_load_2d(sm.q[b] + ch * (kHeads * kAtom), &tm_q, ch * C::kChunkElems,
-                                    c.t * kHeads, &sm.q_full[b]);
+                        for (int ch = 0; ch < C::kChunks; ++ch)
+                            tma_load_2d(sm.q[b] + j * C::kQBytes + ch * (kQb * kHeads * kAtom),
+                                        &tm_q, ch * C::kChunkElems, (kQb * c.t + j) * kHeads,
+                                        &sm.q_full[b]);
+                    }
                     if (kMx)
                         bulk_load(sm.q_sf[b],
                                   reinterpret_cast<const uint8_t *>(p.q_index_scale) +
@@ -445,7 +471,7 @@ indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
             __syncwarp();
         } else if (lane == 0) {
             // kind::f8f6f4 format 0 = e4m3; kind::f16 format 1 = bf16
-            constexpr uint32_t idesc = instr_desc(kKeys, kHeads, kBf16 ? 1 : 0, 0, 0);
+            constexpr uint32_t idesc = instr_desc(kKeys, C::kN, kBf16 ? 1 : 0, 0, 0);
             TileCursor c;
             c.init_at(a.tile_end, sm.start_t, sm.start_i, k0, k1);
             bool seg_start = true;
@@ -462,14 +488,15 @@ indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
                 tc_fence_after();
                 const uint32_t keys = smem_u32(sm.keys[stage]);
                 const uint32_t qs = smem_u32(sm.q[c.seg & 1]);
-                const uint32_t d = tmem + acc * kHeads;
+                const uint32_t d = tmem + acc * C::kN;
                 // 32 bytes of K per instruction: four per 128-byte chunk (the
                 // descriptor address counts 16-byte units)
 #pragma unroll
                 for (int kk = 0; kk < C::kMmas; ++kk) {
                     const int ch = kk / 4, w = kk % 4;
                     const uint64_t adesc = desc_kmajor_sw128(keys + ch * (kKeys * kAtom)) + 2 * w;
-                    const uint64_t bdesc = desc_kmajor_sw128(qs + ch * (kHeads * kAtom)) + 2 * w;
+                    const uint64_t bdesc =
+                        desc_kmajor_sw128(qs + ch * (kQb * kHeads * kAtom)) + 2 * w;
                     if (kBf16)
                         mma_bf16(d, adesc, bdesc, idesc, kk > 0 ? 1u : 0u);
                     else
@@ -500,19 +527,24 @@ indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
         const bool histo = a.hist != nullptr;
         float *wq = sm.wq[g];
         if (histo) {
-            for (int b = ea; b < kHistBins; b += 256) sm.hist[b] = 0;
+            for (int b = ea; b < kQb * kHistBins; b += 256) (&sm.hist[0][0])[b] = 0;
             named_barrier(1, 256);
         }
-        // add the CTA's counts of query t to the global histogram, then clear;
-        // both groups walk every tile, so they get here at the same query change
-        auto flush = [&](int32_t t) {
+        // add the CTA's counts of unit u's queries to their global histograms,
+        // then clear; both groups walk every tile, so they get here at the same
+        // unit change
+        auto flush = [&](int32_t u) {
             named_barrier(1, 256);
-            uint32_t *gh = a.hist + (int64_t)t * kHistBins;
-            for (int b = ea; b < kHistBins; b += 256) {
-                const uint32_t v = sm.hist[b];
-                if (v != 0) {
-                    atomicAdd(gh + b, v);
-                    sm.hist[b] = 0;
+            for (int j = 0; j < kQb; ++j) {
+                const int32_t t = kQb * u + j;
+                if (t >= p.n_q) break;
+                uint32_t *gh = a.hist + (int64_t)t * kHistBins;
+                for (int b = ea; b < kHistBins; b += 256) {
+                    const uint32_t v = sm.hist[j][b];
+                    if (v != 0) {
+                        atomicAdd(gh + b, v);
+                        sm.hist[j][b] = 0;
+                    }
                 }
             }
             named_barrier(1, 256);
@@ -520,21 +552,34 @@ indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
         TileCursor c;
         c.init_at(a.tile_end, sm.start_t, sm.start_i, k0, k1);
         bool ok = true;
-        int32_t V = 0, t_cur = -1;
+        int32_t Vq[kQb];  // visible length of each query of the unit (0: none)
+#pragma unroll
+        for (int j = 0; j < kQb; ++j) Vq[j] = 0;
+        int32_t t_cur = -1;
         for (int n = 0; c.valid(); ++n, c.next(a.tile_end)) {
-            if (c.t != t_cur) {  // a new query: both groups see it at the same tile
+            if (c.t != t_cur) {  // a new unit: both groups see it at the same tile
                 if (histo && t_cur >= 0) flush(t_cur);
                 named_barrier(bar, 128);  // the old weights are no longer read
                 t_cur = c.t;
-                V = a.vis[c.t];
-                if (et < kHeads)
-                    wq[et] = __ldg(p.w + (int64_t)c.t * kHeads + et) *
-                             ((kBf16 || kMx) ? 1.f
-                                             : __ldg(p.q_index_scale + (int64_t)c.t * kHeads + et));
+#pragma unroll
+                for (int j = 0; j < kQb; ++j) {
+                    const int32_t t = kQb * c.t + j;
+                    Vq[j] = t < p.n_q ? a.vis[t] : 0;
+                }
+                for (int i = et; i < kQb * kHeads; i += 128) {
+                    const int32_t t = kQb * c.t + i / kHeads;
+                    const int64_t wi = (int64_t)kQb * c.t * kHeads + i;
+                    wq[i] = t >= p.n_q ? 0.f
+                                       : __ldg(p.w + wi) *
+                                             ((kBf16 || kMx) ? 1.f : __ldg(p.q_index_scale + wi));
+                }
                 named_barrier(bar, 128);
             }
             if ((n & 1) != g) continue;  // the other group's tile
             const int64_t s = (int64_t)c.i * kKeys + row;
+            int32_t V = 0;  // the unit's longest visible length
+#pragma unroll
+            for (int j = 0; j < kQb; ++j) V = max(V, Vq[j]);
             // key scales and page validity have a ring of their own
             const int slot = n % kScaleSlots;
             if (ok)
@@ -546,38 +591,47 @@ indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
             if (ok && s < V && !page_ok) report(p.status, SA_ERR_DEVICE_FAULT, SA_DETAIL_BAD_PAGE);
             const int acc = n % kAcc;
             if (ok) ok = warp_wait(&sm.acc_full[acc], (n / kAcc) & 1, abort_flag, p.status);
-            float sum = 0.f;
+            float sum[kQb];
+#pragma unroll
+            for (int j = 0; j < kQb; ++j) sum[j] = 0.f;
             if (ok) {
                 tc_fence_after();
-                const uint32_t taddr =
-                    tmem + (static_cast<uint32_t>(quad * 32) << 16) + acc * kHeads;
-                float v[32], u[32];
-                tmem_ld32(taddr, v);
-                tmem_ld32(taddr + 32, u);
-                tmem_wait_ld();
-                const float4 *w4 = reinterpret_cast<const float4 *>(wq);
-                float part[4] = {0.f, 0.f, 0.f, 0.f};  // four independent chains
 #pragma unroll
-                for (int j4 = 0; j4 < 8; ++j4) {
-                    const float4 wa = w4[j4], wb = w4[8 + j4];
-                    part[0] = fmaf(wa.x, relu_keep_nan(v[4 * j4]), part[0]);
-                    part[1] = fmaf(wa.y, relu_keep_nan(v[4 * j4 + 1]), part[1]);
-                    part[2] = fmaf(wa.z, relu_keep_nan(v[4 * j4 + 2]), part[2]);
-                    part[3] = fmaf(wa.w, relu_keep_nan(v[4 * j4 + 3]), part[3]);
-                    part[0] = fmaf(wb.x, relu_keep_nan(u[4 * j4]), part[0]);
-                    part[1] = fmaf(wb.y, relu_keep_nan(u[4 * j4 + 1]), part[1]);
-                    part[2] = fmaf(wb.z, relu_keep_nan(u[4 * j4 + 2]), part[2]);
-                    part[3] = fmaf(wb.w, relu_keep_nan(u[4 * j4 + 3]), part[3]);
+                for (int j = 0; j < kQb; ++j) {
+                    if (!__any_sync(0xffffffffu, s < Vq[j])) continue;  // nothing visible here
+                    const uint32_t taddr = tmem + (static_cast<uint32_t>(quad * 32) << 16) +
+                                           acc * C::kN + j * kHeads;
+                    float v[32], u[32];
+                    tmem_ld32(taddr, v);
+                    tmem_ld32(taddr + 32, u);
+                    tmem_wait_ld();
+                    const float4 *w4 = reinterpret_cast<const float4 *>(wq + j * kHeads);
+                    float part[4] = {0.f, 0.f, 0.f, 0.f};  // four independent chains
+#pragma unroll
+                    for (int j4 = 0; j4 < 8; ++j4) {
+                        const float4 wa = w4[j4], wb = w4[8 + j4];
+                        part[0] = fmaf(wa.x, relu_keep_nan(v[4 * j4]), part[0]);
+                        part[1] = fmaf(wa.y, relu_keep_nan(v[4 * j4 + 1]), part[1]);
+                        part[2] = fmaf(wa.z, relu_keep_nan(v[4 * j4 + 2]), part[2]);
+                        part[3] = fmaf(wa.w, relu_keep_nan(v[4 * j4 + 3]), part[3]);
+                        part[0] = fmaf(wb.x, relu_keep_nan(u[4 * j4]), part[0]);
+                        part[1] = fmaf(wb.y, relu_keep_nan(u[4 * j4 + 1]), part[1]);
+                        part[2] = fmaf(wb.z, relu_keep_nan(u[4 * j4 + 2]), part[2]);
+                        part[3] = fmaf(wb.w, relu_keep_nan(u[4 * j4 + 3]), part[3]);
+                    }
+                    sum[j] = (part[0] + part[1]) + (part[2] + part[3]);
                 }
-                sum = (part[0] + part[1]) + (part[2] + part[3]);
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.acc_empty[acc]);
-            if (s < V) {
-                const float score = page_ok ? sum * kscale : -INFINITY;
-                a.scores[(int64_t)c.t * a.ld + s] = score;
-                if (histo) atomicAdd(&sm.hist[order_key(score) >> (32 - kHistBits)], 1u);
+#pragma unroll
+            for (int j = 0; j < kQb; ++j) {
+                if (s < Vq[j]) {
+                    const float score = page_ok ? sum[j] * kscale : -INFINITY;
+                    a.scores[(int64_t)(kQb * c.t + j) * a.ld + s] = score;
+                    if (histo) atomicAdd(&sm.hist[j][order_key(score) >> (32 - kHistBits)], 1u);
+                }
             }
         }
         if (histo && t_cur >= 0) flush(t_cur);
@@ -587,7 +641,7 @@ indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc(tmem, kTmemCols);
+        tmem_dealloc(tmem, C::kTmemCols);
     }
 }
 
@@ -601,38 +655,45 @@ bool indexer_mma_supported(const PathParams &p) {
 
 namespace {
 
-template <int kMode>
+template <int kMode, int kQb>
 cudaError_t launch_indexer_mma_t(const PathParams &p, const int32_t *vis, const int32_t *tile_end,
                                  float *scores, int64_t ld, uint32_t *hist, cudaStream_t s) {
-    using C = IxCfg<kMode>;
+    using C = IxCfg<kMode, kQb>;
     CUtensorMap tk, tq;
     if (!encode_tmap_2d(&tk, C::kElem, p.k_index, kDim, (uint64_t)p.num_pages * 64,
                         kDim * C::kElem, C::kChunkElems, 64, true) ||
         !encode_tmap_2d(&tq, C::kElem, p.q_index, kDim, (uint64_t)p.n_q * kHeads,
                         kDim * C::kElem, C::kChunkElems, kHeads, true))
         return cudaErrorInvalidValue;
-    IndexerArgs a{p, vis, tile_end, scores, ld, hist};
-    const int64_t max_tiles = (int64_t)p.n_q * ceil_div(p.max_visible, kKeys);
+    const int32_t n_units = static_cast<int32_t>(ceil_div(p.n_q, kQb));
+    IndexerArgs a{p, vis, tile_end, n_units, scores, ld, hist};
+    const int64_t max_tiles = (int64_t)n_units * ceil_div(p.max_visible, kKeys);
     const int64_t grid = std::min<int64_t>((int64_t)C::kCtasPerSm * num_sms(), max_tiles);
-    const size_t smem = sizeof(IndexerSmem<kMode>) + 1024;
-    cudaError_t e = cudaFuncSetAttribute(indexer_mma_kernel<kMode>,
+    const size_t smem = sizeof(IndexerSmem<kMode, kQb>) + 1024;
+    cudaError_t e = cudaFuncSetAttribute(indexer_mma_kernel<kMode, kQb>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     count_launch();
-    return launch_pdl(indexer_mma_kernel<kMode>, dim3(static_cast<unsigned>(grid)),
+    return launch_pdl(indexer_mma_kernel<kMode, kQb>, dim3(static_cast<unsigned>(grid)),
                       dim3(kThreads), smem, s, tk, tq, a);
 }
 
 }  // namespace
 
+int32_t indexer_query_group(const PathParams &p) {
+    return (p.q_group == 4 && p.index_dtype == SA_E4M3 && p.n_q >= 4) ? 4 : 1;
+}
+
 cudaError_t launch_indexer_mma(const PathParams &p, const int32_t *vis, const int32_t *tile_end,
                                float *scores, int64_t ld, uint32_t *hist, cudaStream_t s) {
     if (p.n_q == 0) return cudaSuccess;
     if (p.index_dtype == SA_BF16)
-        return launch_indexer_mma_t<kModeBf16>(p, vis, tile_end, scores, ld, hist, s);
+        return launch_indexer_mma_t<kModeBf16, 1>(p, vis, tile_end, scores, ld, hist, s);
     if (p.index_dtype == SA_MXFP8)
-        return launch_indexer_mma_t<kModeMx>(p, vis, tile_end, scores, ld, hist, s);
-    return launch_indexer_mma_t<kModeE4m3>(p, vis, tile_end, scores, ld, hist, s);
+        return launch_indexer_mma_t<kModeMx, 1>(p, vis, tile_end, scores, ld, hist, s);
+    if (indexer_query_group(p) == 4)
+        return launch_indexer_mma_t<kModeE4m3, 4>(p, vis, tile_end, scores, ld, hist, s);
+    return launch_indexer_mma_t<kModeE4m3, 1>(p, vis, tile_end, scores, ld, hist, s);
 }
 
 }  // namespace sa

@@ -63,6 +63,7 @@ struct PathParams {
     int32_t q_dtype;  // sa_dtype
     int32_t heads;
     float sm_scale;
+    int32_t q_group;  // queries in runs of this many of one sequence (4: chunked prefill)
     // status word (first 2 ints of the workspace)
     int32_t *status;
 };
@@ -88,12 +89,17 @@ bool encode_tmap_2d(CUtensorMap *map, int dtype_bytes, const void *base, uint64_
 // zeroes `zero_words` 32-bit words at `zero` (histograms and counters) and,
 // with `clear_status`, the status word before anything can report into it.
 cudaError_t launch_plan(const PathParams &p, int32_t *vis, int32_t *tile_end, int32_t tile,
-                        uint32_t *zero, size_t zero_words, bool clear_status, cudaStream_t s);
+                        uint32_t *zero, size_t zero_words, bool clear_status, cudaStream_t s,
+                        int32_t group = 1);
 
 cudaError_t launch_indexer_simt(const PathParams &p, float *scores, int64_t ld, cudaStream_t s);
 
 // Tensor-core FP8 indexer (e4m3 keys, 64 heads x 128 dims); needs the plan.
+// indexer_query_group(p): how many consecutive queries share each key tile
+// (4 for flagged chunked prefill with e4m3 keys, else 1); the plan's tile
+// prefix must run over groups of that size.
 bool indexer_mma_supported(const PathParams &p);
+int32_t indexer_query_group(const PathParams &p);
 cudaError_t launch_indexer_mma(const PathParams &p, const int32_t *vis, const int32_t *tile_end,
                                float *scores, int64_t ld, uint32_t *hist, cudaStream_t s);
 

@@ -73,6 +73,7 @@ sa_status check_query(const sa_query *q, const sa_cache *c, bool need_index, boo
     if (need_index) {
         if (!q->q_index || !q->w || q->h_index <= 0) return SA_ERR_INVALID_ARG;
         if (q->h_index > 128) return SA_ERR_UNSUPPORTED;
+        if (q->q_group < 0) return SA_ERR_INVALID_ARG;
         if ((c->index_dtype == SA_E4M3 || c->index_dtype == SA_MXFP8) && !q->q_index_scale)
             return SA_ERR_INVALID_ARG;
         if (c->index_dtype == SA_MXFP8 && !aligned16(q->q_index_scale)) return SA_ERR_INVALID_ARG;
@@ -117,6 +118,7 @@ PathParams make_params(const sa_cache *c, const sa_query *q, void *ws) {
     p.q_dtype = q->q_dtype;
     p.heads = q->heads;
     p.sm_scale = q->sm_scale;
+    p.q_group = q->q_group;
     p.status = static_cast<int32_t *>(ws);
     return p;
 }
@@ -204,8 +206,8 @@ sa_status run_indexer(const PathParams &p, const Layout &l, void *ws, float *sco
         int32_t *tile_end = reinterpret_cast<int32_t *>(base + l.tile_end);
         uint32_t *hist = want_hist ? reinterpret_cast<uint32_t *>(base + l.hist) : nullptr;
         const size_t zero_words = want_hist ? (l.sel - l.hist) / 4 : 0;
-        sa_status st =
-            cuda_status(launch_plan(p, vis, tile_end, 128, hist, zero_words, clear, s));
+        sa_status st = cuda_status(launch_plan(p, vis, tile_end, 128, hist, zero_words, clear, s,
+                                               indexer_query_group(p)));
         if (st != SA_OK) return st;
         st = cuda_status(launch_indexer_mma(p, vis, tile_end, scores, ld, hist, s));
         *have_hist = want_hist && st == SA_OK;

@@ -239,6 +239,46 @@ def test_mxfp8_headline_decode_matches_oracle():
           f"max_abs={err['max_abs']:.3g} mean_rel={err['mean_rel']:.3g}")
 
 
+def test_prefill_query_groups_match_single_queries():
+    """Chunked prefill with the query-group promise (q_group = 4: four
+    consecutive queries share every key tile, N = 256 MMAs) must give the same
+    scores, selection and output as one query at a time, bit for bit, including
+    a last group of two queries."""
+    sp = W.WorkloadSpec(name="prefill_groups", seed=45, batch=1, seq_len=("fixed", 6000),
+                        queries=("prefill", 2900, 38), keys=("planted", 0.05, 3.0))
+    wl = workload(sp)
+    cache, queries = api.upload(wl)
+    assert queries.q_group == 4
+    single = dataclasses.replace(queries, q_group=1)
+    s4 = api.indexer_score(cache, queries).cpu().numpy()
+    s1 = api.indexer_score(cache, single).cpu().numpy()
+    for t in range(wl.n_q):
+        V = int(wl.visible[t])
+        assert np.array_equal(s4[t, :V], s1[t, :V]), t
+    outs = []
+    for q in (queries, single):
+        idx = torch.empty((wl.n_q, sp.top_k), dtype=torch.int32, device="cuda")
+        ws = api.workspace(api.workspace_size(cache, q, sp.top_k, _abi.SA_WS_DECODE))
+        out, lse, _ = api.decode(cache, q, sp.top_k, idx=idx, ws=ws)
+        assert api.device_status(ws) == (_abi.SA_OK, 0)
+        outs.append((idx.cpu().numpy(), out.float().cpu().numpy(), lse.cpu().numpy()))
+    for a, b in zip(outs[0], outs[1]):
+        assert np.array_equal(a, b)
+    scores = oracle.index_scores(wl)
+    parity.check_topk(outs[0][0], scores, wl.visible, sp.top_k)
+
+
+def test_query_group_mixing_sequences_is_reported():
+    """A q_group = 4 promise that the queries break (four different sequences
+    in one group) is reported on the device, not scored against the wrong keys."""
+    wl = workload(W.DECODE_B8_8K)
+    cache, queries = api.upload(wl)
+    bad = dataclasses.replace(queries, q_group=4)
+    ws = api.workspace(api.workspace_size(cache, bad, wl.spec.top_k, _abi.SA_WS_DECODE))
+    api.decode(cache, bad, wl.spec.top_k, ws=ws)
+    assert api.device_status(ws) == (_abi.SA_ERR_DEVICE_FAULT, _abi.SA_DETAIL_BAD_POSITION)
+
+
 # ------------------------------------------------ device-side data errors ---
 
 def test_bad_page_id_is_reported_not_faulted():
