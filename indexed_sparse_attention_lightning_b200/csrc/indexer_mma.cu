@@ -56,8 +56,6 @@ constexpr int kKeys = 128;    // MMA M: keys per tile (two pages)
 constexpr int kHeads = 64;    // MMA N: indexer heads
 constexpr int kDim = 128;     // MMA K: index dimension
 constexpr int kScaleSlots = 8;  // key-scale ring: the epilogue frees these, not the key stages
-constexpr int kEpiGroups = 2;  // epilogue warp groups, alternating tiles
-constexpr int kThreads = 64 + kEpiGroups * 128;
 constexpr uint32_t kAtom = 128;  // bytes of a row in one 128-byte swizzle atom
 
 // Numerical paths: e4m3 codes with one fp32 scale per key and per (query,
@@ -97,6 +95,13 @@ struct IxCfg {
     // for the scale factors; query groups keep two of 256 columns
     static constexpr int kAcc = kMx ? 3 : (kQb > 1 ? 2 : 4);
     static constexpr uint32_t kTmemCols = kQb > 1 ? 512 : 256;
+    // epilogue warp groups: two take alternate tiles; with query groups two
+    // more share the tiles, each group summing half of the unit's queries
+    static constexpr int kSplit = kQb > 1 ? 2 : 1;
+    static constexpr int kEpiGroups = 2 * kSplit;
+    static constexpr int kQPerGroup = kQb / kSplit;
+    static constexpr int kEpiThreads = 128 * kEpiGroups;
+    static constexpr int kThreads = 64 + kEpiThreads;
 };
 
 template <int kMode, int kQb = 1>
@@ -105,7 +110,7 @@ struct IndexerSmem {
     uint8_t keys[C::kStages][C::kTileBytes];  // 1024-byte aligned (swizzle atoms)
     uint32_t hist[kQb][kHistBins];            // score-key histograms of the current queries
     uint8_t q[2][kQb * C::kQBytes];           // 1024-byte aligned like the key stages
-    float wq[kEpiGroups][kQb * kHeads];       // head weights x query scales of those queries
+    float wq[C::kEpiGroups][C::kQPerGroup * kHeads];  // head weights x query scales, per group
     // key scales of the staged pages: one fp32 per key (e4m3), or four E8M0
     // bytes per key (MXFP8), 512 bytes a slot either way
     alignas(16) float kscale[kScaleSlots][kKeys];
@@ -231,7 +236,7 @@ __host__ __device__ constexpr uint32_t mx_instr_desc(uint32_t m, uint32_t n, uin
 }
 
 template <int kMode, int kQb>
-__global__ void __launch_bounds__(kThreads, IxCfg<kMode, kQb>::kCtasPerSm)
+__global__ void __launch_bounds__(IxCfg<kMode, kQb>::kThreads, IxCfg<kMode, kQb>::kCtasPerSm)
 indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
                    const __grid_constant__ CUtensorMap tm_q, const IndexerArgs a) {
     using C = IxCfg<kMode, kQb>;
@@ -257,13 +262,13 @@ indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
         }
         for (int s = 0; s < kScaleSlots; ++s) {
             mbar_init(&sm.sc_full[s], 1);
-            // the epilogue group's four warps (and the MMA warp, which reads
-            // the MXFP8 scale bytes)
-            mbar_init(&sm.sc_empty[s], kMx ? 5 : 4);
+            // the four warps of each epilogue group on the tile (and the MMA
+            // warp, which reads the MXFP8 scale bytes)
+            mbar_init(&sm.sc_empty[s], 4 * C::kSplit + (kMx ? 1 : 0));
         }
         for (int c = 0; c < kAcc; ++c) {
             mbar_init(&sm.acc_full[c], 1);
-            mbar_init(&sm.acc_empty[c], 4);
+            mbar_init(&sm.acc_empty[c], 4 * C::kSplit);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sm.q_full[b], 1);
@@ -514,32 +519,38 @@ indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
         // --------------------------------------------------- epilogue ---
         // Two groups of four warps take alternate tiles, so two tiles' chains
         // (scale wait, accumulator wait, TMEM loads, weighted ReLU sum, score
-        // store, histogram) run side by side.  Within a group, warp w reads
-        // TMEM lanes 32 (w % 4) .. +31: one key row per thread.  The loop
-        // never leaves early: after a failed (timed-out) wait it carries on
-        // without waiting, so a group's warps meet at the same named barriers.
+        // store, histogram) run side by side; with query groups a second pair
+        // of groups shares the tiles, each group summing half of the unit's
+        // queries, so every SM sub-partition has four epilogue warps to
+        // interleave.  Within a group, warp w reads TMEM lanes 32 (w % 4) ..
+        // +31: one key row per thread.  The loop never leaves early: after a
+        // failed (timed-out) wait it carries on without waiting, so a group's
+        // warps meet at the same named barriers.
+        constexpr int kQg = C::kQPerGroup;
         const int g = (warp - 2) >> 2;          // epilogue group
+        const int tp = g & 1;                   // the parity of the tiles it takes
+        const int q0 = (g >> 1) * kQg;          // its first query within the unit
         const int quad = warp & 3;              // TMEM lanes this warp may read
         const int row = quad * 32 + lane;       // key row of the tile
-        const int ea = threadIdx.x - 64;        // 0..255 over both groups
-        const int et = ea - 128 * g;            // 0..127 within the group
-        const int bar = 2 + g;                  // the group's named barrier (1: both groups)
+        const int ea = threadIdx.x - 64;        // 0 .. kEpiThreads - 1 over all groups
+        const int et = ea & 127;                // 0..127 within the group
+        const int bar = 2 + g;                  // the group's named barrier (1: all groups)
         const bool histo = a.hist != nullptr;
         float *wq = sm.wq[g];
         if (histo) {
-            for (int b = ea; b < kQb * kHistBins; b += 256) (&sm.hist[0][0])[b] = 0;
-            named_barrier(1, 256);
+            for (int b = ea; b < kQb * kHistBins; b += C::kEpiThreads) (&sm.hist[0][0])[b] = 0;
+            named_barrier(1, C::kEpiThreads);
         }
         // add the CTA's counts of unit u's queries to their global histograms,
-        // then clear; both groups walk every tile, so they get here at the same
-        // unit change
+        // then clear; every group walks every tile, so they all get here at
+        // the same unit change
         auto flush = [&](int32_t u) {
-            named_barrier(1, 256);
+            named_barrier(1, C::kEpiThreads);
             for (int j = 0; j < kQb; ++j) {
                 const int32_t t = kQb * u + j;
                 if (t >= p.n_q) break;
                 uint32_t *gh = a.hist + (int64_t)t * kHistBins;
-                for (int b = ea; b < kHistBins; b += 256) {
+                for (int b = ea; b < kHistBins; b += C::kEpiThreads) {
                     const uint32_t v = sm.hist[j][b];
                     if (v != 0) {
                         atomicAdd(gh + b, v);
@@ -547,39 +558,39 @@ indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
                     }
                 }
             }
-            named_barrier(1, 256);
+            named_barrier(1, C::kEpiThreads);
         };
         TileCursor c;
         c.init_at(a.tile_end, sm.start_t, sm.start_i, k0, k1);
         bool ok = true;
-        int32_t Vq[kQb];  // visible length of each query of the unit (0: none)
+        int32_t Vq[kQg];  // visible length of each of the group's queries (0: none)
 #pragma unroll
-        for (int j = 0; j < kQb; ++j) Vq[j] = 0;
+        for (int j = 0; j < kQg; ++j) Vq[j] = 0;
         int32_t t_cur = -1;
         for (int n = 0; c.valid(); ++n, c.next(a.tile_end)) {
-            if (c.t != t_cur) {  // a new unit: both groups see it at the same tile
+            if (c.t != t_cur) {  // a new unit: every group sees it at the same tile
                 if (histo && t_cur >= 0) flush(t_cur);
                 named_barrier(bar, 128);  // the old weights are no longer read
                 t_cur = c.t;
 #pragma unroll
-                for (int j = 0; j < kQb; ++j) {
-                    const int32_t t = kQb * c.t + j;
+                for (int j = 0; j < kQg; ++j) {
+                    const int32_t t = kQb * c.t + q0 + j;
                     Vq[j] = t < p.n_q ? a.vis[t] : 0;
                 }
-                for (int i = et; i < kQb * kHeads; i += 128) {
-                    const int32_t t = kQb * c.t + i / kHeads;
-                    const int64_t wi = (int64_t)kQb * c.t * kHeads + i;
+                for (int i = et; i < kQg * kHeads; i += 128) {
+                    const int32_t t = kQb * c.t + q0 + i / kHeads;
+                    const int64_t wi = ((int64_t)kQb * c.t + q0) * kHeads + i;
                     wq[i] = t >= p.n_q ? 0.f
                                        : __ldg(p.w + wi) *
                                              ((kBf16 || kMx) ? 1.f : __ldg(p.q_index_scale + wi));
                 }
                 named_barrier(bar, 128);
             }
-            if ((n & 1) != g) continue;  // the other group's tile
+            if ((n & 1) != tp) continue;  // the other groups' tile
             const int64_t s = (int64_t)c.i * kKeys + row;
-            int32_t V = 0;  // the unit's longest visible length
+            int32_t V = 0;  // the longest visible length of the group's queries
 #pragma unroll
-            for (int j = 0; j < kQb; ++j) V = max(V, Vq[j]);
+            for (int j = 0; j < kQg; ++j) V = max(V, Vq[j]);
             // key scales and page validity have a ring of their own
             const int slot = n % kScaleSlots;
             if (ok)
@@ -591,46 +602,93 @@ indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
             if (ok && s < V && !page_ok) report(p.status, SA_ERR_DEVICE_FAULT, SA_DETAIL_BAD_PAGE);
             const int acc = n % kAcc;
             if (ok) ok = warp_wait(&sm.acc_full[acc], (n / kAcc) & 1, abort_flag, p.status);
-            float sum[kQb];
+            float sum[kQg];
 #pragma unroll
-            for (int j = 0; j < kQb; ++j) sum[j] = 0.f;
+            for (int j = 0; j < kQg; ++j) sum[j] = 0.f;
             if (ok) {
                 tc_fence_after();
-#pragma unroll
-                for (int j = 0; j < kQb; ++j) {
-                    if (!__any_sync(0xffffffffu, s < Vq[j])) continue;  // nothing visible here
-                    const uint32_t taddr = tmem + (static_cast<uint32_t>(quad * 32) << 16) +
-                                           acc * C::kN + j * kHeads;
-                    float v[32], u[32];
-                    tmem_ld32(taddr, v);
-                    tmem_ld32(taddr + 32, u);
-                    tmem_wait_ld();
-                    const float4 *w4 = reinterpret_cast<const float4 *>(wq + j * kHeads);
-                    float part[4] = {0.f, 0.f, 0.f, 0.f};  // four independent chains
+                const uint32_t tbase =
+                    tmem + (static_cast<uint32_t>(quad * 32) << 16) + acc * C::kN + q0 * kHeads;
+                // eight independent chains per query: heads 4i + {0, 1} and 4i +
+                // {2, 3} of each 32-head half; the query-group kernel runs them
+                // as packed fp32 FMAs (one half after the other), the
+                // 2-CTA-per-SM kernels (96 registers) as scalar ones (halves
+                // interleaved); both round the same products and sums in the same
+                // order, so a query's scores do not depend on the kernel
+                auto half_sum = [&](const float (&x)[32], const float4 *w4, float2 &p0,
+                                    float2 &p1) {
 #pragma unroll
                     for (int j4 = 0; j4 < 8; ++j4) {
-                        const float4 wa = w4[j4], wb = w4[8 + j4];
-                        part[0] = fmaf(wa.x, relu_keep_nan(v[4 * j4]), part[0]);
-                        part[1] = fmaf(wa.y, relu_keep_nan(v[4 * j4 + 1]), part[1]);
-                        part[2] = fmaf(wa.z, relu_keep_nan(v[4 * j4 + 2]), part[2]);
-                        part[3] = fmaf(wa.w, relu_keep_nan(v[4 * j4 + 3]), part[3]);
-                        part[0] = fmaf(wb.x, relu_keep_nan(u[4 * j4]), part[0]);
-                        part[1] = fmaf(wb.y, relu_keep_nan(u[4 * j4 + 1]), part[1]);
-                        part[2] = fmaf(wb.z, relu_keep_nan(u[4 * j4 + 2]), part[2]);
-                        part[3] = fmaf(wb.w, relu_keep_nan(u[4 * j4 + 3]), part[3]);
+                        const float4 w = w4[j4];
+                        const float2 x0 = make_float2(relu_keep_nan(x[4 * j4]),
+                                                      relu_keep_nan(x[4 * j4 + 1]));
+                        const float2 x1 = make_float2(relu_keep_nan(x[4 * j4 + 2]),
+                                                      relu_keep_nan(x[4 * j4 + 3]));
+                        p0 = __ffma2_rn(make_float2(w.x, w.y), x0, p0);
+                        p1 = __ffma2_rn(make_float2(w.z, w.w), x1, p1);
                     }
-                    sum[j] = (part[0] + part[1]) + (part[2] + part[3]);
+                };
+                if constexpr (kQb > 1) {
+                    // 2 kQg chunks of 32 columns (query j = i / 2, heads 32 (i % 2) ..):
+                    // the load of chunk i + 1 is in flight while chunk i is summed
+                    float ca[32], cb[32];
+                    float2 part[4] = {};
+                    tmem_ld32(tbase, ca);
+                    tmem_wait_ld_keep(ca);
+#pragma unroll
+                    for (int i = 0; i < 2 * kQg; ++i) {
+                        float(&cur)[32] = (i & 1) ? cb : ca;
+                        float(&nxt)[32] = (i & 1) ? ca : cb;
+                        if (i + 1 < 2 * kQg) tmem_ld32(tbase + 32 * (i + 1), nxt);
+                        const int j = i >> 1, hf = i & 1;
+                        const float4 *w4 = reinterpret_cast<const float4 *>(wq + j * kHeads) + 8 * hf;
+                        half_sum(cur, w4, part[2 * hf], part[2 * hf + 1]);
+                        if (hf == 1) {
+                            sum[j] = ((part[0].x + part[0].y) + (part[1].x + part[1].y)) +
+                                     ((part[2].x + part[2].y) + (part[3].x + part[3].y));
+#pragma unroll
+                            for (int c = 0; c < 4; ++c) part[c] = make_float2(0.f, 0.f);
+                        }
+                        if (i + 1 < 2 * kQg) tmem_wait_ld_keep(nxt);
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < kQg; ++j) {
+                        if (!__any_sync(0xffffffffu, s < Vq[j])) continue;  // nothing visible here
+                        const uint32_t taddr = tbase + j * kHeads;
+                        float v[32], u[32];
+                        tmem_ld32(taddr, v);
+                        tmem_ld32(taddr + 32, u);
+                        tmem_wait_ld();
+                        const float4 *w4 = reinterpret_cast<const float4 *>(wq + j * kHeads);
+                        float2 part[4] = {};
+#pragma unroll
+                        for (int j4 = 0; j4 < 8; ++j4) {  // the two halves interleaved
+                            const float4 wa = w4[j4], wb = w4[8 + j4];
+                            part[0].x = fmaf(wa.x, relu_keep_nan(v[4 * j4]), part[0].x);
+                            part[0].y = fmaf(wa.y, relu_keep_nan(v[4 * j4 + 1]), part[0].y);
+                            part[1].x = fmaf(wa.z, relu_keep_nan(v[4 * j4 + 2]), part[1].x);
+                            part[1].y = fmaf(wa.w, relu_keep_nan(v[4 * j4 + 3]), part[1].y);
+                            part[2].x = fmaf(wb.x, relu_keep_nan(u[4 * j4]), part[2].x);
+                            part[2].y = fmaf(wb.y, relu_keep_nan(u[4 * j4 + 1]), part[2].y);
+                            part[3].x = fmaf(wb.z, relu_keep_nan(u[4 * j4 + 2]), part[3].x);
+                            part[3].y = fmaf(wb.w, relu_keep_nan(u[4 * j4 + 3]), part[3].y);
+                        }
+                        sum[j] = ((part[0].x + part[0].y) + (part[1].x + part[1].y)) +
+                                 ((part[2].x + part[2].y) + (part[3].x + part[3].y));
+                    }
                 }
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.acc_empty[acc]);
 #pragma unroll
-            for (int j = 0; j < kQb; ++j) {
+            for (int j = 0; j < kQg; ++j) {
                 if (s < Vq[j]) {
                     const float score = page_ok ? sum[j] * kscale : -INFINITY;
-                    a.scores[(int64_t)(kQb * c.t + j) * a.ld + s] = score;
-                    if (histo) atomicAdd(&sm.hist[j][order_key(score) >> (32 - kHistBits)], 1u);
+                    a.scores[(int64_t)(kQb * c.t + q0 + j) * a.ld + s] = score;
+                    if (histo)
+                        atomicAdd(&sm.hist[q0 + j][order_key(score) >> (32 - kHistBits)], 1u);
                 }
             }
         }
@@ -675,7 +733,7 @@ cudaError_t launch_indexer_mma_t(const PathParams &p, const int32_t *vis, const 
     if (e != cudaSuccess) return e;
     count_launch();
     return launch_pdl(indexer_mma_kernel<kMode, kQb>, dim3(static_cast<unsigned>(grid)),
-                      dim3(kThreads), smem, s, tk, tq, a);
+                      dim3(C::kThreads), smem, s, tk, tq, a);
 }
 
 }  // namespace
