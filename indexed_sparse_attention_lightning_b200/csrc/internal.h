@@ -111,8 +111,9 @@ cudaError_t launch_topk_rowwise(const float *scores, int64_t ld, const int32_t *
 
 // Histogram-guided exact top-K for rows scored by the tensor-core indexer
 // (which filled `hist`, [n_q, kHistBins]).  Scratch: sel [n_q, top_k],
-// counts [n_q, 2] (zeroed), cand [n_q, cap].
+// counts [n_q, kTopkCountsPerQuery] (zeroed), cand [n_q, cap].
 constexpr int32_t kTopkCandCap = 8192;
+constexpr int32_t kTopkCountsPerQuery = 8;
 // With `rows` non-null it also writes the physical cache rows of the
 // selection for the tensor-core attention (compact_rows layout, tile 64,
 // leading dimension ld_rows) and their count n_valid [n_q].

@@ -124,7 +124,7 @@ PathParams make_params(const sa_cache *c, const sa_query *q, void *ws) {
 }
 
 // Workspace: status | vis [n_q] | tile_end [n_q] | scores [n_q, ld] | idx [n_q, K]
-// | hist [n_q, 4096] | counts [n_q, 2] | sel [n_q, K] | cand [n_q, cap]
+// | hist [n_q, 4096] | counts [n_q, 8] | sel [n_q, K] | cand [n_q, cap]
 // | rows [n_q, R] | n_valid [n_q] | o_part [n_q, S, 128, 512]
 // | lse_part [n_q, S, 128]; the indexer needs the first three, the fused path
 // all of them; the attention alone needs the status, the compacted rows and
@@ -156,7 +156,7 @@ Layout make_layout(const sa_query *q, int32_t top_k) {
     l.idx = align_up(l.scores + sizeof(float) * nq * (size_t)l.ld);
     l.hist = align_up(l.idx + sizeof(int32_t) * nq * kk);
     l.counts = align_up(l.hist + sizeof(uint32_t) * nq * kHistBins);  // follows hist: one clear
-    l.sel = align_up(l.counts + sizeof(int32_t) * 2 * nq);
+    l.sel = align_up(l.counts + sizeof(int32_t) * kTopkCountsPerQuery * nq);
     l.cand = align_up(l.sel + sizeof(int32_t) * nq * kk);
     const size_t rows_bytes = sizeof(int32_t) * nq * (size_t)sfa_rows_ld(top_k);
     l.rows = align_up(l.cand + sizeof(uint64_t) * nq * kTopkCandCap);

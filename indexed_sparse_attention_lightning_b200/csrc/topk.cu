@@ -17,7 +17,6 @@ namespace sa {
 namespace {
 
 constexpr int kThreads = 1024;
-constexpr size_t kTopkSmemLimit = 200 * 1024;  // dynamic shared memory of the finalize CTA
 
 // Exclusive prefix of `flag` over the block in thread order; returns the
 // block total through *total.  Uses warp ballots plus one scan of the warp
@@ -272,100 +271,108 @@ __device__ __forceinline__ int collect_prefix(int v, int *warp_sums, int *total)
     return before + incl - v;
 }
 
-// Collects one chunk of a long row: its keys above the threshold bucket into
-// sel (positions) and its keys inside the bucket into cand (composite keys).
-// The chunk's scores are loaded once, all in flight together (each thread
-// 8 x 4 consecutive scores), kept in registers for both the count and the
-// write; one global reservation per list and CTA.
-constexpr int kCollectPer = 8;  // float4 per thread: a chunk of 256 x 32 = 8192 positions
+// Long rows (more than kSingleMaxV positions) take three kernels, each with
+// many CTAs per query where the work is per position:
+//   count      per 8192-position chunk: keys above the threshold bucket are
+//              counted (per chunk), keys inside it are collected as composite
+//              candidates;
+//   threshold  one CTA per query: the exact need-th largest candidate (so an
+//              exact composite threshold for the whole row) and each chunk's
+//              first output slot;
+//   emit       per chunk again: its selected positions, in ascending order,
+//              and their physical cache rows, written straight to their slots.
+// Per-query state (counts, [n_q, 8] int32, zeroed with the histograms):
+//   [0] keys above the bucket, [1] candidates, [2] emit CTAs finished,
+//   [3] an unmapped page was met, [4..5] threshold mask, [6..7] threshold
+//   prefix (mask 0: the threshold kernel selected the whole row itself).
+constexpr int kChunk = 8192;                             // positions per count / emit CTA
+constexpr int kChunkPer = kChunk / kCollectThreads;      // 32 consecutive positions a thread
+constexpr int kCountsPerQuery = kTopkCountsPerQuery;
+
+// The 32 scores of positions [p0, p0 + 32) of `row` (entries at or past V
+// are never selected; they read as 0).
+__device__ __forceinline__ void load_run(const float *row, int64_t p0, int64_t V, float (&x)[32]) {
+    if (p0 + 32 <= V) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const float4 v = *reinterpret_cast<const float4 *>(row + p0 + 4 * u);
+            x[4 * u] = v.x;
+            x[4 * u + 1] = v.y;
+            x[4 * u + 2] = v.z;
+            x[4 * u + 3] = v.w;
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) x[i] = p0 + i < V ? row[p0 + i] : 0.f;
+    }
+}
+
 __global__ void __launch_bounds__(kCollectThreads)
-topk_collect_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *__restrict__ vis,
-                    const uint32_t *__restrict__ hist, int32_t top_k, int32_t chunk,
-                    int32_t *__restrict__ sel, int32_t *__restrict__ counts,
-                    uint64_t *__restrict__ cand, int32_t cap) {
+topk_count_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *__restrict__ vis,
+                  const uint32_t *__restrict__ hist, int32_t top_k, int32_t *__restrict__ chunk_slot,
+                  int32_t ld_chunks, int32_t *__restrict__ counts, uint64_t *__restrict__ cand,
+                  int32_t cap) {
     pdl_wait();
     pdl_trigger();
     __shared__ int warp_sums[kCollectThreads / 32];
-    __shared__ int32_t base_s[2];
+    __shared__ int32_t base_s;
     const int t = blockIdx.y, tid = threadIdx.x;
     const int32_t V = vis[t];
-    const int64_t c0 = (int64_t)blockIdx.x * chunk;
+    const int64_t c0 = (int64_t)blockIdx.x * kChunk;
     if (V <= top_k || c0 >= V) return;
-    const int64_t c1 = min((int64_t)V, c0 + chunk);
-    const float *row = scores + (int64_t)t * ld;
-    float4 xs[kCollectPer];
-#pragma unroll
-    for (int u = 0; u < kCollectPer; ++u) {
-        const int64_t i0 = c0 + 4 * (tid + (int64_t)u * kCollectThreads);
-        if (i0 + 4 <= c1) {
-            xs[u] = *reinterpret_cast<const float4 *>(row + i0);
-        } else {
-            xs[u].x = i0 < c1 ? row[i0] : 0.f;
-            xs[u].y = i0 + 1 < c1 ? row[i0 + 1] : 0.f;
-            xs[u].z = i0 + 2 < c1 ? row[i0 + 2] : 0.f;
-            xs[u].w = i0 + 3 < c1 ? row[i0 + 3] : 0.f;
-        }
-    }
+    const int64_t p0 = c0 + (int64_t)kChunkPer * tid;
+    float x[32];
+    load_run(scores + (int64_t)t * ld, p0, V, x);
     int bstar;
     uint32_t above;
     threshold_bucket(hist + (int64_t)t * kHistBins, top_k, &bstar, &above);
     int nh = 0, ne = 0;
 #pragma unroll
-    for (int u = 0; u < kCollectPer; ++u) {
-        const int64_t i0 = c0 + 4 * (tid + (int64_t)u * kCollectThreads);
-        const float x[4] = {xs[u].x, xs[u].y, xs[u].z, xs[u].w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int b = static_cast<int>(order_key(x[e]) >> (32 - kHistBits));
-            nh += (i0 + e < c1 && b > bstar) ? 1 : 0;
-            ne += (i0 + e < c1 && b == bstar) ? 1 : 0;
-        }
+    for (int i = 0; i < 32; ++i) {
+        const int b = static_cast<int>(order_key(x[i]) >> (32 - kHistBits));
+        nh += (p0 + i < V && b > bstar) ? 1 : 0;
+        ne += (p0 + i < V && b == bstar) ? 1 : 0;
     }
     int tot_h, tot_e;
-    int oh = collect_prefix(nh, warp_sums, &tot_h);
+    collect_prefix(nh, warp_sums, &tot_h);
     int oe = collect_prefix(ne, warp_sums, &tot_e);
+    int32_t *ct = counts + (int64_t)t * kCountsPerQuery;
     if (tid == 0) {
-        base_s[0] = tot_h > 0 ? atomicAdd(&counts[2 * t], tot_h) : 0;
-        base_s[1] = tot_e > 0 ? atomicAdd(&counts[2 * t + 1], tot_e) : 0;
+        // a row of more chunks than slots is left to the threshold kernel's fallback
+        if ((int)blockIdx.x < ld_chunks) chunk_slot[(int64_t)t * ld_chunks + blockIdx.x] = tot_h;
+        if (tot_h > 0) atomicAdd(&ct[0], tot_h);
+        base_s = tot_e > 0 ? atomicAdd(&ct[1], tot_e) : 0;
     }
     __syncthreads();
-    oh += base_s[0];
-    oe += base_s[1];
-    int32_t *sel_t = sel + (int64_t)t * top_k;
+    if (ne == 0) return;
+    oe += base_s;
     uint64_t *cand_t = cand + (int64_t)t * cap;
 #pragma unroll
-    for (int u = 0; u < kCollectPer; ++u) {
-        const int64_t i0 = c0 + 4 * (tid + (int64_t)u * kCollectThreads);
-        const float x[4] = {xs[u].x, xs[u].y, xs[u].z, xs[u].w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            if (i0 + e >= c1) continue;
-            const uint32_t key = order_key(x[e]);
-            const int b = static_cast<int>(key >> (32 - kHistBits));
-            const int32_t i = static_cast<int32_t>(i0 + e);
-            if (b > bstar) {
-                if (oh < top_k) sel_t[oh] = i;
-                ++oh;
-            } else if (b == bstar) {
-                if (oe < cap)
-                    cand_t[oe] = (static_cast<uint64_t>(key) << 32) | (0xFFFFFFFFu - static_cast<uint32_t>(i));
-                ++oe;
-            }
+    for (int i = 0; i < 32; ++i) {
+        const uint32_t key = order_key(x[i]);
+        if (p0 + i < V && static_cast<int>(key >> (32 - kHistBits)) == bstar) {
+            if (oe < cap)
+                cand_t[oe] = (static_cast<uint64_t>(key) << 32) |
+                             (0xFFFFFFFFu - static_cast<uint32_t>(p0 + i));
+            ++oe;
         }
     }
 }
 
-// Marks in `bits` (by position) the `need` largest of the n_cand composite
-// candidate keys cs[] -- order-preserving score key in the high word, inverted
-// position in the low word, so all distinct and ties go to the lower position --
-// which all share their top kHistBits bits (the threshold bucket `bstar`).
-// Radix passes of 10-bit digits below the bucket bits find the need-th
-// largest key, stopping as soon as a whole digit bin is taken (normally after
-// two passes); the bucket bits themselves are never counted, so no pass piles
-// every candidate onto one histogram bin.  1 <= need <= n_cand.  All threads
-// of the block call it; dh holds 1024 counters.
-__device__ void mark_top_candidates(const uint64_t *cs, int n_cand, int need, int bstar,
-                                    uint32_t *bits, unsigned *dh, int *warp_sums) {
+// The `need` largest of the n_cand composite candidate keys cs[] --
+// order-preserving score key in the high word, inverted position in the low
+// word, so all distinct and ties go to the lower position -- which all share
+// their top kHistBits bits (the threshold bucket `bstar`): on return exactly
+// `need` of them satisfy (k & *mask) >= *prefix.  Radix passes of 10-bit
+// digits below the bucket bits find the need-th largest key, stopping as soon
+// as a whole digit bin is taken (normally after two passes); the bucket bits
+// themselves are never counted, so no pass piles every candidate onto one
+// histogram bin.  Any composite key of the row above the bucket also passes
+// the test, any below fails it.  1 <= need <= n_cand.  All threads of the
+// block call it; dh holds 1024 counters.
+__device__ void candidate_threshold(const uint64_t *cs, int n_cand, int need, int bstar,
+                                    unsigned *dh, int *warp_sums, uint64_t *mask_out,
+                                    uint64_t *prefix_out) {
     __shared__ int sel_digit_s, sel_above_s, sel_count_s;
     const int tid = threadIdx.x;
     uint64_t prefix = static_cast<uint64_t>(bstar) << (64 - kHistBits);
@@ -403,7 +410,17 @@ __device__ void mark_top_candidates(const uint64_t *cs, int n_cand, int need, in
             shift = 0;
         }
     }
-    // exactly `need` candidates satisfy (k & mask) >= prefix
+    *mask_out = mask;
+    *prefix_out = prefix;
+}
+
+// Marks in `bits` (by position) the `need` largest candidates (see
+// candidate_threshold).  All threads of the block call it.
+__device__ void mark_top_candidates(const uint64_t *cs, int n_cand, int need, int bstar,
+                                    uint32_t *bits, unsigned *dh, int *warp_sums) {
+    const int tid = threadIdx.x;
+    uint64_t mask, prefix;
+    candidate_threshold(cs, n_cand, need, bstar, dh, warp_sums, &mask, &prefix);
     for (int i = tid; i < n_cand; i += kThreads) {
         const uint64_t k = cs[i];
         if ((k & mask) >= prefix) {
@@ -476,30 +493,35 @@ __device__ void emit_selection(const uint32_t *bits, int words, int32_t top_k, i
     if (threadIdx.x == 0) *n_valid = nv;
 }
 
-// One CTA per query: exact order inside the threshold bucket, then every
-// selected position set in a bitmap and read back in ascending order.  Rows
-// the candidate buffer or the bitmap cannot hold (massive exact ties, very
-// long rows) take the row-wise radix select instead.
+// One CTA per query: the exact composite threshold among the candidates and
+// every chunk's first output slot (chunk_slot: the count kernel's per-chunk
+// counts of keys above the bucket, replaced by the exclusive prefix of the
+// chunks' selected counts).  Rows the candidate buffer cannot hold (massive
+// exact ties), short rows and rows of more chunks than one CTA scans take the
+// row-wise radix select here, whole.
+constexpr int kMaxChunks = kThreads;
 __global__ void __launch_bounds__(kThreads)
-topk_finalize_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *__restrict__ vis,
-                     int32_t top_k, const int32_t *__restrict__ sel,
-                     const int32_t *__restrict__ counts, const uint64_t *__restrict__ cand,
-                     int32_t cap, int32_t bitmap_words, int32_t *__restrict__ idx,
-                     const PathParams p, int32_t *__restrict__ rows_all, int32_t ld_rows,
-                     int32_t *__restrict__ n_valid_all) {
+topk_threshold_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *__restrict__ vis,
+                      int32_t top_k, int32_t *__restrict__ chunk_slot, int32_t ld_chunks,
+                      int32_t *__restrict__ counts, const uint64_t *__restrict__ cand, int32_t cap,
+                      int32_t *__restrict__ idx, const PathParams p, int32_t *__restrict__ rows_all,
+                      int32_t ld_rows, int32_t *__restrict__ n_valid_all) {
     pdl_wait();
     pdl_trigger();
-    extern __shared__ uint64_t fin_smem[];
+    extern __shared__ uint64_t cs[];  // [cap]
     __shared__ unsigned dh[1024];
     __shared__ int warp_sums[33];
-    const int t = blockIdx.x;
+    __shared__ int chunk_sel[kMaxChunks];
+    const int t = blockIdx.x, tid = threadIdx.x;
     const int32_t V = vis[t];
     int32_t *out = idx + (int64_t)t * top_k;
-    const int32_t n_sel = counts[2 * t], n_cand = counts[2 * t + 1];
-    const int32_t need = top_k - n_sel;
-    const bool fits = V > top_k && n_cand <= cap && V <= bitmap_words * 32 && need > 0 &&
-                      need <= n_cand;
-    if (!fits) {
+    int32_t *ct = counts + (int64_t)t * kCountsPerQuery;
+    const int32_t n_above = ct[0], n_cand = ct[1];
+    const int32_t need = top_k - n_above;
+    const int chunks = static_cast<int>((V + kChunk - 1) / kChunk);
+    const bool fits = V > top_k && n_cand <= cap && need > 0 && need <= n_cand &&
+                      chunks <= min(kMaxChunks, ld_chunks);
+    if (!fits) {  // threshold mask stays 0: the emit kernel leaves the row alone
         select_row(scores + (int64_t)t * ld, V, top_k, out);
         if (rows_all != nullptr) {
             __syncthreads();
@@ -508,26 +530,100 @@ topk_finalize_kernel(const float *__restrict__ scores, int64_t ld, const int32_t
         }
         return;
     }
-    int32_t *rows = rows_all != nullptr ? rows_all + (int64_t)t * ld_rows : nullptr;
-    uint64_t *cs = fin_smem;                                       // [cap]
-    uint32_t *bits = reinterpret_cast<uint32_t *>(fin_smem + cap);  // [bitmap_words]
     const uint64_t *cg = cand + (int64_t)t * cap;
-    for (int i = threadIdx.x; i < n_cand; i += kThreads) cs[i] = cg[i];
-    const int words = (V + 31) / 32;
-    for (int w = threadIdx.x; w < words; w += kThreads) bits[w] = 0;
+    for (int i = tid; i < n_cand; i += kThreads) cs[i] = cg[i];
+    for (int c = tid; c < chunks; c += kThreads) chunk_sel[c] = 0;
     __syncthreads();
-    // the need largest candidates (all in the threshold bucket, whose bits
-    // every candidate key carries on top)
-    mark_top_candidates(cs, n_cand, need, static_cast<int>(cs[0] >> (64 - kHistBits)), bits,
-                        dh, warp_sums);
-    const int32_t *st = sel + (int64_t)t * top_k;
-    for (int i = threadIdx.x; i < n_sel; i += kThreads) {
-        const uint32_t pos = static_cast<uint32_t>(st[i]);
-        atomicOr(&bits[pos >> 5], 1u << (pos & 31));
+    uint64_t mask, prefix;
+    candidate_threshold(cs, n_cand, need, static_cast<int>(cs[0] >> (64 - kHistBits)), dh,
+                        warp_sums, &mask, &prefix);
+    for (int i = tid; i < n_cand; i += kThreads) {
+        const uint64_t k = cs[i];
+        if ((k & mask) >= prefix) {
+            const uint32_t pos = 0xFFFFFFFFu - static_cast<uint32_t>(k);
+            atomicAdd(&chunk_sel[pos / kChunk], 1);
+        }
     }
     __syncthreads();
-    emit_selection(bits, words, top_k, out, p, t, rows,
-                   n_valid_all != nullptr ? n_valid_all + t : nullptr, warp_sums);
+    int32_t *slot = chunk_slot + (int64_t)t * ld_chunks;
+    const int mine = tid < chunks ? slot[tid] + chunk_sel[tid] : 0;
+    int total;
+    const int first = block_exclusive_prefix(mine, warp_sums, &total);
+    if (tid < chunks) slot[tid] = first;
+    if (tid == 0) {
+        uint64_t *thr = reinterpret_cast<uint64_t *>(ct + 4);
+        thr[0] = mask;
+        thr[1] = prefix;
+    }
+}
+
+// Per chunk: its selected positions (composite key at or above the row's
+// threshold) in ascending order at the chunk's slot, with their physical
+// cache rows.  A thread's 32 consecutive positions lie in one 64-token page,
+// so one page-table lookup serves them all.  The last CTA of a query to finish
+// writes the row count and padding -- or, when a page id was invalid, redoes
+// the rows with compact_rows, which drops and reports the unmapped ones.
+__global__ void __launch_bounds__(kCollectThreads)
+topk_emit_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *__restrict__ vis,
+                 int32_t top_k, const int32_t *__restrict__ chunk_slot, int32_t ld_chunks,
+                 int32_t *__restrict__ counts, int32_t *__restrict__ idx, const PathParams p,
+                 int32_t *__restrict__ rows_all, int32_t ld_rows,
+                 int32_t *__restrict__ n_valid_all) {
+    pdl_wait();
+    pdl_trigger();
+    __shared__ int warp_sums[33];
+    __shared__ int last_s;
+    const int t = blockIdx.y, tid = threadIdx.x;
+    const int32_t V = vis[t];
+    int32_t *ct = counts + (int64_t)t * kCountsPerQuery;
+    const uint64_t *thr = reinterpret_cast<const uint64_t *>(ct + 4);
+    const uint64_t mask = thr[0], prefix = thr[1];
+    const int chunks = static_cast<int>((V + kChunk - 1) / kChunk);
+    if (mask == 0 || (int)blockIdx.x >= chunks) return;  // uniform over the CTA
+    const int64_t p0 = (int64_t)blockIdx.x * kChunk + (int64_t)kChunkPer * tid;
+    float x[32];
+    load_run(scores + (int64_t)t * ld, p0, V, x);
+    uint32_t sel = 0;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        const uint64_t k = (static_cast<uint64_t>(order_key(x[i])) << 32) |
+                           (0xFFFFFFFFu - static_cast<uint32_t>(p0 + i));
+        if (p0 + i < V && (k & mask) >= prefix) sel |= 1u << i;
+    }
+    int total;
+    int q = chunk_slot[(int64_t)t * ld_chunks + blockIdx.x] +
+            collect_prefix(__popc(sel), warp_sums, &total);
+    int32_t *out = idx + (int64_t)t * top_k;
+    int32_t *rows = rows_all != nullptr ? rows_all + (int64_t)t * ld_rows : nullptr;
+    int64_t r0 = 0;
+    if (rows != nullptr && sel != 0) {
+        r0 = phys_row(p.page_table, p.max_pages, p.num_pages, __ldg(p.q_seq + t), p0);
+        if (r0 < 0) atomicOr(&ct[3], 1);
+    }
+    while (sel != 0) {
+        const int i = __ffs(sel) - 1;
+        sel &= sel - 1;
+        if (q < top_k) {
+            out[q] = static_cast<int32_t>(p0 + i);
+            if (rows != nullptr && r0 >= 0) rows[q] = static_cast<int32_t>(r0 + i);
+        }
+        ++q;
+    }
+    if (rows == nullptr) return;
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) last_s = atomicAdd(&ct[2], 1) == chunks - 1;
+    __syncthreads();
+    if (!last_s) return;
+    __threadfence();  // every chunk's positions and rows are visible from here
+    if (*reinterpret_cast<volatile int32_t *>(&ct[3]) != 0) {
+        compact_rows(p, t, out, top_k, 64, rows, n_valid_all + t, warp_sums);
+        return;
+    }
+    const int32_t padded = (top_k + 63) / 64 * 64;
+    const int32_t first = *reinterpret_cast<volatile int32_t *>(rows);
+    for (int c = top_k + tid; c < padded; c += kCollectThreads) rows[c] = first;
+    if (tid == 0) n_valid_all[t] = top_k;
 }
 
 // ---------------------------------------------------------------------------
@@ -698,24 +794,28 @@ cudaError_t launch_topk_hist(const float *scores, int64_t ld, const int32_t *vis
         return launch_pdl(topk_single_kernel, dim3(n_q), dim3(kThreads), kSingleSmem, s, scores,
                           ld, vis, hist, top_k, idx, p, rows, ld_rows, n_valid);
     }
-    constexpr int32_t kChunk = 8192;
-    static_assert(kChunk == kCollectThreads * kCollectPer * 4, "one float4 batch per thread");
-    const dim3 grid_c(static_cast<unsigned>(ceil_div(std::max(max_valid, 1), kChunk)), n_q);
+    const int32_t chunks = static_cast<int32_t>(ceil_div(std::max(max_valid, 1), kChunk));
+    const dim3 grid_c(static_cast<unsigned>(chunks), n_q);
+    // per-chunk counts, then slots, in `sel` ([n_q, top_k]; rows of more
+    // chunks than top_k fall back to the row-wise select)
+    const int32_t ld_chunks = top_k;
     count_launch();
-    cudaError_t e = launch_pdl(topk_collect_kernel, grid_c, dim3(kCollectThreads), 0, s, scores, ld,
-                               vis, hist, top_k, kChunk, sel, counts, cand, cap);
+    cudaError_t e = launch_pdl(topk_count_kernel, grid_c, dim3(kCollectThreads), 0, s, scores, ld,
+                               vis, hist, top_k, sel, ld_chunks, counts, cand, cap);
     if (e != cudaSuccess) return e;
-    // candidates plus a bitmap of the longest row, within one CTA's shared memory
-    const int32_t words = static_cast<int32_t>(ceil_div(std::max(max_valid, 1), 32));
-    const int32_t max_words = static_cast<int32_t>((kTopkSmemLimit - (size_t)cap * 8) / 4);
-    const int32_t bw = std::min(words, max_words);
-    const size_t smem = (size_t)cap * 8 + (size_t)bw * 4;
-    e = cudaFuncSetAttribute(topk_finalize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    const size_t smem = (size_t)cap * 8;
+    e = cudaFuncSetAttribute(topk_threshold_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem);
     if (e != cudaSuccess) return e;
     count_launch();
-    return launch_pdl(topk_finalize_kernel, dim3(n_q), dim3(kThreads), smem, s, scores, ld, vis,
-                      top_k, sel, counts, cand, cap, bw, idx, p, rows, ld_rows, n_valid);
+    e = launch_pdl(topk_threshold_kernel, dim3(n_q), dim3(kThreads), smem, s, scores, ld, vis,
+                   top_k, sel, ld_chunks, counts, (const uint64_t *)cand, cap, idx, p, rows,
+                   ld_rows, n_valid);
+    if (e != cudaSuccess) return e;
+    count_launch();
+    return launch_pdl(topk_emit_kernel, grid_c, dim3(kCollectThreads), 0, s, scores, ld, vis,
+                      top_k, (const int32_t *)sel, ld_chunks, counts, idx, p, rows, ld_rows,
+                      n_valid);
 }
 
 cudaError_t launch_topk_rowwise(const float *scores, int64_t ld, const int32_t *valid_len,

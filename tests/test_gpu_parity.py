@@ -279,6 +279,66 @@ def test_query_group_mixing_sequences_is_reported():
     assert api.device_status(ws) == (_abi.SA_ERR_DEVICE_FAULT, _abi.SA_DETAIL_BAD_POSITION)
 
 
+# ------------------------------------------------------- long contexts ---
+# Rows longer than 64K positions take the multi-CTA top-K (count, threshold,
+# emit): a batch mixing a row shorter than K, which falls back to the row-wise
+# select, with two long rows; massive ties in a long row; and an unmapped page
+# inside a long row.
+LONG = W.WorkloadSpec(name="long_rows_mixed", seed=47, batch=3,
+                      seq_len=("list", (1500, 70000, 140000)), keys=("planted", 0.05, 3.0))
+
+
+def test_long_rows_match_oracle():
+    wl = workload(LONG)
+    res = run_fused(wl)
+    assert res["status"] == (_abi.SA_OK, 0)
+    scores = oracle.index_scores(wl)
+    parity.check_topk(res["idx"], scores, wl.visible, LONG.top_k)
+    ref_out, ref_lse = oracle.sparse_attn(wl, res["idx"])
+    parity.check_attention(res["out"], ref_out, LONG.kv_dtype)
+    parity.check_lse(res["lse"], ref_lse)
+    # the unfused top-K on the fused path's own scores picks the same set
+    cache, queries = api.upload(wl)
+    s = api.indexer_score(cache, queries)
+    idx = api.topk(s, torch.from_numpy(wl.visible).cuda(), LONG.top_k, wl.max_visible)
+    assert np.array_equal(idx.cpu().numpy(), res["idx"])
+
+
+def test_long_rows_with_massive_ties_take_lowest_positions():
+    wl = workload(LONG)
+    k = wl.k_index.copy()
+    valid = np.isfinite(wl.k_index_scale)
+    rng = np.random.default_rng(6)
+    protos = rng.integers(0, 0x7E, size=(3, LONG.d_index), dtype=np.uint8)
+    k[valid] = protos[rng.integers(0, 3, size=valid.sum())]
+    scale = np.where(valid, np.float32(0.01), wl.k_index_scale).astype(np.float32)
+    wl = dataclasses.replace(wl, k_index=k, k_index_scale=scale)
+    res = run_fused(wl)
+    assert res["status"] == (_abi.SA_OK, 0)
+    ref = oracle.topk(oracle.index_scores(wl), wl.visible, LONG.top_k)
+    assert np.array_equal(res["idx"], ref)
+
+
+def test_long_row_unmapped_page_is_reported_and_skipped():
+    """An unmapped page inside a long row: reported, none of its positions
+    selected, and the attention over the rest matches the oracle."""
+    wl = workload(LONG)
+    base = run_fused(wl)
+    t = 2
+    page = int(base["idx"][t, 0]) // 64          # a page holding a selected position
+    cache, queries = api.upload(wl)
+    cache.page_table[int(wl.q_seq[t]), page] = wl.num_pages + 5
+    idx = torch.full((wl.n_q, LONG.top_k), -7, dtype=torch.int32, device="cuda")
+    ws = api.workspace(api.workspace_size(cache, queries, LONG.top_k, _abi.SA_WS_DECODE))
+    out, lse, _ = api.decode(cache, queries, LONG.top_k, idx=idx, ws=ws)
+    assert api.device_status(ws) == (_abi.SA_ERR_DEVICE_FAULT, _abi.SA_DETAIL_BAD_PAGE)
+    got = idx.cpu().numpy()
+    assert not np.any(got[t] // 64 == page) and np.all(got[t] >= 0)
+    ref_out, ref_lse = oracle.sparse_attn(W.subset_queries(wl, np.array([t])), got[t:t + 1])
+    parity.check_attention(out.float().cpu().numpy()[t:t + 1], ref_out, LONG.kv_dtype)
+    parity.check_lse(lse.cpu().numpy()[t:t + 1], ref_lse)
+
+
 # ------------------------------------------------ device-side data errors ---
 
 def test_bad_page_id_is_reported_not_faulted():
