@@ -111,17 +111,21 @@ cudaError_t launch_topk_rowwise(const float *scores, int64_t ld, const int32_t *
 
 // Histogram-guided exact top-K for rows scored by the tensor-core indexer
 // (which filled `hist`, [n_q, kHistBins]).  Scratch: sel [n_q, top_k],
-// counts [n_q, kTopkCountsPerQuery] (zeroed), cand [n_q, cap].
+// counts [n_q, kTopkCountsPerQuery] (zeroed), cand [n_q, cap], chunk_info.
 constexpr int32_t kTopkCandCap = 8192;
-constexpr int32_t kTopkCountsPerQuery = 8;
+constexpr int32_t kTopkCountsPerQuery = 2;
+// Rows longer than this many positions per chunk split into chunks; chunk_info
+// [n_q, topk_chunk_slots(ld)] (int4) holds each chunk's list slots.
+constexpr int32_t kTopkChunk = 8192;
+inline int64_t topk_chunk_slots(int64_t ld) { return (ld + kTopkChunk - 1) / kTopkChunk; }
 // With `rows` non-null it also writes the physical cache rows of the
 // selection for the tensor-core attention (compact_rows layout, tile 64,
 // leading dimension ld_rows) and their count n_valid [n_q].
 cudaError_t launch_topk_hist(const float *scores, int64_t ld, const int32_t *vis,
                              const uint32_t *hist, int32_t n_q, int32_t max_valid, int32_t top_k,
                              int32_t *sel, int32_t *counts, uint64_t *cand, int32_t cap,
-                             int32_t *idx, const PathParams &p, int32_t *rows, int32_t ld_rows,
-                             int32_t *n_valid, cudaStream_t s);
+                             int4 *chunk_info, int32_t *idx, const PathParams &p, int32_t *rows,
+                             int32_t ld_rows, int32_t *n_valid, cudaStream_t s);
 
 cudaError_t launch_attn_simt(const PathParams &p, const int32_t *idx, int32_t top_k, void *out,
                              int32_t out_dtype, float *lse, cudaStream_t s);

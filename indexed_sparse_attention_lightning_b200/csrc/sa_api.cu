@@ -124,15 +124,16 @@ PathParams make_params(const sa_cache *c, const sa_query *q, void *ws) {
 }
 
 // Workspace: status | vis [n_q] | tile_end [n_q] | scores [n_q, ld] | idx [n_q, K]
-// | hist [n_q, 4096] | counts [n_q, 8] | sel [n_q, K] | cand [n_q, cap]
-// | rows [n_q, R] | n_valid [n_q] | o_part [n_q, S, 128, 512]
+// | hist [n_q, 4096] | counts [n_q, 2] | sel [n_q, K] | cand [n_q, cap]
+// | chunk_info [n_q, C] | rows [n_q, R] | n_valid [n_q] | o_part [n_q, S, 128, 512]
 // | lse_part [n_q, S, 128]; the indexer needs the first three, the fused path
 // all of them; the attention alone needs the status, the compacted rows and
 // the split-KV partials (placed right after the status).
 struct Layout {
     int64_t ld;
     int32_t splits;
-    size_t vis, tile_end, scores, idx, hist, counts, sel, cand, rows, n_valid, o_part, lse_part;
+    size_t vis, tile_end, scores, idx, hist, counts, sel, cand, chunk_info, rows, n_valid, o_part,
+        lse_part;
     size_t indexer_total, decode_total;
     size_t attn_rows, attn_n_valid, attn_o_part, attn_lse_part, attn_total;
 };
@@ -159,7 +160,8 @@ Layout make_layout(const sa_query *q, int32_t top_k) {
     l.sel = align_up(l.counts + sizeof(int32_t) * kTopkCountsPerQuery * nq);
     l.cand = align_up(l.sel + sizeof(int32_t) * nq * kk);
     const size_t rows_bytes = sizeof(int32_t) * nq * (size_t)sfa_rows_ld(top_k);
-    l.rows = align_up(l.cand + sizeof(uint64_t) * nq * kTopkCandCap);
+    l.chunk_info = align_up(l.cand + sizeof(uint64_t) * nq * kTopkCandCap);
+    l.rows = align_up(l.chunk_info + sizeof(int4) * nq * (size_t)topk_chunk_slots(l.ld));
     l.n_valid = align_up(l.rows + rows_bytes);
     l.o_part = align_up(l.n_valid + sizeof(int32_t) * nq);
     l.lse_part = align_up(l.o_part + o_bytes);
@@ -344,7 +346,8 @@ static sa_status decode_impl(const sa_cache *cache, const sa_query *query, int32
                 reinterpret_cast<const uint32_t *>(base + l.hist), query->n_q, query->max_visible,
                 top_k, reinterpret_cast<int32_t *>(base + l.sel),
                 reinterpret_cast<int32_t *>(base + l.counts),
-                reinterpret_cast<uint64_t *>(base + l.cand), kTopkCandCap, idx, p,
+                reinterpret_cast<uint64_t *>(base + l.cand), kTopkCandCap,
+                reinterpret_cast<int4 *>(base + l.chunk_info), idx, p,
                 rows_ready ? reinterpret_cast<int32_t *>(base + l.rows) : nullptr,
                 sfa_rows_ld(top_k),
                 rows_ready ? reinterpret_cast<int32_t *>(base + l.n_valid) : nullptr, s));

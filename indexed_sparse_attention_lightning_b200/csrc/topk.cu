@@ -271,23 +271,23 @@ __device__ __forceinline__ int collect_prefix(int v, int *warp_sums, int *total)
     return before + incl - v;
 }
 
-// Long rows (more than kSingleMaxV positions) take three kernels, each with
-// many CTAs per query where the work is per position:
-//   count      per 8192-position chunk: keys above the threshold bucket are
-//              counted (per chunk), keys inside it are collected as composite
-//              candidates;
-//   threshold  one CTA per query: the exact need-th largest candidate (so an
-//              exact composite threshold for the whole row) and each chunk's
-//              first output slot;
-//   emit       per chunk again: its selected positions, in ascending order,
-//              and their physical cache rows, written straight to their slots.
-// Per-query state (counts, [n_q, 8] int32, zeroed with the histograms):
-//   [0] keys above the bucket, [1] candidates, [2] emit CTAs finished,
-//   [3] an unmapped page was met, [4..5] threshold mask, [6..7] threshold
-//   prefix (mask 0: the threshold kernel selected the whole row itself).
-constexpr int kChunk = 8192;                             // positions per count / emit CTA
+// Long rows (more than kSingleMaxV positions) take two kernels:
+//   count     many CTAs per query, one per 8192-position chunk: the chunk's keys
+//             above the threshold bucket go, in ascending position order, to
+//             a per-query list (one reservation per chunk), its keys inside the
+//             bucket to the candidate list as composite keys (likewise), and
+//             the chunk's four numbers (first slot and count in each list) to
+//             chunk_info;
+//   finalize  one CTA per query: the exact need-th largest candidate (an exact
+//             composite threshold), then every selected position's output slot
+//             from its chunk's first slot, its place in its own list and a
+//             binary search in the chunk's other list -- positions ascending,
+//             no pass over the row -- with its physical cache row.
+// Per-query counters (counts, [n_q, kTopkCountsPerQuery] int32, zeroed with
+// the histograms): [0] keys above the bucket, [1] candidates.
+constexpr int kChunk = kTopkChunk;                       // positions per count CTA
 constexpr int kChunkPer = kChunk / kCollectThreads;      // 32 consecutive positions a thread
-constexpr int kCountsPerQuery = kTopkCountsPerQuery;
+static_assert(kChunkPer == 32, "a thread's run is one 32-bit selection mask");
 
 // The 32 scores of positions [p0, p0 + 32) of `row` (entries at or past V
 // are never selected; they read as 0).
@@ -309,13 +309,13 @@ __device__ __forceinline__ void load_run(const float *row, int64_t p0, int64_t V
 
 __global__ void __launch_bounds__(kCollectThreads)
 topk_count_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *__restrict__ vis,
-                  const uint32_t *__restrict__ hist, int32_t top_k, int32_t *__restrict__ chunk_slot,
-                  int32_t ld_chunks, int32_t *__restrict__ counts, uint64_t *__restrict__ cand,
-                  int32_t cap) {
+                  const uint32_t *__restrict__ hist, int32_t top_k, int32_t *__restrict__ above_pos,
+                  int4 *__restrict__ chunk_info, int32_t ld_chunks, int32_t *__restrict__ counts,
+                  uint64_t *__restrict__ cand, int32_t cap) {
     pdl_wait();
     pdl_trigger();
     __shared__ int warp_sums[kCollectThreads / 32];
-    __shared__ int32_t base_s;
+    __shared__ int32_t base_s[2];
     const int t = blockIdx.y, tid = threadIdx.x;
     const int32_t V = vis[t];
     const int64_t c0 = (int64_t)blockIdx.x * kChunk;
@@ -326,33 +326,42 @@ topk_count_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *_
     int bstar;
     uint32_t above;
     threshold_bucket(hist + (int64_t)t * kHistBins, top_k, &bstar, &above);
-    int nh = 0, ne = 0;
+    uint32_t hi = 0, eq = 0;  // this thread's keys above / inside the bucket
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
         const int b = static_cast<int>(order_key(x[i]) >> (32 - kHistBits));
-        nh += (p0 + i < V && b > bstar) ? 1 : 0;
-        ne += (p0 + i < V && b == bstar) ? 1 : 0;
+        if (p0 + i < V && b > bstar) hi |= 1u << i;
+        if (p0 + i < V && b == bstar) eq |= 1u << i;
     }
     int tot_h, tot_e;
-    collect_prefix(nh, warp_sums, &tot_h);
-    int oe = collect_prefix(ne, warp_sums, &tot_e);
-    int32_t *ct = counts + (int64_t)t * kCountsPerQuery;
+    int oh = collect_prefix(__popc(hi), warp_sums, &tot_h);
+    int oe = collect_prefix(__popc(eq), warp_sums, &tot_e);
+    int32_t *ct = counts + (int64_t)t * kTopkCountsPerQuery;
     if (tid == 0) {
-        // a row of more chunks than slots is left to the threshold kernel's fallback
-        if ((int)blockIdx.x < ld_chunks) chunk_slot[(int64_t)t * ld_chunks + blockIdx.x] = tot_h;
-        if (tot_h > 0) atomicAdd(&ct[0], tot_h);
-        base_s = tot_e > 0 ? atomicAdd(&ct[1], tot_e) : 0;
+        base_s[0] = tot_h > 0 ? atomicAdd(&ct[0], tot_h) : 0;
+        base_s[1] = tot_e > 0 ? atomicAdd(&ct[1], tot_e) : 0;
+        // a row of more chunks than slots is left to the finalize kernel's fallback
+        if ((int)blockIdx.x < ld_chunks)
+            chunk_info[(int64_t)t * ld_chunks + blockIdx.x] =
+                make_int4(base_s[0], tot_h, base_s[1], tot_e);
     }
     __syncthreads();
-    if (ne == 0) return;
-    oe += base_s;
+    oh += base_s[0];
+    oe += base_s[1];
+    int32_t *sel_t = above_pos + (int64_t)t * top_k;
+    while (hi != 0) {
+        const int i = __ffs(hi) - 1;
+        hi &= hi - 1;
+        if (oh < top_k) sel_t[oh] = static_cast<int32_t>(p0 + i);
+        ++oh;
+    }
+    if (eq == 0) return;
     uint64_t *cand_t = cand + (int64_t)t * cap;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-        const uint32_t key = order_key(x[i]);
-        if (p0 + i < V && static_cast<int>(key >> (32 - kHistBits)) == bstar) {
+    for (int i = 0; i < 32; ++i) {  // static indices: x stays in registers
+        if ((eq >> i) & 1u) {
             if (oe < cap)
-                cand_t[oe] = (static_cast<uint64_t>(key) << 32) |
+                cand_t[oe] = (static_cast<uint64_t>(order_key(x[i])) << 32) |
                              (0xFFFFFFFFu - static_cast<uint32_t>(p0 + i));
             ++oe;
         }
@@ -493,136 +502,140 @@ __device__ void emit_selection(const uint32_t *bits, int words, int32_t top_k, i
     if (threadIdx.x == 0) *n_valid = nv;
 }
 
-// One CTA per query: the exact composite threshold among the candidates and
-// every chunk's first output slot (chunk_slot: the count kernel's per-chunk
-// counts of keys above the bucket, replaced by the exclusive prefix of the
-// chunks' selected counts).  Rows the candidate buffer cannot hold (massive
-// exact ties), short rows and rows of more chunks than one CTA scans take the
-// row-wise radix select here, whole.
+// First index of the ascending list v[0, n) holding a value >= x.
+__device__ __forceinline__ int lower_bound(const int32_t *v, int n, int32_t x) {
+    int lo = 0;
+    while (n > 0) {
+        const int half = n >> 1;
+        if (v[lo + half] < x) {
+            lo += half + 1;
+            n -= half + 1;
+        } else {
+            n = half;
+        }
+    }
+    return lo;
+}
+
+// One CTA per query (see topk_count_kernel).  Rows the candidate buffer or the
+// above list cannot hold (massive exact ties, very large K), short rows and
+// rows of more chunks than one CTA handles take the row-wise radix select,
+// whole.
 constexpr int kMaxChunks = kThreads;
+constexpr int kMaxAbove = 8192;
+__host__ __device__ constexpr size_t finalize_smem_bytes(int cap) {
+    return (size_t)cap * 8 + (size_t)kMaxAbove * 4 + (size_t)(cap + 1) * 4 + (size_t)cap * 4 +
+           (size_t)kMaxChunks * 16 + 16;
+}
 __global__ void __launch_bounds__(kThreads)
-topk_threshold_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *__restrict__ vis,
-                      int32_t top_k, int32_t *__restrict__ chunk_slot, int32_t ld_chunks,
-                      int32_t *__restrict__ counts, const uint64_t *__restrict__ cand, int32_t cap,
-                      int32_t *__restrict__ idx, const PathParams p, int32_t *__restrict__ rows_all,
-                      int32_t ld_rows, int32_t *__restrict__ n_valid_all) {
+topk_finalize_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *__restrict__ vis,
+                     int32_t top_k, const int32_t *__restrict__ above_pos,
+                     const int4 *__restrict__ chunk_info, int32_t ld_chunks,
+                     const int32_t *__restrict__ counts, const uint64_t *__restrict__ cand,
+                     int32_t cap, int32_t *__restrict__ idx, const PathParams p,
+                     int32_t *__restrict__ rows_all, int32_t ld_rows,
+                     int32_t *__restrict__ n_valid_all) {
     pdl_wait();
     pdl_trigger();
-    extern __shared__ uint64_t cs[];  // [cap]
+    extern __shared__ uint64_t fin_smem[];
     __shared__ unsigned dh[1024];
     __shared__ int warp_sums[33];
-    __shared__ int chunk_sel[kMaxChunks];
+    __shared__ int slot_s[kMaxChunks], bbase_s[kMaxChunks], bcount_s[kMaxChunks];
     const int t = blockIdx.x, tid = threadIdx.x;
     const int32_t V = vis[t];
     int32_t *out = idx + (int64_t)t * top_k;
-    int32_t *ct = counts + (int64_t)t * kCountsPerQuery;
+    int32_t *rows = rows_all != nullptr ? rows_all + (int64_t)t * ld_rows : nullptr;
+    const int32_t *ct = counts + (int64_t)t * kTopkCountsPerQuery;
     const int32_t n_above = ct[0], n_cand = ct[1];
     const int32_t need = top_k - n_above;
     const int chunks = static_cast<int>((V + kChunk - 1) / kChunk);
-    const bool fits = V > top_k && n_cand <= cap && need > 0 && need <= n_cand &&
-                      chunks <= min(kMaxChunks, ld_chunks);
-    if (!fits) {  // threshold mask stays 0: the emit kernel leaves the row alone
+    const bool fits = V > top_k && n_cand <= cap && n_above <= kMaxAbove && need > 0 &&
+                      need <= n_cand && chunks <= min(kMaxChunks, ld_chunks);
+    if (!fits) {
         select_row(scores + (int64_t)t * ld, V, top_k, out);
-        if (rows_all != nullptr) {
+        if (rows != nullptr) {
             __syncthreads();
-            compact_rows(p, t, out, top_k, 64, rows_all + (int64_t)t * ld_rows, n_valid_all + t,
-                         warp_sums);
+            compact_rows(p, t, out, top_k, 64, rows, n_valid_all + t, warp_sums);
         }
         return;
     }
+    uint64_t *cs = fin_smem;                                    // [cap] candidates
+    int32_t *A = reinterpret_cast<int32_t *>(cs + cap);         // [kMaxAbove] above positions
+    int32_t *pre = A + kMaxAbove;                               // [cap + 1] selected before i
+    int32_t *B = pre + cap + 1;                                 // [cap] selected positions
+    int4 *ci = reinterpret_cast<int4 *>(
+        (reinterpret_cast<uintptr_t>(B + cap) + 15) & ~uintptr_t(15));  // [kMaxChunks]
     const uint64_t *cg = cand + (int64_t)t * cap;
+    const int32_t *ag = above_pos + (int64_t)t * top_k;
     for (int i = tid; i < n_cand; i += kThreads) cs[i] = cg[i];
-    for (int c = tid; c < chunks; c += kThreads) chunk_sel[c] = 0;
+    for (int i = tid; i < n_above; i += kThreads) A[i] = ag[i];
+    if (tid < chunks) ci[tid] = chunk_info[(int64_t)t * ld_chunks + tid];
     __syncthreads();
     uint64_t mask, prefix;
     candidate_threshold(cs, n_cand, need, static_cast<int>(cs[0] >> (64 - kHistBits)), dh,
                         warp_sums, &mask, &prefix);
-    for (int i = tid; i < n_cand; i += kThreads) {
-        const uint64_t k = cs[i];
-        if ((k & mask) >= prefix) {
-            const uint32_t pos = 0xFFFFFFFFu - static_cast<uint32_t>(k);
-            atomicAdd(&chunk_sel[pos / kChunk], 1);
-        }
+    // the selected candidates, compacted in list order (each chunk's stay
+    // contiguous and ascending)
+    const int per = (n_cand + kThreads - 1) / kThreads;
+    const int i0 = tid * per;
+    int mine = 0;
+    for (int k = 0; k < per; ++k) {
+        const int i = i0 + k;
+        if (i < n_cand && (cs[i] & mask) >= prefix) ++mine;
     }
+    int total;
+    int q = block_exclusive_prefix(mine, warp_sums, &total);
+    for (int k = 0; k < per; ++k) {
+        const int i = i0 + k;
+        if (i >= n_cand) break;
+        pre[i] = q;
+        if ((cs[i] & mask) >= prefix) B[q++] = static_cast<int32_t>(0xFFFFFFFFu - static_cast<uint32_t>(cs[i]));
+    }
+    if (tid == 0) pre[n_cand] = total;
     __syncthreads();
-    int32_t *slot = chunk_slot + (int64_t)t * ld_chunks;
-    const int mine = tid < chunks ? slot[tid] + chunk_sel[tid] : 0;
-    int total;
-    const int first = block_exclusive_prefix(mine, warp_sums, &total);
-    if (tid < chunks) slot[tid] = first;
-    if (tid == 0) {
-        uint64_t *thr = reinterpret_cast<uint64_t *>(ct + 4);
-        thr[0] = mask;
-        thr[1] = prefix;
+    // each chunk's first output slot
+    int cnt = 0;
+    if (tid < chunks) {
+        const int4 f = ci[tid];
+        bbase_s[tid] = pre[f.z];
+        bcount_s[tid] = pre[f.z + f.w] - pre[f.z];
+        cnt = f.y + bcount_s[tid];
     }
-}
-
-// Per chunk: its selected positions (composite key at or above the row's
-// threshold) in ascending order at the chunk's slot, with their physical
-// cache rows.  A thread's 32 consecutive positions lie in one 64-token page,
-// so one page-table lookup serves them all.  The last CTA of a query to finish
-// writes the row count and padding -- or, when a page id was invalid, redoes
-// the rows with compact_rows, which drops and reports the unmapped ones.
-__global__ void __launch_bounds__(kCollectThreads)
-topk_emit_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *__restrict__ vis,
-                 int32_t top_k, const int32_t *__restrict__ chunk_slot, int32_t ld_chunks,
-                 int32_t *__restrict__ counts, int32_t *__restrict__ idx, const PathParams p,
-                 int32_t *__restrict__ rows_all, int32_t ld_rows,
-                 int32_t *__restrict__ n_valid_all) {
-    pdl_wait();
-    pdl_trigger();
-    __shared__ int warp_sums[33];
-    __shared__ int last_s;
-    const int t = blockIdx.y, tid = threadIdx.x;
-    const int32_t V = vis[t];
-    int32_t *ct = counts + (int64_t)t * kCountsPerQuery;
-    const uint64_t *thr = reinterpret_cast<const uint64_t *>(ct + 4);
-    const uint64_t mask = thr[0], prefix = thr[1];
-    const int chunks = static_cast<int>((V + kChunk - 1) / kChunk);
-    if (mask == 0 || (int)blockIdx.x >= chunks) return;  // uniform over the CTA
-    const int64_t p0 = (int64_t)blockIdx.x * kChunk + (int64_t)kChunkPer * tid;
-    float x[32];
-    load_run(scores + (int64_t)t * ld, p0, V, x);
-    uint32_t sel = 0;
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-        const uint64_t k = (static_cast<uint64_t>(order_key(x[i])) << 32) |
-                           (0xFFFFFFFFu - static_cast<uint32_t>(p0 + i));
-        if (p0 + i < V && (k & mask) >= prefix) sel |= 1u << i;
-    }
-    int total;
-    int q = chunk_slot[(int64_t)t * ld_chunks + blockIdx.x] +
-            collect_prefix(__popc(sel), warp_sums, &total);
-    int32_t *out = idx + (int64_t)t * top_k;
-    int32_t *rows = rows_all != nullptr ? rows_all + (int64_t)t * ld_rows : nullptr;
-    int64_t r0 = 0;
-    if (rows != nullptr && sel != 0) {
-        r0 = phys_row(p.page_table, p.max_pages, p.num_pages, __ldg(p.q_seq + t), p0);
-        if (r0 < 0) atomicOr(&ct[3], 1);
-    }
-    while (sel != 0) {
-        const int i = __ffs(sel) - 1;
-        sel &= sel - 1;
-        if (q < top_k) {
-            out[q] = static_cast<int32_t>(p0 + i);
-            if (rows != nullptr && r0 >= 0) rows[q] = static_cast<int32_t>(r0 + i);
+    const int first = block_exclusive_prefix(cnt, warp_sums, &total);
+    if (tid < chunks) slot_s[tid] = first;
+    __syncthreads();
+    // every selected position to its slot, with its physical row
+    const int32_t seq = __ldg(p.q_seq + t);
+    int bad = 0;
+    for (int e = tid; e < n_above + need; e += kThreads) {
+        int32_t pos;
+        int slot;
+        if (e < n_above) {
+            pos = A[e];
+            const int c = pos / kChunk;
+            slot = slot_s[c] + (e - ci[c].x) + lower_bound(B + bbase_s[c], bcount_s[c], pos);
+        } else {
+            const int j = e - n_above;
+            pos = B[j];
+            const int c = pos / kChunk;
+            const int4 f = ci[c];
+            slot = slot_s[c] + (j - bbase_s[c]) + lower_bound(A + f.x, f.y, pos);
         }
-        ++q;
+        if (slot < 0 || slot >= top_k) continue;  // only if the lists disagree with the counts
+        out[slot] = pos;
+        if (rows != nullptr) {
+            const int64_t r = phys_row(p.page_table, p.max_pages, p.num_pages, seq, pos);
+            if (r < 0) bad = 1;
+            else rows[slot] = static_cast<int32_t>(r);
+        }
     }
     if (rows == nullptr) return;
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) last_s = atomicAdd(&ct[2], 1) == chunks - 1;
-    __syncthreads();
-    if (!last_s) return;
-    __threadfence();  // every chunk's positions and rows are visible from here
-    if (*reinterpret_cast<volatile int32_t *>(&ct[3]) != 0) {
+    if (__syncthreads_or(bad)) {  // rare: drop (and report) the unmapped rows
         compact_rows(p, t, out, top_k, 64, rows, n_valid_all + t, warp_sums);
         return;
     }
     const int32_t padded = (top_k + 63) / 64 * 64;
-    const int32_t first = *reinterpret_cast<volatile int32_t *>(rows);
-    for (int c = top_k + tid; c < padded; c += kCollectThreads) rows[c] = first;
+    for (int c = top_k + tid; c < padded; c += kThreads) rows[c] = rows[0];
     if (tid == 0) n_valid_all[t] = top_k;
 }
 
@@ -783,8 +796,8 @@ topk_single_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *
 cudaError_t launch_topk_hist(const float *scores, int64_t ld, const int32_t *vis,
                              const uint32_t *hist, int32_t n_q, int32_t max_valid, int32_t top_k,
                              int32_t *sel, int32_t *counts, uint64_t *cand, int32_t cap,
-                             int32_t *idx, const PathParams &p, int32_t *rows, int32_t ld_rows,
-                             int32_t *n_valid, cudaStream_t s) {
+                             int4 *chunk_info, int32_t *idx, const PathParams &p, int32_t *rows,
+                             int32_t ld_rows, int32_t *n_valid, cudaStream_t s) {
     if (n_q == 0) return cudaSuccess;
     if (max_valid <= kSingleMaxV) {
         cudaError_t e = cudaFuncSetAttribute(
@@ -796,26 +809,20 @@ cudaError_t launch_topk_hist(const float *scores, int64_t ld, const int32_t *vis
     }
     const int32_t chunks = static_cast<int32_t>(ceil_div(std::max(max_valid, 1), kChunk));
     const dim3 grid_c(static_cast<unsigned>(chunks), n_q);
-    // per-chunk counts, then slots, in `sel` ([n_q, top_k]; rows of more
-    // chunks than top_k fall back to the row-wise select)
-    const int32_t ld_chunks = top_k;
+    const int32_t ld_chunks = static_cast<int32_t>(topk_chunk_slots(ld));
     count_launch();
     cudaError_t e = launch_pdl(topk_count_kernel, grid_c, dim3(kCollectThreads), 0, s, scores, ld,
-                               vis, hist, top_k, sel, ld_chunks, counts, cand, cap);
+                               vis, hist, top_k, sel, chunk_info, ld_chunks, counts, cand, cap);
     if (e != cudaSuccess) return e;
-    const size_t smem = (size_t)cap * 8;
-    e = cudaFuncSetAttribute(topk_threshold_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    const size_t smem = finalize_smem_bytes(cap);
+    e = cudaFuncSetAttribute(topk_finalize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem);
     if (e != cudaSuccess) return e;
     count_launch();
-    e = launch_pdl(topk_threshold_kernel, dim3(n_q), dim3(kThreads), smem, s, scores, ld, vis,
-                   top_k, sel, ld_chunks, counts, (const uint64_t *)cand, cap, idx, p, rows,
-                   ld_rows, n_valid);
-    if (e != cudaSuccess) return e;
-    count_launch();
-    return launch_pdl(topk_emit_kernel, grid_c, dim3(kCollectThreads), 0, s, scores, ld, vis,
-                      top_k, (const int32_t *)sel, ld_chunks, counts, idx, p, rows, ld_rows,
-                      n_valid);
+    return launch_pdl(topk_finalize_kernel, dim3(n_q), dim3(kThreads), smem, s, scores, ld, vis,
+                      top_k, (const int32_t *)sel, (const int4 *)chunk_info, ld_chunks,
+                      (const int32_t *)counts, (const uint64_t *)cand, cap, idx, p, rows,
+                      ld_rows, n_valid);
 }
 
 cudaError_t launch_topk_rowwise(const float *scores, int64_t ld, const int32_t *valid_len,
