@@ -447,7 +447,7 @@ __device__ void mark_top_candidates(const uint64_t *cs, int n_cand, int need, in
 // serialises many page-table loads.  All threads call it.
 __device__ void emit_selection(const uint32_t *bits, int words, int32_t top_k, int32_t *out,
                                const PathParams &p, int32_t t, int32_t *rows, int32_t *n_valid,
-                               int *warp_sums) {
+                               int *warp_sums, const int32_t *pt_smem = nullptr) {
     // each warp owns a run of words and walks it 32 words at a time, one
     // word per lane, so a run dense with selected keys is shared by 32 lanes
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -488,7 +488,14 @@ __device__ void emit_selection(const uint32_t *bits, int words, int32_t top_k, i
     const int32_t seq = __ldg(p.q_seq + t);
     int bad_page = 0;
     for (int i = threadIdx.x; i < nv; i += kThreads) {
-        const int64_t row = phys_row(p.page_table, p.max_pages, p.num_pages, seq, out[i]);
+        const int32_t s = out[i];
+        int64_t row;
+        if (pt_smem != nullptr) {  // the sequence's page-table row, staged by the caller
+            const int32_t page = pt_smem[s >> 6];
+            row = (page < 0 || page >= p.num_pages) ? -1 : (int64_t)page * 64 + (s & 63);
+        } else {
+            row = phys_row(p.page_table, p.max_pages, p.num_pages, seq, s);
+        }
         if (row < 0) bad_page = 1;
         else rows[i] = static_cast<int32_t>(row);
     }
@@ -642,15 +649,39 @@ topk_finalize_kernel(const float *__restrict__ scores, int64_t ld, const int32_t
 // ---------------------------------------------------------------------------
 // Rows of at most kSingleMaxV positions (decode at up to 64K context): the
 // whole selection in one CTA per query.  One pass over the row (from L2: the
-// indexer has just written it) marks the keys above the threshold bucket in
-// a shared-memory bitmap and collects the bucket's keys; the need-th largest
-// candidate follows from 10-bit radix passes over composite keys (score key,
-// inverted position: distinct, ties to the lower position), normally two;
-// the bitmap is then read back in ascending order.
+// indexer has just written it; the first 32K positions' loads are issued
+// before the threshold bucket is even known) marks the keys above the
+// threshold bucket in a shared-memory bitmap and collects the bucket's keys,
+// each thread's at a slot from one block-wide prefix (no shared counter); the
+// need-th largest candidate follows from 10-bit radix passes over composite
+// keys (score key, inverted position: distinct, ties to the lower position),
+// normally two; the bitmap is then read back in ascending order, the physical
+// rows looked up in a copy of the sequence's page-table row in shared memory.
 // ---------------------------------------------------------------------------
 constexpr int32_t kSingleMaxV = 65536;
 constexpr int32_t kSingleCap = 8192;  // candidates held in shared memory
-constexpr size_t kSingleSmem = (size_t)kSingleCap * 8 + (size_t)kSingleMaxV / 8;
+constexpr size_t kSingleSmem =
+    (size_t)kSingleCap * 8 + (size_t)kSingleMaxV / 8 + (size_t)kSingleMaxV / 64 * 4;
+
+// Scores b0 + 4 (threadIdx.x + u kThreads) .. + 3 of `row` for u < kSingleBatch
+// (entries at or past V read as 0 and are never selected), all loads issued
+// before any is used.
+constexpr int kSingleBatch = 8;
+__device__ __forceinline__ void load_single_batch(const float *row, int32_t b0, int32_t V,
+                                                  float4 (&xs)[kSingleBatch]) {
+#pragma unroll
+    for (int u = 0; u < kSingleBatch; ++u) {
+        const int32_t i0 = b0 + 4 * (threadIdx.x + u * kThreads);
+        if (i0 + 4 <= V) {
+            xs[u] = *reinterpret_cast<const float4 *>(row + i0);
+        } else {
+            xs[u].x = i0 < V ? row[i0] : 0.f;
+            xs[u].y = i0 + 1 < V ? row[i0 + 1] : 0.f;
+            xs[u].z = i0 + 2 < V ? row[i0 + 2] : 0.f;
+            xs[u].w = i0 + 3 < V ? row[i0 + 3] : 0.f;
+        }
+    }
+}
 
 __global__ void __launch_bounds__(kThreads)
 topk_single_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *__restrict__ vis,
@@ -660,24 +691,39 @@ topk_single_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *
     pdl_wait();
     pdl_trigger();
     extern __shared__ uint64_t single_smem[];
-    uint64_t *cs = single_smem;                                           // [kSingleCap]
+    uint64_t *cs = single_smem;                                               // [kSingleCap]
     uint32_t *bits = reinterpret_cast<uint32_t *>(single_smem + kSingleCap);  // [V / 32]
+    int32_t *pt = reinterpret_cast<int32_t *>(bits + kSingleMaxV / 32);       // [V / 64]
     __shared__ unsigned dh[1024];
     __shared__ int warp_sums[33];
-    __shared__ int n_cand_s, bstar_s, above_s;
+    __shared__ int bstar_s, above_s;
     const int t = blockIdx.x, tid = threadIdx.x, lane = tid & 31;
     const int32_t V = vis[t];
     int32_t *out = idx + (int64_t)t * top_k;
     int32_t *rows = rows_all != nullptr ? rows_all + (int64_t)t * ld_rows : nullptr;
     int32_t *nv_out = n_valid_all != nullptr ? n_valid_all + t : nullptr;
     const int words = (V + 31) / 32;
+    // the sequence's page-table row, for the physical rows at the end (rows
+    // past max_pages are looked up, and reported, the usual way)
+    const int slots = min((V + 63) / 64, p.max_pages);
+    if (rows != nullptr) {
+        const int32_t *ptg = p.page_table + (int64_t)__ldg(p.q_seq + t) * p.max_pages;
+        for (int i = tid; i < slots; i += kThreads) pt[i] = __ldg(ptg + i);
+    }
+    const int32_t *pts = (rows != nullptr && (V + 63) / 64 <= p.max_pages) ? pt : nullptr;
     if (V <= top_k) {  // everything visible is selected
         for (int w = tid; w < words; w += kThreads)
             bits[w] = (32 * w + 32 <= V) ? 0xFFFFFFFFu : ((1u << (V & 31)) - 1u);
         __syncthreads();
-        emit_selection(bits, words, top_k, out, p, t, rows, nv_out, warp_sums);
+        emit_selection(bits, words, top_k, out, p, t, rows, nv_out, warp_sums, pts);
         return;
     }
+    // the first batch of the row (a row of up to 32K positions is one batch;
+    // the trip count is the same in every lane) -- issued before the bucket
+    // search
+    const float *row = scores + (int64_t)t * ld;
+    float4 xs[kSingleBatch];
+    load_single_batch(row, 0, V, xs);
     // threshold bucket b*: thread i holds the buckets of rank 4i .. 4i+3 from the top
     const uint32_t *h = hist + (int64_t)t * kHistBins;
     uint32_t c[4], mine = 0;
@@ -689,7 +735,6 @@ topk_single_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *
     if (tid == 0) {
         bstar_s = -1;
         above_s = 0;
-        n_cand_s = 0;
     }
     int tot;
     int excl = block_exclusive_prefix((int)mine, warp_sums, &tot);
@@ -710,40 +755,23 @@ topk_single_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *
     const int bstar = bstar_s;
     const int32_t need = top_k - above_s;
     bool fallback = bstar < 0;
+    int n_cand = 0;
     if (!fallback) {
         // one pass over the row: keys above b* into the bitmap, b*'s keys collected
-        const float *row = scores + (int64_t)t * ld;
-        // all loads of a batch in flight before any is used (a row of up to
-        // 32K positions is one batch); the trip count is the same in every lane
-        constexpr int kBatch = 8;
-        for (int32_t b0 = 0; b0 < V; b0 += 4 * kThreads * kBatch) {
-            float4 xs[kBatch];
+        for (int32_t b0 = 0; b0 < V; b0 += 4 * kThreads * kSingleBatch) {
+            if (b0 > 0) load_single_batch(row, b0, V, xs);
+            uint32_t cmask = 0;  // this thread's keys in the bucket: bit 4u + e
 #pragma unroll
-            for (int u = 0; u < kBatch; ++u) {
-                const int32_t i0 = b0 + 4 * (tid + u * kThreads);
-                if (i0 + 4 <= V) {
-                    xs[u] = *reinterpret_cast<const float4 *>(row + i0);
-                } else {
-                    xs[u].x = i0 < V ? row[i0] : 0.f;
-                    xs[u].y = i0 + 1 < V ? row[i0 + 1] : 0.f;
-                    xs[u].z = i0 + 2 < V ? row[i0 + 2] : 0.f;
-                    xs[u].w = i0 + 3 < V ? row[i0 + 3] : 0.f;
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < kBatch; ++u) {
+            for (int u = 0; u < kSingleBatch; ++u) {
                 const int32_t i0 = b0 + 4 * (tid + u * kThreads);
                 const float x[4] = {xs[u].x, xs[u].y, xs[u].z, xs[u].w};
                 uint32_t above_mask = 0;
-                int n_eq = 0;
-                uint32_t keys[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    keys[e] = order_key(x[e]);
-                    const int b = static_cast<int>(keys[e] >> (32 - kHistBits));
+                    const int b = static_cast<int>(order_key(x[e]) >> (32 - kHistBits));
                     const bool valid = i0 + e < V;
                     if (valid && b > bstar) above_mask |= 1u << e;
-                    if (valid && b == bstar) ++n_eq;
+                    if (valid && b == bstar) cmask |= 1u << (4 * u + e);
                 }
                 // the 8 lanes of a 32-position word combine their 4-bit masks
                 // (lane l holds positions 4l .. 4l + 3 of the warp's 128), and
@@ -753,30 +781,24 @@ topk_single_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *
                 word |= __shfl_xor_sync(0xffffffffu, word, 2);
                 word |= __shfl_xor_sync(0xffffffffu, word, 4);
                 if ((lane & 7) == 0 && i0 < V) bits[i0 >> 5] = word;
-                // warp-aggregated slots for the bucket's keys
-                int incl = n_eq;
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const int n = __shfl_up_sync(0xffffffffu, incl, o);
-                    if (lane >= o) incl += n;
-                }
-                int base = 0;
-                if (lane == 31 && incl > 0) base = atomicAdd(&n_cand_s, incl);
-                base = __shfl_sync(0xffffffffu, base, 31) + incl - n_eq;
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int b = static_cast<int>(keys[e] >> (32 - kHistBits));
-                    if (i0 + e < V && b == bstar) {
-                        if (base < kSingleCap)
-                            cs[base] = (static_cast<uint64_t>(keys[e]) << 32) |
-                                       (0xFFFFFFFFu - static_cast<uint32_t>(i0 + e));
-                        ++base;
-                    }
-                }
+            }
+            // the bucket's keys (a few per thread, their scores read again from
+            // L2): every thread's at its slot of one block prefix
+            int total;
+            int base = n_cand + block_exclusive_prefix(__popc(cmask), warp_sums, &total);
+            n_cand += total;
+            while (cmask != 0) {
+                const int j = __ffs(cmask) - 1;
+                cmask &= cmask - 1;
+                const int32_t pos = b0 + 4 * (tid + (j >> 2) * kThreads) + (j & 3);
+                if (base < kSingleCap)
+                    cs[base] = (static_cast<uint64_t>(order_key(row[pos])) << 32) |
+                               (0xFFFFFFFFu - static_cast<uint32_t>(pos));
+                ++base;
             }
         }
         __syncthreads();
-        fallback = n_cand_s > kSingleCap || need < 1 || need > n_cand_s;
+        fallback = n_cand > kSingleCap || need < 1 || need > n_cand;
     }
     if (fallback) {  // histogram and scores disagree, or too many candidates
         select_row(scores + (int64_t)t * ld, V, top_k, out);
@@ -786,9 +808,9 @@ topk_single_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *
         }
         return;
     }
-    mark_top_candidates(cs, n_cand_s, need, bstar, bits, dh, warp_sums);
+    mark_top_candidates(cs, n_cand, need, bstar, bits, dh, warp_sums);
     __syncthreads();
-    emit_selection(bits, words, top_k, out, p, t, rows, nv_out, warp_sums);
+    emit_selection(bits, words, top_k, out, p, t, rows, nv_out, warp_sums, pts);
 }
 
 }  // namespace
