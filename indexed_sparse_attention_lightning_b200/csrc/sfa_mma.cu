@@ -60,7 +60,9 @@ constexpr int kDl = 512, kDr = 64, kD = kDl + kDr;
 constexpr int kBlocks = kD / 64;  // 64-dim (128-byte) column blocks of a row
 constexpr int kTile = 64;         // selected keys per tile
 constexpr int kStages = 3;
-constexpr int kPrefetch = 4;      // tiles of rows prefetched into L2 ahead of the copies
+// tiles of rows prefetched into L2 ahead of the copies (1 measured faster
+// than 2, 3, 4 or 6 on the 32K decode: 0.0945 against 0.0977 ms at 4)
+constexpr int kPrefetch = 1;
 constexpr int kProducerWarps = 7;
 constexpr int kSoftmaxWarp0 = 8;  // warps 8-11, one per TMEM subpartition
 constexpr int kThreads = 384;
@@ -426,7 +428,7 @@ sfa_mma_kernel(const __grid_constant__ CUtensorMap tm_q, const SfaArgs a) {
         // The ring holds about one tile in flight per SM, too little to cover
         // the latency of random row reads from HBM; so the rows of tile
         // n + kPrefetch are pulled into L2 (one bulk prefetch per row, by
-        // warps 1-2) while tile n is copied, and the copies mostly hit L2.
+        // warps 1-2) while tile n is copied, and the next copies start from L2.
         // Row indices are loaded one iteration before they are used, so no
         // global load latency sits between a freed stage and its copies.
         const int pk = pw * 32 + lane;  // key prefetched by this thread

@@ -304,6 +304,21 @@ def test_long_rows_match_oracle():
     assert np.array_equal(idx.cpu().numpy(), res["idx"])
 
 
+@pytest.mark.parametrize("top_k", [1000, 16])
+def test_long_rows_other_k(top_k):
+    """K = 1000 (rows padded to whole 64-row tiles for the attention) and K = 16
+    (more 8K-position chunks than K slots: the row-wise select takes the row)."""
+    sp = dataclasses.replace(LONG, name=f"long_rows_k{top_k}", top_k=top_k)
+    wl = workload(sp)
+    res = run_fused(wl)
+    assert res["status"] == (_abi.SA_OK, 0)
+    scores = oracle.index_scores(wl)
+    parity.check_topk(res["idx"], scores, wl.visible, top_k)
+    ref_out, ref_lse = oracle.sparse_attn(wl, res["idx"])
+    parity.check_attention(res["out"], ref_out, sp.kv_dtype)
+    parity.check_lse(res["lse"], ref_lse)
+
+
 def test_long_rows_with_massive_ties_take_lowest_positions():
     wl = workload(LONG)
     k = wl.k_index.copy()
