@@ -91,7 +91,11 @@ struct SfaSmem {
     // rows, each 8 x 128 bytes with the 128-byte swizzle (see kGroupBytes)
     uint8_t kv[kStages][kStageBytes];
     uint64_t kv_full[kStages], kv_empty[kStages];
-    uint64_t s_full[2], p_full[kStages], o_done, q_full, q_ready;
+    // o_done: one phase per P V (a rescale waits for the previous tile's);
+    // o_final: once, after the last P V, for the final read of O (P V of the
+    // last two tiles may both be in flight then, which o_done's parity cannot
+    // tell apart)
+    uint64_t s_full[2], p_full[kStages], o_done, o_final, q_full, q_ready;
     uint32_t tmem_base;
     int abort;
 };
@@ -173,6 +177,7 @@ sfa_mma_kernel(const __grid_constant__ CUtensorMap tm_q, const SfaArgs a) {
         for (int b = 0; b < 2; ++b) mbar_init(&sm.s_full[b], 1);
         for (int s = 0; s < kStages; ++s) mbar_init(&sm.p_full[s], 4);  // the four softmax warps
         mbar_init(&sm.o_done, 1);
+        mbar_init(&sm.o_final, 1);
         mbar_init(&sm.q_full, 1);
         mbar_init(&sm.q_ready, 4);
         sm.abort = 0;
@@ -340,7 +345,7 @@ sfa_mma_kernel(const __grid_constant__ CUtensorMap tm_q, const SfaArgs a) {
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.p_full[n % kStages]);
         }
-        if (ok && T > 0) ok = warp_wait(&sm.o_done, (T - 1) & 1, abort_flag, status);
+        if (ok && T > 0) ok = warp_wait(&sm.o_final, 0, abort_flag, status);
         tc_fence_after();
         // full row sums: the four threads of a head each hold a quarter
         l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
@@ -583,6 +588,11 @@ sfa_mma_kernel(const __grid_constant__ CUtensorMap tm_q, const SfaArgs a) {
                 break;
             }
         }
+        // o_final: every MMA issued above (all P V of the tiles) has completed;
+        // after a timeout too, so that TMEM is never released under an MMA
+        mma_commit(&sm.o_final);
+        int never = 0;
+        mbar_wait(&sm.o_final, 0, &never, status);
     }
     // with no tiles nobody waited for Q: its copy must land before the CTA ends
     if (warp == 0 && lane == 0 && T == 0) mbar_wait(&sm.q_full, 0, abort_flag, status);
