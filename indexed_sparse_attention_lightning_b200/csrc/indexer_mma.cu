@@ -313,6 +313,7 @@ indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
             TileCursor c;
             c.init_at(a.tile_end, sm.start_t, sm.start_i, k0, k1);
             bool seg_start = true;
+            const uint64_t key_policy = l2_evict_first_policy();
             // a unit's keys: its (first) query's sequence, up to its longest query
             auto unit_vis = [&](int32_t u) {
                 int32_t v = 0;
@@ -393,9 +394,18 @@ indexer_mma_kernel(const __grid_constant__ CUtensorMap tm_keys,
                 for (int h = 0; h < 2; ++h)
                     if (rows[h] >= 0) {
 #pragma unroll
-                        for (int ch = 0; ch < C::kChunks; ++ch)
-                            tma_load_2d(sm.keys[stage] + ch * (kKeys * kAtom) + h * (64 * kAtom),
-                                        &tm_keys, ch * C::kChunkElems, rows[h], &sm.full[stage]);
+                        for (int ch = 0; ch < C::kChunks; ++ch) {
+                            void *dst = sm.keys[stage] + ch * (kKeys * kAtom) + h * (64 * kAtom);
+                            // one query per tile: its keys are read once, so they
+                            // leave L2 first (the scores and the rows the next
+                            // kernels read stay); query groups share key tiles
+                            if constexpr (kQb == 1)
+                                tma_load_2d_hint(dst, &tm_keys, ch * C::kChunkElems, rows[h],
+                                                 &sm.full[stage], key_policy);
+                            else
+                                tma_load_2d(dst, &tm_keys, ch * C::kChunkElems, rows[h],
+                                            &sm.full[stage]);
+                        }
                         // 256 bytes a page either way: 64 fp32 scales, or 64 x 4
                         // E8M0 bytes (MXFP8, [num_pages, 64, 4] in memory)
                         if (!kBf16)
