@@ -148,7 +148,8 @@ typedef struct sa_query {
     float sm_scale;              /* softmax scale applied to q . kv */
 
     /* A promise for chunked prefill: queries 4i .. 4i+3 belong to one sequence
-     * (0 or 1: no promise).  With 4 and e4m3 index keys, the indexer scores
+     * (the last group may be shorter).  Any value but 4 makes no promise;
+     * negative values are rejected.  With 4 and e4m3 index keys, the indexer scores
      * each group against every key tile once (the tile shared by the four
      * queries); a group that breaks the promise is skipped and reported as
      * SA_DETAIL_BAD_POSITION. */
